@@ -1,0 +1,167 @@
+/*
+ * disco.h -- C ABI of libdisco, the B200 (sm_100a) DISCO convolution on the 2-sphere.
+ *
+ * The operation is the discrete-continuous convolution of the page
+ * "torch_harmonics.DiscreteContinuousConvS2" (forward equation and the
+ * definition of Psi below it):
+ *
+ *   out[b,o,j,q] = bias[o] + sum_{c in group(o)} sum_k w[o,c',k] * y[b,c,k,j,q]
+ *   y[b,c,k,j,q] = sum_{(i,p)} Psi[k,j,(i,p)] * x[b,c,i,(q*s + p) mod nlon_in]
+ *
+ * with s = nlon_in / nlon_out.  Psi is the filter basis evaluated at the
+ * input grid points rotated so that output point (j, 0) sits at the north
+ * pole, times the quadrature weights, normalised per (k, j) row ("nodal");
+ * equispaced longitudes make it independent of the output longitude
+ * (p-shift symmetry).  The constructor arguments of that page map onto
+ * disco_spec_t; input (B, C_in, nlat_in, nlon_in) and output
+ * (B, C_out, nlat_out, nlon_out) shapes are as printed there.
+ *
+ * Conventions for every compute call:
+ *   - Tensors are dense row-major (C order) in device memory, base 16-byte
+ *     aligned, in the storage dtype given (fp32 or bf16); the caller owns them.
+ *       x    (B, C_in, nlat_in, nlon_in)
+ *       w    (C_out, C_in/groups, K)
+ *       bias (C_out)                      may be NULL (no bias)
+ *       y    (B, C_in, K, nlat_out, nlon_out)   the K-expanded intermediate
+ *       out  (B, C_out, nlat_out, nlon_out)
+ *       dout like out, dx like x, dw like w, dbias like bias
+ *   - Output channel o belongs to group o / (C_out/groups) and reads input
+ *     channels of the same group (standard grouped convolution).
+ *   - Arithmetic is fp32 accumulate.  bf16 layers store x, w, y, out, dout,
+ *     dx, dw and dbias in bf16 (round to nearest even on store).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*,
+ *     NULL = legacy default stream).  They never synchronise and never
+ *     allocate device memory; scratch comes in through `workspace` of at
+ *     least disco_workspace_size() bytes (256-byte aligned).
+ *   - Errors are reported as a disco_status; nothing is thrown across the
+ *     ABI.  disco_last_error() returns a thread-local message for the last
+ *     non-OK status on the calling thread.
+ *   - A launch error is reported as DISCO_ERR_CUDA.  Faults that surface
+ *     later (asynchronously) are seen by the caller's next synchronisation.
+ */
+#ifndef DISCO_H
+#define DISCO_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DISCO_OK = 0,
+  DISCO_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, groups not dividing C_in/C_out,
+                                theta_cutoff <= 0, nlat < 2, n_r < 2 */
+  DISCO_ERR_UNSUPPORTED = 2, /* grid/basis/normalisation other than the ones below; nlon_in not a
+                                multiple of nlon_out (the p-shift needs output longitudes on input
+                                longitudes); stride nlon_in/nlon_out above 4; channel counts or
+                                K beyond the kernels' limits */
+  DISCO_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  DISCO_ERR_ALLOC = 4,       /* host allocation or the one-off Psi upload failed */
+  DISCO_ERR_TIMEOUT = 5,     /* a bounded device-side wait expired */
+  DISCO_ERR_GEOMETRY = 6     /* a distance or basis value fell inside the tie reject band
+                                (see disco_psi_build) */
+} disco_status;
+
+typedef enum { DISCO_F32 = 0, DISCO_BF16 = 1 } disco_dtype;
+
+enum { DISCO_GRID_EQUIANGULAR = 0 };           /* theta_i = pi*i/(nlat-1), poles included */
+enum { DISCO_BASIS_PIECEWISE_LINEAR = 0 };
+enum { DISCO_NORM_NODAL = 0 };                 /* every (k, j) row of Psi sums to one */
+
+/* Operation codes for disco_workspace_size. */
+enum {
+  DISCO_OP_FWD = 0,
+  DISCO_OP_FWD_FUSED = 1,
+  DISCO_OP_BWD_INPUT = 2,
+  DISCO_OP_BWD_WEIGHT = 3,           /* with y given */
+  DISCO_OP_BWD_WEIGHT_RECOMPUTE = 4  /* with y == NULL: y is recomputed from x */
+};
+
+/* Layer geometry: the in_shape / out_shape / kernel_shape / basis_type /
+ * basis_norm_mode / grid_in / grid_out / theta_cutoff arguments of the
+ * DiscreteContinuousConvS2 constructor.  kernel_shape = {n_r, n_alpha};
+ * n_alpha == 1 is the isotropic basis with K = n_r radial hats at
+ * r_k = k*theta_cutoff/(n_r-1); n_alpha > 1 is the anisotropic basis with
+ * K = 1 + (n_r-1)*n_alpha (the r = 0 hat merged, the outer radial hats times
+ * n_alpha azimuthal hats of the bearing east of local north).  The pages give
+ * no default cutoff, so theta_cutoff is required. */
+typedef struct {
+  int nlat_in, nlon_in, nlat_out, nlon_out;
+  int grid_in, grid_out;      /* DISCO_GRID_EQUIANGULAR only */
+  int kernel_shape[2];        /* {n_r, n_alpha} */
+  int basis_type;             /* DISCO_BASIS_PIECEWISE_LINEAR only */
+  int basis_norm_mode;        /* DISCO_NORM_NODAL only */
+  double theta_cutoff;        /* radians, > 0 */
+} disco_spec_t;
+
+/* Opaque Psi: owns a host copy (fp64 values) and the device plans. */
+typedef struct disco_psi disco_psi;
+
+/* Builds Psi on the host (synchronous; Clenshaw-Curtis quadrature, inclusive
+ * cutoff r <= theta_c + 1e-10, entries kept when phi_k > 1e-10, a computed
+ * r - theta_c or phi inside [1e-11, 1e-9] is DISCO_ERR_GEOMETRY) and uploads
+ * the kernels' plans to `device`.  On success *out owns everything until
+ * disco_psi_destroy.  On failure *out is NULL. */
+disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** out);
+
+/* Frees host and device memory of a Psi (synchronises the device first).  NULL is a no-op. */
+disco_status disco_psi_destroy(disco_psi* psi);
+
+/* K (number of basis functions) and nnz (number of non-zero Psi entries). */
+disco_status disco_psi_info(const disco_psi* psi, int* K, long long* nnz);
+
+/* Copies the nnz Psi entries to caller-owned HOST arrays of length nnz,
+ * sorted by (j, k, i, p), p in [0, nlon_in), values in fp64. */
+disco_status disco_psi_export(const disco_psi* psi, int* k, int* j, int* i, int* p, double* val);
+
+/* Bytes of scratch the operation needs (0 when none). */
+disco_status disco_workspace_size(const disco_psi* psi, int op, int B, int C_in, int C_out, int groups,
+                                  disco_dtype dtype, size_t* bytes);
+
+/* Forward, unfused: writes the K-expanded y (saved for backward) and out. */
+disco_status disco_fwd(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                       const void* x, const void* w, const void* bias, void* y, void* out,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* Forward, fused: out only; the K-expanded y is formed tile by tile on chip
+ * and never written to device memory (the `fused=True` mode of the page). */
+disco_status disco_fwd_fused(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                             const void* x, const void* w, const void* bias, void* out,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward with respect to x: dx = A^T dout, A the forward map without bias
+ * (the exact adjoint of contraction followed by the weight einsum). */
+disco_status disco_bwd_input(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                             const void* dout, const void* w, void* dx,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward with respect to w and bias:
+ *   dw[o,c',k] = sum_{b,j,q} dout[b,o,j,q] * y[b,c,k,j,q],  dbias[o] = sum_{b,j,q} dout[b,o,j,q].
+ * When y is NULL it is recomputed from x (the fused mode's one extra
+ * contraction).  dbias may be NULL.  The reduction order is fixed, so results
+ * are bitwise reproducible from run to run. */
+disco_status disco_bwd_weight(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                              const void* dout, const void* y, const void* x, void* dw, void* dbias,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/* Diagnostics: the host copy of a gather plan, for inspection by tests.
+ * which = 0 is the forward contraction plan (output rows j), which = 1 the
+ * adjoint plan used by disco_bwd_input (output rows i).  disco_plan_info fills
+ * dims[8] = {rows, source rows, chunks, values, value sets per chunk, source
+ * step per output, residue classes, ints per row record}.  disco_plan_export
+ * copies the records into caller-owned HOST arrays sized from dims: rows
+ * (rows x ints-per-row: row, src_begin, src_end, chunk_start[4], chunk_end[4],
+ * cost as float bits), source rows (x4: row, start, span, 0), chunks (x4: src,
+ * t0, voff, width | kmask << 8) and values. */
+disco_status disco_plan_info(const disco_psi* psi, int which, int* dims);
+disco_status disco_plan_export(const disco_psi* psi, int which, int* rows, int* srcs, int* chunks, float* vals);
+
+/* Thread-local description of the last non-OK status on this thread. */
+const char* disco_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DISCO_H */

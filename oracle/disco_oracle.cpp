@@ -290,16 +290,65 @@ void orc_mix(const void* hv, int B, int C_in, int C_out, int G, const double* y,
     }
 }
 
-// Full forward: y (optional) and out.
+namespace {
+
+// y planes of one input channel plane bc: yk[k][j][q] (the contraction of one channel).
+void contract_plane(const Psi* h, const double* xb, double* yk) {
+  const Spec& s = h->s;
+  const int K = h->K, sft = s.nlon_in / s.nlon_out;
+  const size_t yout = (size_t)s.nlat_out * s.nlon_out;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+  for (int k = 0; k < K; ++k)
+    for (int j = 0; j < s.nlat_out; ++j) {
+      double* yr = yk + (size_t)k * yout + (size_t)j * s.nlon_out;
+      const long long e0 = h->row[(size_t)j * K + k], e1 = h->row[(size_t)j * K + k + 1];
+      for (int q = 0; q < s.nlon_out; ++q) {
+        double acc = 0.0;
+        for (long long t = e0; t < e1; ++t) {
+          const Entry& e = h->e[t];
+          acc += e.val * xb[(size_t)e.i * s.nlon_in + (q * sft + e.p) % s.nlon_in];
+        }
+        yr[q] = acc;
+      }
+    }
+}
+
+}  // namespace
+
+// Full forward: y (optional) and out.  Channels are taken one plane at a
+// time (y of one channel, then its share of every output of its group), so
+// memory stays at one K-expanded plane; the sum over (c, k) runs in a fixed
+// order, the same for every output point.
 void orc_forward(const void* hv, int B, int C_in, int C_out, int G, const double* x, const double* w,
                  const double* bias, double* y_opt, double* out) {
   const Psi* h = static_cast<const Psi*>(hv);
-  const size_t ny = (size_t)B * C_in * h->K * h->s.nlat_out * h->s.nlon_out;
-  std::vector<double> tmp;
-  double* y = y_opt;
-  if (!y) { tmp.resize(ny); y = tmp.data(); }
-  orc_contract(hv, B, C_in, x, y);
-  orc_mix(hv, B, C_in, C_out, G, y, w, bias, out);
+  const Spec& s = h->s;
+  const int K = h->K, cg = C_in / G, og = C_out / G;
+  const size_t nin = (size_t)s.nlat_in * s.nlon_in, n = (size_t)s.nlat_out * s.nlon_out;
+  std::vector<double> yk((size_t)K * n);
+  std::fill(out, out + (size_t)B * C_out * n, 0.0);
+  for (int b = 0; b < B; ++b)
+    for (int c = 0; c < C_in; ++c) {
+      contract_plane(h, x + ((size_t)b * C_in + c) * nin, yk.data());
+      if (y_opt) std::copy(yk.begin(), yk.end(), y_opt + ((size_t)b * C_in + c) * K * n);
+      const int g = group_of(c, C_in, G), cl = c - g * cg;
+#pragma omp parallel for
+      for (int ol = 0; ol < og; ++ol) {
+        const int o = g * og + ol;
+        double* ob = out + ((size_t)b * C_out + o) * n;
+        for (int k = 0; k < K; ++k) {
+          const double wv = w[((size_t)o * cg + cl) * K + k];
+          const double* yr = yk.data() + (size_t)k * n;
+          for (size_t t = 0; t < n; ++t) ob[t] += wv * yr[t];
+        }
+      }
+    }
+  if (bias)
+    for (int b = 0; b < B; ++b)
+      for (int o = 0; o < C_out; ++o) {
+        double* ob = out + ((size_t)b * C_out + o) * n;
+        for (size_t t = 0; t < n; ++t) ob[t] += bias[o];
+      }
 }
 
 // dx = adjoint of the forward map (without bias) applied to dout.
@@ -335,25 +384,29 @@ void orc_backward_input(const void* hv, int B, int C_in, int C_out, int G, const
 }
 
 // dw[o, c', k] = sum_{b,j,q} dout[b,o,j,q] y[b,c,k,j,q];  dbias[o] = sum dout[b,o,:,:]
+// y is recomputed one channel plane at a time from x.
 void orc_backward_weight(const void* hv, int B, int C_in, int C_out, int G, const double* dout,
                          const double* x, double* dw, double* dbias) {
   const Psi* h = static_cast<const Psi*>(hv);
-  const int K = h->K, cg = C_in / G;
-  const size_t nout = (size_t)h->s.nlat_out * h->s.nlon_out;
-  std::vector<double> y((size_t)B * C_in * K * nout);
-  orc_contract(hv, B, C_in, x, y.data());
-#pragma omp parallel for collapse(2)
-  for (int o = 0; o < C_out; ++o)
-    for (int cl = 0; cl < cg; ++cl) {
-      const int g = group_of(o, C_out, G), c = g * cg + cl;
-      for (int k = 0; k < K; ++k) {
-        double acc = 0.0;
-        for (int b = 0; b < B; ++b) {
-          const double* db = dout + ((size_t)b * C_out + o) * nout;
-          const double* yb = y.data() + (((size_t)b * C_in + c) * K + k) * nout;
-          for (size_t t = 0; t < nout; ++t) acc += db[t] * yb[t];
+  const Spec& s = h->s;
+  const int K = h->K, cg = C_in / G, og = C_out / G;
+  const size_t nin = (size_t)s.nlat_in * s.nlon_in, nout = (size_t)s.nlat_out * s.nlon_out;
+  std::vector<double> yk((size_t)K * nout);
+  std::fill(dw, dw + (size_t)C_out * cg * K, 0.0);
+  for (int b = 0; b < B; ++b)
+    for (int c = 0; c < C_in; ++c) {
+      contract_plane(h, x + ((size_t)b * C_in + c) * nin, yk.data());
+      const int g = group_of(c, C_in, G), cl = c - g * cg;
+#pragma omp parallel for
+      for (int ol = 0; ol < og; ++ol) {
+        const int o = g * og + ol;
+        const double* db = dout + ((size_t)b * C_out + o) * nout;
+        for (int k = 0; k < K; ++k) {
+          const double* yr = yk.data() + (size_t)k * nout;
+          double acc = 0.0;
+          for (size_t t = 0; t < nout; ++t) acc += db[t] * yr[t];
+          dw[((size_t)o * cg + cl) * K + k] += acc;
         }
-        dw[((size_t)o * cg + cl) * K + k] = acc;
       }
     }
   if (dbias)

@@ -1,0 +1,190 @@
+"""PyTorch-facing DISCO layer on top of the libdisco C ABI.
+
+PyTorch supplies device memory, streams and autograd bookkeeping; every step
+of the convolution runs in libdisco's CUDA kernels (there is no CPU path).
+The layer mirrors the constructor of the page
+"torch_harmonics.DiscreteContinuousConvS2": in/out channels and shapes,
+kernel_shape, basis_type='piecewise linear', basis_norm_mode='nodal',
+groups, equiangular grids, bias, theta_cutoff and `fused`.  With
+fused=False the K-expanded intermediate is saved for backward; with
+fused=True only x is saved and the intermediate is recomputed in backward
+(K times less activation memory, one extra contraction).
+"""
+
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import disco as D
+
+_DTYPES = {torch.float32: D.DISCO_F32, torch.bfloat16: D.DISCO_BF16}
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+    return _DTYPES[t.dtype]
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("libdisco takes contiguous CUDA tensors")
+
+
+class Psi:
+    """Precomputed sparse convolution tensor of one layer geometry, on one device."""
+
+    def __init__(self, nlat_in: int, nlon_in: int, nlat_out: int, nlon_out: int, kernel_shape, theta_cutoff: float,
+                 device=None):
+        dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.device = dev
+        self.index = dev.index if dev.index is not None else torch.cuda.current_device()
+        self.in_shape = (nlat_in, nlon_in)
+        self.out_shape = (nlat_out, nlon_out)
+        self.kernel_shape = kernel_shape
+        self.theta_cutoff = float(theta_cutoff)
+        self.spec = D.make_spec(nlat_in, nlon_in, nlat_out, nlon_out, kernel_shape, theta_cutoff)
+        with torch.cuda.device(self.index):
+            self.handle = D.disco_psi_build(self.spec, self.index)
+        self.K, self.nnz = D.disco_psi_info(self.handle)
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h is not None and D is not None:
+            try:
+                D.disco_psi_destroy(h)
+            except Exception:
+                pass
+            self.handle = None
+
+    def workspace(self, op: int, B: int, C_in: int, C_out: int, groups: int, dtype: int):
+        n = D.disco_workspace_size(self.handle, op, B, C_in, C_out, groups, dtype)
+        if n == 0:
+            return None, 0
+        return torch.empty(n, dtype=torch.uint8, device=self.device), n
+
+
+def disco_forward(psi: Psi, x: torch.Tensor, w: torch.Tensor, bias=None, groups: int = 1, fused: bool = False):
+    """Returns (out, y); y is None when fused."""
+    _need_cuda(x, w, bias)
+    B, C_in = x.shape[:2]
+    C_out = w.shape[0]
+    dt = _dtype_code(x)
+    out = torch.empty((B, C_out) + psi.out_shape, dtype=x.dtype, device=x.device)
+    st = _stream(x.device)
+    if fused:
+        ws, n = psi.workspace(D.DISCO_OP_FWD_FUSED, B, C_in, C_out, groups, dt)
+        D.disco_fwd_fused(psi.handle, B, C_in, C_out, groups, dt, _ptr(x), _ptr(w), _ptr(bias), _ptr(out),
+                          _ptr(ws), n, st)
+        return out, None
+    y = torch.empty((B, C_in, psi.K) + psi.out_shape, dtype=x.dtype, device=x.device)
+    ws, n = psi.workspace(D.DISCO_OP_FWD, B, C_in, C_out, groups, dt)
+    D.disco_fwd(psi.handle, B, C_in, C_out, groups, dt, _ptr(x), _ptr(w), _ptr(bias), _ptr(y), _ptr(out),
+                _ptr(ws), n, st)
+    return out, y
+
+
+def disco_backward_input(psi: Psi, dout: torch.Tensor, w: torch.Tensor, C_in: int, groups: int = 1):
+    _need_cuda(dout, w)
+    B, C_out = dout.shape[:2]
+    dt = _dtype_code(dout)
+    dx = torch.empty((B, C_in) + psi.in_shape, dtype=dout.dtype, device=dout.device)
+    ws, n = psi.workspace(D.DISCO_OP_BWD_INPUT, B, C_in, C_out, groups, dt)
+    D.disco_bwd_input(psi.handle, B, C_in, C_out, groups, dt, _ptr(dout), _ptr(w), _ptr(dx), _ptr(ws), n,
+                      _stream(dout.device))
+    return dx
+
+
+def disco_backward_weight(psi: Psi, dout: torch.Tensor, y=None, x=None, groups: int = 1, C_in: int = None,
+                          need_bias: bool = True):
+    """(dw, dbias); y given, or x to recompute y."""
+    _need_cuda(dout, y, x)
+    B, C_out = dout.shape[:2]
+    C_in = y.shape[1] if y is not None else x.shape[1]
+    dt = _dtype_code(dout)
+    dw = torch.empty((C_out, C_in // groups, psi.K), dtype=dout.dtype, device=dout.device)
+    db = torch.empty((C_out,), dtype=dout.dtype, device=dout.device) if need_bias else None
+    op = D.DISCO_OP_BWD_WEIGHT if y is not None else D.DISCO_OP_BWD_WEIGHT_RECOMPUTE
+    ws, n = psi.workspace(op, B, C_in, C_out, groups, dt)
+    D.disco_bwd_weight(psi.handle, B, C_in, C_out, groups, dt, _ptr(dout), _ptr(y), _ptr(x), _ptr(dw), _ptr(db),
+                       _ptr(ws), n, _stream(dout.device))
+    return dw, db
+
+
+class _DiscoFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, w, bias, psi, groups):
+        out, y = disco_forward(psi, x.contiguous(), w.contiguous(), None if bias is None else bias.contiguous(),
+                               groups, fused=False)
+        ctx.save_for_backward(y, w)
+        ctx.psi, ctx.groups, ctx.C_in, ctx.has_bias = psi, groups, x.shape[1], bias is not None
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        y, w = ctx.saved_tensors
+        dout = dout.contiguous()
+        dx = disco_backward_input(ctx.psi, dout, w, ctx.C_in, ctx.groups) if ctx.needs_input_grad[0] else None
+        dw, db = disco_backward_weight(ctx.psi, dout, y=y, groups=ctx.groups, need_bias=ctx.has_bias)
+        return dx, dw, db, None, None
+
+
+class _DiscoFusedFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, w, bias, psi, groups):
+        x = x.contiguous()
+        out, _ = disco_forward(psi, x, w.contiguous(), None if bias is None else bias.contiguous(), groups,
+                               fused=True)
+        ctx.save_for_backward(x, w)
+        ctx.psi, ctx.groups, ctx.has_bias = psi, groups, bias is not None
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        x, w = ctx.saved_tensors
+        dout = dout.contiguous()
+        dx = disco_backward_input(ctx.psi, dout, w, x.shape[1], ctx.groups) if ctx.needs_input_grad[0] else None
+        dw, db = disco_backward_weight(ctx.psi, dout, x=x, groups=ctx.groups, need_bias=ctx.has_bias)
+        return dx, dw, db, None, None
+
+
+class DiscreteContinuousConvS2(torch.nn.Module):
+    """DISCO convolution on the 2-sphere (equiangular grids, piecewise-linear basis, nodal norm)."""
+
+    def __init__(self, in_channels, out_channels, in_shape, out_shape, kernel_shape, basis_type="piecewise linear",
+                 basis_norm_mode="nodal", groups=1, grid_in="equiangular", grid_out="equiangular", bias=True,
+                 theta_cutoff=None, optimized_kernel=True, fused=False, device=None, dtype=torch.float32):
+        super().__init__()
+        if basis_type != "piecewise linear" or basis_norm_mode != "nodal":
+            raise NotImplementedError("only basis_type='piecewise linear' with basis_norm_mode='nodal'")
+        if grid_in != "equiangular" or grid_out != "equiangular":
+            raise NotImplementedError("only equiangular grids")
+        if theta_cutoff is None:
+            raise ValueError("theta_cutoff is required (no default is defined for it)")
+        if not optimized_kernel:
+            raise NotImplementedError("only the CUDA kernels exist")
+        if in_channels % groups or out_channels % groups:
+            raise ValueError("groups must divide in_channels and out_channels")
+        self.groups, self.fused = groups, fused
+        self.psi = Psi(in_shape[0], in_shape[1], out_shape[0], out_shape[1], kernel_shape, theta_cutoff, device)
+        K = self.psi.K
+        scale = 1.0 / math.sqrt((in_channels // groups) * K)
+        self.weight = torch.nn.Parameter(
+            torch.randn(out_channels, in_channels // groups, K, device=self.psi.device, dtype=dtype) * scale)
+        self.bias = torch.nn.Parameter(torch.zeros(out_channels, device=self.psi.device, dtype=dtype)) if bias \
+            else None
+
+    def forward(self, x):
+        fn = _DiscoFusedFn if self.fused else _DiscoFn
+        return fn.apply(x, self.weight, self.bias, self.psi, self.groups)

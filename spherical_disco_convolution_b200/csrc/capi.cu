@@ -1,0 +1,444 @@
+// C ABI of libdisco: argument checks, workspace layout and kernel dispatch.
+// See include/disco.h for the contract of every entry point.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/disco.h"
+#include "kernels.h"
+#include "psi_builder.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+disco_status fail(disco_status s, const std::string& msg) {
+  g_last_error = msg;
+  return s;
+}
+
+disco_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(DISCO_ERR_CUDA, std::string(where) + ": " + cudaGetErrorString(e));
+}
+
+struct DevPlan {
+  disco::RowPlan* rows = nullptr;
+  disco::SrcRow* srcs = nullptr;
+  disco::Chunk* chunks = nullptr;
+  float* vals = nullptr;
+  int n_rows = 0;
+};
+
+template <typename T>
+cudaError_t upload(const std::vector<T>& v, T** dst) {
+  *dst = nullptr;
+  if (v.empty()) return cudaSuccess;
+  cudaError_t e = cudaMalloc(reinterpret_cast<void**>(dst), v.size() * sizeof(T));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpy(*dst, v.data(), v.size() * sizeof(T), cudaMemcpyHostToDevice);
+}
+
+cudaError_t upload_plan(const disco::GatherPlan& P, DevPlan* d) {
+  d->n_rows = (int)P.rows.size();
+  cudaError_t e;
+  if ((e = upload(P.rows, &d->rows)) != cudaSuccess) return e;
+  if ((e = upload(P.src, &d->srcs)) != cudaSuccess) return e;
+  if ((e = upload(P.chunks, &d->chunks)) != cudaSuccess) return e;
+  return upload(P.vals, &d->vals);
+}
+
+void free_plan(DevPlan* d) {
+  cudaFree(d->rows);
+  cudaFree(d->srcs);
+  cudaFree(d->chunks);
+  cudaFree(d->vals);
+  *d = DevPlan{};
+}
+
+constexpr int kChannelsPerCta = 16;
+constexpr int kStageFloats = 12288;          // 48 KB of staging for the unfused gathers
+constexpr size_t kSmemLimit = 227 * 1024;    // dynamic shared memory per CTA on sm_100
+constexpr size_t kFusedTileBytes = 160 * 1024;
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+}  // namespace
+
+struct disco_psi {
+  disco::Geometry g;
+  int device = -1;
+  std::vector<disco::PsiEntry> entries;
+  disco::GatherPlan fwd, adj;
+  DevPlan dfwd, dadj;
+};
+
+namespace {
+
+// Block of outputs per CTA: at most `cap` (a multiple of kTaskR), balanced over the row.
+void block_shape(int n, int cap, int* qb, int* nblk) {
+  int nb = (n + cap - 1) / cap;
+  const int per = (n + nb - 1) / nb;
+  *qb = (per + disco::kTaskR - 1) / disco::kTaskR * disco::kTaskR;
+  *nblk = (n + *qb - 1) / *qb;
+}
+
+int max_stage(const disco::GatherPlan& P, int qb) {
+  int m = 0;
+  for (const disco::RowPlan& r : P.rows) m = std::max(m, disco::stage_elems(P, r, qb));
+  return m;
+}
+
+disco::GatherArgs gather_args(const DevPlan& d, int BC, int qb, int nblk, int n_src, int n_src_rows, int n_out,
+                              int n_out_rows, int budget) {
+  disco::GatherArgs a;
+  a.rows = d.rows;
+  a.srcs = d.srcs;
+  a.chunks = d.chunks;
+  a.vals = d.vals;
+  a.n_rows = d.n_rows;
+  a.BC = BC;
+  a.cb = kChannelsPerCta;
+  a.qb = qb;
+  a.nblk = nblk;
+  a.n_src = n_src;
+  a.n_src_rows = n_src_rows;
+  a.n_out = n_out;
+  a.n_out_rows = n_out_rows;
+  a.stage_budget = budget;
+  return a;
+}
+
+disco_status check_common(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype) {
+  if (!psi) return fail(DISCO_ERR_INVALID_ARG, "psi is NULL");
+  if (psi->device < 0) return fail(DISCO_ERR_INVALID_ARG, "psi was built host-only (device < 0)");
+  if (B <= 0 || C_in <= 0 || C_out <= 0 || groups <= 0)
+    return fail(DISCO_ERR_INVALID_ARG, "B, C_in, C_out and groups must be positive");
+  if (C_in % groups || C_out % groups)
+    return fail(DISCO_ERR_INVALID_ARG, "groups must divide both C_in and C_out");
+  if (dtype != DISCO_F32 && dtype != DISCO_BF16) return fail(DISCO_ERR_INVALID_ARG, "unknown dtype");
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev != psi->device) return fail(DISCO_ERR_INVALID_ARG, "current device differs from the device of psi");
+  return DISCO_OK;
+}
+
+struct WsLayout {
+  size_t wt = 0, dy = 0, ybuf = 0, part = 0, bpart = 0, total = 0;
+  int nchunk = 0, nc = 0;
+};
+
+WsLayout layout(const disco_psi* psi, int op, int B, int C_in, int C_out, int groups, disco_dtype dtype) {
+  WsLayout L;
+  const size_t es = dtype == DISCO_BF16 ? 2 : 4;
+  const disco::Geometry& g = psi->g;
+  const size_t n_out = (size_t)g.nlat_out * g.nlon_out;
+  const size_t y_elems = (size_t)B * C_in * g.K * n_out;
+  if (op == DISCO_OP_BWD_INPUT) {
+    L.wt = 0;
+    L.dy = align256((size_t)C_out * (C_in / groups) * g.K * es);
+    L.total = L.dy + align256(y_elems * es);
+  } else if (op == DISCO_OP_BWD_WEIGHT || op == DISCO_OP_BWD_WEIGHT_RECOMPUTE) {
+    const int N = (int)n_out;
+    L.nc = 4096;
+    L.nchunk = (N + L.nc - 1) / L.nc;
+    const size_t nsplit = (size_t)B * L.nchunk;
+    size_t off = 0;
+    if (op == DISCO_OP_BWD_WEIGHT_RECOMPUTE) {
+      L.ybuf = 0;
+      off = align256(y_elems * es);
+    }
+    L.part = off;
+    off += align256(nsplit * (size_t)C_out * (C_in / groups) * g.K * sizeof(float));
+    L.bpart = off;
+    off += align256(nsplit * (size_t)C_out * sizeof(float));
+    L.total = off;
+  }
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* disco_last_error(void) { return g_last_error.c_str(); }
+
+disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** out) {
+  if (!out) return fail(DISCO_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!spec) return fail(DISCO_ERR_INVALID_ARG, "spec is NULL");
+  if (spec->grid_in != DISCO_GRID_EQUIANGULAR || spec->grid_out != DISCO_GRID_EQUIANGULAR)
+    return fail(DISCO_ERR_UNSUPPORTED, "only equiangular grids are supported");
+  if (spec->basis_type != DISCO_BASIS_PIECEWISE_LINEAR)
+    return fail(DISCO_ERR_UNSUPPORTED, "only the piecewise-linear basis is supported");
+  if (spec->basis_norm_mode != DISCO_NORM_NODAL)
+    return fail(DISCO_ERR_UNSUPPORTED, "only nodal basis normalisation is supported");
+  if (spec->nlat_in < 2 || spec->nlat_out < 2 || spec->nlon_in < 1 || spec->nlon_out < 1)
+    return fail(DISCO_ERR_INVALID_ARG, "grids need nlat >= 2 and nlon >= 1");
+  if (!(spec->theta_cutoff > 0.0)) return fail(DISCO_ERR_INVALID_ARG, "theta_cutoff must be > 0");
+  if (spec->kernel_shape[0] < 2 || spec->kernel_shape[1] < 1)
+    return fail(DISCO_ERR_INVALID_ARG, "kernel_shape needs n_r >= 2 and n_alpha >= 1");
+  if (spec->nlon_in % spec->nlon_out)
+    return fail(DISCO_ERR_UNSUPPORTED, "nlon_in must be a multiple of nlon_out (p-shift symmetry)");
+  disco::Geometry g;
+  g.nlat_in = spec->nlat_in;
+  g.nlon_in = spec->nlon_in;
+  g.nlat_out = spec->nlat_out;
+  g.nlon_out = spec->nlon_out;
+  g.n_r = spec->kernel_shape[0];
+  g.n_alpha = spec->kernel_shape[1];
+  g.theta_cutoff = spec->theta_cutoff;
+  g.K = g.n_alpha == 1 ? g.n_r : 1 + (g.n_r - 1) * g.n_alpha;
+  g.stride = g.nlon_in / g.nlon_out;
+  if (g.K > disco::kMaxK) return fail(DISCO_ERR_UNSUPPORTED, "more basis functions than the kernels support");
+  if (g.stride > disco::kMaxStride) return fail(DISCO_ERR_UNSUPPORTED, "nlon_in / nlon_out above 4");
+  disco_psi* h = new (std::nothrow) disco_psi;
+  if (!h) return fail(DISCO_ERR_ALLOC, "host allocation failed");
+  h->g = g;
+  std::string msg;
+  const int st = disco::build_psi_entries(g, h->entries, msg);
+  if (st) {
+    delete h;
+    return fail(static_cast<disco_status>(st), msg);
+  }
+  h->fwd = disco::make_forward_plan(g, h->entries);
+  h->adj = disco::make_adjoint_plan(g, h->entries);
+  if (h->fwd.max_src > disco::kMaxSrc || h->adj.max_src > disco::kMaxSrc) {
+    delete h;
+    return fail(DISCO_ERR_UNSUPPORTED, "an output row reaches more source rows than the kernels support");
+  }
+  h->device = device;
+  if (device >= 0) {
+    int prev = -1;
+    cudaGetDevice(&prev);
+    cudaError_t e = cudaSetDevice(device);
+    if (e == cudaSuccess) e = upload_plan(h->fwd, &h->dfwd);
+    if (e == cudaSuccess) e = upload_plan(h->adj, &h->dadj);
+    if (prev >= 0) cudaSetDevice(prev);
+    if (e != cudaSuccess) {
+      free_plan(&h->dfwd);
+      free_plan(&h->dadj);
+      delete h;
+      return fail(DISCO_ERR_ALLOC, std::string("Psi upload failed: ") + cudaGetErrorString(e));
+    }
+  }
+  *out = h;
+  return DISCO_OK;
+}
+
+disco_status disco_psi_destroy(disco_psi* psi) {
+  if (!psi) return DISCO_OK;
+  if (psi->device >= 0) {
+    int prev = -1;
+    cudaGetDevice(&prev);
+    cudaSetDevice(psi->device);
+    cudaDeviceSynchronize();
+    free_plan(&psi->dfwd);
+    free_plan(&psi->dadj);
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+  delete psi;
+  return DISCO_OK;
+}
+
+disco_status disco_psi_info(const disco_psi* psi, int* K, long long* nnz) {
+  if (!psi) return fail(DISCO_ERR_INVALID_ARG, "psi is NULL");
+  if (K) *K = psi->g.K;
+  if (nnz) *nnz = (long long)psi->entries.size();
+  return DISCO_OK;
+}
+
+disco_status disco_psi_export(const disco_psi* psi, int* k, int* j, int* i, int* p, double* val) {
+  if (!psi || !k || !j || !i || !p || !val) return fail(DISCO_ERR_INVALID_ARG, "NULL argument");
+  for (size_t t = 0; t < psi->entries.size(); ++t) {
+    const disco::PsiEntry& e = psi->entries[t];
+    k[t] = e.k;
+    j[t] = e.j;
+    i[t] = e.i;
+    p[t] = e.p;
+    val[t] = e.v;
+  }
+  return DISCO_OK;
+}
+
+disco_status disco_plan_info(const disco_psi* psi, int which, int* dims) {
+  if (!psi || !dims || (which != 0 && which != 1)) return fail(DISCO_ERR_INVALID_ARG, "bad plan query");
+  const disco::GatherPlan& P = which == 0 ? psi->fwd : psi->adj;
+  dims[0] = (int)P.rows.size();
+  dims[1] = (int)P.src.size();
+  dims[2] = (int)P.chunks.size();
+  dims[3] = (int)P.vals.size();
+  dims[4] = P.nk;
+  dims[5] = P.step;
+  dims[6] = P.residues;
+  dims[7] = (int)(sizeof(disco::RowPlan) / sizeof(int));
+  return DISCO_OK;
+}
+
+disco_status disco_plan_export(const disco_psi* psi, int which, int* rows, int* srcs, int* chunks, float* vals) {
+  if (!psi || !rows || !srcs || !chunks || !vals || (which != 0 && which != 1))
+    return fail(DISCO_ERR_INVALID_ARG, "bad plan export");
+  const disco::GatherPlan& P = which == 0 ? psi->fwd : psi->adj;
+  std::memcpy(rows, P.rows.data(), P.rows.size() * sizeof(disco::RowPlan));
+  std::memcpy(srcs, P.src.data(), P.src.size() * sizeof(disco::SrcRow));
+  std::memcpy(chunks, P.chunks.data(), P.chunks.size() * sizeof(disco::Chunk));
+  std::memcpy(vals, P.vals.data(), P.vals.size() * sizeof(float));
+  return DISCO_OK;
+}
+
+disco_status disco_workspace_size(const disco_psi* psi, int op, int B, int C_in, int C_out, int groups,
+                                  disco_dtype dtype, size_t* bytes) {
+  if (!psi || !bytes) return fail(DISCO_ERR_INVALID_ARG, "NULL argument");
+  if (B <= 0 || C_in <= 0 || C_out <= 0 || groups <= 0 || C_in % groups || C_out % groups)
+    return fail(DISCO_ERR_INVALID_ARG, "bad sizes");
+  if (op < DISCO_OP_FWD || op > DISCO_OP_BWD_WEIGHT_RECOMPUTE) return fail(DISCO_ERR_INVALID_ARG, "unknown op");
+  *bytes = layout(psi, op, B, C_in, C_out, groups, dtype).total;
+  return DISCO_OK;
+}
+
+disco_status disco_fwd(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                       const void* x, const void* w, const void* bias, void* y, void* out, void* workspace,
+                       size_t ws_bytes, void* stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  disco_status s = check_common(psi, B, C_in, C_out, groups, dtype);
+  if (s) return s;
+  if (!x || !w || !y || !out) return fail(DISCO_ERR_INVALID_ARG, "x, w, y and out must be non-NULL");
+  const disco::Geometry& g = psi->g;
+  if (!disco::gather_supports(g.K, g.stride)) return fail(DISCO_ERR_UNSUPPORTED, "K or stride not compiled");
+  const bool bf16 = dtype == DISCO_BF16;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int qb, nblk;
+  block_shape(g.nlon_out, 128, &qb, &nblk);
+  const int need = max_stage(psi->fwd, qb);
+  const int budget = std::max(kStageFloats, need);
+  if ((size_t)(disco::kMaxSrc + 4 + budget) * 4 > kSmemLimit)
+    return fail(DISCO_ERR_UNSUPPORTED, "a Psi row needs more staging than shared memory holds");
+  disco::GatherArgs a = gather_args(psi->dfwd, B * C_in, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget);
+  cudaError_t e = disco::launch_fwd_gather(bf16, g.K, g.stride, a, x, y, st);
+  if (e != cudaSuccess) return cuda_fail(e, "contraction launch");
+  disco::MixArgs m{y, w, bias, out, B, groups, C_out / groups, (C_in / groups) * g.K, g.nlat_out * g.nlon_out};
+  e = disco::launch_mix_simt(bf16, m, st);
+  if (e != cudaSuccess) return cuda_fail(e, "einsum launch");
+  return DISCO_OK;
+}
+
+disco_status disco_fwd_fused(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                             const void* x, const void* w, const void* bias, void* out, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  disco_status s = check_common(psi, B, C_in, C_out, groups, dtype);
+  if (s) return s;
+  if (!x || !w || !out) return fail(DISCO_ERR_INVALID_ARG, "x, w and out must be non-NULL");
+  const disco::Geometry& g = psi->g;
+  if (!disco::gather_supports(g.K, g.stride)) return fail(DISCO_ERR_UNSUPPORTED, "K or stride not compiled");
+  const bool bf16 = dtype == DISCO_BF16;
+  const int Cg = C_in / groups;
+  const size_t per_q = (size_t)Cg * g.K * 4;
+  int cap = (int)std::min<size_t>(128, kFusedTileBytes / per_q) / disco::kTaskR * disco::kTaskR;
+  if (cap < disco::kTaskR) return fail(DISCO_ERR_UNSUPPORTED, "C_in/groups * K too large for the fused tile");
+  int qb, nblk;
+  block_shape(g.nlon_out, cap, &qb, &nblk);
+  const int need = max_stage(psi->fwd, qb);
+  const int ytile = Cg * g.K * qb;
+  int budget = std::max(need, (int)std::min<size_t>(16384, (kSmemLimit / 4) - (disco::kMaxSrc + 4) - ytile));
+  if ((size_t)(disco::kMaxSrc + 4 + ytile + budget) * 4 > kSmemLimit)
+    return fail(DISCO_ERR_UNSUPPORTED, "fused tile and staging exceed shared memory");
+  disco::FusedArgs f;
+  f.g = gather_args(psi->dfwd, B * C_in, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget);
+  f.x = x;
+  f.w = w;
+  f.bias = bias;
+  f.out = out;
+  f.B = B;
+  f.C_in = C_in;
+  f.C_out = C_out;
+  f.G = groups;
+  f.K = g.K;
+  f.ytile_floats = ytile;
+  cudaError_t e = disco::launch_fused_simt(bf16, g.K, g.stride, f, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "fused launch");
+  return DISCO_OK;
+}
+
+disco_status disco_bwd_input(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                             const void* dout, const void* w, void* dx, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  disco_status s = check_common(psi, B, C_in, C_out, groups, dtype);
+  if (s) return s;
+  if (!dout || !w || !dx) return fail(DISCO_ERR_INVALID_ARG, "dout, w and dx must be non-NULL");
+  const disco::Geometry& g = psi->g;
+  if (!disco::gather_supports(g.K, g.stride)) return fail(DISCO_ERR_UNSUPPORTED, "K or stride not compiled");
+  const WsLayout L = layout(psi, DISCO_OP_BWD_INPUT, B, C_in, C_out, groups, dtype);
+  if (!workspace || ws_bytes < L.total) return fail(DISCO_ERR_INVALID_ARG, "workspace missing or too small");
+  const bool bf16 = dtype == DISCO_BF16;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  void* wt = ws + L.wt;
+  void* dy = ws + L.dy;
+  const int Cg = C_in / groups, Og = C_out / groups;
+  cudaError_t e = disco::launch_transpose_weight(bf16, w, wt, groups, Og, Cg, g.K, st);
+  if (e != cudaSuccess) return cuda_fail(e, "weight transpose launch");
+  disco::MixArgs m{dout, wt, nullptr, dy, B, groups, Cg * g.K, Og, g.nlat_out * g.nlon_out};
+  e = disco::launch_mix_simt(bf16, m, st);
+  if (e != cudaSuccess) return cuda_fail(e, "transposed einsum launch");
+  int qb, nblk;
+  block_shape(g.nlon_out, 128, &qb, &nblk);
+  const int need = max_stage(psi->adj, qb);
+  const int budget = std::max(kStageFloats, need);
+  if ((size_t)(disco::kMaxSrc + 4 + budget) * 4 > kSmemLimit)
+    return fail(DISCO_ERR_UNSUPPORTED, "a Psi column needs more staging than shared memory holds");
+  disco::GatherArgs a =
+      gather_args(psi->dadj, B * C_in, qb, nblk, g.nlon_out, g.K * g.nlat_out, g.nlon_in, g.nlat_in, budget);
+  e = disco::launch_adj_gather(bf16, g.stride, a, dy, dx, st);
+  if (e != cudaSuccess) return cuda_fail(e, "adjoint contraction launch");
+  return DISCO_OK;
+}
+
+disco_status disco_bwd_weight(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                              const void* dout, const void* y, const void* x, void* dw, void* dbias, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  disco_status s = check_common(psi, B, C_in, C_out, groups, dtype);
+  if (s) return s;
+  if (!dout || !dw || (!y && !x)) return fail(DISCO_ERR_INVALID_ARG, "dout, dw and one of y/x must be non-NULL");
+  const disco::Geometry& g = psi->g;
+  if (!disco::gather_supports(g.K, g.stride)) return fail(DISCO_ERR_UNSUPPORTED, "K or stride not compiled");
+  const int op = y ? DISCO_OP_BWD_WEIGHT : DISCO_OP_BWD_WEIGHT_RECOMPUTE;
+  const WsLayout L = layout(psi, op, B, C_in, C_out, groups, dtype);
+  if (!workspace || ws_bytes < L.total) return fail(DISCO_ERR_INVALID_ARG, "workspace missing or too small");
+  const bool bf16 = dtype == DISCO_BF16;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  cudaError_t e;
+  const void* yv = y;
+  if (!y) {
+    int qb, nblk;
+    block_shape(g.nlon_out, 128, &qb, &nblk);
+    const int need = max_stage(psi->fwd, qb);
+    const int budget = std::max(kStageFloats, need);
+    if ((size_t)(disco::kMaxSrc + 4 + budget) * 4 > kSmemLimit)
+      return fail(DISCO_ERR_UNSUPPORTED, "a Psi row needs more staging than shared memory holds");
+    disco::GatherArgs a =
+        gather_args(psi->dfwd, B * C_in, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget);
+    e = disco::launch_fwd_gather(bf16, g.K, g.stride, a, x, ws + L.ybuf, st);
+    if (e != cudaSuccess) return cuda_fail(e, "recompute contraction launch");
+    yv = ws + L.ybuf;
+  }
+  const int Og = C_out / groups, Rg = (C_in / groups) * g.K;
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  float* bpart = dbias ? reinterpret_cast<float*>(ws + L.bpart) : nullptr;
+  disco::DwArgs d{dout, yv, part, bpart, B, groups, Og, Rg, g.nlat_out * g.nlon_out, L.nc, L.nchunk};
+  e = disco::launch_dw_partial_simt(bf16, d, st);
+  if (e != cudaSuccess) return cuda_fail(e, "weight-gradient launch");
+  e = disco::launch_dw_reduce(bf16, part, bpart, dw, dbias, B * L.nchunk, groups, Og, Rg, st);
+  if (e != cudaSuccess) return cuda_fail(e, "weight-gradient reduce launch");
+  return DISCO_OK;
+}
+
+}  // extern "C"

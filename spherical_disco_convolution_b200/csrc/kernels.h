@@ -1,0 +1,70 @@
+// Launch interfaces of the libdisco kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "plan.h"
+
+namespace disco {
+
+struct GatherArgs {
+  const RowPlan* rows;
+  const SrcRow* srcs;
+  const Chunk* chunks;
+  const float* vals;
+  int n_rows;        // output rows in the plan (grid.z)
+  int BC;            // channel planes (batch * channels)
+  int cb;            // channel planes per CTA
+  int qb, nblk;      // outputs per block, blocks per row
+  int n_src, n_src_rows;  // source row length, source rows per channel plane
+  int n_out, n_out_rows;  // output row length, output rows per channel plane
+  int stage_budget;  // staged floats per CTA (>= the largest row's per-channel need)
+};
+
+bool gather_supports(int K, int stride);
+cudaError_t launch_fwd_gather(bool bf16, int K, int S, const GatherArgs& a, const void* x, void* y, cudaStream_t st);
+cudaError_t launch_adj_gather(bool bf16, int S, const GatherArgs& a, const void* dy, void* dx, cudaStream_t st);
+
+// Grouped channel mix (SIMT):
+//   out[b, g*Mg + m, n] = bias[g*Mg + m] + sum_{r < Rg} wm[g, m, r] * in[b, g*Rg + r, n]
+struct MixArgs {
+  const void* in;
+  const void* wm;
+  const void* bias;  // may be null
+  void* out;
+  int B, G, Mg, Rg, N;
+};
+cudaError_t launch_mix_simt(bool bf16, const MixArgs& a, cudaStream_t st);
+
+// wt[g, c*K + k, o] = w[g*Og + o, c, k]   (the transposed weight of the dx einsum)
+cudaError_t launch_transpose_weight(bool bf16, const void* w, void* wt, int G, int Og, int Cg, int K, cudaStream_t st);
+
+// Split-K weight gradient partials (SIMT):
+//   part[split, g, o, r] = sum_{n in chunk} dout[b, g*Og + o, n] * yv[b, g*Rg + r, n]
+//   bpart[split, g*Og + o] = sum_{n in chunk} dout[b, g*Og + o, n]          (when bpart != null)
+// split = b * nchunk + chunk, chunk covers n in [chunk*nc, chunk*nc + nc).
+struct DwArgs {
+  const void* dout;
+  const void* yv;
+  float* part;
+  float* bpart;
+  int B, G, Og, Rg, N, nc, nchunk;
+};
+cudaError_t launch_dw_partial_simt(bool bf16, const DwArgs& a, cudaStream_t st);
+// dw[g*Og + o, r] = sum_split part[split, g, o, r]; dbias[o] = sum_split bpart[split, o]; fixed order.
+cudaError_t launch_dw_reduce(bool bf16, const float* part, const float* bpart, void* dw, void* dbias, int nsplit,
+                             int G, int Og, int Rg, cudaStream_t st);
+
+// Fused forward (SIMT): contraction into an on-chip y tile, then the channel mix.
+struct FusedArgs {
+  GatherArgs g;       // forward gather plan; BC unused, qb/nblk for the fused block
+  const void* x;
+  const void* w;      // (C_out, Cg, K)
+  const void* bias;   // may be null
+  void* out;
+  int B, C_in, C_out, G, K;
+  int ytile_floats;   // Cg*K*qb
+};
+cudaError_t launch_fused_simt(bool bf16, int K, int S, const FusedArgs& a, cudaStream_t st);
+
+}  // namespace disco

@@ -1,0 +1,67 @@
+// Host/device plan structures of the DISCO gather kernels.
+//
+// A "plan" is Psi re-laid out for one kernel family.  Psi itself (page
+// "torch_harmonics.DiscreteContinuousConvS2", definition below the forward
+// equation) is a sparse tensor Psi[k, j, (i, p)]; the p-shift symmetry stated
+// there means one row per output latitude j serves every output longitude q.
+//
+// Gather plans group the entries of one output row into "source rows" (the
+// rows of the source tensor it reaches) and "chunks" (windows of at most
+// kChunkW consecutive longitude offsets of one source row, holding the values
+// of all nk basis functions densely, zeros included).  A CTA stages every
+// source row of its output row in shared memory as a straight run of
+// longitudes that already contains the wrap-around, so the inner loop never
+// takes a modulo.
+//
+// For a block of outputs starting at m0 (0 <= m < qb), staged element t of a
+// source row holds source longitude  (m0*step + start + t) mod n_src, and a
+// chunk with column offset t0 reads, for block-relative output m, the staged
+// elements  t0 + m*step + u,  u = 0 .. w-1  (step = s for the forward, where
+// output q reads input longitude q*s + d; step = 1 for the adjoint).
+#pragma once
+
+#include <cstdint>
+
+#if defined(__CUDACC__)
+#define DISCO_HD __host__ __device__
+#else
+#define DISCO_HD
+#endif
+
+namespace disco {
+
+constexpr int kChunkW = 8;      // longitude offsets per chunk
+constexpr int kTaskR = 8;       // consecutive outputs per thread
+constexpr int kMaxStride = 4;   // nlon_in / nlon_out supported by the kernels
+constexpr int kMaxK = 16;       // basis functions supported by the kernels
+constexpr int kMaxSrc = 512;    // source rows per output row supported by the kernels
+
+struct SrcRow {
+  int row;     // row index into the source tensor's (row, longitude) plane of one channel
+  int start;   // offset of staged element 0 relative to m0*step (may be negative)
+  int span;    // longitude offsets covered by the row's chunks
+  int pad;
+};
+
+struct Chunk {
+  int src;     // source row, relative to RowPlan::src_begin
+  int t0;      // first column (staged element for m = 0)
+  int voff;    // offset (floats) of the values, laid out [nk][kChunkW]
+  int wk;      // width (1..kChunkW) in bits 0..7, kmask (bit k: basis k non-zero) from bit 8
+};
+
+// One output row of a gather plan.
+struct RowPlan {
+  int row;                      // output row (j for the forward, i for the adjoint)
+  int src_begin, src_end;
+  int chunk_start[kMaxStride];  // chunk list of residue class rho: [chunk_start[rho], chunk_end[rho])
+  int chunk_end[kMaxStride];    // (the forward plan only has rho = 0)
+  float cost;                   // relative work, used to order heavy rows first
+};
+
+// Staged elements of one source row for a block of qb outputs.
+DISCO_HD inline int staged_len(int span, int qb, int step) {
+  return (((qb + kTaskR - 1) * step + span + kChunkW) + 3) & ~3;
+}
+
+}  // namespace disco

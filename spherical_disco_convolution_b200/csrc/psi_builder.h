@@ -1,0 +1,48 @@
+// Host-side Psi builder and plan construction for libdisco.
+#pragma once
+
+#include <string>
+#include <vector>
+
+#include "plan.h"
+
+namespace disco {
+
+struct Geometry {
+  int nlat_in, nlon_in, nlat_out, nlon_out;
+  int n_r, n_alpha;
+  double theta_cutoff;
+  int K;        // number of basis functions
+  int stride;   // nlon_in / nlon_out
+};
+
+struct PsiEntry {
+  int k, j, i, p;   // basis, output row, input row, longitude offset in [0, nlon_in)
+  double v;
+};
+
+// Status codes mirror disco_status (0 ok, 1 invalid, 2 unsupported, 6 geometry).
+int build_psi_entries(const Geometry& g, std::vector<PsiEntry>& out, std::string& msg);
+
+struct GatherPlan {
+  std::vector<RowPlan> rows;   // ordered heaviest first
+  std::vector<SrcRow> src;
+  std::vector<Chunk> chunks;
+  std::vector<float> vals;
+  int nk = 1;          // value sets per chunk (K for the forward, 1 for the adjoint)
+  int step = 1;        // source positions advance by `step` per output (forward: s; adjoint: 1)
+  int residues = 1;    // output residue classes (adjoint: s)
+  int max_src = 0;     // most source rows of any output row
+};
+
+// Elements staged per channel for output row `r` and a block of qb outputs.
+int stage_elems(const GatherPlan& P, const RowPlan& r, int qb);
+
+// Forward gather plan: output rows j, sources x rows i, K accumulators.
+GatherPlan make_forward_plan(const Geometry& g, const std::vector<PsiEntry>& e);
+
+// Adjoint gather plan: output rows i of dx, sources rows (k, j) of dy, one accumulator,
+// output longitude l = stride*m + rho.
+GatherPlan make_adjoint_plan(const Geometry& g, const std::vector<PsiEntry>& e);
+
+}  // namespace disco

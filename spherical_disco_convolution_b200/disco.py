@@ -1,0 +1,190 @@
+"""Thin ctypes binding of libdisco (the C ABI declared in include/disco.h).
+
+Every function here marshals arguments and calls the entry point of the same
+name; all arithmetic of the DISCO convolution runs in the library's CUDA
+kernels.  Pointers are passed as Python ints (device pointers from
+``tensor.data_ptr()``, streams from ``torch.cuda.Stream.cuda_stream``).  The
+library must have been built (``python -m spherical_disco_convolution_b200.build``);
+if it is missing, importing this module raises: there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdisco.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "disco.h")
+
+DISCO_OK = 0
+DISCO_ERR_INVALID_ARG = 1
+DISCO_ERR_UNSUPPORTED = 2
+DISCO_ERR_CUDA = 3
+DISCO_ERR_ALLOC = 4
+DISCO_ERR_TIMEOUT = 5
+DISCO_ERR_GEOMETRY = 6
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "ALLOC", 5: "TIMEOUT", 6: "GEOMETRY"}
+
+DISCO_F32 = 0
+DISCO_BF16 = 1
+DISCO_GRID_EQUIANGULAR = 0
+DISCO_BASIS_PIECEWISE_LINEAR = 0
+DISCO_NORM_NODAL = 0
+
+DISCO_OP_FWD = 0
+DISCO_OP_FWD_FUSED = 1
+DISCO_OP_BWD_INPUT = 2
+DISCO_OP_BWD_WEIGHT = 3
+DISCO_OP_BWD_WEIGHT_RECOMPUTE = 4
+
+
+class DiscoError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"disco status {STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class disco_spec_t(ctypes.Structure):
+    _fields_ = [
+        ("nlat_in", ctypes.c_int), ("nlon_in", ctypes.c_int),
+        ("nlat_out", ctypes.c_int), ("nlon_out", ctypes.c_int),
+        ("grid_in", ctypes.c_int), ("grid_out", ctypes.c_int),
+        ("kernel_shape", ctypes.c_int * 2),
+        ("basis_type", ctypes.c_int), ("basis_norm_mode", ctypes.c_int),
+        ("theta_cutoff", ctypes.c_double),
+    ]
+
+
+def make_spec(nlat_in, nlon_in, nlat_out, nlon_out, kernel_shape, theta_cutoff,
+              grid_in=DISCO_GRID_EQUIANGULAR, grid_out=DISCO_GRID_EQUIANGULAR,
+              basis_type=DISCO_BASIS_PIECEWISE_LINEAR, basis_norm_mode=DISCO_NORM_NODAL) -> disco_spec_t:
+    ks = (kernel_shape, 1) if isinstance(kernel_shape, int) else tuple(kernel_shape)
+    if len(ks) == 1:
+        ks = (ks[0], 1)
+    s = disco_spec_t()
+    s.nlat_in, s.nlon_in, s.nlat_out, s.nlon_out = nlat_in, nlon_in, nlat_out, nlon_out
+    s.grid_in, s.grid_out = grid_in, grid_out
+    s.kernel_shape[0], s.kernel_shape[1] = ks
+    s.basis_type, s.basis_norm_mode = basis_type, basis_norm_mode
+    s.theta_cutoff = float(theta_cutoff)
+    return s
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libdisco.so not built at {LIB_PATH}; run python -m spherical_disco_convolution_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, LL, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t
+    IP = ctypes.POINTER(ctypes.c_int)
+    DP = ctypes.POINTER(ctypes.c_double)
+    sig = {
+        "disco_psi_build": [ctypes.POINTER(disco_spec_t), I, ctypes.POINTER(P)],
+        "disco_psi_destroy": [P],
+        "disco_psi_info": [P, IP, ctypes.POINTER(LL)],
+        "disco_psi_export": [P, IP, IP, IP, IP, DP],
+        "disco_workspace_size": [P, I, I, I, I, I, I, ctypes.POINTER(Z)],
+        "disco_fwd": [P, I, I, I, I, I, P, P, P, P, P, P, Z, P],
+        "disco_fwd_fused": [P, I, I, I, I, I, P, P, P, P, P, Z, P],
+        "disco_bwd_input": [P, I, I, I, I, I, P, P, P, P, Z, P],
+        "disco_bwd_weight": [P, I, I, I, I, I, P, P, P, P, P, P, Z, P],
+        "disco_plan_info": [P, I, IP],
+        "disco_plan_export": [P, I, IP, IP, IP, ctypes.POINTER(ctypes.c_float)],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    lib.disco_last_error.argtypes = []
+    lib.disco_last_error.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+def header_functions() -> list:
+    """Names of every function that include/disco.h declares."""
+    text = open(HEADER_PATH).read()
+    return sorted(set(re.findall(r"^\s*(?:disco_status|const char\*)\s+(disco_\w+)\s*\(", text, re.M)))
+
+
+def library():
+    return _lib
+
+
+def _check(status: int):
+    if status != DISCO_OK:
+        raise DiscoError(status, _lib.disco_last_error().decode())
+
+
+def disco_last_error() -> str:
+    return _lib.disco_last_error().decode()
+
+
+def disco_psi_build(spec: disco_spec_t, device: int) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(_lib.disco_psi_build(ctypes.byref(spec), device, ctypes.byref(h)))
+    return h
+
+
+def disco_psi_destroy(psi) -> None:
+    _check(_lib.disco_psi_destroy(psi))
+
+
+def disco_psi_info(psi):
+    K = ctypes.c_int()
+    nnz = ctypes.c_longlong()
+    _check(_lib.disco_psi_info(psi, ctypes.byref(K), ctypes.byref(nnz)))
+    return K.value, nnz.value
+
+
+def disco_psi_export(psi):
+    """(k, j, i, p, val) host arrays sorted by (j, k, i, p)."""
+    _, nnz = disco_psi_info(psi)
+    k, j, i, p = (np.empty(nnz, dtype=np.int32) for _ in range(4))
+    v = np.empty(nnz, dtype=np.float64)
+    ip = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))  # noqa: E731
+    _check(_lib.disco_psi_export(psi, ip(k), ip(j), ip(i), ip(p), v.ctypes.data_as(ctypes.POINTER(ctypes.c_double))))
+    return k, j, i, p, v
+
+
+def disco_plan_export(psi, which: int):
+    """Plan arrays of the forward (which=0) or adjoint (which=1) gather kernels."""
+    dims = np.zeros(8, dtype=np.int32)
+    _check(_lib.disco_plan_info(psi, which, dims.ctypes.data_as(ctypes.POINTER(ctypes.c_int))))
+    n_rows, n_src, n_chunks, n_vals, nk, step, residues, row_ints = (int(v) for v in dims)
+    rows = np.zeros((n_rows, row_ints), dtype=np.int32)
+    srcs = np.zeros((n_src, 4), dtype=np.int32)
+    chunks = np.zeros((n_chunks, 4), dtype=np.int32)
+    vals = np.zeros(n_vals, dtype=np.float32)
+    ip = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))  # noqa: E731
+    _check(_lib.disco_plan_export(psi, which, ip(rows), ip(srcs), ip(chunks),
+                                  vals.ctypes.data_as(ctypes.POINTER(ctypes.c_float))))
+    return dict(rows=rows, srcs=srcs, chunks=chunks, vals=vals, nk=nk, step=step, residues=residues)
+
+
+def disco_workspace_size(psi, op, B, C_in, C_out, groups, dtype) -> int:
+    n = ctypes.c_size_t()
+    _check(_lib.disco_workspace_size(psi, op, B, C_in, C_out, groups, dtype, ctypes.byref(n)))
+    return n.value
+
+
+def disco_fwd(psi, B, C_in, C_out, groups, dtype, x, w, bias, y, out, workspace, ws_bytes, stream) -> None:
+    _check(_lib.disco_fwd(psi, B, C_in, C_out, groups, dtype, x, w, bias, y, out, workspace, ws_bytes, stream))
+
+
+def disco_fwd_fused(psi, B, C_in, C_out, groups, dtype, x, w, bias, out, workspace, ws_bytes, stream) -> None:
+    _check(_lib.disco_fwd_fused(psi, B, C_in, C_out, groups, dtype, x, w, bias, out, workspace, ws_bytes, stream))
+
+
+def disco_bwd_input(psi, B, C_in, C_out, groups, dtype, dout, w, dx, workspace, ws_bytes, stream) -> None:
+    _check(_lib.disco_bwd_input(psi, B, C_in, C_out, groups, dtype, dout, w, dx, workspace, ws_bytes, stream))
+
+
+def disco_bwd_weight(psi, B, C_in, C_out, groups, dtype, dout, y, x, dw, dbias, workspace, ws_bytes, stream) -> None:
+    _check(_lib.disco_bwd_weight(psi, B, C_in, C_out, groups, dtype, dout, y, x, dw, dbias, workspace, ws_bytes,
+                                 stream))

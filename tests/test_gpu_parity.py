@@ -1,0 +1,198 @@
+"""GPU parity: libdisco's CUDA path against the CPU oracle, element by element.
+
+Tolerances (max-abs error relative to the oracle's L-infinity norm): 1e-4 for
+fp32 layers, 2e-2 for bf16-storage layers.  Inputs are the seeded workloads;
+bf16 layers take the same bf16-representable values on both sides.  All five
+workloads run at full size; the K-expanded y of the two largest is compared
+on a subset of channel planes (every element of those planes).
+"""
+
+import functools
+import math
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle  # noqa: E402
+from spherical_disco_convolution_b200 import conv  # noqa: E402
+from spherical_disco_convolution_b200 import disco as D  # noqa: E402
+from spherical_disco_convolution_b200.workloads import WORKLOADS, Workload, make_inputs  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+ALL = ["tiny", "mid", "downsample", "weather", "grouped"]
+
+# Small geometries with ragged tails (nlon_out not a multiple of the 8-output task or of the
+# block), odd latitude counts, stride-2 downsampling, groups, no bias, and channel counts that
+# leave a partial channel block.
+EDGE = {
+    "ragged_iso_f32": Workload("ragged_iso_f32", 3, 6, 9, 3, 13, 20, 13, 20, (3, 1), 0.61, "f32"),
+    "ragged_down_bf16": Workload("ragged_down_bf16", 3, 6, 9, 3, 19, 24, 10, 12, (3, 4), 0.7, "bf16", bias=False),
+    "wide_row_f32": Workload("wide_row_f32", 2, 5, 4, 1, 33, 264, 33, 132, (5, 1), 0.35, "f32"),
+    "aniso_k9_f32": Workload("aniso_k9_f32", 1, 17, 17, 1, 21, 40, 21, 40, (3, 4), 0.5, "f32"),
+}
+
+
+def tol(wl):
+    return 1e-4 if wl.dtype == "f32" else 2e-2
+
+
+def workload(name):
+    return WORKLOADS[name] if name in WORKLOADS else EDGE[name]
+
+
+def ospec(wl):
+    return oracle.Spec(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape[0], wl.kernel_shape[1],
+                       wl.theta_cutoff)
+
+
+@functools.lru_cache(maxsize=None)
+def inputs(name):
+    return make_inputs(workload(name), 0)
+
+
+@functools.lru_cache(maxsize=None)
+def oracle_psi(name):
+    return oracle.Psi(ospec(workload(name)))
+
+
+@functools.lru_cache(maxsize=None)
+def oracle_out(name):
+    wl, inp = workload(name), inputs(name)
+    return oracle_psi(name).forward(inp["x"], inp["w"], inp["bias"], groups=wl.groups)
+
+
+@functools.lru_cache(maxsize=None)
+def oracle_dx(name):
+    wl, inp = workload(name), inputs(name)
+    return oracle_psi(name).backward_input(inp["dout"], inp["w"], wl.C_in, groups=wl.groups)
+
+
+@functools.lru_cache(maxsize=None)
+def oracle_dw(name):
+    wl, inp = workload(name), inputs(name)
+    return oracle_psi(name).backward_weight(inp["dout"], inp["x"], groups=wl.groups)
+
+
+@functools.lru_cache(maxsize=None)
+def gpu_psi(name):
+    wl = workload(name)
+    return conv.Psi(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape, wl.theta_cutoff, "cuda:0")
+
+
+def dev(a, wl):
+    if a is None:
+        return None
+    dt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+    return torch.from_numpy(np.ascontiguousarray(a)).to("cuda:0").to(dt)
+
+
+def host(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def check(got, ref, rel, what):
+    err = np.abs(got - ref).max()
+    scale = np.abs(ref).max()
+    assert np.isfinite(err) and err <= rel * scale, f"{what}: max err {err:.3e} > {rel:g} x {scale:.3e}"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def need_cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def y_channels(wl):
+    """Channel planes of y compared element by element."""
+    if wl.B * wl.C_in * wl.K * wl.nlat_out * wl.nlon_out <= 64_000_000:
+        return None  # all
+    return [0, 1, wl.C_in // 2, wl.C_in - 1]
+
+
+@pytest.mark.parametrize("name", ALL + list(EDGE))
+def test_forward_matches_oracle(name):
+    wl, inp = workload(name), inputs(name)
+    out, y = conv.disco_forward(gpu_psi(name), dev(inp["x"], wl), dev(inp["w"], wl), dev(inp["bias"], wl),
+                                wl.groups)
+    torch.cuda.synchronize()
+    check(host(out), oracle_out(name), tol(wl), "out")
+    sel = y_channels(wl)
+    if sel is None:
+        y_ref = oracle_psi(name).contract(inp["x"])
+        check(host(y), y_ref, tol(wl), "y")
+    else:
+        y_ref = oracle_psi(name).contract(inp["x"][:, sel])
+        check(host(y[:, sel]), y_ref, tol(wl), "y (sampled channel planes)")
+
+
+@pytest.mark.parametrize("name", ALL + list(EDGE))
+def test_fused_forward_matches_oracle(name):
+    wl, inp = workload(name), inputs(name)
+    out, y = conv.disco_forward(gpu_psi(name), dev(inp["x"], wl), dev(inp["w"], wl), dev(inp["bias"], wl),
+                                wl.groups, fused=True)
+    torch.cuda.synchronize()
+    assert y is None
+    check(host(out), oracle_out(name), tol(wl), "fused out")
+
+
+@pytest.mark.parametrize("name", ALL + list(EDGE))
+def test_backward_input_matches_oracle(name):
+    wl, inp = workload(name), inputs(name)
+    dx = conv.disco_backward_input(gpu_psi(name), dev(inp["dout"], wl), dev(inp["w"], wl), wl.C_in, wl.groups)
+    torch.cuda.synchronize()
+    check(host(dx), oracle_dx(name), tol(wl), "dx")
+
+
+@pytest.mark.parametrize("name", ALL + list(EDGE))
+def test_backward_weight_matches_oracle(name):
+    wl, inp = workload(name), inputs(name)
+    psi = gpu_psi(name)
+    x = dev(inp["x"], wl)
+    _, y = conv.disco_forward(psi, x, dev(inp["w"], wl), dev(inp["bias"], wl), wl.groups)
+    dout = dev(inp["dout"], wl)
+    dw_ref, db_ref = oracle_dw(name)
+    dw, db = conv.disco_backward_weight(psi, dout, y=y, groups=wl.groups)
+    dw2, db2 = conv.disco_backward_weight(psi, dout, x=x, groups=wl.groups)
+    torch.cuda.synchronize()
+    check(host(dw), dw_ref, tol(wl), "dw")
+    check(host(db), db_ref, tol(wl), "dbias")
+    check(host(dw2), dw_ref, tol(wl), "dw (recomputed y)")
+    # deterministic: the split-K reduction runs in a fixed order
+    dw3, _ = conv.disco_backward_weight(psi, dout, y=y, groups=wl.groups)
+    assert torch.equal(dw, dw3)
+
+
+def test_autograd_layer_matches_oracle():
+    name = "ragged_down_bf16"
+    wl, inp = workload(name), inputs(name)
+    for fused in (False, True):
+        layer = conv.DiscreteContinuousConvS2(wl.C_in, wl.C_out, (wl.nlat_in, wl.nlon_in),
+                                              (wl.nlat_out, wl.nlon_out), wl.kernel_shape, groups=wl.groups,
+                                              bias=False, theta_cutoff=wl.theta_cutoff, fused=fused,
+                                              device="cuda:0", dtype=torch.bfloat16)
+        with torch.no_grad():
+            layer.weight.copy_(dev(inp["w"], wl))
+        x = dev(inp["x"], wl).requires_grad_(True)
+        out = layer(x)
+        out.backward(dev(inp["dout"], wl))
+        torch.cuda.synchronize()
+        check(host(out), oracle_out(name), tol(wl), "layer out")
+        check(host(x.grad), oracle_dx(name), tol(wl), "layer dx")
+        check(host(layer.weight.grad), oracle_dw(name)[0], tol(wl), "layer dw")
+
+
+def test_invalid_calls_raise():
+    wl = workload("ragged_iso_f32")
+    psi = gpu_psi("ragged_iso_f32")
+    x = torch.zeros((0, wl.C_in, wl.nlat_in, wl.nlon_in), device="cuda:0")
+    w = torch.zeros((wl.C_out, wl.C_in // wl.groups, wl.K), device="cuda:0")
+    with pytest.raises(D.DiscoError) as e:
+        conv.disco_forward(psi, x, w, None, wl.groups)
+    assert e.value.status == D.DISCO_ERR_INVALID_ARG
+    x = torch.zeros((1, wl.C_in, wl.nlat_in, wl.nlon_in), device="cuda:0")
+    with pytest.raises(D.DiscoError) as e:
+        conv.disco_forward(psi, x, w, None, 4)  # 4 divides neither 6 nor 9
+    assert e.value.status == D.DISCO_ERR_INVALID_ARG

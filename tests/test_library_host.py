@@ -1,0 +1,143 @@
+"""Host-side checks of libdisco (no GPU): symbols, Psi builder vs oracle, plans, status codes."""
+
+import ctypes
+import math
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from spherical_disco_convolution_b200 import disco as D
+from spherical_disco_convolution_b200.workloads import WORKLOADS, make_inputs
+from tests import plan_emulator
+
+
+def spec_pair(wl):
+    s = D.make_spec(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape, wl.theta_cutoff)
+    o = oracle.Spec(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape[0], wl.kernel_shape[1],
+                    wl.theta_cutoff)
+    return s, o
+
+
+def test_library_exports_every_declared_symbol():
+    names = D.header_functions()
+    assert len(names) >= 10
+    out = subprocess.run(["nm", "-D", "--defined-only", D.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in names:
+        assert n in exported, n
+        assert getattr(D.library(), n) is not None
+
+
+QUICK = ["tiny", "mid", "downsample"]
+
+
+@pytest.mark.parametrize("name", QUICK + [pytest.param(n, marks=pytest.mark.slow) for n in ("weather", "grouped")])
+def test_psi_export_matches_oracle(name):
+    s, o = spec_pair(WORKLOADS[name])
+    h = D.disco_psi_build(s, -1)
+    try:
+        k, j, i, p, v = D.disco_psi_export(h)
+    finally:
+        D.disco_psi_destroy(h)
+    ko, jo, io, po, vo = oracle.Psi(o).entries()
+    # same non-zero pattern, bit for bit, in the same (j, k, i, p) order
+    assert np.array_equal(k, ko) and np.array_equal(j, jo) and np.array_equal(i, io) and np.array_equal(p, po)
+    # values: the two distance routes differ by rounding (~1e-17 rad); a small phi near a hat end
+    # point turns that into an absolute error of ~1e-16/width, so the bound is 1e-12 relative plus
+    # 1e-11 of the largest entry
+    np.testing.assert_allclose(v, vo, rtol=1e-12, atol=1e-11 * np.abs(vo).max())
+
+
+def _bc(x):
+    return x.reshape((-1,) + x.shape[2:])
+
+
+@pytest.mark.parametrize("name", ["tiny", "downsample"])
+def test_forward_plan_reproduces_oracle_contraction(name):
+    wl = WORKLOADS[name].scaled(B=1, C_in=2)
+    s, o = spec_pair(wl)
+    h = D.disco_psi_build(s, -1)
+    plan = D.disco_plan_export(h, 0)
+    D.disco_psi_destroy(h)
+    x = make_inputs(wl, 1)["x"].astype(np.float64)
+    y_ref = oracle.Psi(o).contract(x)
+    y = plan_emulator.forward(plan, _bc(x), wl.nlat_out, wl.nlon_out, wl.K)
+    # plan values are fp32: relative rounding 6e-8 per entry
+    np.testing.assert_allclose(y, _bc(y_ref), rtol=0, atol=1e-6 * np.abs(y_ref).max())
+
+
+@pytest.mark.parametrize("name", ["tiny", "downsample"])
+def test_adjoint_plan_reproduces_oracle_backward(name):
+    wl = WORKLOADS[name].scaled(B=1, C_in=2, C_out=3)
+    s, o = spec_pair(wl)
+    h = D.disco_psi_build(s, -1)
+    plan = D.disco_plan_export(h, 1)
+    D.disco_psi_destroy(h)
+    assert plan["residues"] == wl.stride
+    P = oracle.Psi(o)
+    rng = np.random.default_rng(3)
+    dout = rng.standard_normal((1, wl.C_out, wl.nlat_out, wl.nlon_out))
+    w = rng.standard_normal((wl.C_out, wl.C_in, wl.K))
+    dx_ref = P.backward_input(dout, w, wl.C_in)
+    dy = np.einsum("ock,bojq->bckjq", w, dout).reshape(1 * wl.C_in, wl.K * wl.nlat_out, wl.nlon_out)
+    dx = plan_emulator.adjoint(plan, dy, wl.nlat_in, wl.nlon_in, wl.stride)
+    np.testing.assert_allclose(dx, _bc(dx_ref), rtol=0, atol=1e-6 * np.abs(dx_ref).max())
+
+
+def test_plans_respect_kernel_limits():
+    for name in QUICK:
+        s, _ = spec_pair(WORKLOADS[name])
+        h = D.disco_psi_build(s, -1)
+        for which in (0, 1):
+            plan = D.disco_plan_export(h, which)
+            chunks = plan["chunks"]
+            assert np.all((chunks[:, 3] & 0xFF) >= 1) and np.all((chunks[:, 3] & 0xFF) <= 8)
+            assert np.all(chunks[:, 3] >> 8 > 0)
+            rows = plan["rows"]
+            assert np.all(rows[:, 2] - rows[:, 1] <= 512)
+            # every chunk's columns lie inside its source row's span
+            for r in rows:
+                for ch in range(r[3], r[7 + plan["residues"] - 1]):
+                    src, t0, _, wk = chunks[ch]
+                    assert 0 <= src < r[2] - r[1]
+                    assert t0 + (wk & 0xFF) <= plan["srcs"][r[1] + src][2]
+        D.disco_psi_destroy(h)
+
+
+def test_status_codes():
+    lib = D.library()
+    h = ctypes.c_void_p()
+    bad = D.make_spec(17, 32, 17, 32, 3, 0.0)
+    assert lib.disco_psi_build(ctypes.byref(bad), -1, ctypes.byref(h)) == D.DISCO_ERR_INVALID_ARG
+    assert "theta_cutoff" in D.disco_last_error()
+    assert not h.value
+    bad = D.make_spec(17, 32, 17, 24, 3, 0.3)
+    assert lib.disco_psi_build(ctypes.byref(bad), -1, ctypes.byref(h)) == D.DISCO_ERR_UNSUPPORTED
+    bad = D.make_spec(17, 32, 17, 32, 3, 0.3, grid_in=1)
+    assert lib.disco_psi_build(ctypes.byref(bad), -1, ctypes.byref(h)) == D.DISCO_ERR_UNSUPPORTED
+    bad = D.make_spec(1, 32, 17, 32, 3, 0.3)
+    assert lib.disco_psi_build(ctypes.byref(bad), -1, ctypes.byref(h)) == D.DISCO_ERR_INVALID_ARG
+    bad = D.make_spec(17, 32, 17, 32, (1, 1), 0.3)
+    assert lib.disco_psi_build(ctypes.byref(bad), -1, ctypes.byref(h)) == D.DISCO_ERR_INVALID_ARG
+    # a cutoff 5e-11 below a grid distance: the tie is too close to call
+    tie = D.make_spec(17, 32, 17, 32, 3, 2 * math.pi / 16 - 5e-11)
+    assert lib.disco_psi_build(ctypes.byref(tie), -1, ctypes.byref(h)) == D.DISCO_ERR_GEOMETRY
+    ok = D.make_spec(17, 32, 17, 32, 3, 2 * math.pi / 16)
+    h = D.disco_psi_build(ok, -1)
+    try:
+        # host-only handle: compute calls refuse
+        st = lib.disco_fwd(h, 1, 4, 4, 1, D.DISCO_F32, None, None, None, None, None, None, 0, None)
+        assert st == D.DISCO_ERR_INVALID_ARG
+        n = D.disco_workspace_size(h, D.DISCO_OP_FWD, 1, 4, 4, 1, D.DISCO_F32)
+        assert n == 0
+        n_bi = D.disco_workspace_size(h, D.DISCO_OP_BWD_INPUT, 2, 4, 6, 2, D.DISCO_BF16)
+        assert n_bi >= 2 * 4 * 3 * 17 * 32 * 2
+        n_bw = D.disco_workspace_size(h, D.DISCO_OP_BWD_WEIGHT_RECOMPUTE, 2, 4, 6, 2, D.DISCO_F32)
+        assert n_bw > D.disco_workspace_size(h, D.DISCO_OP_BWD_WEIGHT, 2, 4, 6, 2, D.DISCO_F32)
+        with pytest.raises(D.DiscoError):
+            D.disco_workspace_size(h, D.DISCO_OP_FWD, 1, 4, 6, 4, D.DISCO_F32)  # groups do not divide C_in
+    finally:
+        D.disco_psi_destroy(h)
+    assert lib.disco_psi_destroy(None) == D.DISCO_OK
