@@ -119,7 +119,20 @@ disco_status disco_psi_export(const disco_psi* psi, int* k, int* j, int* i, int*
 disco_status disco_workspace_size(const disco_psi* psi, int op, int B, int C_in, int C_out, int groups,
                                   disco_dtype dtype, size_t* bytes);
 
-/* Forward, unfused: writes the K-expanded y (saved for backward) and out. */
+/* The sparse Psi contraction alone (the first sum of the forward equation):
+ *   y[b,c,k,j,q] = sum_{(i,p)} Psi[k,j,(i,p)] * x[b,c,i,(q*s + p) mod nlon_in]
+ * x (B, C, nlat_in, nlon_in) -> y (B, C, K, nlat_out, nlon_out).  No scratch. */
+disco_status disco_contract(const disco_psi* psi, int B, int C, disco_dtype dtype, const void* x, void* y,
+                            void* stream);
+
+/* The weight einsum alone (the sums over c_i and k of the forward equation):
+ *   out[b,o,j,q] = bias[o] + sum_{c in group(o), k} w[o,c',k] * y[b,c,k,j,q]
+ * y (B, C_in, K, nlat_out, nlon_out), w, bias (nullable) -> out.  No scratch. */
+disco_status disco_einsum(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                          const void* y, const void* w, const void* bias, void* out, void* stream);
+
+/* Forward, unfused: writes the K-expanded y (saved for backward) and out;
+ * the same as disco_contract followed by disco_einsum. */
 disco_status disco_fwd(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
                        const void* x, const void* w, const void* bias, void* y, void* out,
                        void* workspace, size_t ws_bytes, void* stream);
@@ -156,6 +169,10 @@ disco_status disco_bwd_weight(const disco_psi* psi, int B, int C_in, int C_out, 
  * t0, voff, width | kmask << 8) and values. */
 disco_status disco_plan_info(const disco_psi* psi, int which, int* dims);
 disco_status disco_plan_export(const disco_psi* psi, int which, int* rows, int* srcs, int* chunks, float* vals);
+
+/* Number of kernels this library has launched in the process so far (all
+ * devices, all threads); a diagnostic for benchmarks. */
+unsigned long long disco_launch_count(void);
 
 /* Thread-local description of the last non-OK status on this thread. */
 const char* disco_last_error(void);

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <new>
@@ -12,6 +13,13 @@
 #include "../../include/disco.h"
 #include "kernels.h"
 #include "psi_builder.h"
+
+namespace disco {
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace disco
 
 namespace {
 
@@ -168,6 +176,8 @@ extern "C" {
 
 const char* disco_last_error(void) { return g_last_error.c_str(); }
 
+unsigned long long disco_launch_count(void) { return disco::g_launches.load(); }
+
 disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** out) {
   if (!out) return fail(DISCO_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
@@ -301,6 +311,37 @@ disco_status disco_workspace_size(const disco_psi* psi, int op, int B, int C_in,
   return DISCO_OK;
 }
 
+disco_status disco_contract(const disco_psi* psi, int B, int C, disco_dtype dtype, const void* x, void* y,
+                            void* stream) {
+  disco_status s = check_common(psi, B, C, C, 1, dtype);
+  if (s) return s;
+  if (!x || !y) return fail(DISCO_ERR_INVALID_ARG, "x and y must be non-NULL");
+  const disco::Geometry& g = psi->g;
+  if (!disco::gather_supports(g.K, g.stride)) return fail(DISCO_ERR_UNSUPPORTED, "K or stride not compiled");
+  int qb, nblk;
+  block_shape(g.nlon_out, 128, &qb, &nblk);
+  const int need = max_stage(psi->fwd, qb);
+  const int budget = std::max(kStageFloats, need);
+  if ((size_t)(disco::kMaxSrc + 4 + budget) * 4 > kSmemLimit)
+    return fail(DISCO_ERR_UNSUPPORTED, "a Psi row needs more staging than shared memory holds");
+  disco::GatherArgs a = gather_args(psi->dfwd, B * C, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget);
+  cudaError_t e = disco::launch_fwd_gather(dtype == DISCO_BF16, g.K, g.stride, a, x, y, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "contraction launch");
+  return DISCO_OK;
+}
+
+disco_status disco_einsum(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                          const void* y, const void* w, const void* bias, void* out, void* stream) {
+  disco_status s = check_common(psi, B, C_in, C_out, groups, dtype);
+  if (s) return s;
+  if (!y || !w || !out) return fail(DISCO_ERR_INVALID_ARG, "y, w and out must be non-NULL");
+  const disco::Geometry& g = psi->g;
+  disco::MixArgs m{y, w, bias, out, B, groups, C_out / groups, (C_in / groups) * g.K, g.nlat_out * g.nlon_out};
+  cudaError_t e = disco::launch_mix_simt(dtype == DISCO_BF16, m, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "einsum launch");
+  return DISCO_OK;
+}
+
 disco_status disco_fwd(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
                        const void* x, const void* w, const void* bias, void* y, void* out, void* workspace,
                        size_t ws_bytes, void* stream) {
@@ -309,23 +350,9 @@ disco_status disco_fwd(const disco_psi* psi, int B, int C_in, int C_out, int gro
   disco_status s = check_common(psi, B, C_in, C_out, groups, dtype);
   if (s) return s;
   if (!x || !w || !y || !out) return fail(DISCO_ERR_INVALID_ARG, "x, w, y and out must be non-NULL");
-  const disco::Geometry& g = psi->g;
-  if (!disco::gather_supports(g.K, g.stride)) return fail(DISCO_ERR_UNSUPPORTED, "K or stride not compiled");
-  const bool bf16 = dtype == DISCO_BF16;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int qb, nblk;
-  block_shape(g.nlon_out, 128, &qb, &nblk);
-  const int need = max_stage(psi->fwd, qb);
-  const int budget = std::max(kStageFloats, need);
-  if ((size_t)(disco::kMaxSrc + 4 + budget) * 4 > kSmemLimit)
-    return fail(DISCO_ERR_UNSUPPORTED, "a Psi row needs more staging than shared memory holds");
-  disco::GatherArgs a = gather_args(psi->dfwd, B * C_in, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget);
-  cudaError_t e = disco::launch_fwd_gather(bf16, g.K, g.stride, a, x, y, st);
-  if (e != cudaSuccess) return cuda_fail(e, "contraction launch");
-  disco::MixArgs m{y, w, bias, out, B, groups, C_out / groups, (C_in / groups) * g.K, g.nlat_out * g.nlon_out};
-  e = disco::launch_mix_simt(bf16, m, st);
-  if (e != cudaSuccess) return cuda_fail(e, "einsum launch");
-  return DISCO_OK;
+  s = disco_contract(psi, B, C_in, dtype, x, y, stream);
+  if (s) return s;
+  return disco_einsum(psi, B, C_in, C_out, groups, dtype, y, w, bias, out, stream);
 }
 
 disco_status disco_fwd_fused(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,

@@ -185,6 +185,7 @@ cudaError_t launch_mix_simt(bool bf16, const MixArgs& a, cudaStream_t st) {
     mix_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
   else
     mix_kernel<float><<<grid, 256, 0, st>>>(a);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -197,6 +198,7 @@ cudaError_t launch_transpose_weight(bool bf16, const void* w, void* wt, int G, i
   else
     transpose_weight_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(w), static_cast<float*>(wt), G,
                                                            Og, Cg, K);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -206,6 +208,7 @@ cudaError_t launch_dw_partial_simt(bool bf16, const DwArgs& a, cudaStream_t st) 
     dw_partial_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
   else
     dw_partial_kernel<float><<<grid, 256, 0, st>>>(a);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -219,6 +222,7 @@ cudaError_t launch_dw_reduce(bool bf16, const float* part, const float* bpart, v
   else
     dw_reduce_kernel<float><<<blocks, 256, 0, st>>>(part, bpart, static_cast<float*>(dw), static_cast<float*>(dbias),
                                                     nsplit, G, Og, Rg);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -133,6 +133,7 @@ cudaError_t launch_t(const FusedArgs& f, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   dim3 grid(f.g.nblk, f.g.n_rows, f.B * f.G);
   kern<<<grid, kThreads, smem, st>>>(f);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -213,6 +213,7 @@ cudaError_t launch_fwd_t(const GatherArgs& a, const void* x, void* y, cudaStream
   if (e != cudaSuccess) return e;
   dim3 grid((a.BC + a.cb - 1) / a.cb, a.nblk, a.n_rows);
   kern<<<grid, kThreads, smem, st>>>(a, static_cast<const T*>(x), static_cast<T*>(y));
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -224,6 +225,7 @@ cudaError_t launch_adj_t(const GatherArgs& a, const void* dy, void* dx, cudaStre
   if (e != cudaSuccess) return e;
   dim3 grid((a.BC + a.cb - 1) / a.cb, a.nblk, a.n_rows);
   kern<<<grid, kThreads, smem, st>>>(a, static_cast<const T*>(dy), static_cast<T*>(dx));
+  count_launch();
   return cudaGetLastError();
 }
 

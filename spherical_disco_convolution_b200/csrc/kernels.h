@@ -7,6 +7,9 @@
 
 namespace disco {
 
+// Counts a kernel launch (reported by disco_launch_count).
+void count_launch();
+
 struct GatherArgs {
   const RowPlan* rows;
   const SrcRow* srcs;

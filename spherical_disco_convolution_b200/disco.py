@@ -87,6 +87,8 @@ def _load():
         "disco_psi_info": [P, IP, ctypes.POINTER(LL)],
         "disco_psi_export": [P, IP, IP, IP, IP, DP],
         "disco_workspace_size": [P, I, I, I, I, I, I, ctypes.POINTER(Z)],
+        "disco_contract": [P, I, I, I, P, P, P],
+        "disco_einsum": [P, I, I, I, I, I, P, P, P, P, P],
         "disco_fwd": [P, I, I, I, I, I, P, P, P, P, P, P, Z, P],
         "disco_fwd_fused": [P, I, I, I, I, I, P, P, P, P, P, Z, P],
         "disco_bwd_input": [P, I, I, I, I, I, P, P, P, P, Z, P],
@@ -98,6 +100,8 @@ def _load():
         fn = getattr(lib, name)
         fn.argtypes = args
         fn.restype = ctypes.c_int
+    lib.disco_launch_count.argtypes = []
+    lib.disco_launch_count.restype = ctypes.c_ulonglong
     lib.disco_last_error.argtypes = []
     lib.disco_last_error.restype = ctypes.c_char_p
     return lib
@@ -109,7 +113,8 @@ _lib = _load()
 def header_functions() -> list:
     """Names of every function that include/disco.h declares."""
     text = open(HEADER_PATH).read()
-    return sorted(set(re.findall(r"^\s*(?:disco_status|const char\*)\s+(disco_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:disco_status|const char\*|unsigned long long)\s+(disco_\w+)\s*\(",
+                                 text, re.M)))
 
 
 def library():
@@ -119,6 +124,10 @@ def library():
 def _check(status: int):
     if status != DISCO_OK:
         raise DiscoError(status, _lib.disco_last_error().decode())
+
+
+def disco_launch_count() -> int:
+    return int(_lib.disco_launch_count())
 
 
 def disco_last_error() -> str:
@@ -171,6 +180,14 @@ def disco_workspace_size(psi, op, B, C_in, C_out, groups, dtype) -> int:
     n = ctypes.c_size_t()
     _check(_lib.disco_workspace_size(psi, op, B, C_in, C_out, groups, dtype, ctypes.byref(n)))
     return n.value
+
+
+def disco_contract(psi, B, C, dtype, x, y, stream) -> None:
+    _check(_lib.disco_contract(psi, B, C, dtype, x, y, stream))
+
+
+def disco_einsum(psi, B, C_in, C_out, groups, dtype, y, w, bias, out, stream) -> None:
+    _check(_lib.disco_einsum(psi, B, C_in, C_out, groups, dtype, y, w, bias, out, stream))
 
 
 def disco_fwd(psi, B, C_in, C_out, groups, dtype, x, w, bias, y, out, workspace, ws_bytes, stream) -> None:

@@ -90,7 +90,7 @@ def dev(a, wl):
 
 
 def host(t):
-    return t.float().cpu().numpy().astype(np.float64)
+    return t.detach().float().cpu().numpy().astype(np.float64)
 
 
 def check(got, ref, rel, what):
