@@ -101,8 +101,25 @@ int max_stage(const disco::GatherPlan& P, int qb) {
   return m;
 }
 
+constexpr int kChunkCacheMax = 96;
+
+// Dynamic shared memory of a gather CTA (see gather_common.cuh) plus `extra` floats.
+size_t gather_bytes(int cache, int nk, int stage_floats, size_t extra = 0) {
+  return 4 * ((size_t)(disco::kMaxSrc + 4) + (size_t)cache * 4 + (size_t)cache * nk * disco::kChunkW +
+              (size_t)stage_floats + extra);
+}
+
+// Chunks per row kept in shared memory: enough for the typical row, bounded.
+int chunk_cache(const disco::GatherPlan& P) {
+  std::vector<int> n;
+  for (const disco::RowPlan& r : P.rows) n.push_back(r.chunk_end[disco::kMaxStride - 1] - r.chunk_start[0]);
+  if (n.empty()) return 0;
+  std::sort(n.begin(), n.end());
+  return std::min(kChunkCacheMax, n[n.size() * 9 / 10]);
+}
+
 disco::GatherArgs gather_args(const DevPlan& d, int BC, int qb, int nblk, int n_src, int n_src_rows, int n_out,
-                              int n_out_rows, int budget) {
+                              int n_out_rows, int budget, int cache, bool bf16) {
   disco::GatherArgs a;
   a.rows = d.rows;
   a.srcs = d.srcs;
@@ -118,6 +135,8 @@ disco::GatherArgs gather_args(const DevPlan& d, int BC, int qb, int nblk, int n_
   a.n_out = n_out;
   a.n_out_rows = n_out_rows;
   a.stage_budget = budget;
+  a.chunk_cache = cache;
+  a.vec_stage = (n_src % (bf16 ? 8 : 4)) == 0;
   return a;
 }
 
@@ -322,9 +341,10 @@ disco_status disco_contract(const disco_psi* psi, int B, int C, disco_dtype dtyp
   block_shape(g.nlon_out, 128, &qb, &nblk);
   const int need = max_stage(psi->fwd, qb);
   const int budget = std::max(kStageFloats, need);
-  if ((size_t)(disco::kMaxSrc + 4 + budget) * 4 > kSmemLimit)
+  if (gather_bytes(chunk_cache(psi->fwd), g.K, budget) > kSmemLimit)
     return fail(DISCO_ERR_UNSUPPORTED, "a Psi row needs more staging than shared memory holds");
-  disco::GatherArgs a = gather_args(psi->dfwd, B * C, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget);
+  disco::GatherArgs a = gather_args(psi->dfwd, B * C, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget,
+                                    chunk_cache(psi->fwd), dtype == DISCO_BF16);
   cudaError_t e = disco::launch_fwd_gather(dtype == DISCO_BF16, g.K, g.stride, a, x, y, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "contraction launch");
   return DISCO_OK;
@@ -374,11 +394,14 @@ disco_status disco_fwd_fused(const disco_psi* psi, int B, int C_in, int C_out, i
   block_shape(g.nlon_out, cap, &qb, &nblk);
   const int need = max_stage(psi->fwd, qb);
   const int ytile = Cg * g.K * qb;
-  int budget = std::max(need, (int)std::min<size_t>(16384, (kSmemLimit / 4) - (disco::kMaxSrc + 4) - ytile));
-  if ((size_t)(disco::kMaxSrc + 4 + ytile + budget) * 4 > kSmemLimit)
+  const int cache = chunk_cache(psi->fwd);
+  const long room = (long)(kSmemLimit - gather_bytes(cache, g.K, 0, ytile)) / 4;
+  int budget = std::max(need, (int)std::min<long>(16384, room));
+  if (gather_bytes(cache, g.K, budget, ytile) > kSmemLimit)
     return fail(DISCO_ERR_UNSUPPORTED, "fused tile and staging exceed shared memory");
   disco::FusedArgs f;
-  f.g = gather_args(psi->dfwd, B * C_in, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget);
+  f.g = gather_args(psi->dfwd, B * C_in, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget,
+                    chunk_cache(psi->fwd), bf16);
   f.x = x;
   f.w = w;
   f.bias = bias;
@@ -419,10 +442,11 @@ disco_status disco_bwd_input(const disco_psi* psi, int B, int C_in, int C_out, i
   block_shape(g.nlon_out, 128, &qb, &nblk);
   const int need = max_stage(psi->adj, qb);
   const int budget = std::max(kStageFloats, need);
-  if ((size_t)(disco::kMaxSrc + 4 + budget) * 4 > kSmemLimit)
+  if (gather_bytes(chunk_cache(psi->adj), 1, budget) > kSmemLimit)
     return fail(DISCO_ERR_UNSUPPORTED, "a Psi column needs more staging than shared memory holds");
   disco::GatherArgs a =
-      gather_args(psi->dadj, B * C_in, qb, nblk, g.nlon_out, g.K * g.nlat_out, g.nlon_in, g.nlat_in, budget);
+      gather_args(psi->dadj, B * C_in, qb, nblk, g.nlon_out, g.K * g.nlat_out, g.nlon_in, g.nlat_in, budget,
+                  chunk_cache(psi->adj), bf16);
   e = disco::launch_adj_gather(bf16, g.stride, a, dy, dx, st);
   if (e != cudaSuccess) return cuda_fail(e, "adjoint contraction launch");
   return DISCO_OK;
@@ -449,10 +473,11 @@ disco_status disco_bwd_weight(const disco_psi* psi, int B, int C_in, int C_out, 
     block_shape(g.nlon_out, 128, &qb, &nblk);
     const int need = max_stage(psi->fwd, qb);
     const int budget = std::max(kStageFloats, need);
-    if ((size_t)(disco::kMaxSrc + 4 + budget) * 4 > kSmemLimit)
+    if (gather_bytes(chunk_cache(psi->fwd), g.K, budget) > kSmemLimit)
       return fail(DISCO_ERR_UNSUPPORTED, "a Psi row needs more staging than shared memory holds");
     disco::GatherArgs a =
-        gather_args(psi->dfwd, B * C_in, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget);
+        gather_args(psi->dfwd, B * C_in, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget,
+                    chunk_cache(psi->fwd), bf16);
     e = disco::launch_fwd_gather(bf16, g.K, g.stride, a, x, ws + L.ybuf, st);
     if (e != cudaSuccess) return cuda_fail(e, "recompute contraction launch");
     yv = ws + L.ybuf;

@@ -7,42 +7,19 @@
 // of the group into an on-chip y tile [Cg*K][qb] (rounded to the storage type,
 // exactly as the unfused path stores y), then mixes the tile with w into the
 // out block.  y never reaches device memory.
-#include "common.cuh"
-#include "kernels.h"
-#include "plan.h"
+#include "gather_common.cuh"
 
 namespace disco {
 namespace {
 
 constexpr int kThreads = 256;
 
-template <int K, int S, int W>
-__device__ __forceinline__ void chunk_fma(float (&acc)[K][kTaskR], const float* __restrict__ win_ptr,
-                                          const float* __restrict__ v, int kmask) {
-  constexpr int NW = (kTaskR - 1) * S + W;
-  float win[NW];
-#pragma unroll
-  for (int t = 0; t < NW; ++t) win[t] = win_ptr[t];
-#pragma unroll
-  for (int k = 0; k < K; ++k) {
-    if (kmask & (1 << k)) {
-#pragma unroll
-      for (int u = 0; u < W; ++u) {
-        const float vv = __ldg(v + k * kChunkW + u);
-#pragma unroll
-        for (int r = 0; r < kTaskR; ++r) acc[k][r] = fmaf(vv, win[r * S + u], acc[k][r]);
-      }
-    }
-  }
-}
-
 template <typename T, int K, int S>
 __global__ void __launch_bounds__(kThreads) fused_simt_kernel(FusedArgs f) {
-  extern __shared__ float smem[];
-  int* soff = reinterpret_cast<int*>(smem);
-  float* ytile = smem + kMaxSrc + 4;
-  float* stage = ytile + f.ytile_floats;
+  extern __shared__ __align__(16) float smem[];
   const GatherArgs& a = f.g;
+  const GatherSmem s = gather_smem(smem, a.chunk_cache, K);
+  float* ytile = s.stage + a.stage_budget;
   const T* x = static_cast<const T*>(f.x);
   const T* w = static_cast<const T*>(f.w);
   const T* bias = static_cast<const T*>(f.bias);
@@ -51,59 +28,20 @@ __global__ void __launch_bounds__(kThreads) fused_simt_kernel(FusedArgs f) {
   const int q0 = blockIdx.x * a.qb;
   const int b = blockIdx.z / f.G, g = blockIdx.z % f.G;
   const int Cg = f.C_in / f.G, Og = f.C_out / f.G;
-  int stage_elems;
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int s = rp.src_begin; s < rp.src_end; ++s) {
-      soff[s - rp.src_begin] = acc;
-      acc += staged_len(a.srcs[s].span, a.qb, S);
-    }
-    soff[rp.src_end - rp.src_begin] = acc;
-  }
-  __syncthreads();
-  stage_elems = soff[rp.src_end - rp.src_begin];
-  const int cg = max(1, min(Cg, a.stage_budget / max(1, stage_elems)));
+  const int ch_begin = rp.chunk_start[0], nch = rp.chunk_end[0] - rp.chunk_start[0];
+  const int se = gather_prologue(a, rp, ch_begin, rp.chunk_end[0], S, K, s);
+  const int cg = max(1, min(Cg, a.stage_budget / max(1, se)));
   const int tasks_per_ch = a.qb / kTaskR;
-  const size_t x_chan = (size_t)a.n_src_rows * a.n_src;
   const int cbase = b * f.C_in + g * Cg;
   for (int c0 = 0; c0 < Cg; c0 += cg) {
     const int ncg = min(cg, Cg - c0);
-    for (int s = rp.src_begin; s < rp.src_end; ++s) {
-      const SrcRow sr = a.srcs[s];
-      const int len = staged_len(sr.span, a.qb, S);
-      const int first = q0 * S + sr.start;
-      for (int c = 0; c < ncg; ++c) {
-        const T* row = x + (size_t)(cbase + c0 + c) * x_chan + (size_t)sr.row * a.n_src;
-        float* dst = stage + (size_t)c * stage_elems + soff[s - rp.src_begin];
-        for (int t = threadIdx.x; t < len; t += blockDim.x) dst[t] = to_f32(row[wrap_mod(first + t, a.n_src)]);
-      }
-    }
+    stage_rows<T>(a, rp, s, se, x, cbase + c0, ncg, q0 * S, S);
     __syncthreads();
     for (int task = threadIdx.x; task < ncg * tasks_per_ch; task += blockDim.x) {
       const int c = task / tasks_per_ch;
       const int m0 = (task - c * tasks_per_ch) * kTaskR;
-      const float* sb = stage + (size_t)c * stage_elems + m0 * S;
       float acc[K][kTaskR];
-#pragma unroll
-      for (int k = 0; k < K; ++k)
-#pragma unroll
-        for (int r = 0; r < kTaskR; ++r) acc[k][r] = 0.0f;
-      for (int ch = rp.chunk_start[0]; ch < rp.chunk_end[0]; ++ch) {
-        const Chunk cc = a.chunks[ch];
-        const float* wp = sb + soff[cc.src] + cc.t0;
-        const float* v = a.vals + cc.voff;
-        const int kmask = cc.wk >> 8;
-        switch (cc.wk & 0xff) {
-          case 1: chunk_fma<K, S, 1>(acc, wp, v, kmask); break;
-          case 2: chunk_fma<K, S, 2>(acc, wp, v, kmask); break;
-          case 3: chunk_fma<K, S, 3>(acc, wp, v, kmask); break;
-          case 4: chunk_fma<K, S, 4>(acc, wp, v, kmask); break;
-          case 5: chunk_fma<K, S, 5>(acc, wp, v, kmask); break;
-          case 6: chunk_fma<K, S, 6>(acc, wp, v, kmask); break;
-          case 7: chunk_fma<K, S, 7>(acc, wp, v, kmask); break;
-          default: chunk_fma<K, S, 8>(acc, wp, v, kmask); break;
-        }
-      }
+      fwd_task<K, S>(acc, a, s, s.stage + (size_t)c * se + m0 * S, ch_begin, nch);
 #pragma unroll
       for (int k = 0; k < K; ++k)
 #pragma unroll
@@ -128,7 +66,7 @@ __global__ void __launch_bounds__(kThreads) fused_simt_kernel(FusedArgs f) {
 template <typename T, int K, int S>
 cudaError_t launch_t(const FusedArgs& f, cudaStream_t st) {
   auto kern = fused_simt_kernel<T, K, S>;
-  const size_t smem = (size_t)(kMaxSrc + 4 + f.ytile_floats + f.g.stage_budget) * 4;
+  const size_t smem = (gather_smem_floats(f.g.chunk_cache, K, f.g.stage_budget) + f.ytile_floats) * 4;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(f.g.nblk, f.g.n_rows, f.B * f.G);

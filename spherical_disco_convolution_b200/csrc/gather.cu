@@ -8,116 +8,42 @@
 // which for l = s*m + rho reads dy[bc, k, j, m + e] with e = (rho - d)/s.
 //
 // One CTA owns one output row, a block of qb consecutive outputs and a block
-// of channels.  It stages the source rows that the output row reaches in
-// shared memory (fp32, wrap-around already unrolled), then every thread owns
-// kTaskR consecutive outputs of one channel and walks the row's chunks: a
-// window of (kTaskR-1)*step + w staged values is loaded once into registers
-// and reused by all non-zero basis functions of the chunk.
-#include "common.cuh"
-#include "kernels.h"
-#include "plan.h"
+// of channel planes.  It stages the source rows that the output row reaches
+// in shared memory (fp32, wrap-around already unrolled, 16-byte vector moves),
+// then every thread owns kTaskR consecutive outputs of one channel plane and
+// walks the row's chunks: a window of (kTaskR-1)*step + w staged values is
+// loaded once into registers and reused by all non-zero basis functions of
+// the chunk.
+#include "gather_common.cuh"
 
 namespace disco {
 namespace {
 
 constexpr int kThreads = 256;
 
-// Staging: per channel, every source row of the output row back to back.
-// Returns the staged elements per channel; fills soff[] (shared) for each source.
-__device__ __forceinline__ int stage_offsets(const RowPlan& rp, const SrcRow* __restrict__ srcs, int qb, int step,
-                                             int* soff) {
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int s = rp.src_begin; s < rp.src_end; ++s) {
-      soff[s - rp.src_begin] = acc;
-      acc += staged_len(srcs[s].span, qb, step);
-    }
-    soff[rp.src_end - rp.src_begin] = acc;
-  }
-  __syncthreads();
-  return soff[rp.src_end - rp.src_begin];
-}
-
-template <typename T>
-__device__ __forceinline__ void stage_rows(float* stage, int stage_elems, const RowPlan& rp,
-                                           const SrcRow* __restrict__ srcs, const int* soff, const T* __restrict__ src,
-                                           size_t chan_stride, int n_src, int c0, int ncg, int base, int qb, int step) {
-  for (int s = rp.src_begin; s < rp.src_end; ++s) {
-    const SrcRow sr = srcs[s];
-    const int len = staged_len(sr.span, qb, step);
-    const int first = base + sr.start;
-    for (int c = 0; c < ncg; ++c) {
-      const T* row = src + (size_t)(c0 + c) * chan_stride + (size_t)sr.row * n_src;
-      float* dst = stage + (size_t)c * stage_elems + soff[s - rp.src_begin];
-      for (int t = threadIdx.x; t < len; t += blockDim.x) dst[t] = to_f32(row[wrap_mod(first + t, n_src)]);
-    }
-  }
-}
-
-template <int K, int S, int W>
-__device__ __forceinline__ void fwd_chunk(float (&acc)[K][kTaskR], const float* __restrict__ win_ptr,
-                                          const float* __restrict__ v, int kmask) {
-  constexpr int NW = (kTaskR - 1) * S + W;
-  float win[NW];
-#pragma unroll
-  for (int t = 0; t < NW; ++t) win[t] = win_ptr[t];
-#pragma unroll
-  for (int k = 0; k < K; ++k) {
-    if (kmask & (1 << k)) {
-#pragma unroll
-      for (int u = 0; u < W; ++u) {
-        const float vv = __ldg(v + k * kChunkW + u);
-#pragma unroll
-        for (int r = 0; r < kTaskR; ++r) acc[k][r] = fmaf(vv, win[r * S + u], acc[k][r]);
-      }
-    }
-  }
-}
-
 template <typename T, int K, int S>
 __global__ void __launch_bounds__(kThreads) fwd_gather_kernel(GatherArgs a, const T* __restrict__ x,
                                                               T* __restrict__ y) {
-  extern __shared__ float smem[];
-  int* soff = reinterpret_cast<int*>(smem);
-  float* stage = smem + kMaxSrc + 4;
+  extern __shared__ __align__(16) float smem[];
+  const GatherSmem s = gather_smem(smem, a.chunk_cache, K);
   const RowPlan rp = a.rows[blockIdx.z];
   const int q0 = blockIdx.y * a.qb;
   const int c_begin = blockIdx.x * a.cb;
   const int c_end = min(a.BC, c_begin + a.cb);
-  const int se = stage_offsets(rp, a.srcs, a.qb, S, soff);
+  const int ch_begin = rp.chunk_start[0], nch = rp.chunk_end[0] - rp.chunk_start[0];
+  const int se = gather_prologue(a, rp, ch_begin, rp.chunk_end[0], S, K, s);
   const int cg = max(1, min(a.cb, a.stage_budget / max(1, se)));
   const int tasks_per_ch = a.qb / kTaskR;
-  const size_t x_chan = (size_t)a.n_src_rows * a.n_src;
   for (int c0 = c_begin; c0 < c_end; c0 += cg) {
     const int ncg = min(cg, c_end - c0);
-    stage_rows<T>(stage, se, rp, a.srcs, soff, x, x_chan, a.n_src, c0, ncg, q0 * S, a.qb, S);
+    stage_rows<T>(a, rp, s, se, x, c0, ncg, q0 * S, S);
     __syncthreads();
     for (int task = threadIdx.x; task < ncg * tasks_per_ch; task += blockDim.x) {
       const int c = task / tasks_per_ch;
       const int m0 = (task - c * tasks_per_ch) * kTaskR;
       if (q0 + m0 >= a.n_out) continue;
-      const float* sb = stage + (size_t)c * se + m0 * S;
       float acc[K][kTaskR];
-#pragma unroll
-      for (int k = 0; k < K; ++k)
-#pragma unroll
-        for (int r = 0; r < kTaskR; ++r) acc[k][r] = 0.0f;
-      for (int ch = rp.chunk_start[0]; ch < rp.chunk_end[0]; ++ch) {
-        const Chunk cc = a.chunks[ch];
-        const float* wp = sb + soff[cc.src] + cc.t0;
-        const float* v = a.vals + cc.voff;
-        const int kmask = cc.wk >> 8;
-        switch (cc.wk & 0xff) {
-          case 1: fwd_chunk<K, S, 1>(acc, wp, v, kmask); break;
-          case 2: fwd_chunk<K, S, 2>(acc, wp, v, kmask); break;
-          case 3: fwd_chunk<K, S, 3>(acc, wp, v, kmask); break;
-          case 4: fwd_chunk<K, S, 4>(acc, wp, v, kmask); break;
-          case 5: fwd_chunk<K, S, 5>(acc, wp, v, kmask); break;
-          case 6: fwd_chunk<K, S, 6>(acc, wp, v, kmask); break;
-          case 7: fwd_chunk<K, S, 7>(acc, wp, v, kmask); break;
-          default: fwd_chunk<K, S, 8>(acc, wp, v, kmask); break;
-        }
-      }
+      fwd_task<K, S>(acc, a, s, s.stage + (size_t)c * se + m0 * S, ch_begin, nch);
       const int n = min(kTaskR, a.n_out - (q0 + m0));
 #pragma unroll
       for (int k = 0; k < K; ++k) {
@@ -138,7 +64,7 @@ __device__ __forceinline__ void adj_chunk(float (&acc)[kTaskR], const float* __r
   for (int t = 0; t < NW; ++t) win[t] = win_ptr[t];
 #pragma unroll
   for (int u = 0; u < W; ++u) {
-    const float vv = __ldg(v + u);
+    const float vv = v[u];
 #pragma unroll
     for (int r = 0; r < kTaskR; ++r) acc[r] = fmaf(vv, win[r + u], acc[r]);
   }
@@ -147,36 +73,36 @@ __device__ __forceinline__ void adj_chunk(float (&acc)[kTaskR], const float* __r
 template <typename T, int S>
 __global__ void __launch_bounds__(kThreads) adj_gather_kernel(GatherArgs a, const T* __restrict__ dy,
                                                               T* __restrict__ dx) {
-  extern __shared__ float smem[];
-  int* soff = reinterpret_cast<int*>(smem);
-  float* stage = smem + kMaxSrc + 4;
+  extern __shared__ __align__(16) float smem[];
+  const GatherSmem s = gather_smem(smem, a.chunk_cache, 1);
   const RowPlan rp = a.rows[blockIdx.z];
   const int m_blk = blockIdx.y * a.qb;
   const int c_begin = blockIdx.x * a.cb;
   const int c_end = min(a.BC, c_begin + a.cb);
-  const int se = stage_offsets(rp, a.srcs, a.qb, 1, soff);
+  const int ch_begin = rp.chunk_start[0];
+  const int se = gather_prologue(a, rp, ch_begin, rp.chunk_end[S - 1], 1, 1, s);
   const int cg = max(1, min(a.cb, a.stage_budget / max(1, se)));
   const int tasks_per_ch = a.qb / kTaskR;
-  const size_t dy_chan = (size_t)a.n_src_rows * a.n_src;
   const int n_m = a.n_out / S;  // outputs l = S*m + rho, m < n_m
   for (int c0 = c_begin; c0 < c_end; c0 += cg) {
     const int ncg = min(cg, c_end - c0);
-    stage_rows<T>(stage, se, rp, a.srcs, soff, dy, dy_chan, a.n_src, c0, ncg, m_blk, a.qb, 1);
+    stage_rows<T>(a, rp, s, se, dy, c0, ncg, m_blk, 1);
     __syncthreads();
     for (int task = threadIdx.x; task < ncg * tasks_per_ch; task += blockDim.x) {
       const int c = task / tasks_per_ch;
       const int m0 = (task - c * tasks_per_ch) * kTaskR;
       if (m_blk + m0 >= n_m) continue;
-      const float* sb = stage + (size_t)c * se + m0;
+      const float* sb = s.stage + (size_t)c * se + m0;
       float acc[S][kTaskR];
 #pragma unroll
       for (int rho = 0; rho < S; ++rho) {
 #pragma unroll
         for (int r = 0; r < kTaskR; ++r) acc[rho][r] = 0.0f;
-        for (int ch = rp.chunk_start[rho]; ch < rp.chunk_end[rho]; ++ch) {
-          const Chunk cc = a.chunks[ch];
-          const float* wp = sb + soff[cc.src] + cc.t0;
-          const float* v = a.vals + cc.voff;
+        for (int ch = rp.chunk_start[rho] - ch_begin; ch < rp.chunk_end[rho] - ch_begin; ++ch) {
+          Chunk cc;
+          const float* v;
+          chunk_at(a, s, ch_begin, ch, 1, &cc, &v);
+          const float* wp = sb + s.soff[cc.src] + cc.t0;
           switch (cc.wk & 0xff) {
             case 1: adj_chunk<1>(acc[rho], wp, v); break;
             case 2: adj_chunk<2>(acc[rho], wp, v); break;
@@ -208,7 +134,7 @@ __global__ void __launch_bounds__(kThreads) adj_gather_kernel(GatherArgs a, cons
 template <typename T, int K, int S>
 cudaError_t launch_fwd_t(const GatherArgs& a, const void* x, void* y, cudaStream_t st) {
   auto kern = fwd_gather_kernel<T, K, S>;
-  const size_t smem = (size_t)(kMaxSrc + 4) * 4 + (size_t)a.stage_budget * 4;
+  const size_t smem = gather_smem_floats(a.chunk_cache, K, a.stage_budget) * 4;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.BC + a.cb - 1) / a.cb, a.nblk, a.n_rows);
@@ -220,7 +146,7 @@ cudaError_t launch_fwd_t(const GatherArgs& a, const void* x, void* y, cudaStream
 template <typename T, int S>
 cudaError_t launch_adj_t(const GatherArgs& a, const void* dy, void* dx, cudaStream_t st) {
   auto kern = adj_gather_kernel<T, S>;
-  const size_t smem = (size_t)(kMaxSrc + 4) * 4 + (size_t)a.stage_budget * 4;
+  const size_t smem = gather_smem_floats(a.chunk_cache, 1, a.stage_budget) * 4;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.BC + a.cb - 1) / a.cb, a.nblk, a.n_rows);

@@ -1,0 +1,171 @@
+// Shared pieces of the gather kernels: source-row staging and the per-row chunk cache.
+#pragma once
+
+#include "common.cuh"
+#include "kernels.h"
+#include "plan.h"
+
+namespace disco {
+
+// Dynamic shared memory layout of a gather CTA:
+//   int   soff[kMaxSrc + 4]              staging offset of every source row (+ total)
+//   Chunk cch[chunk_cache]               the first chunk_cache chunks of the row
+//   float cval[chunk_cache * nk * 8]     their values
+//   float stage[...]                     staged source rows, channel after channel
+struct GatherSmem {
+  int* soff;
+  Chunk* cch;
+  float* cval;
+  float* stage;
+};
+
+__device__ __forceinline__ GatherSmem gather_smem(float* smem, int chunk_cache, int nk) {
+  GatherSmem s;
+  s.soff = reinterpret_cast<int*>(smem);
+  s.cch = reinterpret_cast<Chunk*>(smem + kMaxSrc + 4);
+  s.cval = reinterpret_cast<float*>(s.cch + chunk_cache);
+  s.stage = s.cval + (size_t)chunk_cache * nk * kChunkW;
+  return s;
+}
+
+__host__ __device__ inline size_t gather_smem_floats(int chunk_cache, int nk, int stage_floats) {
+  return (size_t)(kMaxSrc + 4) + (size_t)chunk_cache * 4 + (size_t)chunk_cache * nk * kChunkW + stage_floats;
+}
+
+// Staging offsets of the row's source rows; returns the elements staged per channel.
+// Also copies the row's first chunks and their values into shared memory.
+__device__ __forceinline__ int gather_prologue(const GatherArgs& a, const RowPlan& rp, int ch_begin, int ch_end,
+                                               int step, int nk, const GatherSmem& s) {
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int t = rp.src_begin; t < rp.src_end; ++t) {
+      s.soff[t - rp.src_begin] = acc;
+      acc += staged_len(a.srcs[t].span, a.qb, step);
+    }
+    s.soff[rp.src_end - rp.src_begin] = acc;
+  }
+  const int ncache = min(ch_end - ch_begin, a.chunk_cache);
+  for (int t = threadIdx.x; t < ncache; t += blockDim.x) s.cch[t] = a.chunks[ch_begin + t];
+  if (ncache > 0) {
+    const float* v0 = a.vals + a.chunks[ch_begin].voff;  // a row's chunk values are contiguous
+    for (int t = threadIdx.x; t < ncache * nk * kChunkW; t += blockDim.x) s.cval[t] = __ldg(v0 + t);
+  }
+  __syncthreads();
+  return s.soff[rp.src_end - rp.src_begin];
+}
+
+// Chunk ch (row-relative) and its values: from the cache, else from global memory.
+__device__ __forceinline__ void chunk_at(const GatherArgs& a, const GatherSmem& s, int ch_begin, int ch, int nk,
+                                         Chunk* c, const float** v) {
+  if (ch < a.chunk_cache) {
+    *c = s.cch[ch];
+    *v = s.cval + (size_t)ch * nk * kChunkW;
+  } else {
+    *c = a.chunks[ch_begin + ch];
+    *v = a.vals + c->voff;
+  }
+}
+
+__device__ __forceinline__ void to_floats(const uint4& u, float (&f)[8], const __nv_bfloat16*) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// Stages every source row of the output row for channel planes c0 .. c0+ncg-1.
+// Staged element t of a source row holds source longitude (base + start + t) mod n_src.
+// With `vec`, starts are multiples of kAlign (the plan guarantees it) and n_src is a
+// multiple of the 16-byte vector, so whole vectors are moved.
+template <typename T>
+__device__ __forceinline__ void stage_rows(const GatherArgs& a, const RowPlan& rp, const GatherSmem& s, int se,
+                                           const T* __restrict__ src, int c0, int ncg, int base, int step) {
+  const size_t chan = (size_t)a.n_src_rows * a.n_src;
+  const int n = a.n_src;
+  for (int t = rp.src_begin; t < rp.src_end; ++t) {
+    const SrcRow sr = a.srcs[t];
+    const int len = staged_len(sr.span, a.qb, step);
+    const int first = wrap_mod(base + sr.start, n);
+    float* dst0 = s.stage + s.soff[t - rp.src_begin];
+    const T* row0 = src + (size_t)sr.row * n;
+    if (a.vec_stage) {
+      constexpr int V = 16 / sizeof(T);
+      const int ng = len / V;
+      for (int idx = threadIdx.x; idx < ncg * ng; idx += blockDim.x) {
+        const int c = idx / ng, g = idx - c * ng;
+        int l = first + g * V;
+        while (l >= n) l -= n;
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(row0 + (size_t)(c0 + c) * chan + l));
+        float* dst = dst0 + (size_t)c * se + g * V;
+        if constexpr (sizeof(T) == 2) {
+          float f[8];
+          to_floats(u, f, static_cast<const __nv_bfloat16*>(nullptr));
+          reinterpret_cast<float4*>(dst)[0] = make_float4(f[0], f[1], f[2], f[3]);
+          reinterpret_cast<float4*>(dst)[1] = make_float4(f[4], f[5], f[6], f[7]);
+        } else {
+          reinterpret_cast<float4*>(dst)[0] =
+              make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
+        }
+      }
+    } else {
+      for (int idx = threadIdx.x; idx < ncg * len; idx += blockDim.x) {
+        const int c = idx / len, e = idx - c * len;
+        int l = first + e;
+        while (l >= n) l -= n;
+        dst0[(size_t)c * se + e] = to_f32(row0[(size_t)(c0 + c) * chan + l]);
+      }
+    }
+  }
+}
+
+// acc[k][r] += sum_u v[k][u] * win[r*S + u] for the basis functions set in kmask.
+template <int K, int S, int W>
+__device__ __forceinline__ void fwd_chunk(float (&acc)[K][kTaskR], const float* __restrict__ win_ptr,
+                                          const float* __restrict__ v, int kmask) {
+  constexpr int NW = (kTaskR - 1) * S + W;
+  float win[NW];
+#pragma unroll
+  for (int t = 0; t < NW; ++t) win[t] = win_ptr[t];
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    if (kmask & (1 << k)) {
+#pragma unroll
+      for (int u = 0; u < W; ++u) {
+        const float vv = v[k * kChunkW + u];
+#pragma unroll
+        for (int r = 0; r < kTaskR; ++r) acc[k][r] = fmaf(vv, win[r * S + u], acc[k][r]);
+      }
+    }
+  }
+}
+
+// All chunks of the row for one task (kTaskR outputs of one channel plane).
+template <int K, int S>
+__device__ __forceinline__ void fwd_task(float (&acc)[K][kTaskR], const GatherArgs& a, const GatherSmem& s,
+                                         const float* sb, int ch_begin, int nch) {
+#pragma unroll
+  for (int k = 0; k < K; ++k)
+#pragma unroll
+    for (int r = 0; r < kTaskR; ++r) acc[k][r] = 0.0f;
+  for (int ch = 0; ch < nch; ++ch) {
+    Chunk cc;
+    const float* v;
+    chunk_at(a, s, ch_begin, ch, K, &cc, &v);
+    const float* wp = sb + s.soff[cc.src] + cc.t0;
+    const int kmask = cc.wk >> 8;
+    switch (cc.wk & 0xff) {
+      case 1: fwd_chunk<K, S, 1>(acc, wp, v, kmask); break;
+      case 2: fwd_chunk<K, S, 2>(acc, wp, v, kmask); break;
+      case 3: fwd_chunk<K, S, 3>(acc, wp, v, kmask); break;
+      case 4: fwd_chunk<K, S, 4>(acc, wp, v, kmask); break;
+      case 5: fwd_chunk<K, S, 5>(acc, wp, v, kmask); break;
+      case 6: fwd_chunk<K, S, 6>(acc, wp, v, kmask); break;
+      case 7: fwd_chunk<K, S, 7>(acc, wp, v, kmask); break;
+      default: fwd_chunk<K, S, 8>(acc, wp, v, kmask); break;
+    }
+  }
+}
+
+}  // namespace disco

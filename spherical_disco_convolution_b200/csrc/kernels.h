@@ -22,6 +22,8 @@ struct GatherArgs {
   int n_src, n_src_rows;  // source row length, source rows per channel plane
   int n_out, n_out_rows;  // output row length, output rows per channel plane
   int stage_budget;  // staged floats per CTA (>= the largest row's per-channel need)
+  int chunk_cache;   // chunks (and their values) of a row kept in shared memory
+  int vec_stage;     // 1: stage whole 16-byte vectors (n_src a multiple of the vector)
 };
 
 bool gather_supports(int K, int stride);

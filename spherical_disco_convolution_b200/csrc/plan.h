@@ -35,6 +35,7 @@ constexpr int kTaskR = 8;       // consecutive outputs per thread
 constexpr int kMaxStride = 4;   // nlon_in / nlon_out supported by the kernels
 constexpr int kMaxK = 16;       // basis functions supported by the kernels
 constexpr int kMaxSrc = 512;    // source rows per output row supported by the kernels
+constexpr int kAlign = 8;       // staged rows start on a multiple of 8 longitudes (16 bytes of bf16)
 
 struct SrcRow {
   int row;     // row index into the source tensor's (row, longitude) plane of one channel
@@ -59,9 +60,9 @@ struct RowPlan {
   float cost;                   // relative work, used to order heavy rows first
 };
 
-// Staged elements of one source row for a block of qb outputs.
+// Staged elements of one source row for a block of qb outputs (a multiple of kAlign).
 DISCO_HD inline int staged_len(int span, int qb, int step) {
-  return (((qb + kTaskR - 1) * step + span + kChunkW) + 3) & ~3;
+  return (((qb + kTaskR - 1) * step + span + kChunkW) + kAlign - 1) & ~(kAlign - 1);
 }
 
 }  // namespace disco

@@ -242,12 +242,16 @@ GatherPlan make_forward_plan(const Geometry& g, const std::vector<PsiEntry>& e) 
       ps.erase(std::unique(ps.begin(), ps.end()), ps.end());
       int d0, span;
       circular_interval(ps, g.nlon_in, &d0, &span);
-      P.src.push_back(SrcRow{i, d0, span, 0});
+      // stage from a multiple of kAlign so that staging moves 16-byte vectors
+      const int lead = pos_mod(d0, kAlign);
+      const int a0 = d0 - lead;
+      span += lead;
+      P.src.push_back(SrcRow{i, a0, span, 0});
       staged += (float)(span + 128 * g.stride);
       std::vector<double> tab((size_t)g.K * span, 0.0);
       std::vector<char> has(span, 0);
       for (size_t t = u; t < v; ++t) {
-        const int col = pos_mod(rowe[t]->p - d0, g.nlon_in);
+        const int col = lead + pos_mod(rowe[t]->p - d0, g.nlon_in);
         tab[(size_t)rowe[t]->k * span + col] = rowe[t]->v;
         has[col] = 1;
       }
@@ -310,6 +314,8 @@ GatherPlan make_adjoint_plan(const Geometry& g, const std::vector<PsiEntry>& e) 
           emin = std::min(emin, ev);
           emax = std::max(emax, ev);
         }
+        const int lead = pos_mod(emin, kAlign);
+        emin -= lead;
         const int espan = emax - emin + 1;
         P.src.push_back(SrcRow{k * g.nlat_out + j, emin, espan, 0});
         staged += (float)(espan + 128);
