@@ -161,14 +161,17 @@ disco_status disco_bwd_weight(const disco_psi* psi, int B, int C_in, int C_out, 
 /* Diagnostics: the host copy of a gather plan, for inspection by tests.
  * which = 0 is the forward contraction plan (output rows j), which = 1 the
  * adjoint plan used by disco_bwd_input (output rows i).  disco_plan_info fills
- * dims[8] = {rows, source rows, chunks, values, value sets per chunk, source
- * step per output, residue classes, ints per row record}.  disco_plan_export
- * copies the records into caller-owned HOST arrays sized from dims: rows
- * (rows x ints-per-row: row, src_begin, src_end, chunk_start[4], chunk_end[4],
- * cost as float bits), source rows (x4: row, start, span, 0), chunks (x4: src,
- * t0, voff, width | kmask << 8) and values. */
+ * dims[9] = {rows, source rows, chunks, values, value sets per chunk, source
+ * step per output, residue classes, ints per row record, ring terms}.
+ * disco_plan_export copies the records into caller-owned HOST arrays sized
+ * from dims: rows (rows x ints-per-row: row, src_begin, src_end,
+ * chunk_start[4], chunk_end[4], ring_begin, ring_end, cost as float bits),
+ * source rows (x4: row, start, span, 0), chunks (x4: src, t0, voff,
+ * width | kmask << 8), values, and ring terms (x4: source row, k, value as
+ * float bits, 0). */
 disco_status disco_plan_info(const disco_psi* psi, int which, int* dims);
-disco_status disco_plan_export(const disco_psi* psi, int which, int* rows, int* srcs, int* chunks, float* vals);
+disco_status disco_plan_export(const disco_psi* psi, int which, int* rows, int* srcs, int* chunks, float* vals,
+                               int* rings);
 
 /* Number of kernels this library has launched in the process so far (all
  * devices, all threads); a diagnostic for benchmarks. */

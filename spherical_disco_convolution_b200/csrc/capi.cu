@@ -11,6 +11,7 @@
 #include <vector>
 
 #include "../../include/disco.h"
+#include "gather_common.cuh"
 #include "kernels.h"
 #include "psi_builder.h"
 
@@ -39,6 +40,7 @@ struct DevPlan {
   disco::SrcRow* srcs = nullptr;
   disco::Chunk* chunks = nullptr;
   float* vals = nullptr;
+  disco::Ring* rings = nullptr;
   int n_rows = 0;
 };
 
@@ -57,6 +59,7 @@ cudaError_t upload_plan(const disco::GatherPlan& P, DevPlan* d) {
   if ((e = upload(P.rows, &d->rows)) != cudaSuccess) return e;
   if ((e = upload(P.src, &d->srcs)) != cudaSuccess) return e;
   if ((e = upload(P.chunks, &d->chunks)) != cudaSuccess) return e;
+  if ((e = upload(P.rings, &d->rings)) != cudaSuccess) return e;
   return upload(P.vals, &d->vals);
 }
 
@@ -65,6 +68,7 @@ void free_plan(DevPlan* d) {
   cudaFree(d->srcs);
   cudaFree(d->chunks);
   cudaFree(d->vals);
+  cudaFree(d->rings);
   *d = DevPlan{};
 }
 
@@ -103,10 +107,9 @@ int max_stage(const disco::GatherPlan& P, int qb) {
 
 constexpr int kChunkCacheMax = 96;
 
-// Dynamic shared memory of a gather CTA (see gather_common.cuh) plus `extra` floats.
+// Dynamic shared memory of a gather CTA (layout in gather_common.cuh) plus `extra` floats.
 size_t gather_bytes(int cache, int nk, int stage_floats, size_t extra = 0) {
-  return 4 * ((size_t)(disco::kMaxSrc + 4) + (size_t)cache * 4 + (size_t)cache * nk * disco::kChunkW +
-              (size_t)stage_floats + extra);
+  return 4 * (disco::gather_smem_floats(cache, nk, stage_floats) + extra);
 }
 
 // Chunks per row kept in shared memory: enough for the typical row, bounded.
@@ -125,6 +128,7 @@ disco::GatherArgs gather_args(const DevPlan& d, int BC, int qb, int nblk, int n_
   a.srcs = d.srcs;
   a.chunks = d.chunks;
   a.vals = d.vals;
+  a.rings = d.rings;
   a.n_rows = d.n_rows;
   a.BC = BC;
   a.cb = kChannelsPerCta;
@@ -237,7 +241,8 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
   }
   h->fwd = disco::make_forward_plan(g, h->entries);
   h->adj = disco::make_adjoint_plan(g, h->entries);
-  if (h->fwd.max_src > disco::kMaxSrc || h->adj.max_src > disco::kMaxSrc) {
+  if (h->fwd.max_src > disco::kMaxSrc || h->adj.max_src > disco::kMaxSrc || h->fwd.max_ring > disco::kMaxRing ||
+      h->adj.max_ring > disco::kMaxRing) {
     delete h;
     return fail(DISCO_ERR_UNSUPPORTED, "an output row reaches more source rows than the kernels support");
   }
@@ -306,13 +311,16 @@ disco_status disco_plan_info(const disco_psi* psi, int which, int* dims) {
   dims[5] = P.step;
   dims[6] = P.residues;
   dims[7] = (int)(sizeof(disco::RowPlan) / sizeof(int));
+  dims[8] = (int)P.rings.size();
   return DISCO_OK;
 }
 
-disco_status disco_plan_export(const disco_psi* psi, int which, int* rows, int* srcs, int* chunks, float* vals) {
-  if (!psi || !rows || !srcs || !chunks || !vals || (which != 0 && which != 1))
+disco_status disco_plan_export(const disco_psi* psi, int which, int* rows, int* srcs, int* chunks, float* vals,
+                               int* rings) {
+  if (!psi || !rows || !srcs || !chunks || !vals || !rings || (which != 0 && which != 1))
     return fail(DISCO_ERR_INVALID_ARG, "bad plan export");
   const disco::GatherPlan& P = which == 0 ? psi->fwd : psi->adj;
+  std::memcpy(rings, P.rings.data(), P.rings.size() * sizeof(disco::Ring));
   std::memcpy(rows, P.rows.data(), P.rows.size() * sizeof(disco::RowPlan));
   std::memcpy(srcs, P.src.data(), P.src.size() * sizeof(disco::SrcRow));
   std::memcpy(chunks, P.chunks.data(), P.chunks.size() * sizeof(disco::Chunk));

@@ -30,25 +30,18 @@ __global__ void __launch_bounds__(kThreads) fused_simt_kernel(FusedArgs f) {
   const int Cg = f.C_in / f.G, Og = f.C_out / f.G;
   const int ch_begin = rp.chunk_start[0], nch = rp.chunk_end[0] - rp.chunk_start[0];
   const int se = gather_prologue(a, rp, ch_begin, rp.chunk_end[0], S, K, s);
-  const int cg = max(1, min(Cg, a.stage_budget / max(1, se)));
-  const int tasks_per_ch = a.qb / kTaskR;
+  const int cg = max(1, min(min(Cg, kMaxCb), a.stage_budget / max(1, se)));
   const int cbase = b * f.C_in + g * Cg;
   for (int c0 = 0; c0 < Cg; c0 += cg) {
     const int ncg = min(cg, Cg - c0);
-    stage_rows<T>(a, rp, s, se, x, cbase + c0, ncg, q0 * S, S);
-    __syncthreads();
-    for (int task = threadIdx.x; task < ncg * tasks_per_ch; task += blockDim.x) {
-      const int c = task / tasks_per_ch;
-      const int m0 = (task - c * tasks_per_ch) * kTaskR;
-      float acc[K][kTaskR];
-      fwd_task<K, S>(acc, a, s, s.stage + (size_t)c * se + m0 * S, ch_begin, nch);
+    auto sink = [&](int c, int m0, float (&acc)[K][kTaskR]) {
 #pragma unroll
       for (int k = 0; k < K; ++k)
 #pragma unroll
         for (int r = 0; r < kTaskR; ++r)
           ytile[((size_t)(c0 + c) * K + k) * a.qb + m0 + r] = round_trip<T>(acc[k][r]);
-    }
-    __syncthreads();
+    };
+    fwd_block<T, K, S>(a, rp, s, se, x, cbase + c0, ncg, q0 * S, ch_begin, nch, sink);
   }
   const int R = Cg * K;
   for (int idx = threadIdx.x; idx < Og * a.qb; idx += blockDim.x) {

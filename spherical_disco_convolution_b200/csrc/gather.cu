@@ -13,13 +13,30 @@
 // then every thread owns kTaskR consecutive outputs of one channel plane and
 // walks the row's chunks: a window of (kTaskR-1)*step + w staged values is
 // loaded once into registers and reused by all non-zero basis functions of
-// the chunk.
+// the chunk.  Full circles of one constant value (rings) enter as value x
+// row sum.  Rows with many chunks and few staged channels split their chunk
+// list over idle threads and combine the partial sums in a fixed order.
 #include "gather_common.cuh"
 
 namespace disco {
 namespace {
 
 constexpr int kThreads = 256;
+
+template <typename T, int K>
+struct YSink {
+  T* y;
+  int c0, n_out_rows, row, n_out, q0;
+  __device__ __forceinline__ void operator()(int c, int m0, float (&acc)[K][kTaskR]) const {
+    if (q0 + m0 >= n_out) return;
+    const int n = min(kTaskR, n_out - (q0 + m0));
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      T* dst = y + (((size_t)(c0 + c) * K + k) * n_out_rows + row) * n_out + q0 + m0;
+      store_run<T, kTaskR>(dst, acc[k], n);
+    }
+  }
+};
 
 template <typename T, int K, int S>
 __global__ void __launch_bounds__(kThreads) fwd_gather_kernel(GatherArgs a, const T* __restrict__ x,
@@ -32,26 +49,11 @@ __global__ void __launch_bounds__(kThreads) fwd_gather_kernel(GatherArgs a, cons
   const int c_end = min(a.BC, c_begin + a.cb);
   const int ch_begin = rp.chunk_start[0], nch = rp.chunk_end[0] - rp.chunk_start[0];
   const int se = gather_prologue(a, rp, ch_begin, rp.chunk_end[0], S, K, s);
-  const int cg = max(1, min(a.cb, a.stage_budget / max(1, se)));
-  const int tasks_per_ch = a.qb / kTaskR;
+  const int cg = max(1, min(min(a.cb, kMaxCb), a.stage_budget / max(1, se)));
   for (int c0 = c_begin; c0 < c_end; c0 += cg) {
     const int ncg = min(cg, c_end - c0);
-    stage_rows<T>(a, rp, s, se, x, c0, ncg, q0 * S, S);
-    __syncthreads();
-    for (int task = threadIdx.x; task < ncg * tasks_per_ch; task += blockDim.x) {
-      const int c = task / tasks_per_ch;
-      const int m0 = (task - c * tasks_per_ch) * kTaskR;
-      if (q0 + m0 >= a.n_out) continue;
-      float acc[K][kTaskR];
-      fwd_task<K, S>(acc, a, s, s.stage + (size_t)c * se + m0 * S, ch_begin, nch);
-      const int n = min(kTaskR, a.n_out - (q0 + m0));
-#pragma unroll
-      for (int k = 0; k < K; ++k) {
-        T* dst = y + (((size_t)(c0 + c) * K + k) * a.n_out_rows + rp.row) * a.n_out + q0 + m0;
-        store_run<T, kTaskR>(dst, acc[k], n);
-      }
-    }
-    __syncthreads();
+    YSink<T, K> sink{y, c0, a.n_out_rows, rp.row, a.n_out, q0};
+    fwd_block<T, K, S>(a, rp, s, se, x, c0, ncg, q0 * S, ch_begin, nch, sink);
   }
 }
 
@@ -70,6 +72,33 @@ __device__ __forceinline__ void adj_chunk(float (&acc)[kTaskR], const float* __r
   }
 }
 
+template <int S>
+__device__ __forceinline__ void adj_task(float (&acc)[S][kTaskR], const GatherArgs& a, const GatherSmem& s,
+                                         const RowPlan& rp, const float* sb, int ch_begin, int sl, int nsl) {
+#pragma unroll
+  for (int rho = 0; rho < S; ++rho) {
+#pragma unroll
+    for (int r = 0; r < kTaskR; ++r) acc[rho][r] = 0.0f;
+    const int lo = rp.chunk_start[rho] - ch_begin, n = rp.chunk_end[rho] - rp.chunk_start[rho];
+    for (int ch = lo + (sl * n) / nsl; ch < lo + ((sl + 1) * n) / nsl; ++ch) {
+      Chunk cc;
+      const float* v;
+      chunk_at(a, s, ch_begin, ch, 1, &cc, &v);
+      const float* wp = sb + s.soff[cc.src] + cc.t0;
+      switch (cc.wk & 0xff) {
+        case 1: adj_chunk<1>(acc[rho], wp, v); break;
+        case 2: adj_chunk<2>(acc[rho], wp, v); break;
+        case 3: adj_chunk<3>(acc[rho], wp, v); break;
+        case 4: adj_chunk<4>(acc[rho], wp, v); break;
+        case 5: adj_chunk<5>(acc[rho], wp, v); break;
+        case 6: adj_chunk<6>(acc[rho], wp, v); break;
+        case 7: adj_chunk<7>(acc[rho], wp, v); break;
+        default: adj_chunk<8>(acc[rho], wp, v); break;
+      }
+    }
+  }
+}
+
 template <typename T, int S>
 __global__ void __launch_bounds__(kThreads) adj_gather_kernel(GatherArgs a, const T* __restrict__ dy,
                                                               T* __restrict__ dx) {
@@ -79,52 +108,73 @@ __global__ void __launch_bounds__(kThreads) adj_gather_kernel(GatherArgs a, cons
   const int m_blk = blockIdx.y * a.qb;
   const int c_begin = blockIdx.x * a.cb;
   const int c_end = min(a.BC, c_begin + a.cb);
-  const int ch_begin = rp.chunk_start[0];
+  const int ch_begin = rp.chunk_start[0], nch = rp.chunk_end[S - 1] - rp.chunk_start[0];
   const int se = gather_prologue(a, rp, ch_begin, rp.chunk_end[S - 1], 1, 1, s);
-  const int cg = max(1, min(a.cb, a.stage_budget / max(1, se)));
-  const int tasks_per_ch = a.qb / kTaskR;
+  const int cg = max(1, min(min(a.cb, kMaxCb), a.stage_budget / max(1, se)));
+  const int tpc = a.qb / kTaskR;
   const int n_m = a.n_out / S;  // outputs l = S*m + rho, m < n_m
+  const int nring = rp.ring_end - rp.ring_begin;
   for (int c0 = c_begin; c0 < c_end; c0 += cg) {
     const int ncg = min(cg, c_end - c0);
     stage_rows<T>(a, rp, s, se, dy, c0, ncg, m_blk, 1);
+    ring_sums<T>(a, s, nring, dy, c0, ncg);
     __syncthreads();
-    for (int task = threadIdx.x; task < ncg * tasks_per_ch; task += blockDim.x) {
-      const int c = task / tasks_per_ch;
-      const int m0 = (task - c * tasks_per_ch) * kTaskR;
-      if (m_blk + m0 >= n_m) continue;
-      const float* sb = s.stage + (size_t)c * se + m0;
-      float acc[S][kTaskR];
-#pragma unroll
-      for (int rho = 0; rho < S; ++rho) {
-#pragma unroll
-        for (int r = 0; r < kTaskR; ++r) acc[rho][r] = 0.0f;
-        for (int ch = rp.chunk_start[rho] - ch_begin; ch < rp.chunk_end[rho] - ch_begin; ++ch) {
-          Chunk cc;
-          const float* v;
-          chunk_at(a, s, ch_begin, ch, 1, &cc, &v);
-          const float* wp = sb + s.soff[cc.src] + cc.t0;
-          switch (cc.wk & 0xff) {
-            case 1: adj_chunk<1>(acc[rho], wp, v); break;
-            case 2: adj_chunk<2>(acc[rho], wp, v); break;
-            case 3: adj_chunk<3>(acc[rho], wp, v); break;
-            case 4: adj_chunk<4>(acc[rho], wp, v); break;
-            case 5: adj_chunk<5>(acc[rho], wp, v); break;
-            case 6: adj_chunk<6>(acc[rho], wp, v); break;
-            case 7: adj_chunk<7>(acc[rho], wp, v); break;
-            default: adj_chunk<8>(acc[rho], wp, v); break;
-          }
-        }
-      }
+    const int tasks = ncg * tpc;
+    const int nsl = slice_count(tasks, nch, S * kTaskR, a.stage_budget);
+    auto finish = [&](int c, int m0, float (&acc)[S][kTaskR]) {
+      if (m_blk + m0 >= n_m) return;
+      float ring = 0.0f;
+      for (int t = 0; t < nring; ++t) ring += s.rings[t].v * s.rsum[c * nring + t];
       const int nm = min(kTaskR, n_m - (m_blk + m0));
       T* dst = dx + ((size_t)(c0 + c) * a.n_out_rows + rp.row) * a.n_out + (size_t)S * (m_blk + m0);
       if constexpr (S == 1) {
+#pragma unroll
+        for (int r = 0; r < kTaskR; ++r) acc[0][r] += ring;
         store_run<T, kTaskR>(dst, acc[0], nm);
       } else {
 #pragma unroll
         for (int r = 0; r < kTaskR; ++r)
 #pragma unroll
           for (int rho = 0; rho < S; ++rho)
-            if (r < nm) dst[r * S + rho] = from_f32<T>(acc[rho][r]);
+            if (r < nm) dst[r * S + rho] = from_f32<T>(acc[rho][r] + ring);
+      }
+    };
+    if (nsl == 1) {
+      for (int task = threadIdx.x; task < tasks; task += blockDim.x) {
+        const int c = task / tpc, m0 = (task - c * tpc) * kTaskR;
+        float acc[S][kTaskR];
+        adj_task<S>(acc, a, s, rp, s.stage + (size_t)c * se + m0, ch_begin, 0, 1);
+        finish(c, m0, acc);
+      }
+    } else {
+      const int tg = threadIdx.x;
+      const bool active = tg < nsl * tasks;
+      const int sl = tg / tasks, task = tg - sl * tasks;
+      float acc[S][kTaskR];
+      if (active) {
+        const int c = task / tpc, m0 = (task - c * tpc) * kTaskR;
+        adj_task<S>(acc, a, s, rp, s.stage + (size_t)c * se + m0, ch_begin, sl, nsl);
+      }
+      __syncthreads();  // staging consumed: reuse it for the partial sums
+      float* red = s.stage;
+      if (active)
+#pragma unroll
+        for (int rho = 0; rho < S; ++rho)
+#pragma unroll
+          for (int r = 0; r < kTaskR; ++r) red[((size_t)(sl * tasks + task) * S + rho) * kTaskR + r] = acc[rho][r];
+      __syncthreads();
+      for (int t = threadIdx.x; t < tasks; t += blockDim.x) {
+        const int c = t / tpc, m0 = (t - c * tpc) * kTaskR;
+        float sum[S][kTaskR];
+#pragma unroll
+        for (int rho = 0; rho < S; ++rho)
+#pragma unroll
+          for (int r = 0; r < kTaskR; ++r) {
+            float v = 0.0f;
+            for (int q = 0; q < nsl; ++q) v += red[((size_t)(q * tasks + t) * S + rho) * kTaskR + r];
+            sum[rho][r] = v;
+          }
+        finish(c, m0, sum);
       }
     }
     __syncthreads();

@@ -15,6 +15,7 @@ struct GatherArgs {
   const SrcRow* srcs;
   const Chunk* chunks;
   const float* vals;
+  const Ring* rings;
   int n_rows;        // output rows in the plan (grid.z)
   int BC;            // channel planes (batch * channels)
   int cb;            // channel planes per CTA

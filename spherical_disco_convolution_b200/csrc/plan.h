@@ -35,6 +35,7 @@ constexpr int kTaskR = 8;       // consecutive outputs per thread
 constexpr int kMaxStride = 4;   // nlon_in / nlon_out supported by the kernels
 constexpr int kMaxK = 16;       // basis functions supported by the kernels
 constexpr int kMaxSrc = 512;    // source rows per output row supported by the kernels
+constexpr int kMaxRing = 64;    // ring terms per output row supported by the kernels
 constexpr int kAlign = 8;       // staged rows start on a multiple of 8 longitudes (16 bytes of bf16)
 
 struct SrcRow {
@@ -51,12 +52,24 @@ struct Chunk {
   int wk;      // width (1..kChunkW) in bits 0..7, kmask (bit k: basis k non-zero) from bit 8
 };
 
+// A full longitude circle of one source row that enters with one constant
+// value (an input pole row, or any row seen from an output pole with an
+// isotropic basis): its contribution is value * (sum of the source row), the
+// same for every output longitude.
+struct Ring {
+  int row;     // source row index (as SrcRow::row)
+  int k;       // accumulator (basis function; 0 for the adjoint)
+  float v;     // the constant value
+  int pad;
+};
+
 // One output row of a gather plan.
 struct RowPlan {
   int row;                      // output row (j for the forward, i for the adjoint)
   int src_begin, src_end;
   int chunk_start[kMaxStride];  // chunk list of residue class rho: [chunk_start[rho], chunk_end[rho])
   int chunk_end[kMaxStride];    // (the forward plan only has rho = 0)
+  int ring_begin, ring_end;     // ring terms of the row
   float cost;                   // relative work, used to order heavy rows first
 };
 

@@ -171,7 +171,10 @@ int build_psi_entries(const Geometry& g, std::vector<PsiEntry>& out, std::string
 namespace {
 
 void order_rows(GatherPlan& P) {
-  for (const RowPlan& rp : P.rows) P.max_src = std::max(P.max_src, rp.src_end - rp.src_begin);
+  for (const RowPlan& rp : P.rows) {
+    P.max_src = std::max(P.max_src, rp.src_end - rp.src_begin);
+    P.max_ring = std::max(P.max_ring, rp.ring_end - rp.ring_begin);
+  }
   std::stable_sort(P.rows.begin(), P.rows.end(),
                    [](const RowPlan& a, const RowPlan& b) { return a.cost > b.cost; });
 }
@@ -205,6 +208,19 @@ void emit_chunks(GatherPlan& P, const std::vector<double>& tab, const std::vecto
   }
 }
 
+// True when `vals` covers all n longitudes of a circle with one value (to 1e-12 relative).
+bool constant_ring(const std::vector<double>& vals, int n, double* mean) {
+  if ((int)vals.size() != n) return false;
+  double s = 0.0, lo = vals[0], hi = vals[0];
+  for (double v : vals) {
+    s += v;
+    lo = std::min(lo, v);
+    hi = std::max(hi, v);
+  }
+  *mean = s / n;
+  return hi - lo <= 1e-12 * std::fabs(*mean);
+}
+
 }  // namespace
 
 int stage_elems(const GatherPlan& P, const RowPlan& r, int qb) {
@@ -230,14 +246,35 @@ GatherPlan make_forward_plan(const Geometry& g, const std::vector<PsiEntry>& e) 
     rp.row = j;
     rp.src_begin = (int)P.src.size();
     rp.chunk_start[0] = (int)P.chunks.size();
+    rp.ring_begin = (int)P.rings.size();
     float cost = 0.0f, staged = 0.0f;
     size_t u = 0;
     while (u < rowe.size()) {
       const int i = rowe[u]->i;
       size_t v = u;
       while (v < rowe.size() && rowe[v]->i == i) ++v;
+      // full circles of one constant value become ring terms
+      std::vector<char> is_ring(g.K, 0);
+      for (int k = 0; k < g.K; ++k) {
+        std::vector<double> vk;
+        for (size_t t = u; t < v; ++t)
+          if (rowe[t]->k == k) vk.push_back(rowe[t]->v);
+        double mean;
+        if (constant_ring(vk, g.nlon_in, &mean)) {
+          is_ring[k] = 1;
+          P.rings.push_back(Ring{i, k, (float)mean, 0});
+          cost += 0.01f * g.nlon_in / std::max(1, g.nlon_out);
+        }
+      }
+      std::vector<const PsiEntry*> keep;
+      for (size_t t = u; t < v; ++t)
+        if (!is_ring[rowe[t]->k]) keep.push_back(rowe[t]);
+      if (keep.empty()) {
+        u = v;
+        continue;
+      }
       std::vector<int> ps;
-      for (size_t t = u; t < v; ++t) ps.push_back(rowe[t]->p);
+      for (const PsiEntry* e : keep) ps.push_back(e->p);
       std::sort(ps.begin(), ps.end());
       ps.erase(std::unique(ps.begin(), ps.end()), ps.end());
       int d0, span;
@@ -250,9 +287,9 @@ GatherPlan make_forward_plan(const Geometry& g, const std::vector<PsiEntry>& e) 
       staged += (float)(span + 128 * g.stride);
       std::vector<double> tab((size_t)g.K * span, 0.0);
       std::vector<char> has(span, 0);
-      for (size_t t = u; t < v; ++t) {
-        const int col = lead + pos_mod(rowe[t]->p - d0, g.nlon_in);
-        tab[(size_t)rowe[t]->k * span + col] = rowe[t]->v;
+      for (const PsiEntry* e : keep) {
+        const int col = lead + pos_mod(e->p - d0, g.nlon_in);
+        tab[(size_t)e->k * span + col] = e->v;
         has[col] = 1;
       }
       emit_chunks(P, tab, has, span, g.K, (int)P.src.size() - 1 - rp.src_begin, &cost);
@@ -260,6 +297,7 @@ GatherPlan make_forward_plan(const Geometry& g, const std::vector<PsiEntry>& e) 
     }
     rp.src_end = (int)P.src.size();
     rp.chunk_end[0] = (int)P.chunks.size();
+    rp.ring_end = (int)P.rings.size();
     for (int rho = 1; rho < kMaxStride; ++rho) rp.chunk_start[rho] = rp.chunk_end[rho] = rp.chunk_end[0];
     rp.cost = cost + 0.02f * staged;
     P.rows.push_back(rp);
@@ -286,6 +324,7 @@ GatherPlan make_adjoint_plan(const Geometry& g, const std::vector<PsiEntry>& e) 
     RowPlan rp{};
     rp.row = i;
     rp.src_begin = (int)P.src.size();
+    rp.ring_begin = (int)P.rings.size();
     float cost = 0.0f, staged = 0.0f;
     struct Pending { int rho; std::vector<double> tab; std::vector<char> has; int span; int src_rel; };
     std::vector<Pending> pend;
@@ -306,6 +345,18 @@ GatherPlan make_adjoint_plan(const Geometry& g, const std::vector<PsiEntry>& e) 
         const int k = ent[w0]->k;
         size_t w1 = w0;
         while (w1 < v && ent[w1]->k == k) ++w1;
+        {
+          // a constant full circle: every dx[l] takes v * (sum of the dy row)
+          std::vector<double> vk;
+          for (size_t t = w0; t < w1; ++t) vk.push_back(ent[t]->v);
+          double mean;
+          if (constant_ring(vk, g.nlon_in, &mean)) {
+            P.rings.push_back(Ring{k * g.nlat_out + j, 0, (float)mean, 0});
+            cost += 0.01f * g.nlon_out;
+            w0 = w1;
+            continue;
+          }
+        }
         // dx[l = s*m + rho] takes dy[m + e] with e = (rho - d)/s, d the signed offset, rho = d mod s
         int emin = 1 << 30, emax = -(1 << 30);
         for (size_t t = w0; t < w1; ++t) {
@@ -344,6 +395,7 @@ GatherPlan make_adjoint_plan(const Geometry& g, const std::vector<PsiEntry>& e) 
       rp.chunk_end[rho] = (int)P.chunks.size();
     }
     rp.src_end = (int)P.src.size();
+    rp.ring_end = (int)P.rings.size();
     rp.cost = cost + 0.02f * staged;
     P.rows.push_back(rp);
   }

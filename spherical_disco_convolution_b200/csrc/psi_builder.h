@@ -29,10 +29,12 @@ struct GatherPlan {
   std::vector<SrcRow> src;
   std::vector<Chunk> chunks;
   std::vector<float> vals;
+  std::vector<Ring> rings;
   int nk = 1;          // value sets per chunk (K for the forward, 1 for the adjoint)
   int step = 1;        // source positions advance by `step` per output (forward: s; adjoint: 1)
   int residues = 1;    // output residue classes (adjoint: s)
   int max_src = 0;     // most source rows of any output row
+  int max_ring = 0;    // most ring terms of any output row
 };
 
 // Elements staged per channel for output row `r` and a block of qb outputs.

@@ -94,7 +94,7 @@ def _load():
         "disco_bwd_input": [P, I, I, I, I, I, P, P, P, P, Z, P],
         "disco_bwd_weight": [P, I, I, I, I, I, P, P, P, P, P, P, Z, P],
         "disco_plan_info": [P, I, IP],
-        "disco_plan_export": [P, I, IP, IP, IP, ctypes.POINTER(ctypes.c_float)],
+        "disco_plan_export": [P, I, IP, IP, IP, ctypes.POINTER(ctypes.c_float), IP],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -163,17 +163,20 @@ def disco_psi_export(psi):
 
 def disco_plan_export(psi, which: int):
     """Plan arrays of the forward (which=0) or adjoint (which=1) gather kernels."""
-    dims = np.zeros(8, dtype=np.int32)
+    dims = np.zeros(9, dtype=np.int32)
     _check(_lib.disco_plan_info(psi, which, dims.ctypes.data_as(ctypes.POINTER(ctypes.c_int))))
-    n_rows, n_src, n_chunks, n_vals, nk, step, residues, row_ints = (int(v) for v in dims)
+    n_rows, n_src, n_chunks, n_vals, nk, step, residues, row_ints, n_rings = (int(v) for v in dims)
     rows = np.zeros((n_rows, row_ints), dtype=np.int32)
     srcs = np.zeros((n_src, 4), dtype=np.int32)
     chunks = np.zeros((n_chunks, 4), dtype=np.int32)
     vals = np.zeros(n_vals, dtype=np.float32)
+    rings = np.zeros((max(n_rings, 1), 4), dtype=np.int32)
     ip = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))  # noqa: E731
     _check(_lib.disco_plan_export(psi, which, ip(rows), ip(srcs), ip(chunks),
-                                  vals.ctypes.data_as(ctypes.POINTER(ctypes.c_float))))
-    return dict(rows=rows, srcs=srcs, chunks=chunks, vals=vals, nk=nk, step=step, residues=residues)
+                                  vals.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), ip(rings)))
+    ring_v = rings[:n_rings, 2].copy().view(np.float32)
+    return dict(rows=rows, srcs=srcs, chunks=chunks, vals=vals, nk=nk, step=step, residues=residues,
+                rings=rings[:n_rings], ring_v=ring_v)
 
 
 def disco_workspace_size(psi, op, B, C_in, C_out, groups, dtype) -> int:

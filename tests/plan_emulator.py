@@ -2,7 +2,8 @@
 
 The CUDA gather kernels read, for output m of a row, the staged element
 t0 + m*step + u of a chunk's source row, where staged element t holds source
-longitude (start + t) mod n_src (block offset zero).  This module applies
+longitude (start + t) mod n_src (block offset zero), and add value x (sum of
+the source row) for every ring term.  This module applies
 exactly that rule to the plan records exported by libdisco, in fp64, so a
 wrong offset, wrap, residue class or value layout in the host plans shows up
 against the oracle on the CPU, before any kernel runs.
@@ -19,6 +20,9 @@ def forward(plan, x, nlat_out, nlon_out, K):
     step = plan["step"]
     for r in plan["rows"]:
         row, sb = r[0], r[1]
+        for t in range(r[11], r[12]):
+            srow, k = plan["rings"][t][:2]
+            y[:, k, row, :] += float(plan["ring_v"][t]) * x[:, srow, :].sum(axis=-1)[:, None]
         for ch in range(r[3], r[7]):
             src, t0, voff, wk = plan["chunks"][ch]
             srow, start = plan["srcs"][sb + src][:2]
@@ -39,6 +43,9 @@ def adjoint(plan, dy, nlat_in, nlon_in, stride):
     m = np.arange(n_src)
     for r in plan["rows"]:
         row, sb = r[0], r[1]
+        for t in range(r[11], r[12]):
+            srow = plan["rings"][t][0]
+            dx[:, row, :] += float(plan["ring_v"][t]) * dy[:, srow, :].sum(axis=-1)[:, None]
         for rho in range(stride):
             for ch in range(r[3 + rho], r[7 + rho]):
                 src, t0, voff, wk = plan["chunks"][ch]
