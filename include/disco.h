@@ -158,6 +158,35 @@ disco_status disco_bwd_weight(const disco_psi* psi, int B, int C_in, int C_out, 
                               const void* dout, const void* y, const void* x, void* dw, void* dbias,
                               void* workspace, size_t ws_bytes, void* stream);
 
+/* Weight gradient that allocates nothing (the pages have no counterpart to this entry point).
+ *
+ * disco_bwd_weight needs a caller-provided workspace for its split-K partial sums.  Some
+ * callers cannot provide one: code that runs inside a host application whose device
+ * memory is all owned by that application's allocator, and code that must not allocate
+ * once it has started (a cudaMalloc can synchronise the device, fail under memory
+ * pressure, or be forbidden by the surrounding framework).  This variant computes the
+ * same dw and dbias with its partial sums in a fixed 8 MiB array built into the library;
+ * every GPU that loads the library holds that array until the process exits.  It calls
+ * no cudaMalloc, cudaFree or other allocating routine.
+ *
+ *   - Arguments as for disco_bwd_weight, except that y is required (no recompute from x:
+ *     that would need a y-sized buffer) and there is no workspace.
+ *   - Limit: B * (C_out * (C_in/groups) * K + C_out) <= 2^21 (floats of the array);
+ *     larger layers get DISCO_ERR_UNSUPPORTED with a message, and nothing is launched.
+ *   - Results equal disco_bwd_weight's up to the order of the split-K additions (this
+ *     variant may use fewer, longer splits); the order is fixed, so repeated calls give
+ *     identical bits.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call before any
+ *     stream capture.
+ *   - All calls share the one array and each call overwrites every entry it later reads,
+ *     so nothing from an earlier call leaks into a result.  Calls that can overlap on the
+ *     GPU (on different streams, or from threads that do not order their streams) race on
+ *     the array and produce wrong results: serialise them. */
+disco_status disco_bwd_weight_noalloc(const disco_psi* psi, int B, int C_in, int C_out, int groups,
+                                      disco_dtype dtype, const void* dout, const void* y, void* dw, void* dbias,
+                                      void* stream);
+
 /* Diagnostics: the host copy of a gather plan, for inspection by tests.
  * which = 0 is the forward contraction plan (output rows j), which = 1 the
  * adjoint plan used by disco_bwd_input (output rows i).  disco_plan_info fills

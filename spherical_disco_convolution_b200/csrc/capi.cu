@@ -6,6 +6,7 @@
 #include <atomic>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -502,3 +503,77 @@ disco_status disco_bwd_weight(const disco_psi* psi, int B, int C_in, int C_out, 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Weight gradient without any device allocation.
+//
+// The split-K partial sums of disco_bwd_weight normally live in a workspace
+// that the caller allocates.  This variant keeps them in a fixed array that is
+// part of the library image instead, for callers that may not allocate device
+// memory at all.  The array is reached from host code only through the device
+// address that cudaGetSymbolAddress returns (the host-side name of a
+// __device__ array is not a device address).
+
+static constexpr size_t kNoAllocScratchFloats = size_t(1) << 21;  // 8 MiB of fp32
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+constexpr int kNoAllocMaxDevices = 64;
+float* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device `dev` (looked up once per device).
+disco_status noalloc_scratch(int dev, float** out) {
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(DISCO_ERR_UNSUPPORTED, "device ordinal above 63");
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static scratch");
+    g_noalloc_addr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_addr[dev];
+  return DISCO_OK;
+}
+
+}  // namespace
+
+extern "C" disco_status disco_bwd_weight_noalloc(const disco_psi* psi, int B, int C_in, int C_out, int groups,
+                                                 disco_dtype dtype, const void* dout, const void* y, void* dw,
+                                                 void* dbias, void* stream) {
+  disco_status s = check_common(psi, B, C_in, C_out, groups, dtype);
+  if (s) return s;
+  if (!dout || !y || !dw) return fail(DISCO_ERR_INVALID_ARG, "dout, y and dw must be non-NULL");
+  const disco::Geometry& g = psi->g;
+  const int Og = C_out / groups, Rg = (C_in / groups) * g.K, N = g.nlat_out * g.nlon_out;
+  // one split needs C_out*Rg partial weights plus C_out partial biases; every batch needs a split
+  const size_t per_split = (size_t)C_out * Rg + (size_t)C_out;
+  const size_t max_splits = kNoAllocScratchFloats / per_split;
+  if (max_splits < (size_t)B)
+    return fail(DISCO_ERR_UNSUPPORTED,
+                "B * (C_out * (C_in/groups) * K + C_out) floats exceed the 8 MiB static scratch of "
+                "disco_bwd_weight_noalloc; use disco_bwd_weight with a workspace");
+  int nchunk = std::min<long>((N + 4095) / 4096, (long)(max_splits / B));
+  nchunk = std::max(nchunk, 1);
+  const int nc = (N + nchunk - 1) / nchunk;
+  nchunk = (N + nc - 1) / nc;
+  int dev = -1;
+  cudaGetDevice(&dev);
+  float* scratch = nullptr;
+  s = noalloc_scratch(dev, &scratch);
+  if (s) return s;
+  const size_t nsplit = (size_t)B * nchunk;
+  // The partial kernel writes every (split, o, r) entry and every (split, o) bias entry that the
+  // reduction reads, so nothing left by an earlier call is used and nothing needs clearing.
+  float* part = scratch;
+  float* bpart = dbias ? scratch + nsplit * (size_t)C_out * Rg : nullptr;
+  const bool bf16 = dtype == DISCO_BF16;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  disco::DwArgs d{dout, y, part, bpart, B, groups, Og, Rg, N, nc, nchunk};
+  cudaError_t e = disco::launch_dw_partial_simt(bf16, d, st);
+  if (e != cudaSuccess) return cuda_fail(e, "weight-gradient launch");
+  e = disco::launch_dw_reduce(bf16, part, bpart, dw, dbias, (int)nsplit, groups, Og, Rg, st);
+  if (e != cudaSuccess) return cuda_fail(e, "weight-gradient reduce launch");
+  return DISCO_OK;
+}

@@ -93,6 +93,7 @@ def _load():
         "disco_fwd_fused": [P, I, I, I, I, I, P, P, P, P, P, Z, P],
         "disco_bwd_input": [P, I, I, I, I, I, P, P, P, P, Z, P],
         "disco_bwd_weight": [P, I, I, I, I, I, P, P, P, P, P, P, Z, P],
+        "disco_bwd_weight_noalloc": [P, I, I, I, I, I, P, P, P, P, P],
         "disco_plan_info": [P, I, IP],
         "disco_plan_export": [P, I, IP, IP, IP, ctypes.POINTER(ctypes.c_float), IP],
     }
@@ -208,3 +209,7 @@ def disco_bwd_input(psi, B, C_in, C_out, groups, dtype, dout, w, dx, workspace, 
 def disco_bwd_weight(psi, B, C_in, C_out, groups, dtype, dout, y, x, dw, dbias, workspace, ws_bytes, stream) -> None:
     _check(_lib.disco_bwd_weight(psi, B, C_in, C_out, groups, dtype, dout, y, x, dw, dbias, workspace, ws_bytes,
                                  stream))
+
+
+def disco_bwd_weight_noalloc(psi, B, C_in, C_out, groups, dtype, dout, y, dw, dbias, stream) -> None:
+    _check(_lib.disco_bwd_weight_noalloc(psi, B, C_in, C_out, groups, dtype, dout, y, dw, dbias, stream))
