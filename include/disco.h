@@ -202,6 +202,12 @@ disco_status disco_plan_info(const disco_psi* psi, int which, int* dims);
 disco_status disco_plan_export(const disco_psi* psi, int which, int* rows, int* srcs, int* chunks, float* vals,
                                int* rings);
 
+/* Synchronises `stream` and reports device-side failures of the calls queued on it
+ * before: DISCO_ERR_CUDA for an asynchronous CUDA error, DISCO_ERR_TIMEOUT when a
+ * tensor-core kernel gave up a bounded wait (its results are then invalid).  Clears the
+ * timeout record. */
+disco_status disco_sync_status(void* stream);
+
 /* Number of kernels this library has launched in the process so far (all
  * devices, all threads); a diagnostic for benchmarks. */
 unsigned long long disco_launch_count(void);

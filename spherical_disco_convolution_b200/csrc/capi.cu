@@ -163,7 +163,14 @@ disco_status check_common(const disco_psi* psi, int B, int C_in, int C_out, int 
 struct WsLayout {
   size_t wt = 0, dy = 0, ybuf = 0, part = 0, bpart = 0, total = 0;
   int nchunk = 0, nc = 0;
+  bool tc = false;  // weight gradient on tensor cores
 };
+
+// Weight einsum (and its transpose): tensor cores for bf16 when TMA can address the rows.
+cudaError_t launch_mix(bool bf16, const disco::MixArgs& m, cudaStream_t st) {
+  if (bf16 && disco::mix_tc_supported(m.Mg, m.Rg, m.N)) return disco::launch_mix_tc(m, st);
+  return disco::launch_mix_simt(bf16, m, st);
+}
 
 WsLayout layout(const disco_psi* psi, int op, int B, int C_in, int C_out, int groups, disco_dtype dtype) {
   WsLayout L;
@@ -177,7 +184,8 @@ WsLayout layout(const disco_psi* psi, int op, int B, int C_in, int C_out, int gr
     L.total = L.dy + align256(y_elems * es);
   } else if (op == DISCO_OP_BWD_WEIGHT || op == DISCO_OP_BWD_WEIGHT_RECOMPUTE) {
     const int N = (int)n_out;
-    L.nc = 4096;
+    L.tc = dtype == DISCO_BF16 && disco::dw_tc_supported(C_out / groups, (C_in / groups) * g.K, N);
+    L.nc = L.tc ? 8192 : 4096;
     L.nchunk = (N + L.nc - 1) / L.nc;
     const size_t nsplit = (size_t)B * L.nchunk;
     size_t off = 0;
@@ -201,6 +209,13 @@ extern "C" {
 const char* disco_last_error(void) { return g_last_error.c_str(); }
 
 unsigned long long disco_launch_count(void) { return disco::g_launches.load(); }
+
+disco_status disco_sync_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronisation");
+  if (disco::take_mix_tc_status()) return fail(DISCO_ERR_TIMEOUT, "a bounded device-side wait expired");
+  return DISCO_OK;
+}
 
 disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** out) {
   if (!out) return fail(DISCO_ERR_INVALID_ARG, "out is NULL");
@@ -366,7 +381,7 @@ disco_status disco_einsum(const disco_psi* psi, int B, int C_in, int C_out, int 
   if (!y || !w || !out) return fail(DISCO_ERR_INVALID_ARG, "y, w and out must be non-NULL");
   const disco::Geometry& g = psi->g;
   disco::MixArgs m{y, w, bias, out, B, groups, C_out / groups, (C_in / groups) * g.K, g.nlat_out * g.nlon_out};
-  cudaError_t e = disco::launch_mix_simt(dtype == DISCO_BF16, m, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_mix(dtype == DISCO_BF16, m, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "einsum launch");
   return DISCO_OK;
 }
@@ -445,7 +460,7 @@ disco_status disco_bwd_input(const disco_psi* psi, int B, int C_in, int C_out, i
   cudaError_t e = disco::launch_transpose_weight(bf16, w, wt, groups, Og, Cg, g.K, st);
   if (e != cudaSuccess) return cuda_fail(e, "weight transpose launch");
   disco::MixArgs m{dout, wt, nullptr, dy, B, groups, Cg * g.K, Og, g.nlat_out * g.nlon_out};
-  e = disco::launch_mix_simt(bf16, m, st);
+  e = launch_mix(bf16, m, st);
   if (e != cudaSuccess) return cuda_fail(e, "transposed einsum launch");
   int qb, nblk;
   block_shape(g.nlon_out, 128, &qb, &nblk);
@@ -495,7 +510,7 @@ disco_status disco_bwd_weight(const disco_psi* psi, int B, int C_in, int C_out, 
   float* part = reinterpret_cast<float*>(ws + L.part);
   float* bpart = dbias ? reinterpret_cast<float*>(ws + L.bpart) : nullptr;
   disco::DwArgs d{dout, yv, part, bpart, B, groups, Og, Rg, g.nlat_out * g.nlon_out, L.nc, L.nchunk};
-  e = disco::launch_dw_partial_simt(bf16, d, st);
+  e = L.tc ? disco::launch_dw_tc(d, st) : disco::launch_dw_partial_simt(bf16, d, st);
   if (e != cudaSuccess) return cuda_fail(e, "weight-gradient launch");
   e = disco::launch_dw_reduce(bf16, part, bpart, dw, dbias, B * L.nchunk, groups, Og, Rg, st);
   if (e != cudaSuccess) return cuda_fail(e, "weight-gradient reduce launch");

@@ -41,6 +41,12 @@ struct MixArgs {
   int B, G, Mg, Rg, N;
 };
 cudaError_t launch_mix_simt(bool bf16, const MixArgs& a, cudaStream_t st);
+// Tensor-core (tcgen05) form for bf16: needs Mg % 16 == 0, Rg % 8 == 0 and N % 8 == 0
+// (TMA rows start on 16-byte boundaries).
+bool mix_tc_supported(int Mg, int Rg, int N);
+cudaError_t launch_mix_tc(const MixArgs& a, cudaStream_t st);
+// Device status word of the tensor-core kernels (5 after an expired wait); read and clear.
+int take_mix_tc_status();
 
 // wt[g, c*K + k, o] = w[g*Og + o, c, k]   (the transposed weight of the dx einsum)
 cudaError_t launch_transpose_weight(bool bf16, const void* w, void* wt, int G, int Og, int Cg, int K, cudaStream_t st);
@@ -57,6 +63,9 @@ struct DwArgs {
   int B, G, Og, Rg, N, nc, nchunk;
 };
 cudaError_t launch_dw_partial_simt(bool bf16, const DwArgs& a, cudaStream_t st);
+// Tensor-core form for bf16 (Og % 16 == 0, Og <= 256, N % 8 == 0); nc must be a multiple of 64.
+bool dw_tc_supported(int Og, int Rg, int N);
+cudaError_t launch_dw_tc(const DwArgs& a, cudaStream_t st);
 // dw[g*Og + o, r] = sum_split part[split, g, o, r]; dbias[o] = sum_split bpart[split, o]; fixed order.
 cudaError_t launch_dw_reduce(bool bf16, const float* part, const float* bpart, void* dw, void* dbias, int nsplit,
                              int G, int Og, int Rg, cudaStream_t st);

@@ -1,0 +1,363 @@
+// Tensor-core (tcgen05) forms of the dense channel contractions, bf16 in, fp32 accumulate.
+//
+// The weight einsum of the forward equation on the page
+// "torch_harmonics.DiscreteContinuousConvS2" (the sums over c_i and k of
+// w_k^{co,ci} times the contracted signal) and the transposed einsum of the
+// input gradient are one GEMM per (batch, group):
+//     out[g*Mg + m, n] = sum_r wm[g, m, r] * in[g*Rg + r, n]  (+ bias)
+// computed here as D[n, m] with M = 128 grid points per tile (A = `in`,
+// MN-major: n is contiguous) and N = a tile of up to 256 output channels
+// (B = `wm`, K-major: r is contiguous).  The weight gradient is the split-K GEMM
+//     part[split, g, o, r] = sum_{n in split} y[g*Rg + r, n] * dout[g*Og + o, n]
+// computed as D[r, o] with both operands K-major (n contiguous).
+//
+// One CTA = 4 warps: lane 0 of warp 0 issues the TMA loads through a ring of
+// stages, lane 0 of warp 1 issues the MMAs (fp32 accumulator in tensor
+// memory), all four warps read the accumulator back (one TMEM lane per thread)
+// and store.  Every wait is bounded (tc_common.cuh).
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace disco {
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kBK = 64;                      // K elements per stage (one 128-byte swizzle row)
+constexpr uint32_t kHalfTile = 64 * 128;     // one [64 K][64 M] MN-major box, bytes
+
+struct MixTcArgs {
+  void* out;
+  const void* bias;
+  int G, Mg, Rg, N, BN;
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__host__ __device__ inline uint32_t tmem_cols(int n) {
+  uint32_t c = 32;
+  while ((int)c < n) c <<= 1;
+  return c;
+}
+
+__global__ void __launch_bounds__(128, 1) mix_tc_kernel(const __grid_constant__ CUtensorMap map_in,
+                                                        const __grid_constant__ CUtensorMap map_w, MixTcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const int BN = a.BN;
+  const uint32_t a_bytes = 2 * kHalfTile;
+  const uint32_t b_bytes = (uint32_t)BN * 128;
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * a_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * b_bytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* done = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+  const int n0 = blockIdx.x * 128;
+  const int m0 = blockIdx.y * BN;
+  const int bg = blockIdx.z;
+  const int g = bg % a.G;
+  const int nk = (a.Rg + kBK - 1) / kBK;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ncols = tmem_cols(BN);
+
+  if (threadIdx.x == 0) {
+    tc::prefetch_map(&map_in);
+    tc::prefetch_map(&map_w);
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(done, 1);
+    tc::fence_barrier_init();
+  }
+  if (warp == 2) {
+    tc::tmem_alloc(tmem_slot, ncols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    for (int kc = 0; kc < nk; ++kc) {
+      const int s = kc % kStages;
+      if (kc >= kStages && !tc::mbar_wait(&empty[s], ((kc / kStages) & 1) ^ 1)) break;
+      tc::mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes);
+      tc::tma_load_3d(sA + s * a_bytes, &map_in, &full[s], n0, kc * kBK, bg);
+      tc::tma_load_3d(sA + s * a_bytes + kHalfTile, &map_in, &full[s], n0 + 64, kc * kBK, bg);
+      tc::tma_load_2d(sB + s * b_bytes, &map_w, &full[s], kc * kBK, g * a.Mg + m0);
+    }
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t idesc = tc::idesc_bf16(128, BN, true, false);
+    bool ok = true;
+    for (int kc = 0; kc < nk && ok; ++kc) {
+      const int s = kc % kStages;
+      ok = tc::mbar_wait(&full[s], (kc / kStages) & 1);
+      if (!ok) break;
+      tc::fence_after_sync();
+      const uint32_t a0 = tc::smem_u32(sA + s * a_bytes);
+      const uint32_t b0 = tc::smem_u32(sB + s * b_bytes);
+#pragma unroll
+      for (int kk = 0; kk < kBK / 16; ++kk) {
+        // A (MN-major): 16 K-rows of 128 B per step; the two 64-wide M halves are 8 KB apart
+        const uint64_t ad = tc::desc_sw128(a0 + kk * 2048, kHalfTile, 1024);
+        // B (K-major): 16 K-elements = 32 B per step inside the 128-byte swizzled rows
+        const uint64_t bd = tc::desc_sw128(b0 + kk * 32, 16, 1024);
+        tc::mma_bf16(tmem, ad, bd, idesc, (kc | kk) != 0);
+      }
+      tc::mma_commit(&empty[s]);
+    }
+    tc::mma_commit(done);
+  }
+  __syncwarp();
+  const bool ok = tc::mbar_wait(done, 0);
+  tc::fence_after_sync();
+  if (ok) {
+    const int row = warp * 32 + lane;
+    const int n = n0 + row;
+    const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) + ((size_t)bg * a.Mg) * a.N;
+    for (int c = 0; c < BN; c += 16) {
+      float v[16];
+      tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+      if (n < a.N) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int m = m0 + c + i;
+          if (m < a.Mg) {
+            const float bv = bias ? __bfloat162float(bias[g * a.Mg + m]) : 0.0f;
+            out[(size_t)m * a.N + n] = __float2bfloat16_rn(v[i] + bv);
+          }
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 2) tc::tmem_dealloc(tmem, ncols);
+}
+
+struct DwTcArgs {
+  float* part;
+  int G, Og, Rg, N, nc, nchunk;
+};
+
+__global__ void __launch_bounds__(128, 1) dw_tc_kernel(const __grid_constant__ CUtensorMap map_y,
+                                                       const __grid_constant__ CUtensorMap map_d, DwTcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const int BN = a.Og;
+  const uint32_t a_bytes = 128 * 128;
+  const uint32_t b_bytes = (uint32_t)BN * 128;
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * a_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * b_bytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* done = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+
+  const int chunk = blockIdx.x;
+  const int r0 = blockIdx.y * 128;
+  const int bg = blockIdx.z;
+  const int g = bg % a.G, b = bg / a.G;
+  const int nb = chunk * a.nc;
+  const int nk = (min(a.N, nb + a.nc) - nb + kBK - 1) / kBK;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ncols = tmem_cols(BN);
+
+  if (threadIdx.x == 0) {
+    tc::prefetch_map(&map_y);
+    tc::prefetch_map(&map_d);
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(done, 1);
+    tc::fence_barrier_init();
+  }
+  if (warp == 2) {
+    tc::tmem_alloc(tmem_slot, ncols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    for (int kc = 0; kc < nk; ++kc) {
+      const int s = kc % kStages;
+      if (kc >= kStages && !tc::mbar_wait(&empty[s], ((kc / kStages) & 1) ^ 1)) break;
+      tc::mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes);
+      tc::tma_load_3d(sA + s * a_bytes, &map_y, &full[s], nb + kc * kBK, r0, bg);
+      tc::tma_load_3d(sB + s * b_bytes, &map_d, &full[s], nb + kc * kBK, 0, bg);
+    }
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t idesc = tc::idesc_bf16(128, BN, false, false);
+    for (int kc = 0; kc < nk; ++kc) {
+      const int s = kc % kStages;
+      if (!tc::mbar_wait(&full[s], (kc / kStages) & 1)) break;
+      tc::fence_after_sync();
+      const uint32_t a0 = tc::smem_u32(sA + s * a_bytes);
+      const uint32_t b0 = tc::smem_u32(sB + s * b_bytes);
+#pragma unroll
+      for (int kk = 0; kk < kBK / 16; ++kk)
+        tc::mma_bf16(tmem, tc::desc_sw128(a0 + kk * 32, 16, 1024), tc::desc_sw128(b0 + kk * 32, 16, 1024), idesc,
+                     (kc | kk) != 0);
+      tc::mma_commit(&empty[s]);
+    }
+    tc::mma_commit(done);
+  }
+  __syncwarp();
+  const bool ok = tc::mbar_wait(done, 0);
+  tc::fence_after_sync();
+  if (ok) {
+    const int r = r0 + warp * 32 + lane;
+    const size_t split = (size_t)b * a.nchunk + chunk;
+    float* P = a.part + ((split * a.G + g) * a.Og) * (size_t)a.Rg;
+    for (int c = 0; c < BN; c += 16) {
+      float v[16];
+      tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+      if (r < a.Rg)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) P[(size_t)(c + i) * a.Rg + r] = nk > 0 ? v[i] : 0.0f;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 2) tc::tmem_dealloc(tmem, ncols);
+}
+
+// bpart[split, g*Og + o] = sum over the split's n of dout[b, g*Og + o, n]; one warp per row,
+// fixed lane striding and shuffle tree.
+__global__ void __launch_bounds__(256) bias_partial_kernel(const __nv_bfloat16* __restrict__ dout,
+                                                           float* __restrict__ bpart, int G, int Og, int N, int nc,
+                                                           int nchunk) {
+  const int chunk = blockIdx.x, bg = blockIdx.y;
+  const int b = bg / G, g = bg % G;
+  const int nb = chunk * nc, ne = min(N, nb + nc);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int o = warp; o < Og; o += blockDim.x >> 5) {
+    const __nv_bfloat16* row = dout + ((size_t)bg * Og + o) * N;
+    float acc = 0.0f;
+    for (int n = nb + lane * 8; n < ne; n += 256) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(row + n));
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc += __uint_as_float(w[i] << 16) + __uint_as_float(w[i] & 0xffff0000u);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) bpart[((size_t)b * nchunk + chunk) * (G * Og) + g * Og + o] = acc;
+  }
+}
+
+// ------------------------------------------------------------------- host
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims innermost first, strides in bytes for dims 1..
+bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+              const cuuint32_t* box) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  cuuint32_t es[3] = {1, 1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t mix_smem(int BN) { return 1024 + kStages * (2 * kHalfTile + (size_t)BN * 128) + (2 * kStages + 2) * 8; }
+size_t dw_smem(int BN) { return 1024 + kStages * (128 * 128 + (size_t)BN * 128) + (2 * kStages + 2) * 8; }
+
+int mix_bn(int Mg) {
+  if (Mg <= 256) return Mg;
+  for (int bn = 256; bn >= 16; bn -= 16)
+    if (Mg % bn == 0) return bn;
+  return 256;
+}
+
+}  // namespace
+
+bool mix_tc_supported(int Mg, int Rg, int N) {
+  return encode_fn() != nullptr && Mg % 16 == 0 && Rg % 8 == 0 && N % 8 == 0 && (mix_bn(Mg) % 16 == 0);
+}
+
+cudaError_t launch_mix_tc(const MixArgs& a, cudaStream_t st) {
+  CUtensorMap mi, mw;
+  const int BN = mix_bn(a.Mg);
+  const cuuint64_t di[3] = {(cuuint64_t)a.N, (cuuint64_t)a.Rg, (cuuint64_t)a.B * a.G};
+  const cuuint64_t si[2] = {(cuuint64_t)a.N * 2, (cuuint64_t)a.Rg * a.N * 2};
+  const cuuint32_t bi[3] = {64, 64, 1};
+  const cuuint64_t dw[2] = {(cuuint64_t)a.Rg, (cuuint64_t)a.G * a.Mg};
+  const cuuint64_t sw[1] = {(cuuint64_t)a.Rg * 2};
+  const cuuint32_t bw[2] = {64, (cuuint32_t)BN};
+  if (!make_map(&mi, a.in, 3, di, si, bi) || !make_map(&mw, a.wm, 2, dw, sw, bw)) return cudaErrorInvalidValue;
+  MixTcArgs t{a.out, a.bias, a.G, a.Mg, a.Rg, a.N, BN};
+  const size_t smem = mix_smem(BN);
+  cudaError_t e = cudaFuncSetAttribute(mix_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.N + 127) / 128, (a.Mg + BN - 1) / BN, a.B * a.G);
+  mix_tc_kernel<<<grid, 128, smem, st>>>(mi, mw, t);
+  count_launch();
+  return cudaGetLastError();
+}
+
+bool dw_tc_supported(int Og, int Rg, int N) {
+  return encode_fn() != nullptr && Og % 16 == 0 && Og <= 256 && N % 8 == 0 && Rg >= 1;
+}
+
+cudaError_t launch_dw_tc(const DwArgs& a, cudaStream_t st) {
+  CUtensorMap my, md;
+  const cuuint64_t dy[3] = {(cuuint64_t)a.N, (cuuint64_t)a.Rg, (cuuint64_t)a.B * a.G};
+  const cuuint64_t sy[2] = {(cuuint64_t)a.N * 2, (cuuint64_t)a.Rg * a.N * 2};
+  const cuuint32_t by[3] = {64, 128, 1};
+  const cuuint64_t dd[3] = {(cuuint64_t)a.N, (cuuint64_t)a.Og, (cuuint64_t)a.B * a.G};
+  const cuuint64_t sd[2] = {(cuuint64_t)a.N * 2, (cuuint64_t)a.Og * a.N * 2};
+  const cuuint32_t bd[3] = {64, (cuuint32_t)a.Og, 1};
+  if (!make_map(&my, a.yv, 3, dy, sy, by) || !make_map(&md, a.dout, 3, dd, sd, bd)) return cudaErrorInvalidValue;
+  DwTcArgs t{a.part, a.G, a.Og, a.Rg, a.N, a.nc, a.nchunk};
+  const size_t smem = dw_smem(a.Og);
+  cudaError_t e = cudaFuncSetAttribute(dw_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.nchunk, (a.Rg + 127) / 128, a.B * a.G);
+  dw_tc_kernel<<<grid, 128, smem, st>>>(my, md, t);
+  count_launch();
+  if (a.bpart) {
+    dim3 g2(a.nchunk, a.B * a.G);
+    bias_partial_kernel<<<g2, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.dout), a.bpart, a.G, a.Og, a.N, a.nc,
+                                            a.nchunk);
+    count_launch();
+  }
+  return cudaGetLastError();
+}
+
+int take_mix_tc_status() {
+  int v = 0, z = 0;
+  cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int));
+  if (v) cudaMemcpyToSymbol(g_device_status, &z, sizeof(int));
+  return v;
+}
+
+}  // namespace disco

@@ -95,6 +95,7 @@ def _load():
         "disco_bwd_weight": [P, I, I, I, I, I, P, P, P, P, P, P, Z, P],
         "disco_bwd_weight_noalloc": [P, I, I, I, I, I, P, P, P, P, P],
         "disco_plan_info": [P, I, IP],
+        "disco_sync_status": [P],
         "disco_plan_export": [P, I, IP, IP, IP, ctypes.POINTER(ctypes.c_float), IP],
     }
     for name, args in sig.items():
@@ -125,6 +126,10 @@ def library():
 def _check(status: int):
     if status != DISCO_OK:
         raise DiscoError(status, _lib.disco_last_error().decode())
+
+
+def disco_sync_status(stream) -> None:
+    _check(_lib.disco_sync_status(stream))
 
 
 def disco_launch_count() -> int:
