@@ -213,7 +213,8 @@ unsigned long long disco_launch_count(void) { return disco::g_launches.load(); }
 disco_status disco_sync_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronisation");
-  if (disco::take_mix_tc_status()) return fail(DISCO_ERR_TIMEOUT, "a bounded device-side wait expired");
+  if (disco::take_mix_tc_status() | disco::take_fused_tc_status())
+    return fail(DISCO_ERR_TIMEOUT, "a bounded device-side wait expired");
   return DISCO_OK;
 }
 
@@ -410,7 +411,25 @@ disco_status disco_fwd_fused(const disco_psi* psi, int B, int C_in, int C_out, i
   const disco::Geometry& g = psi->g;
   if (!disco::gather_supports(g.K, g.stride)) return fail(DISCO_ERR_UNSUPPORTED, "K or stride not compiled");
   const bool bf16 = dtype == DISCO_BF16;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int Cg = C_in / groups;
+  if (bf16) {
+    // tensor-core mix: blocks of exactly 128 outputs
+    const int qb = 128, nblk = (g.nlon_out + qb - 1) / qb;
+    const int need = max_stage(psi->fwd, qb);
+    const int cache = std::min(chunk_cache(psi->fwd), 48);
+    for (int budget : {std::max(need, 12288), std::max(need, 8192), need}) {
+      int pass_ch, a_sbo, w_chunks;
+      size_t smem;
+      if (!disco::fused_tc_plan(C_in, C_out, groups, g.K, cache, budget, &pass_ch, &a_sbo, &w_chunks, &smem)) continue;
+      disco::GatherArgs a = gather_args(psi->dfwd, B * C_in, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out,
+                                        budget, cache, true);
+      cudaError_t e = disco::launch_fused_tc(g.K, g.stride, a, x, w, bias, out, B, C_in, C_out, groups, pass_ch,
+                                             a_sbo, w_chunks, st);
+      if (e != cudaSuccess) return cuda_fail(e, "fused tensor-core launch");
+      return DISCO_OK;
+    }
+  }
   const size_t per_q = (size_t)Cg * g.K * 4;
   int cap = (int)std::min<size_t>(128, kFusedTileBytes / per_q) / disco::kTaskR * disco::kTaskR;
   if (cap < disco::kTaskR) return fail(DISCO_ERR_UNSUPPORTED, "C_in/groups * K too large for the fused tile");
@@ -424,8 +443,7 @@ disco_status disco_fwd_fused(const disco_psi* psi, int B, int C_in, int C_out, i
   if (gather_bytes(cache, g.K, budget, ytile) > kSmemLimit)
     return fail(DISCO_ERR_UNSUPPORTED, "fused tile and staging exceed shared memory");
   disco::FusedArgs f;
-  f.g = gather_args(psi->dfwd, B * C_in, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget,
-                    chunk_cache(psi->fwd), bf16);
+  f.g = gather_args(psi->dfwd, B * C_in, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget, cache, bf16);
   f.x = x;
   f.w = w;
   f.bias = bias;
@@ -436,7 +454,7 @@ disco_status disco_fwd_fused(const disco_psi* psi, int B, int C_in, int C_out, i
   f.G = groups;
   f.K = g.K;
   f.ytile_floats = ytile;
-  cudaError_t e = disco::launch_fused_simt(bf16, g.K, g.stride, f, static_cast<cudaStream_t>(stream));
+  cudaError_t e = disco::launch_fused_simt(bf16, g.K, g.stride, f, st);
   if (e != cudaSuccess) return cuda_fail(e, "fused launch");
   return DISCO_OK;
 }

@@ -47,6 +47,7 @@ bool mix_tc_supported(int Mg, int Rg, int N);
 cudaError_t launch_mix_tc(const MixArgs& a, cudaStream_t st);
 // Device status word of the tensor-core kernels (5 after an expired wait); read and clear.
 int take_mix_tc_status();
+int take_fused_tc_status();
 
 // wt[g, c*K + k, o] = w[g*Og + o, c, k]   (the transposed weight of the dx einsum)
 cudaError_t launch_transpose_weight(bool bf16, const void* w, void* wt, int G, int Og, int Cg, int K, cudaStream_t st);
@@ -81,5 +82,14 @@ struct FusedArgs {
   int ytile_floats;   // Cg*K*qb
 };
 cudaError_t launch_fused_simt(bool bf16, int K, int S, const FusedArgs& a, cudaStream_t st);
+
+// Fused forward with the channel mix on tensor cores (bf16).  fused_tc_plan decides whether the
+// layer fits (Og a multiple of 32 up to 256, C_in/G a multiple of 16, w staged in <= 96 KB) and
+// fills the pass layout and the shared memory size for a gather block of 128 outputs.
+bool fused_tc_plan(int C_in, int C_out, int G, int K, int chunk_cache, int stage_floats, int* pass_ch, int* a_sbo,
+                   int* w_chunks, size_t* smem);
+cudaError_t launch_fused_tc(int K, int S, const GatherArgs& g, const void* x, const void* w, const void* bias,
+                            void* out, int B, int C_in, int C_out, int G, int pass_ch, int a_sbo, int w_chunks,
+                            cudaStream_t st);
 
 }  // namespace disco

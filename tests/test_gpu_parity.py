@@ -32,6 +32,10 @@ EDGE = {
     "ragged_down_bf16": Workload("ragged_down_bf16", 3, 6, 9, 3, 19, 24, 10, 12, (3, 4), 0.7, "bf16", bias=False),
     "wide_row_f32": Workload("wide_row_f32", 2, 5, 4, 1, 33, 264, 33, 132, (5, 1), 0.35, "f32"),
     "aniso_k9_f32": Workload("aniso_k9_f32", 1, 17, 17, 1, 21, 40, 21, 40, (3, 4), 0.5, "f32"),
+    # bf16 layers small enough to debug that still take the tensor-core paths (TMA-aligned rows,
+    # channel counts in multiples of 16/32) with partial 128-wide tiles
+    "tc_small_bf16": Workload("tc_small_bf16", 2, 32, 64, 2, 33, 64, 33, 64, (3, 1), 0.3, "bf16"),
+    "tc_down_bf16": Workload("tc_down_bf16", 1, 16, 32, 1, 33, 128, 17, 64, (3, 4), 0.5, "bf16"),
 }
 
 
