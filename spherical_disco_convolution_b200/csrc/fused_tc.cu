@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_tc_kernel(const __grid_cons
   uint8_t* ytile = reinterpret_cast<uint8_t*>(s.stage + a.stage_budget);
   const size_t y_bytes = (size_t)16 * f.a_sbo;
   uint8_t* wsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ytile + y_bytes) + 1023) & ~uintptr_t(1023));
-  const int Cg = f.C_in / f.G, Og = f.C_out / f.G, R = Cg * K;
+  const int Cg = f.C_in / f.G, Og = f.C_out / f.G;
   uint64_t* bars = reinterpret_cast<uint64_t*>(wsm + (size_t)f.w_chunks * Og * 128);
   uint64_t* w_full = bars;
   uint64_t* mma_done = bars + 1;

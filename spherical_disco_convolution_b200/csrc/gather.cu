@@ -39,7 +39,7 @@ struct YSink {
 };
 
 template <typename T, int K, int S>
-__global__ void __launch_bounds__(kThreads) fwd_gather_kernel(GatherArgs a, const T* __restrict__ x,
+__global__ void __launch_bounds__(kThreads, (K <= 3 ? 3 : (K <= 5 ? 2 : 1))) fwd_gather_kernel(GatherArgs a, const T* __restrict__ x,
                                                               T* __restrict__ y) {
   extern __shared__ __align__(16) float smem[];
   const GatherSmem s = gather_smem(smem, a.chunk_cache, K);
@@ -57,13 +57,9 @@ __global__ void __launch_bounds__(kThreads) fwd_gather_kernel(GatherArgs a, cons
   }
 }
 
-template <int W>
-__device__ __forceinline__ void adj_chunk(float (&acc)[kTaskR], const float* __restrict__ win_ptr,
+template <int W, int NW>
+__device__ __forceinline__ void adj_chunk(float (&acc)[kTaskR], const float (&win)[NW],
                                           const float* __restrict__ v) {
-  constexpr int NW = kTaskR - 1 + W;
-  float win[NW];
-#pragma unroll
-  for (int t = 0; t < NW; ++t) win[t] = win_ptr[t];
 #pragma unroll
   for (int u = 0; u < W; ++u) {
     const float vv = v[u];
@@ -74,7 +70,8 @@ __device__ __forceinline__ void adj_chunk(float (&acc)[kTaskR], const float* __r
 
 template <int S>
 __device__ __forceinline__ void adj_task(float (&acc)[S][kTaskR], const GatherArgs& a, const GatherSmem& s,
-                                         const RowPlan& rp, const float* sb, int ch_begin, int sl, int nsl) {
+                                         const RowPlan& rp, const float* sc, int m0, int ch_begin, int sl, int nsl) {
+  constexpr int NW = kTaskR - 1 + kChunkW;
 #pragma unroll
   for (int rho = 0; rho < S; ++rho) {
 #pragma unroll
@@ -84,23 +81,24 @@ __device__ __forceinline__ void adj_task(float (&acc)[S][kTaskR], const GatherAr
       Chunk cc;
       const float* v;
       chunk_at(a, s, ch_begin, ch, 1, &cc, &v);
-      const float* wp = sb + s.soff[cc.src] + cc.t0;
+      float win[NW];
+      load_window_any<NW>(win, sc + s.soff[cc.src], cc.t0 + m0);
       switch (cc.wk & 0xff) {
-        case 1: adj_chunk<1>(acc[rho], wp, v); break;
-        case 2: adj_chunk<2>(acc[rho], wp, v); break;
-        case 3: adj_chunk<3>(acc[rho], wp, v); break;
-        case 4: adj_chunk<4>(acc[rho], wp, v); break;
-        case 5: adj_chunk<5>(acc[rho], wp, v); break;
-        case 6: adj_chunk<6>(acc[rho], wp, v); break;
-        case 7: adj_chunk<7>(acc[rho], wp, v); break;
-        default: adj_chunk<8>(acc[rho], wp, v); break;
+        case 1: adj_chunk<1>(acc[rho], win, v); break;
+        case 2: adj_chunk<2>(acc[rho], win, v); break;
+        case 3: adj_chunk<3>(acc[rho], win, v); break;
+        case 4: adj_chunk<4>(acc[rho], win, v); break;
+        case 5: adj_chunk<5>(acc[rho], win, v); break;
+        case 6: adj_chunk<6>(acc[rho], win, v); break;
+        case 7: adj_chunk<7>(acc[rho], win, v); break;
+        default: adj_chunk<8>(acc[rho], win, v); break;
       }
     }
   }
 }
 
 template <typename T, int S>
-__global__ void __launch_bounds__(kThreads) adj_gather_kernel(GatherArgs a, const T* __restrict__ dy,
+__global__ void __launch_bounds__(kThreads, 3) adj_gather_kernel(GatherArgs a, const T* __restrict__ dy,
                                                               T* __restrict__ dx) {
   extern __shared__ __align__(16) float smem[];
   const GatherSmem s = gather_smem(smem, a.chunk_cache, 1);
@@ -143,7 +141,7 @@ __global__ void __launch_bounds__(kThreads) adj_gather_kernel(GatherArgs a, cons
       for (int task = threadIdx.x; task < tasks; task += blockDim.x) {
         const int c = task / tpc, m0 = (task - c * tpc) * kTaskR;
         float acc[S][kTaskR];
-        adj_task<S>(acc, a, s, rp, s.stage + (size_t)c * se + m0, ch_begin, 0, 1);
+        adj_task<S>(acc, a, s, rp, s.stage + (size_t)c * se, m0, ch_begin, 0, 1);
         finish(c, m0, acc);
       }
     } else {
@@ -153,7 +151,7 @@ __global__ void __launch_bounds__(kThreads) adj_gather_kernel(GatherArgs a, cons
       float acc[S][kTaskR];
       if (active) {
         const int c = task / tpc, m0 = (task - c * tpc) * kTaskR;
-        adj_task<S>(acc, a, s, rp, s.stage + (size_t)c * se + m0, ch_begin, sl, nsl);
+        adj_task<S>(acc, a, s, rp, s.stage + (size_t)c * se, m0, ch_begin, sl, nsl);
       }
       __syncthreads();  // staging consumed: reuse it for the partial sums
       float* red = s.stage;

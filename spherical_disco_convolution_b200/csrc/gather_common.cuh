@@ -54,7 +54,7 @@ __device__ __forceinline__ int gather_prologue(const GatherArgs& a, const RowPla
     int acc = 0;
     for (int t = rp.src_begin; t < rp.src_end; ++t) {
       s.soff[t - rp.src_begin] = acc;
-      acc += staged_len(a.srcs[t].span, a.qb, step);
+      acc += staged_words(staged_len(a.srcs[t].span, a.qb, step));
     }
     s.soff[rp.src_end - rp.src_begin] = acc;
   }
@@ -91,9 +91,10 @@ __device__ __forceinline__ void bf16x8_to_floats(const uint4& u, float (&f)[8]) 
 }
 
 // Stages every source row of the output row for channel planes c0 .. c0+ncg-1.
-// Staged element t of a source row holds source longitude (base + start + t) mod n_src.
-// With vec_stage, starts are multiples of kAlign (the plan guarantees it) and n_src is a
-// multiple of the 16-byte vector, so whole vectors are moved.
+// Staged element t of a source row holds source longitude (base + start + t) mod n_src and
+// lives at word t + t/8 of the row (see staged_words).  With vec_stage, starts are multiples
+// of kAlign (the plan guarantees it) and n_src is a multiple of the 16-byte vector, so whole
+// vectors are read.
 template <typename T>
 __device__ __forceinline__ void stage_rows(const GatherArgs& a, const RowPlan& rp, const GatherSmem& s, int se,
                                            const T* __restrict__ src, int c0, int ncg, int base, int step) {
@@ -108,20 +109,24 @@ __device__ __forceinline__ void stage_rows(const GatherArgs& a, const RowPlan& r
     if (a.vec_stage) {
       constexpr int V = 16 / sizeof(T);
       const int ng = len / V;
+#pragma unroll 4
       for (int idx = threadIdx.x; idx < ncg * ng; idx += blockDim.x) {
         const int c = idx / ng, g = idx - c * ng;
         int l = first + g * V;
         while (l >= n) l -= n;
         const uint4 u = __ldg(reinterpret_cast<const uint4*>(row0 + (size_t)(c0 + c) * chan + l));
-        float* dst = dst0 + (size_t)c * se + g * V;
+        const int e = g * V;
+        float* dst = dst0 + (size_t)c * se + e + (e >> 3);
         if constexpr (sizeof(T) == 2) {
           float f[8];
           bf16x8_to_floats(u, f);
-          reinterpret_cast<float4*>(dst)[0] = make_float4(f[0], f[1], f[2], f[3]);
-          reinterpret_cast<float4*>(dst)[1] = make_float4(f[4], f[5], f[6], f[7]);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) dst[i] = f[i];
         } else {
-          reinterpret_cast<float4*>(dst)[0] =
-              make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
+          dst[0] = __uint_as_float(u.x);
+          dst[1] = __uint_as_float(u.y);
+          dst[2] = __uint_as_float(u.z);
+          dst[3] = __uint_as_float(u.w);
         }
       }
     } else {
@@ -129,7 +134,7 @@ __device__ __forceinline__ void stage_rows(const GatherArgs& a, const RowPlan& r
         const int c = idx / len, e = idx - c * len;
         int l = first + e;
         while (l >= n) l -= n;
-        dst0[(size_t)c * se + e] = to_f32(row0[(size_t)(c0 + c) * chan + l]);
+        dst0[(size_t)c * se + e + (e >> 3)] = to_f32(row0[(size_t)(c0 + c) * chan + l]);
       }
     }
   }
@@ -168,14 +173,33 @@ __device__ __forceinline__ void ring_sums(const GatherArgs& a, const GatherSmem&
   }
 }
 
-// acc[k][r] += sum_u v[k][u] * win[r*S + u] for the basis functions set in kmask.
-template <int K, int S, int W>
-__device__ __forceinline__ void fwd_chunk(float (&acc)[K][kTaskR], const float* __restrict__ win_ptr,
-                                          const float* __restrict__ v, int kmask) {
-  constexpr int NW = (kTaskR - 1) * S + W;
-  float win[NW];
+// Loads NW staged elements e0 .. e0+NW-1 of a padded row (word e + e/8); p points at the
+// word of e0 and LO = e0 mod 8, so the pad words inside the window sit at compile-time offsets.
+template <int NW, int LO>
+__device__ __forceinline__ void load_window(float (&win)[NW], const float* __restrict__ p) {
 #pragma unroll
-  for (int t = 0; t < NW; ++t) win[t] = win_ptr[t];
+  for (int t = 0; t < NW; ++t) win[t] = p[t + (LO + t) / 8];
+}
+
+template <int NW>
+__device__ __forceinline__ void load_window_any(float (&win)[NW], const float* __restrict__ row, int e0) {
+  const float* p = row + e0 + (e0 >> 3);
+  switch (e0 & 7) {
+    case 0: load_window<NW, 0>(win, p); break;
+    case 1: load_window<NW, 1>(win, p); break;
+    case 2: load_window<NW, 2>(win, p); break;
+    case 3: load_window<NW, 3>(win, p); break;
+    case 4: load_window<NW, 4>(win, p); break;
+    case 5: load_window<NW, 5>(win, p); break;
+    case 6: load_window<NW, 6>(win, p); break;
+    default: load_window<NW, 7>(win, p); break;
+  }
+}
+
+// acc[k][r] += sum_u v[k][u] * win[r*S + u] for the basis functions set in kmask.
+template <int K, int S, int W, int NW>
+__device__ __forceinline__ void fwd_chunk(float (&acc)[K][kTaskR], const float (&win)[NW],
+                                          const float* __restrict__ v, int kmask) {
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     if (kmask & (1 << k)) {
@@ -189,10 +213,12 @@ __device__ __forceinline__ void fwd_chunk(float (&acc)[K][kTaskR], const float* 
   }
 }
 
-// Chunks [c_lo, c_hi) of the row for one task (kTaskR outputs of one channel plane).
+// Chunks [c_lo, c_hi) of the row for one task (kTaskR outputs of one channel plane whose
+// staging starts at `sc`; the task's first output is m0 of the block).
 template <int K, int S>
 __device__ __forceinline__ void fwd_task(float (&acc)[K][kTaskR], const GatherArgs& a, const GatherSmem& s,
-                                         const float* sb, int ch_begin, int c_lo, int c_hi) {
+                                         const float* sc, int m0, int ch_begin, int c_lo, int c_hi) {
+  constexpr int NW = (kTaskR - 1) * S + kChunkW;
 #pragma unroll
   for (int k = 0; k < K; ++k)
 #pragma unroll
@@ -201,17 +227,18 @@ __device__ __forceinline__ void fwd_task(float (&acc)[K][kTaskR], const GatherAr
     Chunk cc;
     const float* v;
     chunk_at(a, s, ch_begin, ch, K, &cc, &v);
-    const float* wp = sb + s.soff[cc.src] + cc.t0;
+    float win[NW];
+    load_window_any<NW>(win, sc + s.soff[cc.src], cc.t0 + m0 * S);
     const int kmask = cc.wk >> 8;
     switch (cc.wk & 0xff) {
-      case 1: fwd_chunk<K, S, 1>(acc, wp, v, kmask); break;
-      case 2: fwd_chunk<K, S, 2>(acc, wp, v, kmask); break;
-      case 3: fwd_chunk<K, S, 3>(acc, wp, v, kmask); break;
-      case 4: fwd_chunk<K, S, 4>(acc, wp, v, kmask); break;
-      case 5: fwd_chunk<K, S, 5>(acc, wp, v, kmask); break;
-      case 6: fwd_chunk<K, S, 6>(acc, wp, v, kmask); break;
-      case 7: fwd_chunk<K, S, 7>(acc, wp, v, kmask); break;
-      default: fwd_chunk<K, S, 8>(acc, wp, v, kmask); break;
+      case 1: fwd_chunk<K, S, 1>(acc, win, v, kmask); break;
+      case 2: fwd_chunk<K, S, 2>(acc, win, v, kmask); break;
+      case 3: fwd_chunk<K, S, 3>(acc, win, v, kmask); break;
+      case 4: fwd_chunk<K, S, 4>(acc, win, v, kmask); break;
+      case 5: fwd_chunk<K, S, 5>(acc, win, v, kmask); break;
+      case 6: fwd_chunk<K, S, 6>(acc, win, v, kmask); break;
+      case 7: fwd_chunk<K, S, 7>(acc, win, v, kmask); break;
+      default: fwd_chunk<K, S, 8>(acc, win, v, kmask); break;
     }
   }
 }
@@ -231,10 +258,10 @@ __device__ __forceinline__ int slice_count(int tasks, int nch, int red_floats_pe
 template <typename T, int K, int S, typename Sink>
 __device__ __forceinline__ void fwd_block(const GatherArgs& a, const RowPlan& rp, const GatherSmem& s, int se,
                                           const T* __restrict__ x, int c0, int ncg, int base, int ch_begin,
-                                          int nch, Sink& sink) {
+                                          int nch, Sink& sink, bool rings_ready = false) {
   const int nring = rp.ring_end - rp.ring_begin;
   stage_rows<T>(a, rp, s, se, x, c0, ncg, base, S);
-  ring_sums<T>(a, s, nring, x, c0, ncg);
+  if (!rings_ready) ring_sums<T>(a, s, nring, x, c0, ncg);
   __syncthreads();
   const int tpc = a.qb / kTaskR;
   const int tasks = ncg * tpc;
@@ -254,7 +281,7 @@ __device__ __forceinline__ void fwd_block(const GatherArgs& a, const RowPlan& rp
     for (int task = threadIdx.x; task < tasks; task += blockDim.x) {
       const int c = task / tpc, m0 = (task - c * tpc) * kTaskR;
       float acc[K][kTaskR];
-      fwd_task<K, S>(acc, a, s, s.stage + (size_t)c * se + m0 * S, ch_begin, 0, nch);
+      fwd_task<K, S>(acc, a, s, s.stage + (size_t)c * se, m0, ch_begin, 0, nch);
       add_rings(acc, c);
       sink(c, m0, acc);
     }
@@ -268,7 +295,7 @@ __device__ __forceinline__ void fwd_block(const GatherArgs& a, const RowPlan& rp
   float acc[K][kTaskR];
   if (active) {
     const int c = task / tpc, m0 = (task - c * tpc) * kTaskR;
-    fwd_task<K, S>(acc, a, s, s.stage + (size_t)c * se + m0 * S, ch_begin, (sl * nch) / nsl, ((sl + 1) * nch) / nsl);
+    fwd_task<K, S>(acc, a, s, s.stage + (size_t)c * se, m0, ch_begin, (sl * nch) / nsl, ((sl + 1) * nch) / nsl);
   }
   __syncthreads();  // staging consumed: reuse it for the partial sums
   float* red = s.stage;

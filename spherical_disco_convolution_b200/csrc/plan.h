@@ -78,4 +78,8 @@ DISCO_HD inline int staged_len(int span, int qb, int step) {
   return (((qb + kTaskR - 1) * step + span + kChunkW) + kAlign - 1) & ~(kAlign - 1);
 }
 
+// Shared-memory words of a staged row: one pad word after every 8 elements, so that the
+// windows of 32 threads 8 outputs apart fall into 32 different banks.
+DISCO_HD inline int staged_words(int len) { return len + (len >> 3); }
+
 }  // namespace disco

@@ -225,7 +225,7 @@ bool constant_ring(const std::vector<double>& vals, int n, double* mean) {
 
 int stage_elems(const GatherPlan& P, const RowPlan& r, int qb) {
   int n = 0;
-  for (int s = r.src_begin; s < r.src_end; ++s) n += staged_len(P.src[s].span, qb, P.step);
+  for (int s = r.src_begin; s < r.src_end; ++s) n += staged_words(staged_len(P.src[s].span, qb, P.step));
   return n;
 }
 
