@@ -355,24 +355,45 @@ disco_status disco_workspace_size(const disco_psi* psi, int op, int B, int C_in,
   return DISCO_OK;
 }
 
+namespace {
+
+// Forward contraction x -> y with the best gather form for the layer.
+disco_status launch_contract(const disco_psi* psi, int BC, disco_dtype dtype, const void* x, void* y,
+                             cudaStream_t st, const char* what) {
+  const disco::Geometry& g = psi->g;
+  int qb, nblk;
+  block_shape(g.nlon_out, 128, &qb, &nblk);
+  const int need = max_stage(psi->fwd, qb);
+  if (g.K == 3) {
+    const int cache = std::min(chunk_cache(psi->fwd), 48);
+    const int budget = std::max(6656, need);
+    if (disco::gather2_bytes(cache, g.K, budget) <= kSmemLimit) {
+      disco::GatherArgs a = gather_args(psi->dfwd, BC, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget,
+                                        cache, dtype == DISCO_BF16);
+      cudaError_t e = disco::launch_fwd_gather2(dtype == DISCO_BF16, g.K, g.stride, a, x, y, st);
+      if (e != cudaSuccess) return cuda_fail(e, what);
+      return DISCO_OK;
+    }
+  }
+  const int budget = std::max(kStageFloats, need);
+  if (gather_bytes(chunk_cache(psi->fwd), g.K, budget) > kSmemLimit)
+    return fail(DISCO_ERR_UNSUPPORTED, "a Psi row needs more staging than shared memory holds");
+  disco::GatherArgs a = gather_args(psi->dfwd, BC, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget,
+                                    chunk_cache(psi->fwd), dtype == DISCO_BF16);
+  cudaError_t e = disco::launch_fwd_gather(dtype == DISCO_BF16, g.K, g.stride, a, x, y, st);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return DISCO_OK;
+}
+
+}  // namespace
+
 disco_status disco_contract(const disco_psi* psi, int B, int C, disco_dtype dtype, const void* x, void* y,
                             void* stream) {
   disco_status s = check_common(psi, B, C, C, 1, dtype);
   if (s) return s;
   if (!x || !y) return fail(DISCO_ERR_INVALID_ARG, "x and y must be non-NULL");
-  const disco::Geometry& g = psi->g;
-  if (!disco::gather_supports(g.K, g.stride)) return fail(DISCO_ERR_UNSUPPORTED, "K or stride not compiled");
-  int qb, nblk;
-  block_shape(g.nlon_out, 128, &qb, &nblk);
-  const int need = max_stage(psi->fwd, qb);
-  const int budget = std::max(kStageFloats, need);
-  if (gather_bytes(chunk_cache(psi->fwd), g.K, budget) > kSmemLimit)
-    return fail(DISCO_ERR_UNSUPPORTED, "a Psi row needs more staging than shared memory holds");
-  disco::GatherArgs a = gather_args(psi->dfwd, B * C, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget,
-                                    chunk_cache(psi->fwd), dtype == DISCO_BF16);
-  cudaError_t e = disco::launch_fwd_gather(dtype == DISCO_BF16, g.K, g.stride, a, x, y, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "contraction launch");
-  return DISCO_OK;
+  if (!disco::gather_supports(psi->g.K, psi->g.stride)) return fail(DISCO_ERR_UNSUPPORTED, "K or stride not compiled");
+  return launch_contract(psi, B * C, dtype, x, y, static_cast<cudaStream_t>(stream), "contraction launch");
 }
 
 disco_status disco_einsum(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
@@ -511,17 +532,8 @@ disco_status disco_bwd_weight(const disco_psi* psi, int B, int C_in, int C_out, 
   cudaError_t e;
   const void* yv = y;
   if (!y) {
-    int qb, nblk;
-    block_shape(g.nlon_out, 128, &qb, &nblk);
-    const int need = max_stage(psi->fwd, qb);
-    const int budget = std::max(kStageFloats, need);
-    if (gather_bytes(chunk_cache(psi->fwd), g.K, budget) > kSmemLimit)
-      return fail(DISCO_ERR_UNSUPPORTED, "a Psi row needs more staging than shared memory holds");
-    disco::GatherArgs a =
-        gather_args(psi->dfwd, B * C_in, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget,
-                    chunk_cache(psi->fwd), bf16);
-    e = disco::launch_fwd_gather(bf16, g.K, g.stride, a, x, ws + L.ybuf, st);
-    if (e != cudaSuccess) return cuda_fail(e, "recompute contraction launch");
+    s = launch_contract(psi, B * C_in, dtype, x, ws + L.ybuf, st, "recompute contraction launch");
+    if (s) return s;
     yv = ws + L.ybuf;
   }
   const int Og = C_out / groups, Rg = (C_in / groups) * g.K;

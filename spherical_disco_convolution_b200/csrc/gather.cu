@@ -16,6 +16,7 @@
 // the chunk.  Full circles of one constant value (rings) enter as value x
 // row sum.  Rows with many chunks and few staged channels split their chunk
 // list over idle threads and combine the partial sums in a fixed order.
+#include "gather2.cuh"
 #include "gather_common.cuh"
 
 namespace disco {
@@ -54,6 +55,49 @@ __global__ void __launch_bounds__(kThreads, (K <= 3 ? 3 : (K <= 5 ? 2 : 1))) fwd
     const int ncg = min(cg, c_end - c0);
     YSink<T, K> sink{y, c0, a.n_out_rows, rp.row, a.n_out, q0};
     fwd_block<T, K, S>(a, rp, s, se, x, c0, ncg, q0 * S, ch_begin, nch, sink);
+  }
+}
+
+template <typename T, int K>
+struct YSink2 {
+  T* y;
+  int c0, ncg, n_out_rows, row, n_out, q0;
+  __device__ __forceinline__ void operator()(int p, int m0, float2 (&acc)[K][kTaskR]) const {
+    if (q0 + m0 >= n_out) return;
+    const int n = min(kTaskR, n_out - (q0 + m0));
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      float va[kTaskR], vb[kTaskR];
+#pragma unroll
+      for (int r = 0; r < kTaskR; ++r) {
+        va[r] = acc[k][r].x;
+        vb[r] = acc[k][r].y;
+      }
+      const size_t off = ((size_t)k * n_out_rows + row) * n_out + q0 + m0;
+      store_run<T, kTaskR>(y + (size_t)(c0 + 2 * p) * K * n_out_rows * n_out + off, va, n);
+      if (2 * p + 1 < ncg) store_run<T, kTaskR>(y + (size_t)(c0 + 2 * p + 1) * K * n_out_rows * n_out + off, vb, n);
+    }
+  }
+};
+
+// Paired form of the forward gather (K <= 5): 128 threads, each owning 8 outputs of two
+// channel planes; the stage budget counts float2 words.
+template <typename T, int K, int S>
+__global__ void __launch_bounds__(128, 3) fwd_gather2_kernel(GatherArgs a, const T* __restrict__ x,
+                                                              T* __restrict__ y) {
+  extern __shared__ __align__(16) float smem[];
+  const Gather2Smem s = gather2_smem(smem, a.chunk_cache, K);
+  const RowPlan rp = a.rows[blockIdx.z];
+  const int q0 = blockIdx.y * a.qb;
+  const int c_begin = blockIdx.x * a.cb;
+  const int c_end = min(a.BC, c_begin + a.cb);
+  const int ch_begin = rp.chunk_start[0], nch = rp.chunk_end[0] - rp.chunk_start[0];
+  const int se = gather2_prologue(a, rp, ch_begin, rp.chunk_end[0], S, K, s);
+  const int cg = max(1, min(min(a.cb, kMaxCb), 2 * (a.stage_budget / max(1, se))));
+  for (int c0 = c_begin; c0 < c_end; c0 += cg) {
+    const int ncg = min(cg, c_end - c0);
+    YSink2<T, K> sink{y, c0, ncg, a.n_out_rows, rp.row, a.n_out, q0};
+    fwd_block2<T, K, S>(a, rp, s, se, x, c0, ncg, q0 * S, ch_begin, nch, sink);
   }
 }
 
@@ -203,6 +247,18 @@ cudaError_t launch_adj_t(const GatherArgs& a, const void* dy, void* dx, cudaStre
   return cudaGetLastError();
 }
 
+template <typename T, int K, int S>
+cudaError_t launch_fwd2_t(const GatherArgs& a, const void* x, void* y, cudaStream_t st) {
+  auto kern = fwd_gather2_kernel<T, K, S>;
+  const size_t smem = gather2_smem_bytes(a.chunk_cache, K, a.stage_budget);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.BC + a.cb - 1) / a.cb, a.nblk, a.n_rows);
+  kern<<<grid, 128, smem, st>>>(a, static_cast<const T*>(x), static_cast<T*>(y));
+  count_launch();
+  return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t launch_fwd_k(int K, int S, const GatherArgs& a, const void* x, void* y, cudaStream_t st) {
 #define DISCO_FWD_CASE(KK)                                           \
@@ -219,6 +275,24 @@ cudaError_t launch_fwd_k(int K, int S, const GatherArgs& a, const void* x, void*
 }
 
 }  // namespace
+
+cudaError_t launch_fwd_gather2(bool bf16, int K, int S, const GatherArgs& a, const void* x, void* y,
+                               cudaStream_t st) {
+#define DISCO_FWD2_CASE(TT, KK)                                      \
+  if (K == KK) {                                                     \
+    if (S == 1) return launch_fwd2_t<TT, KK, 1>(a, x, y, st);        \
+    if (S == 2) return launch_fwd2_t<TT, KK, 2>(a, x, y, st);        \
+  }
+  if (bf16) {
+    DISCO_FWD2_CASE(__nv_bfloat16, 3)
+  } else {
+    DISCO_FWD2_CASE(float, 3)
+  }
+#undef DISCO_FWD2_CASE
+  return cudaErrorNotSupported;
+}
+
+size_t gather2_bytes(int chunk_cache, int nk, int stage_f2) { return gather2_smem_bytes(chunk_cache, nk, stage_f2); }
 
 bool gather_supports(int K, int stride) {
   return (K == 3 || K == 5 || K == 7 || K == 9) && (stride == 1 || stride == 2);

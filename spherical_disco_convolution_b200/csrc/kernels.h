@@ -30,6 +30,10 @@ struct GatherArgs {
 bool gather_supports(int K, int stride);
 cudaError_t launch_fwd_gather(bool bf16, int K, int S, const GatherArgs& a, const void* x, void* y, cudaStream_t st);
 cudaError_t launch_adj_gather(bool bf16, int S, const GatherArgs& a, const void* dy, void* dx, cudaStream_t st);
+// Paired-plane forward gather (packed fp32 FMAs) for K = 3; stage_budget in float2 words.
+cudaError_t launch_fwd_gather2(bool bf16, int K, int S, const GatherArgs& a, const void* x, void* y,
+                               cudaStream_t st);
+size_t gather2_bytes(int chunk_cache, int nk, int stage_f2);
 
 // Grouped channel mix (SIMT):
 //   out[b, g*Mg + m, n] = bias[g*Mg + m] + sum_{r < Rg} wm[g, m, r] * in[b, g*Rg + r, n]

@@ -73,9 +73,11 @@ struct RowPlan {
   float cost;                   // relative work, used to order heavy rows first
 };
 
-// Staged elements of one source row for a block of qb outputs (a multiple of kAlign).
+// Staged elements of one source row for a block of qb outputs (a multiple of kAlign).  A task's
+// window starts at t0 + m0*step (t0 <= span - 1, m0 <= qb - kTaskR) and holds
+// (kTaskR - 1)*step + kChunkW elements, so the last element read is span + (qb - 1)*step + 6.
 DISCO_HD inline int staged_len(int span, int qb, int step) {
-  return (((qb + kTaskR - 1) * step + span + kChunkW) + kAlign - 1) & ~(kAlign - 1);
+  return ((qb - 1) * step + span + kChunkW - 1 + kAlign - 1) & ~(kAlign - 1);
 }
 
 // Shared-memory words of a staged row: one pad word after every 8 elements, so that the
