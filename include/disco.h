@@ -189,7 +189,9 @@ disco_status disco_bwd_weight_noalloc(const disco_psi* psi, int B, int C_in, int
 
 /* Diagnostics: the host copy of a gather plan, for inspection by tests.
  * which = 0 is the forward contraction plan (output rows j), which = 1 the
- * adjoint plan used by disco_bwd_input (output rows i).  disco_plan_info fills
+ * adjoint plan used by disco_bwd_input (output rows i), which = 2 and 3 the
+ * banded forms of those two (consecutive light rows sharing their staged
+ * source rows; each row record carries its band's source range).  disco_plan_info fills
  * dims[9] = {rows, source rows, chunks, values, value sets per chunk, source
  * step per output, residue classes, ints per row record, ring terms}.
  * disco_plan_export copies the records into caller-owned HOST arrays sized

@@ -42,7 +42,9 @@ struct DevPlan {
   disco::Chunk* chunks = nullptr;
   float* vals = nullptr;
   disco::Ring* rings = nullptr;
+  disco::BandPlan* bands = nullptr;
   int n_rows = 0;
+  int n_bands = 0;
 };
 
 template <typename T>
@@ -56,7 +58,9 @@ cudaError_t upload(const std::vector<T>& v, T** dst) {
 
 cudaError_t upload_plan(const disco::GatherPlan& P, DevPlan* d) {
   d->n_rows = (int)P.rows.size();
+  d->n_bands = (int)P.bands.size();
   cudaError_t e;
+  if ((e = upload(P.bands, &d->bands)) != cudaSuccess) return e;
   if ((e = upload(P.rows, &d->rows)) != cudaSuccess) return e;
   if ((e = upload(P.src, &d->srcs)) != cudaSuccess) return e;
   if ((e = upload(P.chunks, &d->chunks)) != cudaSuccess) return e;
@@ -70,6 +74,7 @@ void free_plan(DevPlan* d) {
   cudaFree(d->chunks);
   cudaFree(d->vals);
   cudaFree(d->rings);
+  cudaFree(d->bands);
   *d = DevPlan{};
 }
 
@@ -85,9 +90,11 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 struct disco_psi {
   disco::Geometry g;
   int device = -1;
+  cudaStream_t side = nullptr;        // heavy-row launches run here, forked from the caller's stream
+  cudaEvent_t fork = nullptr, join = nullptr;
   std::vector<disco::PsiEntry> entries;
-  disco::GatherPlan fwd, adj;
-  DevPlan dfwd, dadj;
+  disco::GatherPlan fwd, adj, fwdb, adjb;
+  DevPlan dfwd, dadj, dfwdb, dadjb;
 };
 
 namespace {
@@ -107,6 +114,13 @@ int max_stage(const disco::GatherPlan& P, int qb) {
 }
 
 constexpr int kChunkCacheMax = 96;
+constexpr int kLightStage = 6656;  // float2 words of staging per CTA for the light bands
+
+int max_stage_bands(const disco::GatherPlan& P, int b0, int b1, int qb) {
+  int m = 1;
+  for (int b = b0; b < b1; ++b) m = std::max(m, disco::stage_elems(P, P.rows[P.bands[b].rp_begin], qb));
+  return m;
+}
 
 // Dynamic shared memory of a gather CTA (layout in gather_common.cuh) plus `extra` floats.
 size_t gather_bytes(int cache, int nk, int stage_floats, size_t extra = 0) {
@@ -130,6 +144,9 @@ disco::GatherArgs gather_args(const DevPlan& d, int BC, int qb, int nblk, int n_
   a.chunks = d.chunks;
   a.vals = d.vals;
   a.rings = d.rings;
+  a.bands = d.bands;
+  a.n_bands = d.n_bands;
+  a.band0 = 0;
   a.n_rows = d.n_rows;
   a.BC = BC;
   a.cb = kChannelsPerCta;
@@ -204,6 +221,76 @@ WsLayout layout(const disco_psi* psi, int op, int B, int C_in, int C_out, int gr
 
 }  // namespace
 
+namespace {
+
+// Runs a banded gather as two launches so that the few bands with long staged rows do not set
+// the shared-memory size (and so the occupancy) of all the others: heavy bands run on the
+// plan's side stream, forked from and joined back to the caller's stream; light bands run on
+// the caller's stream with a small staging area.
+template <typename Launch>
+disco_status run_banded(const disco_psi* psi, const disco::GatherPlan& P, disco::GatherArgs a, int nk,
+                        cudaStream_t st, Launch launch, const char* what) {
+  const int nb = (int)P.bands.size(), nh = P.n_heavy;
+  if (nh > 0) {
+    disco::GatherArgs h = a;
+    h.band0 = 0;
+    h.n_bands = nh;
+    h.stage_budget = max_stage_bands(P, 0, nh, a.qb);
+    if (disco::gather2_bytes(a.chunk_cache, nk, h.stage_budget) > kSmemLimit)
+      return fail(DISCO_ERR_UNSUPPORTED, "a Psi row needs more staging than shared memory holds");
+    cudaError_t e = cudaEventRecord(psi->fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(psi->side, psi->fork, 0);
+    if (e == cudaSuccess) e = launch(h, psi->side);
+    if (e == cudaSuccess) e = cudaEventRecord(psi->join, psi->side);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+  }
+  if (nb > nh) {
+    disco::GatherArgs l = a;
+    l.band0 = nh;
+    l.n_bands = nb - nh;
+    // a staging area larger than the longest light row lets a CTA stage more channel
+    // pairs per round, so fewer rounds (and barriers) per block of outputs
+    l.stage_budget = std::max(kLightStage, max_stage_bands(P, nh, nb, a.qb));
+    cudaError_t e = launch(l, st);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+  }
+  if (nh > 0) {
+    cudaError_t e = cudaStreamWaitEvent(st, psi->join, 0);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+  }
+  return DISCO_OK;
+}
+
+// Forward contraction x -> y with the best gather form for the layer.
+disco_status launch_contract(const disco_psi* psi, int BC, disco_dtype dtype, const void* x, void* y,
+                             cudaStream_t st, const char* what) {
+  const disco::Geometry& g = psi->g;
+  int qb, nblk;
+  block_shape(g.nlon_out, 128, &qb, &nblk);
+  const int need = max_stage(psi->fwd, qb);
+  if (g.K == 3) {
+    // banded paired gather: a band's chunks are cached together
+    const bool bf16 = dtype == DISCO_BF16;
+    disco::GatherArgs a = gather_args(psi->dfwdb, BC, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, 0, 64,
+                                      bf16);
+    return run_banded(psi, psi->fwdb, a, g.K, st,
+                      [&](const disco::GatherArgs& la, cudaStream_t ls) {
+                        return disco::launch_fwd_gather2_band(bf16, g.K, g.stride, la, x, y, ls);
+                      },
+                      what);
+  }
+  const int budget = std::max(kStageFloats, need);
+  if (gather_bytes(chunk_cache(psi->fwd), g.K, budget) > kSmemLimit)
+    return fail(DISCO_ERR_UNSUPPORTED, "a Psi row needs more staging than shared memory holds");
+  disco::GatherArgs a = gather_args(psi->dfwd, BC, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget,
+                                    chunk_cache(psi->fwd), dtype == DISCO_BF16);
+  cudaError_t e = disco::launch_fwd_gather(dtype == DISCO_BF16, g.K, g.stride, a, x, y, st);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return DISCO_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* disco_last_error(void) { return g_last_error.c_str(); }
@@ -258,8 +345,12 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
   }
   h->fwd = disco::make_forward_plan(g, h->entries);
   h->adj = disco::make_adjoint_plan(g, h->entries);
+  h->fwdb = disco::make_band_plan(g.nlat_out, h->fwd, 4, 24);
+  h->adjb = disco::make_band_plan(g.nlat_in, h->adj, 4, 48);
+  disco::split_bands(h->fwdb, 128, kLightStage);
+  disco::split_bands(h->adjb, 128, kLightStage);
   if (h->fwd.max_src > disco::kMaxSrc || h->adj.max_src > disco::kMaxSrc || h->fwd.max_ring > disco::kMaxRing ||
-      h->adj.max_ring > disco::kMaxRing) {
+      h->adj.max_ring > disco::kMaxRing || h->fwdb.max_src > disco::kMaxSrc || h->adjb.max_src > disco::kMaxSrc) {
     delete h;
     return fail(DISCO_ERR_UNSUPPORTED, "an output row reaches more source rows than the kernels support");
   }
@@ -270,10 +361,17 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
     cudaError_t e = cudaSetDevice(device);
     if (e == cudaSuccess) e = upload_plan(h->fwd, &h->dfwd);
     if (e == cudaSuccess) e = upload_plan(h->adj, &h->dadj);
+    if (e == cudaSuccess) e = upload_plan(h->fwdb, &h->dfwdb);
+    if (e == cudaSuccess) e = upload_plan(h->adjb, &h->dadjb);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->join, cudaEventDisableTiming);
     if (prev >= 0) cudaSetDevice(prev);
     if (e != cudaSuccess) {
       free_plan(&h->dfwd);
       free_plan(&h->dadj);
+      free_plan(&h->dfwdb);
+      free_plan(&h->dadjb);
       delete h;
       return fail(DISCO_ERR_ALLOC, std::string("Psi upload failed: ") + cudaGetErrorString(e));
     }
@@ -291,6 +389,11 @@ disco_status disco_psi_destroy(disco_psi* psi) {
     cudaDeviceSynchronize();
     free_plan(&psi->dfwd);
     free_plan(&psi->dadj);
+    free_plan(&psi->dfwdb);
+    free_plan(&psi->dadjb);
+    if (psi->side) cudaStreamDestroy(psi->side);
+    if (psi->fork) cudaEventDestroy(psi->fork);
+    if (psi->join) cudaEventDestroy(psi->join);
     if (prev >= 0) cudaSetDevice(prev);
   }
   delete psi;
@@ -318,8 +421,8 @@ disco_status disco_psi_export(const disco_psi* psi, int* k, int* j, int* i, int*
 }
 
 disco_status disco_plan_info(const disco_psi* psi, int which, int* dims) {
-  if (!psi || !dims || (which != 0 && which != 1)) return fail(DISCO_ERR_INVALID_ARG, "bad plan query");
-  const disco::GatherPlan& P = which == 0 ? psi->fwd : psi->adj;
+  if (!psi || !dims || which < 0 || which > 3) return fail(DISCO_ERR_INVALID_ARG, "bad plan query");
+  const disco::GatherPlan& P = which == 0 ? psi->fwd : which == 1 ? psi->adj : which == 2 ? psi->fwdb : psi->adjb;
   dims[0] = (int)P.rows.size();
   dims[1] = (int)P.src.size();
   dims[2] = (int)P.chunks.size();
@@ -334,9 +437,9 @@ disco_status disco_plan_info(const disco_psi* psi, int which, int* dims) {
 
 disco_status disco_plan_export(const disco_psi* psi, int which, int* rows, int* srcs, int* chunks, float* vals,
                                int* rings) {
-  if (!psi || !rows || !srcs || !chunks || !vals || !rings || (which != 0 && which != 1))
+  if (!psi || !rows || !srcs || !chunks || !vals || !rings || which < 0 || which > 3)
     return fail(DISCO_ERR_INVALID_ARG, "bad plan export");
-  const disco::GatherPlan& P = which == 0 ? psi->fwd : psi->adj;
+  const disco::GatherPlan& P = which == 0 ? psi->fwd : which == 1 ? psi->adj : which == 2 ? psi->fwdb : psi->adjb;
   std::memcpy(rings, P.rings.data(), P.rings.size() * sizeof(disco::Ring));
   std::memcpy(rows, P.rows.data(), P.rows.size() * sizeof(disco::RowPlan));
   std::memcpy(srcs, P.src.data(), P.src.size() * sizeof(disco::SrcRow));
@@ -355,37 +458,6 @@ disco_status disco_workspace_size(const disco_psi* psi, int op, int B, int C_in,
   return DISCO_OK;
 }
 
-namespace {
-
-// Forward contraction x -> y with the best gather form for the layer.
-disco_status launch_contract(const disco_psi* psi, int BC, disco_dtype dtype, const void* x, void* y,
-                             cudaStream_t st, const char* what) {
-  const disco::Geometry& g = psi->g;
-  int qb, nblk;
-  block_shape(g.nlon_out, 128, &qb, &nblk);
-  const int need = max_stage(psi->fwd, qb);
-  if (g.K == 3) {
-    const int cache = std::min(chunk_cache(psi->fwd), 48);
-    const int budget = std::max(6656, need);
-    if (disco::gather2_bytes(cache, g.K, budget) <= kSmemLimit) {
-      disco::GatherArgs a = gather_args(psi->dfwd, BC, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget,
-                                        cache, dtype == DISCO_BF16);
-      cudaError_t e = disco::launch_fwd_gather2(dtype == DISCO_BF16, g.K, g.stride, a, x, y, st);
-      if (e != cudaSuccess) return cuda_fail(e, what);
-      return DISCO_OK;
-    }
-  }
-  const int budget = std::max(kStageFloats, need);
-  if (gather_bytes(chunk_cache(psi->fwd), g.K, budget) > kSmemLimit)
-    return fail(DISCO_ERR_UNSUPPORTED, "a Psi row needs more staging than shared memory holds");
-  disco::GatherArgs a = gather_args(psi->dfwd, BC, qb, nblk, g.nlon_in, g.nlat_in, g.nlon_out, g.nlat_out, budget,
-                                    chunk_cache(psi->fwd), dtype == DISCO_BF16);
-  cudaError_t e = disco::launch_fwd_gather(dtype == DISCO_BF16, g.K, g.stride, a, x, y, st);
-  if (e != cudaSuccess) return cuda_fail(e, what);
-  return DISCO_OK;
-}
-
-}  // namespace
 
 disco_status disco_contract(const disco_psi* psi, int B, int C, disco_dtype dtype, const void* x, void* y,
                             void* stream) {
@@ -503,6 +575,17 @@ disco_status disco_bwd_input(const disco_psi* psi, int B, int C_in, int C_out, i
   if (e != cudaSuccess) return cuda_fail(e, "transposed einsum launch");
   int qb, nblk;
   block_shape(g.nlon_out, 128, &qb, &nblk);
+  if (g.K == 3) {
+    // paired, banded adjoint gather (few basis functions: the staged dy rows of a band
+    // fit with room for several channel pairs)
+    disco::GatherArgs a = gather_args(psi->dadjb, B * C_in, qb, nblk, g.nlon_out, g.K * g.nlat_out, g.nlon_in,
+                                      g.nlat_in, 0, 96, bf16);
+    return run_banded(psi, psi->adjb, a, 1, st,
+                      [&](const disco::GatherArgs& la, cudaStream_t ls) {
+                        return disco::launch_adj_gather2_band(bf16, g.stride, la, dy, dx, ls);
+                      },
+                      "adjoint contraction launch");
+  }
   const int need = max_stage(psi->adj, qb);
   const int budget = std::max(kStageFloats, need);
   if (gather_bytes(chunk_cache(psi->adj), 1, budget) > kSmemLimit)

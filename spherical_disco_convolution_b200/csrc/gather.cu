@@ -101,6 +101,53 @@ __global__ void __launch_bounds__(128, 3) fwd_gather2_kernel(GatherArgs a, const
   }
 }
 
+// Banded paired forward gather: the rows of a band share their staged source rows.
+template <typename T, int K, int S>
+__global__ void __launch_bounds__(128, 3) fwd_gather2_band_kernel(GatherArgs a, const T* __restrict__ x,
+                                                                   T* __restrict__ y) {
+  extern __shared__ __align__(16) float smem[];
+  __shared__ int brow[8][3];  // row, first chunk, end chunk (band-relative) of each member row
+  const Gather2Smem s = gather2_smem(smem, a.chunk_cache, K);
+  const BandPlan bp = a.bands[a.band0 + blockIdx.z];
+  const int nr = bp.rp_end - bp.rp_begin;
+  const RowPlan r0 = a.rows[bp.rp_begin];
+  const int ch_begin = r0.chunk_start[0];
+  const int ch_end = a.rows[bp.rp_end - 1].chunk_end[0];
+  if (threadIdx.x < nr) {
+    const RowPlan& rr = a.rows[bp.rp_begin + threadIdx.x];
+    brow[threadIdx.x][0] = rr.row;
+    brow[threadIdx.x][1] = rr.chunk_start[0] - ch_begin;
+    brow[threadIdx.x][2] = rr.chunk_end[0] - ch_begin;
+  }
+  const int q0 = blockIdx.y * a.qb;
+  const int c_begin = blockIdx.x * a.cb;
+  const int c_end = min(a.BC, c_begin + a.cb);
+  const int se = gather2_prologue(a, r0, ch_begin, ch_end, S, K, s);
+  const int cg = max(1, min(min(a.cb, kMaxCb), 2 * (a.stage_budget / max(1, se))));
+  const int tpc = a.qb / kTaskR;
+  for (int c0 = c_begin; c0 < c_end; c0 += cg) {
+    const int ncg = min(cg, c_end - c0);
+    if (nr == 1) {
+      YSink2<T, K> sink{y, c0, ncg, a.n_out_rows, r0.row, a.n_out, q0};
+      fwd_block2<T, K, S>(a, r0, s, se, x, c0, ncg, q0 * S, ch_begin, ch_end - ch_begin, sink);
+      continue;
+    }
+    stage_rows2<T>(a, r0, s, se, x, c0, ncg, q0 * S, S);
+    __syncthreads();
+    const int npair = (ncg + 1) >> 1;
+    const int per_row = npair * tpc;
+    for (int t = threadIdx.x; t < nr * per_row; t += blockDim.x) {
+      const int r = t / per_row, rem = t - r * per_row;
+      const int p = rem / tpc, m0 = (rem - p * tpc) * kTaskR;
+      float2 acc[K][kTaskR];
+      fwd_task2<K, S>(acc, a, s, s.stage + (size_t)p * se, m0, ch_begin, brow[r][1], brow[r][2]);
+      YSink2<T, K> sink{y, c0, ncg, a.n_out_rows, brow[r][0], a.n_out, q0};
+      sink(p, m0, acc);
+    }
+    __syncthreads();
+  }
+}
+
 template <int W, int NW>
 __device__ __forceinline__ void adj_chunk(float (&acc)[kTaskR], const float (&win)[NW],
                                           const float* __restrict__ v) {
@@ -223,6 +270,199 @@ __global__ void __launch_bounds__(kThreads, 3) adj_gather_kernel(GatherArgs a, c
   }
 }
 
+// ---- paired, banded adjoint gather (dx) ----
+
+template <int W, int NW, typename Vals>
+__device__ __forceinline__ void adj_chunk2(float2 (&acc)[kTaskR], const float2 (&win)[NW], const Vals& v) {
+#pragma unroll
+  for (int u = 0; u < W; ++u) {
+    const float2 vv = v(u);
+#pragma unroll
+    for (int r = 0; r < kTaskR; ++r) acc[r] = __ffma2_rn(vv, win[r + u], acc[r]);
+  }
+}
+
+template <typename Vals>
+__device__ __forceinline__ void adj_apply2(float2 (&acc)[kTaskR], const float2* sc, const Gather2Smem& s,
+                                           const Chunk& cc, int m0, const Vals& v) {
+  constexpr int NW = kTaskR - 1 + kChunkW;
+  float2 win[NW];
+  load_window2_any<NW>(win, sc + s.soff[cc.src], cc.t0 + m0);
+  switch (cc.wk & 0xff) {
+    case 1: adj_chunk2<1>(acc, win, v); break;
+    case 2: adj_chunk2<2>(acc, win, v); break;
+    case 3: adj_chunk2<3>(acc, win, v); break;
+    case 4: adj_chunk2<4>(acc, win, v); break;
+    case 5: adj_chunk2<5>(acc, win, v); break;
+    case 6: adj_chunk2<6>(acc, win, v); break;
+    case 7: adj_chunk2<7>(acc, win, v); break;
+    default: adj_chunk2<8>(acc, win, v); break;
+  }
+}
+
+// Chunk ranges are relative to the band's first chunk; lo/hi per residue class.
+template <int S>
+__device__ __forceinline__ void adj_task2(float2 (&acc)[S][kTaskR], const GatherArgs& a, const Gather2Smem& s,
+                                          const float2* sc, int m0, int ch_begin, const int* lo, const int* hi,
+                                          int sl, int nsl) {
+#pragma unroll
+  for (int rho = 0; rho < S; ++rho) {
+#pragma unroll
+    for (int r = 0; r < kTaskR; ++r) acc[rho][r] = make_float2(0.0f, 0.0f);
+    const int n = hi[rho] - lo[rho];
+    const int ca = lo[rho] + (sl * n) / nsl, cb = lo[rho] + ((sl + 1) * n) / nsl;
+    const int cm = max(ca, min(cb, a.chunk_cache));
+    for (int ch = ca; ch < cm; ++ch) adj_apply2(acc[rho], sc, s, s.cch[ch], m0, CachedValues{s.cval + (size_t)ch * kChunkW});
+    for (int ch = cm; ch < cb; ++ch) {
+      const Chunk cc = a.chunks[ch_begin + ch];
+      adj_apply2(acc[rho], sc, s, cc, m0, GlobalValues{a.vals + cc.voff});
+    }
+  }
+}
+
+template <typename T, int S>
+__global__ void __launch_bounds__(128, 4) adj_gather2_band_kernel(GatherArgs a, const T* __restrict__ dy,
+                                                                   T* __restrict__ dx) {
+  extern __shared__ __align__(16) float smem[];
+  __shared__ int brow[8][1 + 2 * kMaxStride];  // row, then [lo, hi) of each residue class
+  const Gather2Smem s = gather2_smem(smem, a.chunk_cache, 1);
+  const BandPlan bp = a.bands[a.band0 + blockIdx.z];
+  const int nr = bp.rp_end - bp.rp_begin;
+  const RowPlan r0 = a.rows[bp.rp_begin];
+  const int ch_begin = r0.chunk_start[0];
+  const int ch_end = a.rows[bp.rp_end - 1].chunk_end[S - 1];
+  if (threadIdx.x < nr) {
+    const RowPlan& rr = a.rows[bp.rp_begin + threadIdx.x];
+    brow[threadIdx.x][0] = rr.row;
+    for (int rho = 0; rho < S; ++rho) {
+      brow[threadIdx.x][1 + 2 * rho] = rr.chunk_start[rho] - ch_begin;
+      brow[threadIdx.x][2 + 2 * rho] = rr.chunk_end[rho] - ch_begin;
+    }
+  }
+  const int m_blk = blockIdx.y * a.qb;
+  const int c_begin = blockIdx.x * a.cb;
+  const int c_end = min(a.BC, c_begin + a.cb);
+  const int se = gather2_prologue(a, r0, ch_begin, ch_end, 1, 1, s);
+  const int cg = max(1, min(min(a.cb, kMaxCb), 2 * (a.stage_budget / max(1, se))));
+  const int tpc = a.qb / kTaskR;
+  const int n_m = a.n_out / S;  // outputs l = S*m + rho, m < n_m
+  const int nring = nr == 1 ? r0.ring_end - r0.ring_begin : 0;
+  GatherSmem s1;
+  s1.soff = s.soff;
+  s1.rings = s.rings;
+  s1.rsum = s.rsum;
+  for (int c0 = c_begin; c0 < c_end; c0 += cg) {
+    const int ncg = min(cg, c_end - c0);
+    stage_rows2<T>(a, r0, s, se, dy, c0, ncg, m_blk, 1);
+    if (nring) ring_sums<T>(a, s1, nring, dy, c0, ncg);
+    __syncthreads();
+    const int npair = (ncg + 1) >> 1;
+    const int per_row = npair * tpc;
+    const int tasks = nr * per_row;
+    const int nsl = nr == 1 ? slice_count(tasks, ch_end - ch_begin, 2 * S * kTaskR, 2 * a.stage_budget) : 1;
+    auto finish = [&](int r, int p, int m0, float2 (&acc)[S][kTaskR]) {
+      if (m_blk + m0 >= n_m) return;
+      float ra = 0.0f, rb = 0.0f;
+      for (int t = 0; t < nring; ++t) {
+        ra += s.rings[t].v * s.rsum[(2 * p) * nring + t];
+        if (2 * p + 1 < ncg) rb += s.rings[t].v * s.rsum[(2 * p + 1) * nring + t];
+      }
+      const int nm = min(kTaskR, n_m - (m_blk + m0));
+      const size_t off = (size_t)brow[r][0] * a.n_out + (size_t)S * (m_blk + m0);
+      T* da = dx + (size_t)(c0 + 2 * p) * a.n_out_rows * a.n_out + off;
+      T* db = dx + (size_t)(c0 + 2 * p + 1) * a.n_out_rows * a.n_out + off;
+      const bool has_b = 2 * p + 1 < ncg;
+      if constexpr (S == 1) {
+        float va[kTaskR], vb[kTaskR];
+#pragma unroll
+        for (int q = 0; q < kTaskR; ++q) {
+          va[q] = acc[0][q].x + ra;
+          vb[q] = acc[0][q].y + rb;
+        }
+        store_run<T, kTaskR>(da, va, nm);
+        if (has_b) store_run<T, kTaskR>(db, vb, nm);
+      } else {
+#pragma unroll
+        for (int q = 0; q < kTaskR; ++q)
+#pragma unroll
+          for (int rho = 0; rho < S; ++rho)
+            if (q < nm) {
+              da[q * S + rho] = from_f32<T>(acc[rho][q].x + ra);
+              if (has_b) db[q * S + rho] = from_f32<T>(acc[rho][q].y + rb);
+            }
+      }
+    };
+    if (nsl == 1) {
+      for (int t = threadIdx.x; t < tasks; t += blockDim.x) {
+        const int r = t / per_row, rem = t - r * per_row;
+        const int p = rem / tpc, m0 = (rem - p * tpc) * kTaskR;
+        float2 acc[S][kTaskR];
+        int lo[S], hi[S];
+#pragma unroll
+        for (int rho = 0; rho < S; ++rho) {
+          lo[rho] = brow[r][1 + 2 * rho];
+          hi[rho] = brow[r][2 + 2 * rho];
+        }
+        adj_task2<S>(acc, a, s, s.stage + (size_t)p * se, m0, ch_begin, lo, hi, 0, 1);
+        finish(r, p, m0, acc);
+      }
+    } else {
+      const int tg = threadIdx.x;
+      const bool active = tg < nsl * tasks;
+      const int sl = tg / tasks, task = tg - sl * tasks;
+      const int p = task / tpc, m0 = (task - p * tpc) * kTaskR;
+      float2 acc[S][kTaskR];
+      if (active) {
+        int lo[S], hi[S];
+#pragma unroll
+        for (int rho = 0; rho < S; ++rho) {
+          lo[rho] = brow[0][1 + 2 * rho];
+          hi[rho] = brow[0][2 + 2 * rho];
+        }
+        adj_task2<S>(acc, a, s, s.stage + (size_t)p * se, m0, ch_begin, lo, hi, sl, nsl);
+      }
+      __syncthreads();  // staging consumed: reuse it for the partial sums
+      float2* red = s.stage;
+      if (active)
+#pragma unroll
+        for (int rho = 0; rho < S; ++rho)
+#pragma unroll
+          for (int q = 0; q < kTaskR; ++q) red[((size_t)(sl * tasks + task) * S + rho) * kTaskR + q] = acc[rho][q];
+      __syncthreads();
+      for (int t = threadIdx.x; t < tasks; t += blockDim.x) {
+        const int pp = t / tpc, mm = (t - pp * tpc) * kTaskR;
+        float2 sum[S][kTaskR];
+#pragma unroll
+        for (int rho = 0; rho < S; ++rho)
+#pragma unroll
+          for (int q = 0; q < kTaskR; ++q) {
+            float2 v = make_float2(0.0f, 0.0f);
+            for (int z = 0; z < nsl; ++z) {
+              const float2 w = red[((size_t)(z * tasks + t) * S + rho) * kTaskR + q];
+              v.x += w.x;
+              v.y += w.y;
+            }
+            sum[rho][q] = v;
+          }
+        finish(0, pp, mm, sum);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+template <typename T, int S>
+cudaError_t launch_adj2b_t(const GatherArgs& a, const void* dy, void* dx, cudaStream_t st) {
+  auto kern = adj_gather2_band_kernel<T, S>;
+  const size_t smem = gather2_smem_bytes(a.chunk_cache, 1, a.stage_budget);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.BC + a.cb - 1) / a.cb, a.nblk, a.n_bands);
+  kern<<<grid, 128, smem, st>>>(a, static_cast<const T*>(dy), static_cast<T*>(dx));
+  count_launch();
+  return cudaGetLastError();
+}
+
 template <typename T, int K, int S>
 cudaError_t launch_fwd_t(const GatherArgs& a, const void* x, void* y, cudaStream_t st) {
   auto kern = fwd_gather_kernel<T, K, S>;
@@ -259,6 +499,18 @@ cudaError_t launch_fwd2_t(const GatherArgs& a, const void* x, void* y, cudaStrea
   return cudaGetLastError();
 }
 
+template <typename T, int K, int S>
+cudaError_t launch_fwd2b_t(const GatherArgs& a, const void* x, void* y, cudaStream_t st) {
+  auto kern = fwd_gather2_band_kernel<T, K, S>;
+  const size_t smem = gather2_smem_bytes(a.chunk_cache, K, a.stage_budget);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.BC + a.cb - 1) / a.cb, a.nblk, a.n_bands);
+  kern<<<grid, 128, smem, st>>>(a, static_cast<const T*>(x), static_cast<T*>(y));
+  count_launch();
+  return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t launch_fwd_k(int K, int S, const GatherArgs& a, const void* x, void* y, cudaStream_t st) {
 #define DISCO_FWD_CASE(KK)                                           \
@@ -289,6 +541,31 @@ cudaError_t launch_fwd_gather2(bool bf16, int K, int S, const GatherArgs& a, con
     DISCO_FWD2_CASE(float, 3)
   }
 #undef DISCO_FWD2_CASE
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_fwd_gather2_band(bool bf16, int K, int S, const GatherArgs& a, const void* x, void* y,
+                                    cudaStream_t st) {
+  if (K != 3) return cudaErrorNotSupported;
+  if (bf16) {
+    if (S == 1) return launch_fwd2b_t<__nv_bfloat16, 3, 1>(a, x, y, st);
+    if (S == 2) return launch_fwd2b_t<__nv_bfloat16, 3, 2>(a, x, y, st);
+  } else {
+    if (S == 1) return launch_fwd2b_t<float, 3, 1>(a, x, y, st);
+    if (S == 2) return launch_fwd2b_t<float, 3, 2>(a, x, y, st);
+  }
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_adj_gather2_band(bool bf16, int S, const GatherArgs& a, const void* dy, void* dx,
+                                    cudaStream_t st) {
+  if (bf16) {
+    if (S == 1) return launch_adj2b_t<__nv_bfloat16, 1>(a, dy, dx, st);
+    if (S == 2) return launch_adj2b_t<__nv_bfloat16, 2>(a, dy, dx, st);
+  } else {
+    if (S == 1) return launch_adj2b_t<float, 1>(a, dy, dx, st);
+    if (S == 2) return launch_adj2b_t<float, 2>(a, dy, dx, st);
+  }
   return cudaErrorNotSupported;
 }
 

@@ -16,6 +16,9 @@ struct GatherArgs {
   const Chunk* chunks;
   const float* vals;
   const Ring* rings;
+  const BandPlan* bands;  // banded plans only
+  int n_bands;            // bands of this launch: bands[band0 .. band0 + n_bands)
+  int band0;
   int n_rows;        // output rows in the plan (grid.z)
   int BC;            // channel planes (batch * channels)
   int cb;            // channel planes per CTA
@@ -33,7 +36,13 @@ cudaError_t launch_adj_gather(bool bf16, int S, const GatherArgs& a, const void*
 // Paired-plane forward gather (packed fp32 FMAs) for K = 3; stage_budget in float2 words.
 cudaError_t launch_fwd_gather2(bool bf16, int K, int S, const GatherArgs& a, const void* x, void* y,
                                cudaStream_t st);
+// Same over a banded plan (a.bands): one CTA per band, block of outputs and channel block.
+cudaError_t launch_fwd_gather2_band(bool bf16, int K, int S, const GatherArgs& a, const void* x, void* y,
+                                    cudaStream_t st);
 size_t gather2_bytes(int chunk_cache, int nk, int stage_f2);
+// Paired, banded adjoint gather (dx) over a banded adjoint plan; stage_budget in float2 words.
+cudaError_t launch_adj_gather2_band(bool bf16, int S, const GatherArgs& a, const void* dy, void* dx,
+                                    cudaStream_t st);
 
 // Grouped channel mix (SIMT):
 //   out[b, g*Mg + m, n] = bias[g*Mg + m] + sum_{r < Rg} wm[g, m, r] * in[b, g*Rg + r, n]

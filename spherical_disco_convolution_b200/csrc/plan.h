@@ -73,6 +73,14 @@ struct RowPlan {
   float cost;                   // relative work, used to order heavy rows first
 };
 
+// A band of consecutive output rows that share their staged source rows: the RowPlans
+// rows[rp_begin .. rp_end) all carry the band's source range and their chunks refer to it.
+struct BandPlan {
+  int rp_begin, rp_end;
+  float cost;
+  int pad;
+};
+
 // Staged elements of one source row for a block of qb outputs (a multiple of kAlign).  A task's
 // window starts at t0 + m0*step (t0 <= span - 1, m0 <= qb - kTaskR) and holds
 // (kTaskR - 1)*step + kChunkW elements, so the last element read is span + (qb - 1)*step + 6.

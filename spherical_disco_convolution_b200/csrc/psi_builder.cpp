@@ -307,6 +307,99 @@ GatherPlan make_forward_plan(const Geometry& g, const std::vector<PsiEntry>& e) 
   return P;
 }
 
+GatherPlan make_band_plan(int n_rows, const GatherPlan& one, int nb_max, int max_chunks) {
+  GatherPlan P;
+  P.nk = one.nk;
+  P.step = one.step;
+  P.residues = one.residues;
+  std::vector<int> by_row(n_rows, -1);
+  for (size_t t = 0; t < one.rows.size(); ++t) by_row[one.rows[t].row] = (int)t;
+  auto light = [&](const RowPlan& r) {
+    if (r.ring_end > r.ring_begin) return false;
+    if (r.chunk_end[kMaxStride - 1] - r.chunk_start[0] > max_chunks) return false;
+    for (int s = r.src_begin; s < r.src_end; ++s)
+      if (one.src[s].span > 64) return false;
+    return true;
+  };
+  int j = 0;
+  while (j < n_rows) {
+    std::vector<int> members{by_row[j]};
+    if (light(one.rows[by_row[j]]))
+      while ((int)members.size() < nb_max && j + (int)members.size() < n_rows &&
+             light(one.rows[by_row[j + members.size()]]))
+        members.push_back(by_row[j + members.size()]);
+    j += (int)members.size();
+    // union of the members' source intervals, per source row
+    std::vector<SrcRow> band_src;
+    for (int m : members) {
+      const RowPlan& r = one.rows[m];
+      for (int s = r.src_begin; s < r.src_end; ++s) {
+        const SrcRow& sr = one.src[s];
+        auto it = std::find_if(band_src.begin(), band_src.end(), [&](const SrcRow& b) { return b.row == sr.row; });
+        if (it == band_src.end()) {
+          band_src.push_back(sr);
+        } else {
+          const int lo = std::min(it->start, sr.start);
+          const int hi = std::max(it->start + it->span, sr.start + sr.span);
+          it->start = lo;
+          it->span = hi - lo;
+        }
+      }
+    }
+    std::sort(band_src.begin(), band_src.end(), [](const SrcRow& a, const SrcRow& b) { return a.row < b.row; });
+    BandPlan bp{(int)P.rows.size(), 0, 0.0f, 0};
+    const int src_begin = (int)P.src.size();
+    P.src.insert(P.src.end(), band_src.begin(), band_src.end());
+    float cost = 0.0f;
+    for (int m : members) {
+      const RowPlan& r = one.rows[m];
+      RowPlan nr = r;
+      nr.src_begin = src_begin;
+      nr.src_end = (int)P.src.size();
+      for (int rho = 0; rho < kMaxStride; ++rho) {
+        nr.chunk_start[rho] = (int)P.chunks.size();
+        for (int c = r.chunk_start[rho]; c < r.chunk_end[rho]; ++c) {
+          Chunk ch = one.chunks[c];
+          const SrcRow& own = one.src[r.src_begin + ch.src];
+          const int bi = (int)(std::find_if(band_src.begin(), band_src.end(),
+                                            [&](const SrcRow& b) { return b.row == own.row; }) -
+                               band_src.begin());
+          ch.t0 += own.start - band_src[bi].start;
+          ch.src = bi;
+          const int nv = one.nk * kChunkW;
+          const int voff = (int)P.vals.size();
+          P.vals.insert(P.vals.end(), one.vals.begin() + ch.voff, one.vals.begin() + ch.voff + nv);
+          ch.voff = voff;
+          P.chunks.push_back(ch);
+        }
+        nr.chunk_end[rho] = (int)P.chunks.size();
+      }
+      nr.ring_begin = (int)P.rings.size();
+      for (int t = r.ring_begin; t < r.ring_end; ++t) P.rings.push_back(one.rings[t]);
+      nr.ring_end = (int)P.rings.size();
+      cost += r.cost;
+      P.rows.push_back(nr);
+    }
+    bp.rp_end = (int)P.rows.size();
+    bp.cost = cost;
+    P.bands.push_back(bp);
+  }
+  for (const RowPlan& rp : P.rows) {
+    P.max_src = std::max(P.max_src, rp.src_end - rp.src_begin);
+    P.max_ring = std::max(P.max_ring, rp.ring_end - rp.ring_begin);
+  }
+  std::stable_sort(P.bands.begin(), P.bands.end(),
+                   [](const BandPlan& a, const BandPlan& b) { return a.cost > b.cost; });
+  return P;
+}
+
+void split_bands(GatherPlan& P, int qb, int light_words) {
+  auto heavy = [&](const BandPlan& b) { return stage_elems(P, P.rows[b.rp_begin], qb) > light_words; };
+  std::stable_partition(P.bands.begin(), P.bands.end(), heavy);
+  P.n_heavy = 0;
+  for (const BandPlan& b : P.bands) P.n_heavy += heavy(b) ? 1 : 0;
+}
+
 GatherPlan make_adjoint_plan(const Geometry& g, const std::vector<PsiEntry>& e) {
   GatherPlan P;
   const int s = g.stride;

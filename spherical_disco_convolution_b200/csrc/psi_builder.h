@@ -30,6 +30,8 @@ struct GatherPlan {
   std::vector<Chunk> chunks;
   std::vector<float> vals;
   std::vector<Ring> rings;
+  std::vector<BandPlan> bands;  // banded plans only: heavy bands first, then light ones
+  int n_heavy = 0;              // bands whose staging exceeds the light budget
   int nk = 1;          // value sets per chunk (K for the forward, 1 for the adjoint)
   int step = 1;        // source positions advance by `step` per output (forward: s; adjoint: 1)
   int residues = 1;    // output residue classes (adjoint: s)
@@ -42,6 +44,16 @@ int stage_elems(const GatherPlan& P, const RowPlan& r, int qb);
 
 // Forward gather plan: output rows j, sources x rows i, K accumulators.
 GatherPlan make_forward_plan(const Geometry& g, const std::vector<PsiEntry>& e);
+
+// Banded plan: consecutive light output rows (no ring terms, spans <= 64, at most max_chunks
+// chunks) are grouped into bands of up to nb_max rows that share their staged source rows;
+// other rows form bands of one.  Works on the forward plan (rows j) and the adjoint plan
+// (rows i, one chunk list per residue class).
+GatherPlan make_band_plan(int n_rows, const GatherPlan& single, int nb_max, int max_chunks);
+
+// Orders a banded plan's bands as [heavy ..., light ...] where a band is heavy when one channel
+// pair's staging for a block of qb outputs exceeds light_words; sets n_heavy.
+void split_bands(GatherPlan& P, int qb, int light_words);
 
 // Adjoint gather plan: output rows i of dx, sources rows (k, j) of dy, one accumulator,
 // output longitude l = stride*m + rho.

@@ -54,12 +54,13 @@ def _bc(x):
     return x.reshape((-1,) + x.shape[2:])
 
 
-@pytest.mark.parametrize("name", ["tiny", "downsample"])
-def test_forward_plan_reproduces_oracle_contraction(name):
+@pytest.mark.parametrize("which", [0, 2], ids=["rows", "bands"])
+@pytest.mark.parametrize("name", ["tiny", "downsample", "mid"])
+def test_forward_plan_reproduces_oracle_contraction(name, which):
     wl = WORKLOADS[name].scaled(B=1, C_in=2)
     s, o = spec_pair(wl)
     h = D.disco_psi_build(s, -1)
-    plan = D.disco_plan_export(h, 0)
+    plan = D.disco_plan_export(h, which)
     D.disco_psi_destroy(h)
     x = make_inputs(wl, 1)["x"].astype(np.float64)
     y_ref = oracle.Psi(o).contract(x)
@@ -68,12 +69,13 @@ def test_forward_plan_reproduces_oracle_contraction(name):
     np.testing.assert_allclose(y, _bc(y_ref), rtol=0, atol=1e-6 * np.abs(y_ref).max())
 
 
-@pytest.mark.parametrize("name", ["tiny", "downsample"])
-def test_adjoint_plan_reproduces_oracle_backward(name):
+@pytest.mark.parametrize("which", [1, 3], ids=["rows", "bands"])
+@pytest.mark.parametrize("name", ["tiny", "downsample", "mid"])
+def test_adjoint_plan_reproduces_oracle_backward(name, which):
     wl = WORKLOADS[name].scaled(B=1, C_in=2, C_out=3)
     s, o = spec_pair(wl)
     h = D.disco_psi_build(s, -1)
-    plan = D.disco_plan_export(h, 1)
+    plan = D.disco_plan_export(h, which)
     D.disco_psi_destroy(h)
     assert plan["residues"] == wl.stride
     P = oracle.Psi(o)
