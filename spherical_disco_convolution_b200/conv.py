@@ -75,6 +75,15 @@ class Psi:
         return torch.empty(n, dtype=torch.uint8, device=self.device), n
 
 
+def disco_contract(psi: Psi, x: torch.Tensor) -> torch.Tensor:
+    """y = the K-expanded contraction of x with Psi, shape (B, C, K, nlat_out, nlon_out)."""
+    _need_cuda(x)
+    B, C = x.shape[:2]
+    y = torch.empty((B, C, psi.K) + psi.out_shape, dtype=x.dtype, device=x.device)
+    D.disco_contract(psi.handle, B, C, _dtype_code(x), _ptr(x), _ptr(y), _stream(x.device))
+    return y
+
+
 def disco_forward(psi: Psi, x: torch.Tensor, w: torch.Tensor, bias=None, groups: int = 1, fused: bool = False):
     """Returns (out, y); y is None when fused."""
     _need_cuda(x, w, bias)

@@ -1,6 +1,7 @@
 // C ABI of libdisco: argument checks, workspace layout and kernel dispatch.
 // See include/disco.h for the contract of every entry point.
 #include <cuda_runtime.h>
+#include <cstdlib>
 
 #include <algorithm>
 #include <atomic>
@@ -87,6 +88,30 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 }  // namespace
 
+// Device copy of the Toeplitz plan of the tensor-core contraction.
+struct DevTz {
+  disco::TzSlab* slabs = nullptr;
+  int* row_begin = nullptr;
+  int* order = nullptr;
+  uint16_t* b = nullptr;
+};
+
+cudaError_t upload_tz(const disco::ToeplitzPlan& P, DevTz* d) {
+  cudaError_t e;
+  if ((e = upload(P.slabs, &d->slabs)) != cudaSuccess) return e;
+  if ((e = upload(P.row_begin, &d->row_begin)) != cudaSuccess) return e;
+  if ((e = upload(P.order, &d->order)) != cudaSuccess) return e;
+  return upload(P.b, &d->b);
+}
+
+void free_tz(DevTz* d) {
+  cudaFree(d->slabs);
+  cudaFree(d->row_begin);
+  cudaFree(d->order);
+  cudaFree(d->b);
+  *d = DevTz{};
+}
+
 struct disco_psi {
   disco::Geometry g;
   int device = -1;
@@ -95,6 +120,9 @@ struct disco_psi {
   std::vector<disco::PsiEntry> entries;
   disco::GatherPlan fwd, adj, fwdb, adjb;
   DevPlan dfwd, dadj, dfwdb, dadjb;
+  bool tz_ok = false;                 // tensor-core contraction available (bf16 signals)
+  disco::ToeplitzPlan tz;
+  DevTz dtz;
 };
 
 namespace {
@@ -265,6 +293,15 @@ disco_status run_banded(const disco_psi* psi, const disco::GatherPlan& P, disco:
 disco_status launch_contract(const disco_psi* psi, int BC, disco_dtype dtype, const void* x, void* y,
                              cudaStream_t st, const char* what) {
   const disco::Geometry& g = psi->g;
+  if (dtype == DISCO_BF16 && psi->tz_ok && !(reinterpret_cast<uintptr_t>(x) & 15) &&
+      !(reinterpret_cast<uintptr_t>(y) & 15)) {
+    // Toeplitz blocks of Psi on tensor cores
+    disco::TzLaunch L{psi->dtz.slabs, psi->dtz.row_begin, psi->dtz.order, psi->dtz.b, psi->tz.K, psi->tz.parts,
+                      psi->tz.N, BC, g.nlat_in, g.nlat_out, g.nlon_in};
+    cudaError_t e = disco::launch_contract_tc(L, x, y, st);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    return DISCO_OK;
+  }
   int qb, nblk;
   block_shape(g.nlon_out, 128, &qb, &nblk);
   const int need = max_stage(psi->fwd, qb);
@@ -300,7 +337,7 @@ unsigned long long disco_launch_count(void) { return disco::g_launches.load(); }
 disco_status disco_sync_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronisation");
-  if (disco::take_mix_tc_status() | disco::take_fused_tc_status())
+  if (disco::take_mix_tc_status() | disco::take_fused_tc_status() | disco::take_contract_tc_status())
     return fail(DISCO_ERR_TIMEOUT, "a bounded device-side wait expired");
   return DISCO_OK;
 }
@@ -363,6 +400,14 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
     if (e == cudaSuccess) e = upload_plan(h->adj, &h->dadj);
     if (e == cudaSuccess) e = upload_plan(h->fwdb, &h->dfwdb);
     if (e == cudaSuccess) e = upload_plan(h->adjb, &h->dadjb);
+    // tensor-core contraction for bf16 signals (DISCO_SIMT_CONTRACT=1 keeps the gather kernels)
+    const char* simt = std::getenv("DISCO_SIMT_CONTRACT");
+    if (e == cudaSuccess && !(simt && simt[0] == '1') &&
+        disco::contract_tc_supported(g.K, g.stride, g.nlon_in, g.nlon_out)) {
+      h->tz = disco::make_toeplitz_plan(g, h->entries);
+      e = upload_tz(h->tz, &h->dtz);
+      h->tz_ok = e == cudaSuccess;
+    }
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->fork, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->join, cudaEventDisableTiming);
@@ -372,6 +417,7 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
       free_plan(&h->dadj);
       free_plan(&h->dfwdb);
       free_plan(&h->dadjb);
+      free_tz(&h->dtz);
       delete h;
       return fail(DISCO_ERR_ALLOC, std::string("Psi upload failed: ") + cudaGetErrorString(e));
     }
@@ -391,6 +437,7 @@ disco_status disco_psi_destroy(disco_psi* psi) {
     free_plan(&psi->dadj);
     free_plan(&psi->dfwdb);
     free_plan(&psi->dadjb);
+    free_tz(&psi->dtz);
     if (psi->side) cudaStreamDestroy(psi->side);
     if (psi->fork) cudaEventDestroy(psi->fork);
     if (psi->join) cudaEventDestroy(psi->join);

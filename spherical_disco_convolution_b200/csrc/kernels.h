@@ -44,6 +44,20 @@ size_t gather2_bytes(int chunk_cache, int nk, int stage_f2);
 cudaError_t launch_adj_gather2_band(bool bf16, int S, const GatherArgs& a, const void* dy, void* dx,
                                     cudaStream_t st);
 
+// Tensor-core (Toeplitz) contraction x -> y for bf16, stride 1 (contract_tc.cu).
+constexpr size_t kTcSmemLimit = 227 * 1024;
+struct TzLaunch {
+  const TzSlab* slabs;   // device arrays of the Toeplitz plan
+  const int* row_begin;
+  const int* order;
+  const void* b;         // expanded Psi blocks (bf16)
+  int K, parts, N;
+  int BC, nlat_in, nlat_out, nlon;
+};
+bool contract_tc_supported(int K, int stride, int nlon_in, int nlon_out);
+cudaError_t launch_contract_tc(const TzLaunch& L, const void* x, void* y, cudaStream_t st);
+int take_contract_tc_status();
+
 // Grouped channel mix (SIMT):
 //   out[b, g*Mg + m, n] = bias[g*Mg + m] + sum_{r < Rg} wm[g, m, r] * in[b, g*Rg + r, n]
 struct MixArgs {

@@ -81,6 +81,17 @@ struct BandPlan {
   int pad;
 };
 
+// One slab of the tensor-core (Toeplitz) contraction: a window of 16*nk consecutive source
+// longitudes of source row i, starting lon_off longitudes after the first output of a step
+// (lon_off a multiple of 8), together with its expanded Psi block in global memory at 16-byte
+// unit boff: [parts][2*nk octets][N columns][8 longitudes] bf16.  Column n of part h holds the
+// hi (h = 0) or lo (h = 1) bf16 part of Psi_k at offset lon_off + p' - u for output u, with
+// n = (h*K + k)*8 + u when both parts share one block (parts = 1), n = k*8 + u otherwise.
+struct TzSlab {
+  int i, lon_off, nk, boff;
+};
+constexpr int kTzSlabK = 4;  // most 16-longitude K-steps in one slab
+
 // Staged elements of one source row for a block of qb outputs (a multiple of kAlign).  A task's
 // window starts at t0 + m0*step (t0 <= span - 1, m0 <= qb - kTaskR) and holds
 // (kTaskR - 1)*step + kChunkW elements, so the last element read is span + (qb - 1)*step + 6.

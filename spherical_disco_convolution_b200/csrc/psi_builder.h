@@ -1,6 +1,7 @@
 // Host-side Psi builder and plan construction for libdisco.
 #pragma once
 
+#include <cstdint>
 #include <string>
 #include <vector>
 
@@ -54,6 +55,25 @@ GatherPlan make_band_plan(int n_rows, const GatherPlan& single, int nb_max, int 
 // Orders a banded plan's bands as [heavy ..., light ...] where a band is heavy when one channel
 // pair's staging for a block of qb outputs exceeds light_words; sets n_heavy.
 void split_bands(GatherPlan& P, int qb, int light_words);
+
+// Toeplitz plan of the tensor-core contraction (stride 1).  For output row j and source row i,
+// y[c, k, j, q] gets sum_p Psi_k(j, i, p) x[c, i, q + p]: the same correlation for every q, so
+// one expanded block B[p', (h, k, u)] = Psi_k(lon_off + p' - u) serves every group of 8 outputs
+// whose window starts lon_off longitudes after it.
+struct ToeplitzPlan {
+  int K = 0;
+  int N = 0;                         // MMA columns
+  int parts = 1;                     // 1: hi and lo parts side by side in N (N = 16K); 2: one
+                                     // block per part, two MMAs into one accumulator (N = 8K
+                                     // rounded up to 16), for K above 8
+  std::vector<TzSlab> slabs;         // grouped by output row
+  std::vector<int> row_begin;        // slabs of row j: [row_begin[j], row_begin[j + 1])
+  std::vector<int> order;            // output rows, most K-steps first
+  std::vector<uint16_t> b;           // expanded Psi blocks, bf16 bits
+  long long ksteps = 0;              // sum of nk over all slabs
+};
+
+ToeplitzPlan make_toeplitz_plan(const Geometry& g, const std::vector<PsiEntry>& e);
 
 // Adjoint gather plan: output rows i of dx, sources rows (k, j) of dy, one accumulator,
 // output longitude l = stride*m + rho.

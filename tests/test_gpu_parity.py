@@ -200,3 +200,23 @@ def test_invalid_calls_raise():
     with pytest.raises(D.DiscoError) as e:
         conv.disco_forward(psi, x, w, None, 4)  # 4 divides neither 6 nor 9
     assert e.value.status == D.DISCO_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name", ["tc_small_bf16", "weather", "grouped"])
+def test_contract_tensor_core_matches_gather(name, monkeypatch):
+    """The Toeplitz tensor-core contraction (bf16, stride 1) against the gather kernels and the
+    oracle: both paths round y to bf16 once, so they agree to a few bf16 units."""
+    wl, inp = workload(name), inputs(name)
+    sel = y_channels(wl)
+    x = dev(inp["x"], wl)
+    if sel is not None:
+        x = x[:, sel].contiguous()
+    y_tc = conv.disco_contract(gpu_psi(name), x)
+    monkeypatch.setenv("DISCO_SIMT_CONTRACT", "1")
+    psi_simt = conv.Psi(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape, wl.theta_cutoff,
+                        "cuda:0")
+    y_g = conv.disco_contract(psi_simt, x)
+    torch.cuda.synchronize()
+    y_ref = oracle_psi(name).contract(inp["x"] if sel is None else inp["x"][:, sel])
+    check(host(y_tc), y_ref, 4e-3, "y (tensor cores)")
+    check(host(y_tc), host(y_g), 8e-3, "y (tensor cores vs gather)")
