@@ -92,7 +92,7 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 struct DevTz {
   disco::TzSlab* slabs = nullptr;
   int* row_begin = nullptr;
-  int* order = nullptr;
+  int* slots = nullptr;
   uint16_t* b = nullptr;
 };
 
@@ -100,14 +100,14 @@ cudaError_t upload_tz(const disco::ToeplitzPlan& P, DevTz* d) {
   cudaError_t e;
   if ((e = upload(P.slabs, &d->slabs)) != cudaSuccess) return e;
   if ((e = upload(P.row_begin, &d->row_begin)) != cudaSuccess) return e;
-  if ((e = upload(P.order, &d->order)) != cudaSuccess) return e;
+  if ((e = upload(P.slots, &d->slots)) != cudaSuccess) return e;
   return upload(P.b, &d->b);
 }
 
 void free_tz(DevTz* d) {
   cudaFree(d->slabs);
   cudaFree(d->row_begin);
-  cudaFree(d->order);
+  cudaFree(d->slots);
   cudaFree(d->b);
   *d = DevTz{};
 }
@@ -121,8 +121,8 @@ struct disco_psi {
   disco::GatherPlan fwd, adj, fwdb, adjb;
   DevPlan dfwd, dadj, dfwdb, dadjb;
   bool tz_ok = false;                 // tensor-core contraction available (bf16 signals)
-  disco::ToeplitzPlan tz;
-  DevTz dtz;
+  disco::ToeplitzPlan tz, tza;        // forward (x -> y) and adjoint (dy -> dx) Toeplitz plans
+  DevTz dtz, dtza;
 };
 
 namespace {
@@ -296,7 +296,7 @@ disco_status launch_contract(const disco_psi* psi, int BC, disco_dtype dtype, co
   if (dtype == DISCO_BF16 && psi->tz_ok && !(reinterpret_cast<uintptr_t>(x) & 15) &&
       !(reinterpret_cast<uintptr_t>(y) & 15)) {
     // Toeplitz blocks of Psi on tensor cores
-    disco::TzLaunch L{psi->dtz.slabs, psi->dtz.row_begin, psi->dtz.order, psi->dtz.b, psi->tz.K, psi->tz.parts,
+    disco::TzLaunch L{psi->dtz.slabs, psi->dtz.row_begin, psi->dtz.slots, psi->dtz.b, psi->tz.K, psi->tz.parts,
                       psi->tz.N, BC, g.nlat_in, g.nlat_out, g.nlon_in};
     cudaError_t e = disco::launch_contract_tc(L, x, y, st);
     if (e != cudaSuccess) return cuda_fail(e, what);
@@ -405,7 +405,9 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
     if (e == cudaSuccess && !(simt && simt[0] == '1') &&
         disco::contract_tc_supported(g.K, g.stride, g.nlon_in, g.nlon_out)) {
       h->tz = disco::make_toeplitz_plan(g, h->entries);
+      h->tza = disco::make_adjoint_toeplitz_plan(g, h->entries);
       e = upload_tz(h->tz, &h->dtz);
+      if (e == cudaSuccess) e = upload_tz(h->tza, &h->dtza);
       h->tz_ok = e == cudaSuccess;
     }
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
@@ -418,6 +420,7 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
       free_plan(&h->dfwdb);
       free_plan(&h->dadjb);
       free_tz(&h->dtz);
+      free_tz(&h->dtza);
       delete h;
       return fail(DISCO_ERR_ALLOC, std::string("Psi upload failed: ") + cudaGetErrorString(e));
     }
@@ -438,6 +441,7 @@ disco_status disco_psi_destroy(disco_psi* psi) {
     free_plan(&psi->dfwdb);
     free_plan(&psi->dadjb);
     free_tz(&psi->dtz);
+    free_tz(&psi->dtza);
     if (psi->side) cudaStreamDestroy(psi->side);
     if (psi->fork) cudaEventDestroy(psi->fork);
     if (psi->join) cudaEventDestroy(psi->join);
@@ -553,8 +557,19 @@ disco_status disco_fwd_fused(const disco_psi* psi, int B, int C_in, int C_out, i
   const bool bf16 = dtype == DISCO_BF16;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int Cg = C_in / groups;
+  if (bf16 && psi->tz_ok && disco::fused_tz_supported(g.K, C_in, C_out, groups) &&
+      !(reinterpret_cast<uintptr_t>(x) & 15) && !(reinterpret_cast<uintptr_t>(w) & 15)) {
+    // Toeplitz contraction and channel mix, both on tensor cores, y tile in shared memory
+    const disco::ToeplitzPlan& P = psi->tz;
+    disco::TzLaunch L{psi->dtz.slabs, psi->dtz.row_begin, psi->dtz.slots, psi->dtz.b, P.K, P.parts, P.N,
+                      B * C_in, g.nlat_in, g.nlat_out, g.nlon_in};
+    disco::TzFused F{x, w, bias, out, C_in, C_out, groups};
+    cudaError_t e = disco::launch_fused_tz(L, F, st);
+    if (e != cudaSuccess) return cuda_fail(e, "fused tensor-core launch");
+    return DISCO_OK;
+  }
   if (bf16) {
-    // tensor-core mix: blocks of exactly 128 outputs
+    // gather into an on-chip y tile, tensor-core mix: blocks of exactly 128 outputs
     const int qb = 128, nblk = (g.nlon_out + qb - 1) / qb;
     const int need = max_stage(psi->fwd, qb);
     const int cache = std::min(chunk_cache(psi->fwd), 48);
@@ -620,6 +635,15 @@ disco_status disco_bwd_input(const disco_psi* psi, int B, int C_in, int C_out, i
   disco::MixArgs m{dout, wt, nullptr, dy, B, groups, Cg * g.K, Og, g.nlat_out * g.nlon_out};
   e = launch_mix(bf16, m, st);
   if (e != cudaSuccess) return cuda_fail(e, "transposed einsum launch");
+  if (bf16 && psi->tz_ok && !(reinterpret_cast<uintptr_t>(dx) & 15)) {
+    // Toeplitz blocks of the reversed Psi on tensor cores: dy rows (k, j) are the source rows
+    const disco::ToeplitzPlan& P = psi->tza;
+    disco::TzLaunch T{psi->dtza.slabs, psi->dtza.row_begin, psi->dtza.slots, psi->dtza.b, P.K, P.parts, P.N,
+                      B * C_in, g.K * g.nlat_out, g.nlat_in, g.nlon_in};
+    e = disco::launch_contract_tc(T, dy, dx, st);
+    if (e != cudaSuccess) return cuda_fail(e, "adjoint contraction launch");
+    return DISCO_OK;
+  }
   int qb, nblk;
   block_shape(g.nlon_out, 128, &qb, &nblk);
   if (g.K == 3) {

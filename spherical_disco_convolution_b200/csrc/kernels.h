@@ -49,13 +49,24 @@ constexpr size_t kTcSmemLimit = 227 * 1024;
 struct TzLaunch {
   const TzSlab* slabs;   // device arrays of the Toeplitz plan
   const int* row_begin;
-  const int* order;
+  const int* slots;     // {row, first slab, end slab, 0} per row position, heaviest rows first
   const void* b;         // expanded Psi blocks (bf16)
   int K, parts, N;
   int BC, nlat_in, nlat_out, nlon;
 };
 bool contract_tc_supported(int K, int stride, int nlon_in, int nlon_out);
 cudaError_t launch_contract_tc(const TzLaunch& L, const void* x, void* y, cudaStream_t st);
+// Fused forward on the same plan: out = bias + mix(w, contraction(x)) with the y tile kept in
+// shared memory; for K = 3 or 5 and 64 input channels per group (bf16, stride 1).
+struct TzFused {
+  const void* x;
+  const void* w;     // (C_out, C_in / G, K)
+  const void* bias;  // may be null
+  void* out;
+  int C_in, C_out, G;
+};
+bool fused_tz_supported(int K, int C_in, int C_out, int G);
+cudaError_t launch_fused_tz(const TzLaunch& L, const TzFused& F, cudaStream_t st);
 int take_contract_tc_status();
 
 // Grouped channel mix (SIMT):

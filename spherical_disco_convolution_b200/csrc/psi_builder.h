@@ -69,11 +69,17 @@ struct ToeplitzPlan {
   std::vector<TzSlab> slabs;         // grouped by output row
   std::vector<int> row_begin;        // slabs of row j: [row_begin[j], row_begin[j + 1])
   std::vector<int> order;            // output rows, most K-steps first
+  std::vector<int> slots;            // per position in `order`: {row, first slab, end slab, 0}
   std::vector<uint16_t> b;           // expanded Psi blocks, bf16 bits
   long long ksteps = 0;              // sum of nk over all slabs
 };
 
+// Forward plan: output rows j, source rows i of x, K basis functions, offsets p.
 ToeplitzPlan make_toeplitz_plan(const Geometry& g, const std::vector<PsiEntry>& e);
+
+// Adjoint plan (input gradient, stride 1): output rows i of dx, source rows k*nlat_out + j of dy
+// (one basis function), offsets -p:  dx[c, i, l] = sum_{k,j} sum_p Psi_k(j, i, p) dy[c, k, j, l - p].
+ToeplitzPlan make_adjoint_toeplitz_plan(const Geometry& g, const std::vector<PsiEntry>& e);
 
 // Adjoint gather plan: output rows i of dx, sources rows (k, j) of dy, one accumulator,
 // output longitude l = stride*m + rho.

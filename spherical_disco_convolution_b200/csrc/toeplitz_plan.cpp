@@ -39,36 +39,44 @@ float bf16_value(uint16_t h) {
 
 }  // namespace
 
-ToeplitzPlan make_toeplitz_plan(const Geometry& g, const std::vector<PsiEntry>& e) {
+namespace {
+
+// One term of a correlation along the ring: out[.., k, out_row, q] += v * src[.., src_row, q + off].
+struct Term {
+  int out_row, src_row, k, off;
+  double v;
+};
+
+ToeplitzPlan build(int n_out_rows, int nlon, int K, std::vector<Term>& terms) {
   ToeplitzPlan P;
-  P.K = g.K;
-  P.parts = 16 * g.K <= 128 ? 1 : 2;
-  P.N = P.parts == 1 ? 16 * g.K : (8 * g.K + 15) / 16 * 16;
-  const int n = g.nlon_in, K = g.K, N = P.N;
-  // entries grouped by (j, i); offsets centred in (-n/2, n/2] so that an arc around offset 0
-  // is one contiguous range
-  auto centred = [n](int p) { return p > n / 2 ? p - n : p; };
-  std::vector<size_t> idx(e.size());
-  std::iota(idx.begin(), idx.end(), 0);
-  std::sort(idx.begin(), idx.end(), [&](size_t a, size_t b) {
-    if (e[a].j != e[b].j) return e[a].j < e[b].j;
-    if (e[a].i != e[b].i) return e[a].i < e[b].i;
-    return centred(e[a].p) < centred(e[b].p);
+  P.K = K;
+  P.parts = 16 * K <= 128 ? 1 : 2;
+  P.N = P.parts == 1 ? 16 * K : (8 * K + 15) / 16 * 16;
+  const int n = nlon, N = P.N;
+  // offsets centred in (-n/2, n/2] so that an arc around offset 0 is one contiguous range
+  for (Term& t : terms) {
+    t.off = ((t.off % n) + n) % n;
+    if (t.off > n / 2) t.off -= n;
+  }
+  std::sort(terms.begin(), terms.end(), [](const Term& a, const Term& b) {
+    if (a.out_row != b.out_row) return a.out_row < b.out_row;
+    if (a.src_row != b.src_row) return a.src_row < b.src_row;
+    return a.off < b.off;
   });
-  P.row_begin.assign(g.nlat_out + 1, 0);
-  std::vector<long long> row_steps(g.nlat_out, 0);
+  P.row_begin.assign(n_out_rows + 1, 0);
+  std::vector<long long> row_steps(n_out_rows, 0);
   std::vector<double> dense;
   size_t a = 0;
   int row = 0;
-  while (a < idx.size()) {
-    const int j = e[idx[a]].j, i = e[idx[a]].i;
+  while (a < terms.size()) {
+    const int j = terms[a].out_row, i = terms[a].src_row;
     size_t b = a;
-    while (b < idx.size() && e[idx[b]].j == j && e[idx[b]].i == i) ++b;
+    while (b < terms.size() && terms[b].out_row == j && terms[b].src_row == i) ++b;
     while (row <= j) P.row_begin[row++] = (int)P.slabs.size();
-    int pmin = centred(e[idx[a]].p), pmax = centred(e[idx[b - 1]].p);
+    const int pmin = terms[a].off, pmax = terms[b - 1].off;
     const int s = pmax - pmin + 1;
     dense.assign((size_t)K * s, 0.0);
-    for (size_t t = a; t < b; ++t) dense[(size_t)e[idx[t]].k * s + (centred(e[idx[t]].p) - pmin)] += e[idx[t]].v;
+    for (size_t t = a; t < b; ++t) dense[(size_t)terms[t].k * s + (terms[t].off - pmin)] += terms[t].v;
     const int delta = ((pmin % 8) + 8) % 8;
     const int p0 = pmin - delta;
     const int ks = (delta + s + 7 + 15) / 16;  // K-steps of 16 longitudes
@@ -85,7 +93,7 @@ ToeplitzPlan make_toeplitz_plan(const Geometry& g, const std::vector<PsiEntry>& 
             const int k = P.parts == 1 ? (col / 8) % K : col / 8;
             const int h = P.parts == 1 ? col / (8 * K) : part;
             for (int el = 0; el < 8; ++el) {
-              const int off = sl.lon_off + 8 * o + el - u;  // Psi offset of this (p', u)
+              const int off = sl.lon_off + 8 * o + el - u;  // offset of this (p', u)
               double v = 0.0;
               if (k < K && h < 2 && off >= pmin && off <= pmax) v = dense[(size_t)k * s + (off - pmin)];
               const uint16_t hi = bf16_bits((float)v);
@@ -98,12 +106,34 @@ ToeplitzPlan make_toeplitz_plan(const Geometry& g, const std::vector<PsiEntry>& 
     }
     a = b;
   }
-  while (row <= g.nlat_out) P.row_begin[row++] = (int)P.slabs.size();
-  P.order.resize(g.nlat_out);
+  while (row <= n_out_rows) P.row_begin[row++] = (int)P.slabs.size();
+  P.order.resize(n_out_rows);
   std::iota(P.order.begin(), P.order.end(), 0);
   std::stable_sort(P.order.begin(), P.order.end(),
                    [&](int x, int y) { return row_steps[x] > row_steps[y]; });
+  for (int r : P.order) {
+    P.slots.push_back(r);
+    P.slots.push_back(P.row_begin[r]);
+    P.slots.push_back(P.row_begin[r + 1]);
+    P.slots.push_back(0);
+  }
   return P;
+}
+
+}  // namespace
+
+ToeplitzPlan make_toeplitz_plan(const Geometry& g, const std::vector<PsiEntry>& e) {
+  std::vector<Term> t;
+  t.reserve(e.size());
+  for (const PsiEntry& x : e) t.push_back(Term{x.j, x.i, x.k, x.p, x.v});
+  return build(g.nlat_out, g.nlon_in, g.K, t);
+}
+
+ToeplitzPlan make_adjoint_toeplitz_plan(const Geometry& g, const std::vector<PsiEntry>& e) {
+  std::vector<Term> t;
+  t.reserve(e.size());
+  for (const PsiEntry& x : e) t.push_back(Term{x.i, x.k * g.nlat_out + x.j, 0, -x.p, x.v});
+  return build(g.nlat_in, g.nlon_in, 1, t);
 }
 
 }  // namespace disco

@@ -36,6 +36,10 @@ EDGE = {
     # channel counts in multiples of 16/32) with partial 128-wide tiles
     "tc_small_bf16": Workload("tc_small_bf16", 2, 32, 64, 2, 33, 64, 33, 64, (3, 1), 0.3, "bf16"),
     "tc_down_bf16": Workload("tc_down_bf16", 1, 16, 32, 1, 33, 128, 17, 64, (3, 4), 0.5, "bf16"),
+    # layers of the fused tensor-core forward (64 input channels per group): two groups with a
+    # ragged last 128-output block, and K = 5 with one contraction accumulator buffer
+    "tz_fused_k3": Workload("tz_fused_k3", 2, 128, 64, 2, 33, 192, 33, 192, (3, 1), 0.3, "bf16"),
+    "tz_fused_k5": Workload("tz_fused_k5", 1, 64, 48, 1, 25, 64, 25, 64, (5, 1), 0.45, "bf16", bias=False),
 }
 
 
@@ -220,3 +224,32 @@ def test_contract_tensor_core_matches_gather(name, monkeypatch):
     y_ref = oracle_psi(name).contract(inp["x"] if sel is None else inp["x"][:, sel])
     check(host(y_tc), y_ref, 4e-3, "y (tensor cores)")
     check(host(y_tc), host(y_g), 8e-3, "y (tensor cores vs gather)")
+
+
+@pytest.mark.parametrize("name", ["tc_small_bf16", "weather", "grouped"])
+def test_adjoint_tensor_core_matches_gather(name, monkeypatch):
+    """dx through the reversed-Psi Toeplitz blocks on tensor cores against the gather kernels and
+    the oracle (bf16, stride 1)."""
+    wl, inp = workload(name), inputs(name)
+    dout, w = dev(inp["dout"], wl), dev(inp["w"], wl)
+    dx_tc = conv.disco_backward_input(gpu_psi(name), dout, w, wl.C_in, wl.groups)
+    monkeypatch.setenv("DISCO_SIMT_CONTRACT", "1")
+    psi_simt = conv.Psi(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape, wl.theta_cutoff,
+                        "cuda:0")
+    dx_g = conv.disco_backward_input(psi_simt, dout, w, wl.C_in, wl.groups)
+    torch.cuda.synchronize()
+    check(host(dx_tc), oracle_dx(name), 1e-2, "dx (tensor cores)")
+    check(host(dx_tc), host(dx_g), 8e-3, "dx (tensor cores vs gather)")
+
+
+@pytest.mark.parametrize("name", ["tz_fused_k3", "tz_fused_k5", "weather"])
+def test_fused_tensor_core_matches_unfused(name):
+    """The fused forward (Toeplitz contraction and channel mix on tensor cores, y tile on chip)
+    against the unfused path, which rounds the same y to bf16 before the same mix."""
+    wl, inp = workload(name), inputs(name)
+    args = (gpu_psi(name), dev(inp["x"], wl), dev(inp["w"], wl), dev(inp["bias"], wl), wl.groups)
+    out_f, _ = conv.disco_forward(*args, fused=True)
+    out_u, _ = conv.disco_forward(*args)
+    torch.cuda.synchronize()
+    check(host(out_f), host(out_u), 8e-3, "fused vs unfused out")
+    check(host(out_f), oracle_out(name), tol(wl), "fused out")
