@@ -40,7 +40,9 @@ METRIC = "DISCO conv fwd/bwd grid-points·channels/s and % HBM roofline on 1 B20
 UNIT = "grid-points*channels/s"
 PSI_ENTRY_BYTES = 13  # algorithmic Psi bytes per entry: fp32 value + int32 i + int32 p + int8 k
 OPS = ("contract", "einsum", "fused", "dx", "dw")
-LAUNCHES_PER_STEP = {"contract": 1, "einsum": 1, "fused": 1, "dx": 3, "dw": 2}
+# single-launch kernels of the step, timed one by one for the roofline: the contraction, the weight
+# einsum, the fused forward and the adjoint contraction of dx (dx = its dy einsum + this kernel)
+KERNELS = ("contract", "einsum", "fused", "adjoint")
 
 
 def parse():
@@ -73,7 +75,7 @@ def algorithmic_bytes(wl, nnz: int) -> dict:
     b = wl.C_out * es
     psi = nnz * PSI_ENTRY_BYTES
     return {"contract": x + psi + y, "einsum": y + w + b + out, "fused": x + psi + w + b + out,
-            "dx": out + w + psi + x, "dw": out + y + w + b}
+            "dx": out + w + psi + x, "dw": out + y + w + b, "adjoint": y + psi + x}
 
 
 def measured_peaks() -> tuple:
@@ -285,7 +287,8 @@ def run_gpu(args):
     dx = torch.empty(sh["x"], dtype=dt, device=dev)
     dw = torch.empty(sh["w"], dtype=dt, device=dev)
     db = torch.empty(sh["bias"], dtype=dt, device=dev) if bias is not None else None
-    ws_dx, n_dx = psi.workspace(D.DISCO_OP_BWD_INPUT, wl.B, wl.C_in, wl.C_out, wl.groups, dcode)
+    ws_dy, n_dy = psi.workspace(D.DISCO_OP_EINSUM_ADJOINT, wl.B, wl.C_in, wl.C_out, wl.groups, dcode)
+    dy = torch.empty(sh["y"], dtype=dt, device=dev)  # dx = adjoint contraction of dy = w^T dout
     ws_dw, n_dw = psi.workspace(D.DISCO_OP_BWD_WEIGHT, wl.B, wl.C_in, wl.C_out, wl.groups, dcode)
     stream = torch.cuda.current_stream(dev)
     st = stream.cuda_stream
@@ -305,12 +308,16 @@ def run_gpu(args):
         D.disco_fwd_fused(h, B, Ci, Co, G, dcode, p(x), p(w), p(bias), p(out_f), None, 0, st)
         if ev:
             ev[3].record(stream)
-        D.disco_bwd_input(h, B, Ci, Co, G, dcode, p(dout), p(w), p(dx), p(ws_dx), n_dx, st)
+        # dx in its two C-ABI halves (together they are disco_bwd_input), timed apart
+        D.disco_einsum_adjoint(h, B, Ci, Co, G, dcode, p(dout), p(w), p(dy), p(ws_dy), n_dy, st)
         if ev:
             ev[4].record(stream)
-        D.disco_bwd_weight(h, B, Ci, Co, G, dcode, p(dout), p(y), None, p(dw), p(db), p(ws_dw), n_dw, st)
+        D.disco_contract_adjoint(h, B, Ci, dcode, p(dy), p(dx), st)
         if ev:
             ev[5].record(stream)
+        D.disco_bwd_weight(h, B, Ci, Co, G, dcode, p(dout), p(y), None, p(dw), p(db), p(ws_dw), n_dw, st)
+        if ev:
+            ev[6].record(stream)
 
     def barrier():
         if world > 1:
@@ -319,7 +326,7 @@ def run_gpu(args):
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     barrier()
     torch.cuda.synchronize()
@@ -340,7 +347,10 @@ def run_gpu(args):
     ups = units_per_step(wl)
     units = sum(ups.values()) * args.steps
     el_max, units_all = aggregate(elapsed, units, world, dev)
-    op_ms = {op: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, op in enumerate(OPS)}
+    span = lambda i, j: statistics.mean(e[i].elapsed_time(e[j]) for e in evs)  # noqa: E731
+    op_ms = {"contract": span(0, 1), "einsum": span(1, 2), "fused": span(2, 3), "dx": span(3, 5), "dw": span(5, 6)}
+    kern_ms = {"contract": op_ms["contract"], "einsum": op_ms["einsum"], "fused": op_ms["fused"],
+               "adjoint": span(4, 5)}
 
     # end to end through the C ABI from pinned host buffers: inputs in, results out, every step
     e2e = None
@@ -389,16 +399,19 @@ def run_gpu(args):
     alg = algorithmic_bytes(wl, psi.nnz)
     ops = {op: {"ms": op_ms[op], "GBps": alg[op] / (op_ms[op] * 1e-3) / 1e9,
                 "frac_hbm": alg[op] / (op_ms[op] * 1e-3) / 1e9 / peak, "alg_bytes": alg[op]} for op in OPS}
-    dom = max(OPS, key=lambda o: op_ms[o])
+    kernels = {k: {"ms": kern_ms[k], "GBps": alg[k] / (kern_ms[k] * 1e-3) / 1e9,
+                   "frac_hbm": alg[k] / (kern_ms[k] * 1e-3) / 1e9 / peak, "alg_bytes": alg[k]} for k in KERNELS}
+    dom = max(KERNELS, key=lambda k: kern_ms[k])  # the longest single launch of the step
     traffic = recorded_traffic(dom, wl.name)
-    roof = {"bound": "hbm", "kernel": dom, "achieved": ops[dom]["GBps"], "peak": peak, "unit": "GB/s",
-            "frac": ops[dom]["frac_hbm"], "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
-            "headline_contract": {"achieved": ops["contract"]["GBps"], "frac": ops["contract"]["frac_hbm"]}}
+    roof = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["GBps"], "peak": peak, "unit": "GB/s",
+            "frac": kernels[dom]["frac_hbm"], "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
+            "headline_contract": {"achieved": kernels["contract"]["GBps"], "frac": kernels["contract"]["frac_hbm"]}}
     line = {
         "metric": METRIC, "value": units_all / (el_max / 1000.0), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": el_max / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
-        "config": workload_config(wl), "roofline": roof, "ops": ops, "clocks": clk, "gpu_launches": launches,
+        "config": workload_config(wl), "roofline": roof, "ops": ops, "kernels": kernels, "clocks": clk,
+        "gpu_launches": launches,
         "e2e": e2e,
     }
     if cpu is not None:

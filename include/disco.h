@@ -75,7 +75,8 @@ enum {
   DISCO_OP_FWD_FUSED = 1,
   DISCO_OP_BWD_INPUT = 2,
   DISCO_OP_BWD_WEIGHT = 3,           /* with y given */
-  DISCO_OP_BWD_WEIGHT_RECOMPUTE = 4  /* with y == NULL: y is recomputed from x */
+  DISCO_OP_BWD_WEIGHT_RECOMPUTE = 4, /* with y == NULL: y is recomputed from x */
+  DISCO_OP_EINSUM_ADJOINT = 5        /* disco_einsum_adjoint */
 };
 
 /* Layer geometry: the in_shape / out_shape / kernel_shape / basis_type /
@@ -148,6 +149,28 @@ disco_status disco_fwd_fused(const disco_psi* psi, int B, int C_in, int C_out, i
 disco_status disco_bwd_input(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
                              const void* dout, const void* w, void* dx,
                              void* workspace, size_t ws_bytes, void* stream);
+
+/* The two halves of disco_bwd_input, for callers that keep dy or time the steps apart.
+ *
+ * disco_einsum_adjoint: the transposed weight einsum (the adjoint of disco_einsum without bias)
+ *   dy[b,c,k,j,q] = sum_{o in group(c)} w[o,c',k] * dout[b,o,j,q]
+ * dout (B, C_out, nlat_out, nlon_out), w (C_out, C_in/groups, K) -> dy (B, C_in, K, nlat_out,
+ * nlon_out), all caller-owned device memory.  Scratch (the transposed w) comes in through
+ * `workspace`, sized by disco_workspace_size(DISCO_OP_EINSUM_ADJOINT, ...).
+ *
+ * disco_contract_adjoint: the adjoint of the sparse Psi contraction (disco_contract), that is
+ * the transpose of the forward equation's first sum on the page
+ * "torch_harmonics.DiscreteContinuousConvS2", section "Forward":
+ *   dx[b,c,i,l] = sum_{k,j,q,p : (q*s + p) mod nlon_in = l} Psi[k,j,(i,p)] * dy[b,c,k,j,q]
+ * dy (B, C, K, nlat_out, nlon_out) -> dx (B, C, nlat_in, nlon_in).  No scratch.
+ *
+ * Both are asynchronous on `stream` and allocate nothing; errors as for disco_bwd_input.
+ * disco_bwd_input(..) is disco_einsum_adjoint followed by disco_contract_adjoint. */
+disco_status disco_einsum_adjoint(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                                  const void* dout, const void* w, void* dy, void* workspace, size_t ws_bytes,
+                                  void* stream);
+disco_status disco_contract_adjoint(const disco_psi* psi, int B, int C, disco_dtype dtype, const void* dy, void* dx,
+                                    void* stream);
 
 /* Backward with respect to w and bias:
  *   dw[o,c',k] = sum_{b,j,q} dout[b,o,j,q] * y[b,c,k,j,q],  dbias[o] = sum_{b,j,q} dout[b,o,j,q].

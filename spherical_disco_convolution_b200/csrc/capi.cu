@@ -223,7 +223,10 @@ WsLayout layout(const disco_psi* psi, int op, int B, int C_in, int C_out, int gr
   const disco::Geometry& g = psi->g;
   const size_t n_out = (size_t)g.nlat_out * g.nlon_out;
   const size_t y_elems = (size_t)B * C_in * g.K * n_out;
-  if (op == DISCO_OP_BWD_INPUT) {
+  if (op == DISCO_OP_EINSUM_ADJOINT) {
+    L.wt = 0;
+    L.total = align256((size_t)C_out * (C_in / groups) * g.K * es);
+  } else if (op == DISCO_OP_BWD_INPUT) {
     L.wt = 0;
     L.dy = align256((size_t)C_out * (C_in / groups) * g.K * es);
     L.total = L.dy + align256(y_elems * es);
@@ -326,9 +329,62 @@ disco_status launch_contract(const disco_psi* psi, int BC, disco_dtype dtype, co
   return DISCO_OK;
 }
 
+// dy = w^T dout (the transposed weight einsum): w transposed into `wt`, then the channel mix.
+disco_status launch_dy(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                       const void* dout, const void* w, void* wt, void* dy, cudaStream_t st) {
+  const disco::Geometry& g = psi->g;
+  const bool bf16 = dtype == DISCO_BF16;
+  const int Cg = C_in / groups, Og = C_out / groups;
+  cudaError_t e = disco::launch_transpose_weight(bf16, w, wt, groups, Og, Cg, g.K, st);
+  if (e != cudaSuccess) return cuda_fail(e, "weight transpose launch");
+  disco::MixArgs m{dout, wt, nullptr, dy, B, groups, Cg * g.K, Og, g.nlat_out * g.nlon_out};
+  e = launch_mix(bf16, m, st);
+  if (e != cudaSuccess) return cuda_fail(e, "transposed einsum launch");
+  return DISCO_OK;
+}
+
+// dx from dy: the adjoint contraction with the best kernel for the layer.
+disco_status launch_adjoint(const disco_psi* psi, int BC, disco_dtype dtype, const void* dy, void* dx,
+                            cudaStream_t st) {
+  const disco::Geometry& g = psi->g;
+  const bool bf16 = dtype == DISCO_BF16;
+  if (bf16 && psi->tz_ok && !(reinterpret_cast<uintptr_t>(dx) & 15) && !(reinterpret_cast<uintptr_t>(dy) & 15)) {
+    // Toeplitz blocks of the reversed Psi on tensor cores: dy rows (k, j) are the source rows
+    const disco::ToeplitzPlan& P = psi->tza;
+    disco::TzLaunch T{psi->dtza.slabs, psi->dtza.row_begin, psi->dtza.slots, psi->dtza.b, P.K, P.parts, P.N,
+                      BC, g.K * g.nlat_out, g.nlat_in, g.nlon_in};
+    cudaError_t e = disco::launch_contract_tc(T, dy, dx, st);
+    if (e != cudaSuccess) return cuda_fail(e, "adjoint contraction launch");
+    return DISCO_OK;
+  }
+  int qb, nblk;
+  block_shape(g.nlon_out, 128, &qb, &nblk);
+  if (g.K == 3) {
+    // paired, banded adjoint gather (few basis functions: the staged dy rows of a band
+    // fit with room for several channel pairs)
+    disco::GatherArgs a = gather_args(psi->dadjb, BC, qb, nblk, g.nlon_out, g.K * g.nlat_out, g.nlon_in,
+                                      g.nlat_in, 0, 96, bf16);
+    return run_banded(psi, psi->adjb, a, 1, st,
+                      [&](const disco::GatherArgs& la, cudaStream_t ls) {
+                        return disco::launch_adj_gather2_band(bf16, g.stride, la, dy, dx, ls);
+                      },
+                      "adjoint contraction launch");
+  }
+  const int need = max_stage(psi->adj, qb);
+  const int budget = std::max(kStageFloats, need);
+  if (gather_bytes(chunk_cache(psi->adj), 1, budget) > kSmemLimit)
+    return fail(DISCO_ERR_UNSUPPORTED, "a Psi column needs more staging than shared memory holds");
+  disco::GatherArgs a = gather_args(psi->dadj, BC, qb, nblk, g.nlon_out, g.K * g.nlat_out, g.nlon_in, g.nlat_in,
+                                    budget, chunk_cache(psi->adj), bf16);
+  cudaError_t e = disco::launch_adj_gather(bf16, g.stride, a, dy, dx, st);
+  if (e != cudaSuccess) return cuda_fail(e, "adjoint contraction launch");
+  return DISCO_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
 
 const char* disco_last_error(void) { return g_last_error.c_str(); }
 
@@ -504,7 +560,7 @@ disco_status disco_workspace_size(const disco_psi* psi, int op, int B, int C_in,
   if (!psi || !bytes) return fail(DISCO_ERR_INVALID_ARG, "NULL argument");
   if (B <= 0 || C_in <= 0 || C_out <= 0 || groups <= 0 || C_in % groups || C_out % groups)
     return fail(DISCO_ERR_INVALID_ARG, "bad sizes");
-  if (op < DISCO_OP_FWD || op > DISCO_OP_BWD_WEIGHT_RECOMPUTE) return fail(DISCO_ERR_INVALID_ARG, "unknown op");
+  if (op < DISCO_OP_FWD || op > DISCO_OP_EINSUM_ADJOINT) return fail(DISCO_ERR_INVALID_ARG, "unknown op");
   *bytes = layout(psi, op, B, C_in, C_out, groups, dtype).total;
   return DISCO_OK;
 }
@@ -620,53 +676,36 @@ disco_status disco_bwd_input(const disco_psi* psi, int B, int C_in, int C_out, i
   disco_status s = check_common(psi, B, C_in, C_out, groups, dtype);
   if (s) return s;
   if (!dout || !w || !dx) return fail(DISCO_ERR_INVALID_ARG, "dout, w and dx must be non-NULL");
-  const disco::Geometry& g = psi->g;
-  if (!disco::gather_supports(g.K, g.stride)) return fail(DISCO_ERR_UNSUPPORTED, "K or stride not compiled");
+  if (!disco::gather_supports(psi->g.K, psi->g.stride)) return fail(DISCO_ERR_UNSUPPORTED, "K or stride not compiled");
   const WsLayout L = layout(psi, DISCO_OP_BWD_INPUT, B, C_in, C_out, groups, dtype);
   if (!workspace || ws_bytes < L.total) return fail(DISCO_ERR_INVALID_ARG, "workspace missing or too small");
-  const bool bf16 = dtype == DISCO_BF16;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
-  void* wt = ws + L.wt;
   void* dy = ws + L.dy;
-  const int Cg = C_in / groups, Og = C_out / groups;
-  cudaError_t e = disco::launch_transpose_weight(bf16, w, wt, groups, Og, Cg, g.K, st);
-  if (e != cudaSuccess) return cuda_fail(e, "weight transpose launch");
-  disco::MixArgs m{dout, wt, nullptr, dy, B, groups, Cg * g.K, Og, g.nlat_out * g.nlon_out};
-  e = launch_mix(bf16, m, st);
-  if (e != cudaSuccess) return cuda_fail(e, "transposed einsum launch");
-  if (bf16 && psi->tz_ok && !(reinterpret_cast<uintptr_t>(dx) & 15)) {
-    // Toeplitz blocks of the reversed Psi on tensor cores: dy rows (k, j) are the source rows
-    const disco::ToeplitzPlan& P = psi->tza;
-    disco::TzLaunch T{psi->dtza.slabs, psi->dtza.row_begin, psi->dtza.slots, psi->dtza.b, P.K, P.parts, P.N,
-                      B * C_in, g.K * g.nlat_out, g.nlat_in, g.nlon_in};
-    e = disco::launch_contract_tc(T, dy, dx, st);
-    if (e != cudaSuccess) return cuda_fail(e, "adjoint contraction launch");
-    return DISCO_OK;
-  }
-  int qb, nblk;
-  block_shape(g.nlon_out, 128, &qb, &nblk);
-  if (g.K == 3) {
-    // paired, banded adjoint gather (few basis functions: the staged dy rows of a band
-    // fit with room for several channel pairs)
-    disco::GatherArgs a = gather_args(psi->dadjb, B * C_in, qb, nblk, g.nlon_out, g.K * g.nlat_out, g.nlon_in,
-                                      g.nlat_in, 0, 96, bf16);
-    return run_banded(psi, psi->adjb, a, 1, st,
-                      [&](const disco::GatherArgs& la, cudaStream_t ls) {
-                        return disco::launch_adj_gather2_band(bf16, g.stride, la, dy, dx, ls);
-                      },
-                      "adjoint contraction launch");
-  }
-  const int need = max_stage(psi->adj, qb);
-  const int budget = std::max(kStageFloats, need);
-  if (gather_bytes(chunk_cache(psi->adj), 1, budget) > kSmemLimit)
-    return fail(DISCO_ERR_UNSUPPORTED, "a Psi column needs more staging than shared memory holds");
-  disco::GatherArgs a =
-      gather_args(psi->dadj, B * C_in, qb, nblk, g.nlon_out, g.K * g.nlat_out, g.nlon_in, g.nlat_in, budget,
-                  chunk_cache(psi->adj), bf16);
-  e = disco::launch_adj_gather(bf16, g.stride, a, dy, dx, st);
-  if (e != cudaSuccess) return cuda_fail(e, "adjoint contraction launch");
-  return DISCO_OK;
+  s = launch_dy(psi, B, C_in, C_out, groups, dtype, dout, w, ws + L.wt, dy, st);
+  if (s) return s;
+  return launch_adjoint(psi, B * C_in, dtype, dy, dx, st);
+}
+
+disco_status disco_einsum_adjoint(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                                  const void* dout, const void* w, void* dy, void* workspace, size_t ws_bytes,
+                                  void* stream) {
+  disco_status s = check_common(psi, B, C_in, C_out, groups, dtype);
+  if (s) return s;
+  if (!dout || !w || !dy) return fail(DISCO_ERR_INVALID_ARG, "dout, w and dy must be non-NULL");
+  const WsLayout L = layout(psi, DISCO_OP_EINSUM_ADJOINT, B, C_in, C_out, groups, dtype);
+  if (!workspace || ws_bytes < L.total) return fail(DISCO_ERR_INVALID_ARG, "workspace missing or too small");
+  return launch_dy(psi, B, C_in, C_out, groups, dtype, dout, w, static_cast<char*>(workspace) + L.wt, dy,
+                   static_cast<cudaStream_t>(stream));
+}
+
+disco_status disco_contract_adjoint(const disco_psi* psi, int B, int C, disco_dtype dtype, const void* dy, void* dx,
+                                    void* stream) {
+  disco_status s = check_common(psi, B, C, C, 1, dtype);
+  if (s) return s;
+  if (!dy || !dx) return fail(DISCO_ERR_INVALID_ARG, "dy and dx must be non-NULL");
+  if (!disco::gather_supports(psi->g.K, psi->g.stride)) return fail(DISCO_ERR_UNSUPPORTED, "K or stride not compiled");
+  return launch_adjoint(psi, B * C, dtype, dy, dx, static_cast<cudaStream_t>(stream));
 }
 
 disco_status disco_bwd_weight(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,

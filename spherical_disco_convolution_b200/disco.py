@@ -40,6 +40,7 @@ DISCO_OP_FWD_FUSED = 1
 DISCO_OP_BWD_INPUT = 2
 DISCO_OP_BWD_WEIGHT = 3
 DISCO_OP_BWD_WEIGHT_RECOMPUTE = 4
+DISCO_OP_EINSUM_ADJOINT = 5
 
 
 class DiscoError(RuntimeError):
@@ -92,6 +93,8 @@ def _load():
         "disco_fwd": [P, I, I, I, I, I, P, P, P, P, P, P, Z, P],
         "disco_fwd_fused": [P, I, I, I, I, I, P, P, P, P, P, Z, P],
         "disco_bwd_input": [P, I, I, I, I, I, P, P, P, P, Z, P],
+        "disco_einsum_adjoint": [P, I, I, I, I, I, P, P, P, P, Z, P],
+        "disco_contract_adjoint": [P, I, I, I, P, P, P],
         "disco_bwd_weight": [P, I, I, I, I, I, P, P, P, P, P, P, Z, P],
         "disco_bwd_weight_noalloc": [P, I, I, I, I, I, P, P, P, P, P],
         "disco_plan_info": [P, I, IP],
@@ -209,6 +212,14 @@ def disco_fwd_fused(psi, B, C_in, C_out, groups, dtype, x, w, bias, out, workspa
 
 def disco_bwd_input(psi, B, C_in, C_out, groups, dtype, dout, w, dx, workspace, ws_bytes, stream) -> None:
     _check(_lib.disco_bwd_input(psi, B, C_in, C_out, groups, dtype, dout, w, dx, workspace, ws_bytes, stream))
+
+
+def disco_einsum_adjoint(psi, B, C_in, C_out, groups, dtype, dout, w, dy, workspace, ws_bytes, stream) -> None:
+    _check(_lib.disco_einsum_adjoint(psi, B, C_in, C_out, groups, dtype, dout, w, dy, workspace, ws_bytes, stream))
+
+
+def disco_contract_adjoint(psi, B, C, dtype, dy, dx, stream) -> None:
+    _check(_lib.disco_contract_adjoint(psi, B, C, dtype, dy, dx, stream))
 
 
 def disco_bwd_weight(psi, B, C_in, C_out, groups, dtype, dout, y, x, dw, dbias, workspace, ws_bytes, stream) -> None:

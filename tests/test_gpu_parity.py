@@ -253,3 +253,24 @@ def test_fused_tensor_core_matches_unfused(name):
     torch.cuda.synchronize()
     check(host(out_f), host(out_u), 8e-3, "fused vs unfused out")
     check(host(out_f), oracle_out(name), tol(wl), "fused out")
+
+
+@pytest.mark.parametrize("name", ["ragged_iso_f32", "tc_small_bf16", "ragged_down_bf16", "grouped"])
+def test_input_gradient_halves_compose(name):
+    """disco_einsum_adjoint followed by disco_contract_adjoint is disco_bwd_input, bit for bit
+    (the same kernels in the same order)."""
+    wl, inp = workload(name), inputs(name)
+    psi = gpu_psi(name)
+    dout, w = dev(inp["dout"], wl), dev(inp["w"], wl)
+    dx_ref = conv.disco_backward_input(psi, dout, w, wl.C_in, wl.groups)
+    dcode = D.DISCO_BF16 if wl.dtype == "bf16" else D.DISCO_F32
+    ws, n = psi.workspace(D.DISCO_OP_EINSUM_ADJOINT, wl.B, wl.C_in, wl.C_out, wl.groups, dcode)
+    dy = torch.empty(wl.shapes()["y"], dtype=dx_ref.dtype, device="cuda:0")
+    dx = torch.empty_like(dx_ref)
+    st = torch.cuda.current_stream().cuda_stream
+    D.disco_einsum_adjoint(psi.handle, wl.B, wl.C_in, wl.C_out, wl.groups, dcode, dout.data_ptr(), w.data_ptr(),
+                           dy.data_ptr(), ws.data_ptr(), n, st)
+    D.disco_contract_adjoint(psi.handle, wl.B, wl.C_in, dcode, dy.data_ptr(), dx.data_ptr(), st)
+    torch.cuda.synchronize()
+    assert torch.equal(dx, dx_ref)
+    check(host(dx), oracle_dx(name), tol(wl), "dx from the two halves")
