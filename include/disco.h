@@ -227,6 +227,25 @@ disco_status disco_plan_info(const disco_psi* psi, int which, int* dims);
 disco_status disco_plan_export(const disco_psi* psi, int which, int* rows, int* srcs, int* chunks, float* vals,
                                int* rings);
 
+/* Toeplitz plans of the tensor-core kernels (bf16 layers with nlon_in == nlon_out, a
+ * multiple of 8): which = 0 the forward plan (output rows j, source rows i of x), which = 1
+ * the adjoint plan (output rows i, source rows k*nlat_out + j of dy, one basis function).
+ * For an output row and a source row, the correlation along the longitude ring of the
+ * forward equation on the page "torch_harmonics.DiscreteContinuousConvS2" (class
+ * description) has the same coefficients for every output longitude; for 8 outputs q0 + u
+ * and 16*nk input longitudes q0 + lon_off + p' it is the banded block
+ * B[p', (h, k, u)] = part h of Psi_k(lon_off + p' - u), h = 0 the bf16 rounding of the
+ * value and h = 1 the bf16 rounding of the remainder.
+ * disco_toeplitz_info fills dims[8] = {K, parts, N, slabs, row records, bf16 values, most
+ * K-steps per slab, K-steps}.  disco_toeplitz_export copies into caller-owned HOST arrays:
+ * slabs (x4: source row, lon_off, nk, offset of the block in 16-byte units), row records
+ * (x4: output row, first slab, end slab, 0; heaviest rows first) and the blocks (bf16
+ * bits, [parts][2*nk][N][8] per slab; column n = (h*K + k)*8 + u when parts = 1,
+ * n = k*8 + u in part h when parts = 2).  Both return DISCO_ERR_UNSUPPORTED for layers
+ * without a Toeplitz plan.  Host-only handles (device < 0) build the plans too. */
+disco_status disco_toeplitz_info(const disco_psi* psi, int which, int* dims);
+disco_status disco_toeplitz_export(const disco_psi* psi, int which, int* slabs, int* slots, unsigned short* b);
+
 /* Synchronises `stream` and reports device-side failures of the calls queued on it
  * before: DISCO_ERR_CUDA for an asynchronous CUDA error, DISCO_ERR_TIMEOUT when a
  * tensor-core kernel gave up a bounded wait (its results are then invalid).  Clears the

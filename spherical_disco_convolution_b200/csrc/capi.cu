@@ -448,6 +448,11 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
     return fail(DISCO_ERR_UNSUPPORTED, "an output row reaches more source rows than the kernels support");
   }
   h->device = device;
+  if (device < 0 && disco::toeplitz_geometry(g.K, g.stride, g.nlon_in, g.nlon_out)) {
+    // host-only handle: the Toeplitz plans are built for inspection (disco_toeplitz_export)
+    h->tz = disco::make_toeplitz_plan(g, h->entries);
+    h->tza = disco::make_adjoint_toeplitz_plan(g, h->entries);
+  }
   if (device >= 0) {
     int prev = -1;
     cudaGetDevice(&prev);
@@ -552,6 +557,32 @@ disco_status disco_plan_export(const disco_psi* psi, int which, int* rows, int* 
   std::memcpy(srcs, P.src.data(), P.src.size() * sizeof(disco::SrcRow));
   std::memcpy(chunks, P.chunks.data(), P.chunks.size() * sizeof(disco::Chunk));
   std::memcpy(vals, P.vals.data(), P.vals.size() * sizeof(float));
+  return DISCO_OK;
+}
+
+disco_status disco_toeplitz_info(const disco_psi* psi, int which, int* dims) {
+  if (!psi || !dims || which < 0 || which > 1) return fail(DISCO_ERR_INVALID_ARG, "bad Toeplitz plan query");
+  const disco::ToeplitzPlan& P = which == 0 ? psi->tz : psi->tza;
+  if (P.slots.empty()) return fail(DISCO_ERR_UNSUPPORTED, "no Toeplitz plan for this layer");
+  dims[0] = P.K;
+  dims[1] = P.parts;
+  dims[2] = P.N;
+  dims[3] = (int)P.slabs.size();
+  dims[4] = (int)(P.slots.size() / 4);
+  dims[5] = (int)P.b.size();
+  dims[6] = disco::kTzSlabK;
+  dims[7] = (int)P.ksteps;
+  return DISCO_OK;
+}
+
+disco_status disco_toeplitz_export(const disco_psi* psi, int which, int* slabs, int* slots, unsigned short* b) {
+  if (!psi || !slabs || !slots || !b || which < 0 || which > 1)
+    return fail(DISCO_ERR_INVALID_ARG, "bad Toeplitz plan export");
+  const disco::ToeplitzPlan& P = which == 0 ? psi->tz : psi->tza;
+  if (P.slots.empty()) return fail(DISCO_ERR_UNSUPPORTED, "no Toeplitz plan for this layer");
+  std::memcpy(slabs, P.slabs.data(), P.slabs.size() * sizeof(disco::TzSlab));
+  std::memcpy(slots, P.slots.data(), P.slots.size() * sizeof(int));
+  std::memcpy(b, P.b.data(), P.b.size() * sizeof(uint16_t));
   return DISCO_OK;
 }
 

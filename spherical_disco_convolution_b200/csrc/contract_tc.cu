@@ -649,11 +649,14 @@ cudaError_t launch_tz_fused(const TzLaunch& L, const TzFused& F, cudaStream_t st
 
 }  // namespace
 
-bool contract_tc_supported(int K, int stride, int nlon_in, int nlon_out) {
+bool toeplitz_geometry(int K, int stride, int nlon_in, int nlon_out) {
   // compiled for K = 1 (the adjoint) and the forward's K = 3, 5, 7, 9; a staged window may
   // wrap around the ring any number of times, so there is no lower bound on nlon
-  return tc::encode_tiled_fn() != nullptr && stride == 1 && nlon_in == nlon_out && nlon_in % 8 == 0 &&
-         (K == 1 || K == 3 || K == 5 || K == 7 || K == 9);
+  return stride == 1 && nlon_in == nlon_out && nlon_in % 8 == 0 && (K == 1 || K == 3 || K == 5 || K == 7 || K == 9);
+}
+
+bool contract_tc_supported(int K, int stride, int nlon_in, int nlon_out) {
+  return tc::encode_tiled_fn() != nullptr && toeplitz_geometry(K, stride, nlon_in, nlon_out);
 }
 
 cudaError_t launch_contract_tc(const TzLaunch& L, const void* x, void* y, cudaStream_t st) {

@@ -54,6 +54,8 @@ struct TzLaunch {
   int K, parts, N;
   int BC, nlat_in, nlat_out, nlon;
 };
+// Layers the Toeplitz plan serves (host-side geometry only) / that the device can run.
+bool toeplitz_geometry(int K, int stride, int nlon_in, int nlon_out);
 bool contract_tc_supported(int K, int stride, int nlon_in, int nlon_out);
 cudaError_t launch_contract_tc(const TzLaunch& L, const void* x, void* y, cudaStream_t st);
 // Fused forward on the same plan: out = bias + mix(w, contraction(x)) with the y tile kept in

@@ -100,6 +100,8 @@ def _load():
         "disco_plan_info": [P, I, IP],
         "disco_sync_status": [P],
         "disco_plan_export": [P, I, IP, IP, IP, ctypes.POINTER(ctypes.c_float), IP],
+        "disco_toeplitz_info": [P, I, IP],
+        "disco_toeplitz_export": [P, I, IP, IP, ctypes.POINTER(ctypes.c_ushort)],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -186,6 +188,20 @@ def disco_plan_export(psi, which: int):
     ring_v = rings[:n_rings, 2].copy().view(np.float32)
     return dict(rows=rows, srcs=srcs, chunks=chunks, vals=vals, nk=nk, step=step, residues=residues,
                 rings=rings[:n_rings], ring_v=ring_v)
+
+
+def disco_toeplitz_export(psi, which: int):
+    """Toeplitz plan of the tensor-core kernels: which=0 forward, which=1 adjoint."""
+    dims = np.zeros(8, dtype=np.int32)
+    _check(_lib.disco_toeplitz_info(psi, which, dims.ctypes.data_as(ctypes.POINTER(ctypes.c_int))))
+    K, parts, N, n_slabs, n_rows, n_b, kslab, ksteps = (int(v) for v in dims)
+    slabs = np.zeros((n_slabs, 4), dtype=np.int32)
+    slots = np.zeros((n_rows, 4), dtype=np.int32)
+    b = np.zeros(n_b, dtype=np.uint16)
+    ip = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))  # noqa: E731
+    _check(_lib.disco_toeplitz_export(psi, which, ip(slabs), ip(slots),
+                                      b.ctypes.data_as(ctypes.POINTER(ctypes.c_ushort))))
+    return dict(K=K, parts=parts, N=N, slabs=slabs, slots=slots, b=b, kslab=kslab, ksteps=ksteps)
 
 
 def disco_workspace_size(psi, op, B, C_in, C_out, groups, dtype) -> int:

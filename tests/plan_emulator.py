@@ -54,3 +54,34 @@ def adjoint(plan, dy, nlat_in, nlon_in, stride):
                     v = float(plan["vals"][voff + u])
                     dx[:, row, stride * m + rho] += v * dy[:, srow, (start + t0 + m + u) % n_src]
     return dx
+
+
+def _bf16_values(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def toeplitz(plan, src, n_out_rows):
+    """Re-enacts the tensor-core kernel on a Toeplitz plan, in fp64.
+
+    src (B*C, source rows, nlon) -> out (B*C, K, n_out_rows, nlon).  For output q the kernel
+    takes the group of 8 outputs q8 = q - q % 8 and, per slab (i, lon_off, nk, offset), the
+    window of source longitudes (q8 + lon_off + p') mod nlon, p' < 16*nk, against column
+    (k, u = q % 8) of the slab's block, summing the hi and lo parts."""
+    K, parts, N = plan["K"], plan["parts"], plan["N"]
+    BC, _, nlon = src.shape
+    out = np.zeros((BC, K, n_out_rows, nlon))
+    vals = _bf16_values(plan["b"])
+    q = np.arange(nlon)
+    u = q % 8
+    q8 = q - u
+    for row, s0, s1, _ in plan["slots"]:
+        for i, lon_off, nk, boff in plan["slabs"][s0:s1]:
+            n = 16 * nk
+            blk = vals[8 * boff: 8 * boff + parts * 2 * nk * N * 8].reshape(parts, 2 * nk, N, 8)
+            bm = blk.transpose(0, 1, 3, 2).reshape(parts, n, N)  # [part][p' = 8*octet + e][column]
+            wsum = bm[0][:, : 8 * K] + (bm[0][:, 8 * K: 16 * K] if parts == 1 else bm[1][:, : 8 * K])
+            wsum = wsum.reshape(n, K, 8)  # [p', k, u]
+            idx = (q8[:, None] + lon_off + np.arange(n)[None, :]) % nlon  # [q, p']
+            coef = wsum[np.arange(n)[None, :], :, u[:, None]]  # [q, p', k]
+            out[:, :, row, :] += np.einsum("cqp,qpk->ckq", src[:, i, :][:, idx], coef)
+    return out

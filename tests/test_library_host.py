@@ -143,3 +143,63 @@ def test_status_codes():
     finally:
         D.disco_psi_destroy(h)
     assert lib.disco_psi_destroy(None) == D.DISCO_OK
+
+
+# bf16 layers with nlon_in == nlon_out take the tensor-core kernels: their Toeplitz plans must
+# reproduce the contraction and its adjoint (Psi as bf16 hi + lo: relative error <= 2^-17)
+TZ_LAYERS = {
+    "iso_k3": WORKLOADS["tiny"],
+    "aniso_k9": WORKLOADS["tiny"].scaled(nlat_in=21, nlon_in=40, nlat_out=21, nlon_out=40, kernel_shape=(3, 4),
+                                         theta_cutoff=0.5),
+    "iso_k5": WORKLOADS["tiny"].scaled(nlat_in=25, nlon_in=64, nlat_out=25, nlon_out=64, kernel_shape=(5, 1),
+                                       theta_cutoff=0.45),
+}
+
+
+@pytest.mark.parametrize("name", list(TZ_LAYERS))
+def test_toeplitz_plan_reproduces_oracle_contraction(name):
+    wl = TZ_LAYERS[name].scaled(B=1, C_in=3)
+    s, o = spec_pair(wl)
+    h = D.disco_psi_build(s, -1)
+    try:
+        plan = D.disco_toeplitz_export(h, 0)
+    finally:
+        D.disco_psi_destroy(h)
+    assert plan["K"] == wl.K and plan["parts"] == (1 if 16 * wl.K <= 128 else 2)
+    assert np.all((plan["slabs"][:, 2] >= 1) & (plan["slabs"][:, 2] <= plan["kslab"]))
+    assert np.all(plan["slabs"][:, 1] % 8 == 0)  # windows start on 16-byte boundaries
+    assert sorted(plan["slots"][:, 0].tolist()) == list(range(wl.nlat_out))
+    x = make_inputs(wl, 1)["x"].astype(np.float64)
+    y_ref = oracle.Psi(o).contract(x)
+    y = plan_emulator.toeplitz(plan, _bc(x), wl.nlat_out)
+    np.testing.assert_allclose(y, _bc(y_ref), rtol=0, atol=2e-5 * np.abs(y_ref).max())
+
+
+@pytest.mark.parametrize("name", list(TZ_LAYERS))
+def test_adjoint_toeplitz_plan_reproduces_oracle_backward(name):
+    wl = TZ_LAYERS[name].scaled(B=1, C_in=2, C_out=3)
+    s, o = spec_pair(wl)
+    h = D.disco_psi_build(s, -1)
+    try:
+        plan = D.disco_toeplitz_export(h, 1)
+    finally:
+        D.disco_psi_destroy(h)
+    assert plan["K"] == 1 and plan["N"] == 16
+    rng = np.random.default_rng(5)
+    dout = rng.standard_normal((1, wl.C_out, wl.nlat_out, wl.nlon_out))
+    w = rng.standard_normal((wl.C_out, wl.C_in, wl.K))
+    dx_ref = oracle.Psi(o).backward_input(dout, w, wl.C_in)
+    dy = np.einsum("ock,bojq->bckjq", w, dout).reshape(wl.C_in, wl.K * wl.nlat_out, wl.nlon_out)
+    dx = plan_emulator.toeplitz(plan, dy, wl.nlat_in)[:, 0]
+    np.testing.assert_allclose(dx, _bc(dx_ref), rtol=0, atol=2e-5 * np.abs(dx_ref).max())
+
+
+def test_toeplitz_plan_absent_for_stride_two():
+    s, _ = spec_pair(WORKLOADS["downsample"])
+    h = D.disco_psi_build(s, -1)
+    try:
+        with pytest.raises(D.DiscoError) as e:
+            D.disco_toeplitz_export(h, 0)
+        assert e.value.status == D.DISCO_ERR_UNSUPPORTED
+    finally:
+        D.disco_psi_destroy(h)
