@@ -32,6 +32,8 @@ struct MixTcArgs {
   void* out;
   const void* bias;
   int G, Mg, Rg, N, BN;
+  int S;  // pipeline stages: no more than the K loop has chunks, so small tiles leave room
+          // for several CTAs per SM
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -44,18 +46,19 @@ __host__ __device__ inline uint32_t tmem_cols(int n) {
   return c;
 }
 
-__global__ void __launch_bounds__(128, 1) mix_tc_kernel(const __grid_constant__ CUtensorMap map_in,
+__global__ void __launch_bounds__(128, 2) mix_tc_kernel(const __grid_constant__ CUtensorMap map_in,
                                                         const __grid_constant__ CUtensorMap map_w, MixTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const int BN = a.BN;
+  const int nst = a.S;  // stages of this launch
   const uint32_t a_bytes = 2 * kHalfTile;
   const uint32_t b_bytes = (uint32_t)BN * 128;
   uint8_t* sA = smem;
-  uint8_t* sB = smem + kStages * a_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * b_bytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* done = empty + kStages;
+  uint8_t* sB = smem + nst * a_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + nst * b_bytes);
+  uint64_t* empty = full + nst;
+  uint64_t* done = empty + nst;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
   const int n0 = blockIdx.x * 128;
@@ -69,7 +72,7 @@ __global__ void __launch_bounds__(128, 1) mix_tc_kernel(const __grid_constant__ 
   if (threadIdx.x == 0) {
     tc::prefetch_map(&map_in);
     tc::prefetch_map(&map_w);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < nst; ++s) {
       tc::mbar_init(&full[s], 1);
       tc::mbar_init(&empty[s], 1);
     }
@@ -87,8 +90,8 @@ __global__ void __launch_bounds__(128, 1) mix_tc_kernel(const __grid_constant__ 
 
   if (warp == 0 && lane == 0) {
     for (int kc = 0; kc < nk; ++kc) {
-      const int s = kc % kStages;
-      if (kc >= kStages && !tc::mbar_wait(&empty[s], ((kc / kStages) & 1) ^ 1)) break;
+      const int s = kc % nst;
+      if (kc >= nst && !tc::mbar_wait(&empty[s], ((kc / nst) & 1) ^ 1)) break;
       tc::mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes);
       tc::tma_load_3d(sA + s * a_bytes, &map_in, &full[s], n0, kc * kBK, bg);
       tc::tma_load_3d(sA + s * a_bytes + kHalfTile, &map_in, &full[s], n0 + 64, kc * kBK, bg);
@@ -98,8 +101,8 @@ __global__ void __launch_bounds__(128, 1) mix_tc_kernel(const __grid_constant__ 
     const uint32_t idesc = tc::idesc_bf16(128, BN, true, false);
     bool ok = true;
     for (int kc = 0; kc < nk && ok; ++kc) {
-      const int s = kc % kStages;
-      ok = tc::mbar_wait(&full[s], (kc / kStages) & 1);
+      const int s = kc % nst;
+      ok = tc::mbar_wait(&full[s], (kc / nst) & 1);
       if (!ok) break;
       tc::fence_after_sync();
       const uint32_t a0 = tc::smem_u32(sA + s * a_bytes);
@@ -288,7 +291,7 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t mix_smem(int BN) { return 1024 + kStages * (2 * kHalfTile + (size_t)BN * 128) + (2 * kStages + 2) * 8; }
+size_t mix_smem(int BN, int S) { return 1024 + S * (2 * kHalfTile + (size_t)BN * 128) + (2 * S + 2) * 8; }
 size_t dw_smem(int BN) { return 1024 + kStages * (128 * 128 + (size_t)BN * 128) + (2 * kStages + 2) * 8; }
 
 int mix_bn(int Mg) {
@@ -314,8 +317,9 @@ cudaError_t launch_mix_tc(const MixArgs& a, cudaStream_t st) {
   const cuuint64_t sw[1] = {(cuuint64_t)a.Rg * 2};
   const cuuint32_t bw[2] = {64, (cuuint32_t)BN};
   if (!make_map(&mi, a.in, 3, di, si, bi) || !make_map(&mw, a.wm, 2, dw, sw, bw)) return cudaErrorInvalidValue;
-  MixTcArgs t{a.out, a.bias, a.G, a.Mg, a.Rg, a.N, BN};
-  const size_t smem = mix_smem(BN);
+  const int S = std::min(kStages, (a.Rg + kBK - 1) / kBK);
+  MixTcArgs t{a.out, a.bias, a.G, a.Mg, a.Rg, a.N, BN, S};
+  const size_t smem = mix_smem(BN, S);
   cudaError_t e = cudaFuncSetAttribute(mix_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.N + 127) / 128, (a.Mg + BN - 1) / BN, a.B * a.G);
