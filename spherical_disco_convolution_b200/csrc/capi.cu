@@ -80,6 +80,9 @@ void free_plan(DevPlan* d) {
 }
 
 constexpr int kChannelsPerCta = 16;
+constexpr int kPackStrip = 32;  // output rows per strip of a packed plan
+constexpr int kPackKs = 4;      // widest window (K-steps of 16 longitudes) a packed entry takes
+constexpr int kPackPairs = 24;  // slabs per output row from which the adjoint is packed
 constexpr int kStageFloats = 12288;          // 48 KB of staging for the unfused gathers
 constexpr size_t kSmemLimit = 227 * 1024;    // dynamic shared memory per CTA on sm_100
 constexpr size_t kFusedTileBytes = 160 * 1024;
@@ -112,6 +115,42 @@ void free_tz(DevTz* d) {
   *d = DevTz{};
 }
 
+// Device copy of a packed Toeplitz plan and the row records of the rows it leaves to the
+// per-pair kernel.
+struct DevPk {
+  int* ent = nullptr;
+  int* strips = nullptr;
+  uint16_t* b = nullptr;
+  int* rest = nullptr;
+  int n_strips = 0, n_rest = 0;
+  bool ok = false;
+};
+
+cudaError_t upload_pk(const disco::PackedPlan& P, const disco::ToeplitzPlan& per_pair, DevPk* d) {
+  std::vector<char> is_rest(per_pair.row_begin.size(), 0);
+  for (int r : P.rest) is_rest[r] = 1;
+  std::vector<int> rest;  // the per-pair plan's row records of the rest rows, same order
+  for (size_t q = 0; q + 3 < per_pair.slots.size(); q += 4)
+    if (is_rest[per_pair.slots[q]]) rest.insert(rest.end(), per_pair.slots.begin() + q, per_pair.slots.begin() + q + 4);
+  d->n_strips = (int)(P.strips.size() / 4);
+  d->n_rest = (int)(rest.size() / 4);
+  cudaError_t e;
+  if ((e = upload(P.dev, &d->ent)) != cudaSuccess) return e;
+  if ((e = upload(P.strips, &d->strips)) != cudaSuccess) return e;
+  if ((e = upload(P.b, &d->b)) != cudaSuccess) return e;
+  if ((e = upload(rest, &d->rest)) != cudaSuccess) return e;
+  d->ok = true;
+  return cudaSuccess;
+}
+
+void free_pk(DevPk* d) {
+  cudaFree(d->ent);
+  cudaFree(d->strips);
+  cudaFree(d->b);
+  cudaFree(d->rest);
+  *d = DevPk{};
+}
+
 struct disco_psi {
   disco::Geometry g;
   int device = -1;
@@ -123,6 +162,8 @@ struct disco_psi {
   bool tz_ok = false;                 // tensor-core contraction available (bf16 signals)
   disco::ToeplitzPlan tz, tza;        // forward (x -> y) and adjoint (dy -> dx) Toeplitz plans
   DevTz dtz, dtza;
+  disco::PackedPlan pf, pa;           // packed forms of the same (rows they serve)
+  DevPk dpf, dpa;
 };
 
 namespace {
@@ -298,9 +339,20 @@ disco_status launch_contract(const disco_psi* psi, int BC, disco_dtype dtype, co
   const disco::Geometry& g = psi->g;
   if (dtype == DISCO_BF16 && psi->tz_ok && !(reinterpret_cast<uintptr_t>(x) & 15) &&
       !(reinterpret_cast<uintptr_t>(y) & 15)) {
-    // Toeplitz blocks of Psi on tensor cores
+    // Toeplitz blocks of Psi on tensor cores: the packed kernel for the rows its plan serves,
+    // the per-pair kernel for the others (all rows without a packed plan)
     disco::TzLaunch L{psi->dtz.slabs, psi->dtz.row_begin, psi->dtz.slots, psi->dtz.b, psi->tz.K, psi->tz.parts,
                       psi->tz.N, BC, g.nlat_in, g.nlat_out, g.nlon_in};
+    if (psi->dpf.ok) {
+      const disco::PackedPlan& P = psi->pf;
+      disco::TpLaunch T{psi->dpf.ent, psi->dpf.strips, psi->dpf.b, P.K, P.T, P.NR, kPackKs,
+                        BC, g.nlat_in, g.nlat_out, g.nlon_in, psi->dpf.n_strips};
+      cudaError_t e = disco::launch_contract_tcp(T, x, y, st, 1 << 30);
+      if (e != cudaSuccess) return cuda_fail(e, what);
+      L.slots = psi->dpf.rest;
+      L.n_slots = psi->dpf.n_rest;
+      if (L.n_slots == 0) return DISCO_OK;
+    }
     cudaError_t e = disco::launch_contract_tc(L, x, y, st);
     if (e != cudaSuccess) return cuda_fail(e, what);
     return DISCO_OK;
@@ -353,6 +405,16 @@ disco_status launch_adjoint(const disco_psi* psi, int BC, disco_dtype dtype, con
     const disco::ToeplitzPlan& P = psi->tza;
     disco::TzLaunch T{psi->dtza.slabs, psi->dtza.row_begin, psi->dtza.slots, psi->dtza.b, P.K, P.parts, P.N,
                       BC, g.K * g.nlat_out, g.nlat_in, g.nlon_in};
+    if (psi->dpa.ok) {
+      const disco::PackedPlan& Q = psi->pa;
+      disco::TpLaunch L{psi->dpa.ent, psi->dpa.strips, psi->dpa.b, Q.K, Q.T, Q.NR, kPackKs,
+                        BC, g.K * g.nlat_out, g.nlat_in, g.nlon_in, psi->dpa.n_strips};
+      cudaError_t e = disco::launch_contract_tcp(L, dy, dx, st, 1 << 30);
+      if (e != cudaSuccess) return cuda_fail(e, "adjoint contraction launch");
+      T.slots = psi->dpa.rest;
+      T.n_slots = psi->dpa.n_rest;
+      if (T.n_slots == 0) return DISCO_OK;
+    }
     cudaError_t e = disco::launch_contract_tc(T, dy, dx, st);
     if (e != cudaSuccess) return cuda_fail(e, "adjoint contraction launch");
     return DISCO_OK;
@@ -393,7 +455,8 @@ unsigned long long disco_launch_count(void) { return disco::g_launches.load(); }
 disco_status disco_sync_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronisation");
-  if (disco::take_mix_tc_status() | disco::take_fused_tc_status() | disco::take_contract_tc_status())
+  if (disco::take_mix_tc_status() | disco::take_fused_tc_status() | disco::take_contract_tc_status() |
+      disco::take_contract_tcp_status())
     return fail(DISCO_ERR_TIMEOUT, "a bounded device-side wait expired");
   return DISCO_OK;
 }
@@ -470,6 +533,24 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
       e = upload_tz(h->tz, &h->dtz);
       if (e == cudaSuccess) e = upload_tz(h->tza, &h->dtza);
       h->tz_ok = e == cudaSuccess;
+      // Packed forms.  Measured on one B200, packing pays where an output row reaches many
+      // source rows (the K = 9 adjoint: about 63 (k, j) rows per output row); with fewer (the
+      // K = 3 layers: 5 forward, 15 adjoint) the per-pair kernels are faster, because staging,
+      // not the MMA count, bounds both.  So by default the adjoint is packed from kPackPairs
+      // slabs per output row on, the forward never; DISCO_PACKED=1 packs wherever a packed plan
+      // exists, DISCO_PACKED=0 never.
+      const char* pk = std::getenv("DISCO_PACKED");
+      const bool force = pk && pk[0] == '1', never = pk && pk[0] == '0';
+      int T, NR;
+      if (e == cudaSuccess && force && disco::packed_shape(g.K, false, &T, &NR)) {
+        h->pf = disco::make_packed_plan(g, h->entries, false, T, NR, kPackStrip, kPackKs);
+        if (!h->pf.strips.empty()) e = upload_pk(h->pf, h->tz, &h->dpf);
+      }
+      const bool dense_adj = h->tza.slabs.size() >= (size_t)kPackPairs * g.nlat_in;
+      if (e == cudaSuccess && !never && (force || dense_adj) && disco::packed_shape(1, true, &T, &NR)) {
+        h->pa = disco::make_packed_plan(g, h->entries, true, T, NR, kPackStrip, kPackKs);
+        if (!h->pa.strips.empty()) e = upload_pk(h->pa, h->tza, &h->dpa);
+      }
     }
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->fork, cudaEventDisableTiming);
@@ -482,6 +563,8 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
       free_plan(&h->dadjb);
       free_tz(&h->dtz);
       free_tz(&h->dtza);
+      free_pk(&h->dpf);
+      free_pk(&h->dpa);
       delete h;
       return fail(DISCO_ERR_ALLOC, std::string("Psi upload failed: ") + cudaGetErrorString(e));
     }
@@ -503,6 +586,8 @@ disco_status disco_psi_destroy(disco_psi* psi) {
     free_plan(&psi->dadjb);
     free_tz(&psi->dtz);
     free_tz(&psi->dtza);
+    free_pk(&psi->dpf);
+    free_pk(&psi->dpa);
     if (psi->side) cudaStreamDestroy(psi->side);
     if (psi->fork) cudaEventDestroy(psi->fork);
     if (psi->join) cudaEventDestroy(psi->join);

@@ -556,7 +556,7 @@ TzArgs base_args(const TzLaunch& L, const void* x, int QT) {
   a.n_lat_out = L.nlat_out;
   a.n_seg = (L.nlon + QT - 1) / QT;
   a.n_ctile = (L.BC + kCT - 1) / kCT;
-  a.n_tiles = L.nlat_out * a.n_seg * a.n_ctile;
+  a.n_tiles = (L.n_slots > 0 ? L.n_slots : L.nlat_out) * a.n_seg * a.n_ctile;
   return a;
 }
 

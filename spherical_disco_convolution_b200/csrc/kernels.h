@@ -53,11 +53,25 @@ struct TzLaunch {
   const void* b;         // expanded Psi blocks (bf16)
   int K, parts, N;
   int BC, nlat_in, nlat_out, nlon;
+  int n_slots = 0;       // row records to process (0: all nlat_out rows)
 };
 // Layers the Toeplitz plan serves (host-side geometry only) / that the device can run.
 bool toeplitz_geometry(int K, int stride, int nlon_in, int nlon_out);
 bool contract_tc_supported(int K, int stride, int nlon_in, int nlon_out);
 cudaError_t launch_contract_tc(const TzLaunch& L, const void* x, void* y, cudaStream_t st);
+// Packed form (contract_tcp.cu): a source row staged once per tile and applied to all the
+// output rows it reaches in one MMA; the rows of a packed plan only (make_packed_plan).
+struct TpLaunch {
+  const int* ent;      // 8 ints per entry (PackedPlan::dev)
+  const int* strips;   // 4 ints per strip
+  const void* b;       // packed blocks (bf16)
+  int K, T, NR, ksmax;
+  int BC, n_src_rows, n_out_rows, nlon, n_strips;
+};
+bool packed_shape(int K, bool adjoint, int* T, int* NR);
+cudaError_t launch_contract_tcp(const TpLaunch& L, const void* x, void* y, cudaStream_t st, int grid_cap);
+int take_contract_tcp_status();
+
 // Fused forward on the same plan: out = bias + mix(w, contraction(x)) with the y tile kept in
 // shared memory; for K = 3 or 5 and 64 input channels per group (bf16, stride 1).
 struct TzFused {

@@ -152,7 +152,7 @@ struct DwTcArgs {
   int G, Og, Rg, N, nc, nchunk;
 };
 
-__global__ void __launch_bounds__(128, 1) dw_tc_kernel(const __grid_constant__ CUtensorMap map_y,
+__global__ void __launch_bounds__(128, 2) dw_tc_kernel(const __grid_constant__ CUtensorMap map_y,
                                                        const __grid_constant__ CUtensorMap map_d, DwTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
