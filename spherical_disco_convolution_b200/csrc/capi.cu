@@ -515,6 +515,11 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
     // host-only handle: the Toeplitz plans are built for inspection (disco_toeplitz_export)
     h->tz = disco::make_toeplitz_plan(g, h->entries);
     h->tza = disco::make_adjoint_toeplitz_plan(g, h->entries);
+    int T, NR;
+    if (disco::packed_shape(g.K, false, &T, &NR))
+      h->pf = disco::make_packed_plan(g, h->entries, false, T, NR, kPackStrip, kPackKs);
+    if (disco::packed_shape(1, true, &T, &NR))
+      h->pa = disco::make_packed_plan(g, h->entries, true, T, NR, kPackStrip, kPackKs);
   }
   if (device >= 0) {
     int prev = -1;
@@ -668,6 +673,34 @@ disco_status disco_toeplitz_export(const disco_psi* psi, int which, int* slabs, 
   std::memcpy(slabs, P.slabs.data(), P.slabs.size() * sizeof(disco::TzSlab));
   std::memcpy(slots, P.slots.data(), P.slots.size() * sizeof(int));
   std::memcpy(b, P.b.data(), P.b.size() * sizeof(uint16_t));
+  return DISCO_OK;
+}
+
+disco_status disco_packed_info(const disco_psi* psi, int which, int* dims) {
+  if (!psi || !dims || which < 0 || which > 1) return fail(DISCO_ERR_INVALID_ARG, "bad packed plan query");
+  const disco::PackedPlan& P = which == 0 ? psi->pf : psi->pa;
+  if (P.Nr == 0) return fail(DISCO_ERR_UNSUPPORTED, "no packed plan for this layer");
+  dims[0] = P.K;
+  dims[1] = P.Nr;
+  dims[2] = P.NR;
+  dims[3] = P.T;
+  dims[4] = (int)(P.strips.size() / 4);
+  dims[5] = (int)P.entries.size();
+  dims[6] = (int)P.b.size();
+  dims[7] = (int)P.rest.size();
+  return DISCO_OK;
+}
+
+disco_status disco_packed_export(const disco_psi* psi, int which, int* strips, int* entries, unsigned short* b,
+                                 int* rest) {
+  if (!psi || !strips || !entries || !b || !rest || which < 0 || which > 1)
+    return fail(DISCO_ERR_INVALID_ARG, "bad packed plan export");
+  const disco::PackedPlan& P = which == 0 ? psi->pf : psi->pa;
+  if (P.Nr == 0) return fail(DISCO_ERR_UNSUPPORTED, "no packed plan for this layer");
+  std::memcpy(strips, P.strips.data(), P.strips.size() * sizeof(int));
+  std::memcpy(entries, P.dev.data(), P.dev.size() * sizeof(int));
+  std::memcpy(b, P.b.data(), P.b.size() * sizeof(uint16_t));
+  std::memcpy(rest, P.rest.data(), P.rest.size() * sizeof(int));
   return DISCO_OK;
 }
 

@@ -102,6 +102,8 @@ def _load():
         "disco_plan_export": [P, I, IP, IP, IP, ctypes.POINTER(ctypes.c_float), IP],
         "disco_toeplitz_info": [P, I, IP],
         "disco_toeplitz_export": [P, I, IP, IP, ctypes.POINTER(ctypes.c_ushort)],
+        "disco_packed_info": [P, I, IP],
+        "disco_packed_export": [P, I, IP, IP, ctypes.POINTER(ctypes.c_ushort), IP],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -202,6 +204,21 @@ def disco_toeplitz_export(psi, which: int):
     _check(_lib.disco_toeplitz_export(psi, which, ip(slabs), ip(slots),
                                       b.ctypes.data_as(ctypes.POINTER(ctypes.c_ushort))))
     return dict(K=K, parts=parts, N=N, slabs=slabs, slots=slots, b=b, kslab=kslab, ksteps=ksteps)
+
+
+def disco_packed_export(psi, which: int):
+    """Packed Toeplitz plan: which=0 forward, which=1 adjoint."""
+    dims = np.zeros(8, dtype=np.int32)
+    _check(_lib.disco_packed_info(psi, which, dims.ctypes.data_as(ctypes.POINTER(ctypes.c_int))))
+    K, Nr, NR, T, n_strips, n_ent, n_b, n_rest = (int(v) for v in dims)
+    strips = np.zeros((n_strips, 4), dtype=np.int32)
+    ent = np.zeros((n_ent, 8), dtype=np.int32)
+    b = np.zeros(n_b, dtype=np.uint16)
+    rest = np.zeros(max(n_rest, 1), dtype=np.int32)
+    ip = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))  # noqa: E731
+    _check(_lib.disco_packed_export(psi, which, ip(strips), ip(ent), b.ctypes.data_as(ctypes.POINTER(ctypes.c_ushort)),
+                                    ip(rest)))
+    return dict(K=K, Nr=Nr, NR=NR, T=T, strips=strips, entries=ent, b=b, rest=rest[:n_rest])
 
 
 def disco_workspace_size(psi, op, B, C_in, C_out, groups, dtype) -> int:
