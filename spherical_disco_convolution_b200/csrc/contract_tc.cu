@@ -50,7 +50,7 @@ namespace {
 
 constexpr int kCT = 64;                       // channels per tile
 constexpr uint32_t kOctBytes = kCT * 16;      // one staged octet: 64 channels x 8 bf16
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;  // producer, MMA issuer, four epilogue warps, second MMA issuer
 constexpr uint32_t kTmemCols = 512;
 constexpr int kStages = 4;
 constexpr int kMaxSlabs = 24;                 // slab table entries per stage
@@ -140,10 +140,10 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tc_kernel(const __grid_c
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(&full[s], 33);  // 32 producer lanes' copy completions + the closing arrival
-      tc::mbar_init(&empty[s], 1);
+      tc::mbar_init(&empty[s], 2);  // both MMA issuers commit
     }
     for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(&tfull[b], 1);
+      tc::mbar_init(&tfull[b], 2);
       tc::mbar_init(&tempty[b], 4);
     }
     tc::mbar_init(yfull, 1);
@@ -273,9 +273,13 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tc_kernel(const __grid_c
     }
     // no copy may still be in flight when the CTA exits
     tc::cp_async_wait_all();
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 6) {
     if (lane == 0) {
-      // ---------------------------------------------------------------- MMA issuer
+      // ---------------------------------------------------------------- MMA issuers
+      // two threads issue the contraction's MMAs, the even and the odd groups of 16 outputs
+      // (disjoint accumulator columns), which halves each one's issue overhead; the first
+      // also runs the fused mode's channel mix
+      const int gsel = warp == 1 ? 0 : 1;
       constexpr uint32_t idesc = tc::idesc_bf16(128, N, false, false);
       // descriptors differ only in their 14-bit start-address field (address >> 4, below
       // 256 KB, so adding to it never carries into the other fields)
@@ -318,8 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tc_kernel(const __grid_c
 #pragma unroll
               for (int part = 0; part < PARTS; ++part) {
                 const uint64_t bd0 = b_fix | (uint64_t)(sbase4 + (uint32_t)e1 + (uint32_t)(part * nk) * b_step);
-#pragma unroll
-                for (int g = 0; g < T; ++g) {
+                for (int g = gsel; g < T; g += 2) {
                   uint64_t ad = a_fix | (uint64_t)(sbase4 + (uint32_t)(e0 >> 8) + (uint32_t)g * a_step);
                   uint64_t bd = bd0;
                   const uint32_t d = d0 + (uint32_t)(g * N);
@@ -339,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tc_kernel(const __grid_c
           if (!ok) break;
           tc::mma_commit(&tfull[buf]);
         }
-        if (FUSED && ok) {
+        if (FUSED && ok && gsel == 0) {
           // ------------------------------------------------ channel mix of the tile
           const int ct = tile % a.n_ctile, g = ct % a.G;
           if (g != wg) {  // stage w of this group (after the previous mix has read the old one)
