@@ -52,7 +52,7 @@ constexpr int kCT = 64;                       // channels per tile
 constexpr uint32_t kOctBytes = kCT * 16;      // one staged octet: 64 channels x 8 bf16
 constexpr int kThreads = 224;  // producer, MMA issuer, four epilogue warps, second MMA issuer
 constexpr uint32_t kTmemCols = 512;
-constexpr int kStages = 4;
+constexpr int kStages = 4;                    // most stages (barriers are laid out for this many)
 constexpr int kMaxSlabs = 24;                 // slab table entries per stage
 constexpr int kBars = 2 * kStages + 8;        // full/empty per stage, tfull/tempty x2, yfull, d2full, d2empty, w
 
@@ -65,6 +65,7 @@ struct TzArgs {
   int n_lat_in, n_lon, n_lat_out;
   int n_seg, n_ctile, n_tiles;
   uint32_t stage_bytes;
+  int n_stages;        // stages of this launch (at most kStages)
   uint32_t r0_bytes;   // output staging tile (contraction) or y tile (fused)
   uint32_t w_bytes;    // fused: staged w of one group
   // fused forward
@@ -83,7 +84,10 @@ template <int K, int PARTS, bool FUSED>
 struct TzShape {
   static constexpr int N = PARTS == 1 ? 16 * K : (8 * K + 15) / 16 * 16;
   static constexpr int T = FUSED ? 4 : ((256 / N) < 8 ? 256 / N : 8);
-  static constexpr int NH = FUSED ? 2 : 1;               // contraction halves per tile
+  // fused: two contraction halves of 64 outputs (y tile of 128 rows) for K <= 5; one half
+  // for larger K, whose 128-row y tile would not fit shared memory (the mix then runs on
+  // M = 128 with its upper 64 rows discarded)
+  static constexpr int NH = FUSED ? (K <= 5 ? 2 : 1) : 1;
   static constexpr int QT = 16 * T * NH;                 // outputs per tile
   static constexpr int NB = FUSED ? (2 * T * N + 64 <= 512 ? 2 : 1) : 2;  // accumulator buffers
 };
@@ -121,8 +125,9 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tc_kernel(const __grid_c
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sR0 = smem;                 // output staging tile / y tile
   uint8_t* sW = smem + a.r0_bytes;     // fused: w of the current group
-  uint8_t* sS = sW + a.w_bytes;        // kStages stages of stage_bytes
-  uint64_t* full = reinterpret_cast<uint64_t*>(sS + (size_t)kStages * a.stage_bytes);
+  uint8_t* sS = sW + a.w_bytes;        // n_stages stages of stage_bytes
+  const int S = a.n_stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sS + (size_t)S * a.stage_bytes);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;  // [2] contraction accumulator ready for the epilogue
   uint64_t* tempty = tfull + 2;       // [2] contraction accumulator drained by the epilogue
@@ -171,12 +176,12 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tc_kernel(const __grid_c
     uint32_t used = 0;                            // bytes of the open stage
     // opens stage n: waits until the MMAs of its previous use are done
     auto open = [&]() -> bool {
-      st = (int)(n % kStages);
+      st = (int)(n % S);
       cnt = 0;
       used = 0;
-      if (n >= (uint32_t)kStages) {
+      if (n >= (uint32_t)S) {
         int good = 1;
-        if (lane == 0) good = tc::mbar_wait(&empty[st], ((n / kStages) & 1) ^ 1);
+        if (lane == 0) good = tc::mbar_wait(&empty[st], ((n / S) & 1) ^ 1);
         if (!__shfl_sync(0xffffffffu, good, 0)) return false;
         __syncwarp();  // order every lane's copies after lane 0's wait
       }
@@ -303,8 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tc_kernel(const __grid_c
           tc::fence_after_sync();
           const uint32_t d0 = tmem + (uint32_t)buf * TN;
           while (true) {
-            const int st = (int)(n % kStages);
-            if (!tc::mbar_wait(&full[st], (n / kStages) & 1)) {
+            const int st = (int)(n % S);
+            if (!tc::mbar_wait(&full[st], (n / S) & 1)) {
               ok = false;
               break;
             }
@@ -505,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tc_kernel(const __grid_c
       for (int o0 = 0; o0 < a.Og; o0 += 16) {
         float v[16];
         tc::tmem_ld16(d2 + (uint32_t)o0, v);
-        if (q < a.n_lon) {
+        if (m < QT && q < a.n_lon) {  // rows beyond the tile's outputs (one-half tiles) are discarded
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int oc = g * a.Og + o0 + i;
@@ -586,6 +591,7 @@ cudaError_t launch_tz(const TzLaunch& L, const void* x, void* y, cudaStream_t st
   if (!tc::encode_bf16_map(&ym, y, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE)) return cudaErrorInvalidValue;
   TzArgs a = base_args(L, x, Sh::QT);
   a.stage_bytes = stage;
+  a.n_stages = kStages;
   a.r0_bytes = out_bytes;
   a.w_bytes = 0;
   return launch_common(reinterpret_cast<const void*>(&contract_tc_kernel<K, PARTS, false>), a, ym, wm, smem, st);
@@ -595,6 +601,7 @@ cudaError_t launch_tz(const TzLaunch& L, const void* x, void* y, cudaStream_t st
 // the layer does not fit (tensor memory or shared memory).
 struct FusedLayout {
   uint32_t a_sbo, r0, w_bytes, stage;
+  int stages;
   size_t smem;
 };
 
@@ -606,14 +613,21 @@ bool fused_layout(int Og, FusedLayout* f) {
   const int R = kCT * K;
   const size_t extra = tz_extra();
   f->a_sbo = (uint32_t)(R * 16 + 16);
-  f->r0 = (16 * f->a_sbo + 1023u) & ~1023u;
   f->w_bytes = (uint32_t)(K * Og * 128);  // R / 64 = K chunks of [Og][64]
+  // the mix reads 16 blocks of 8 outputs: a one-half tile writes 8 of them and the other 8
+  // must still lie inside shared memory (they read into the staged w, and are discarded)
+  const uint32_t blocks = (uint32_t)(Sh::NH * 8);
+  f->r0 = (blocks * f->a_sbo + 1023u) & ~1023u;
+  if (16 * f->a_sbo > f->r0 + f->w_bytes) f->r0 = (16 * f->a_sbo - f->w_bytes + 1023u) & ~1023u;
   if (f->r0 + f->w_bytes + extra >= kTcSmemLimit) return false;
-  f->stage = (uint32_t)((kTcSmemLimit - extra - f->r0 - f->w_bytes) / kStages) & ~1023u;
   const uint32_t max_slab =
       (uint32_t)(2 * T + 2 * kTzSlabK - 1) * kOctBytes + (uint32_t)(PARTS * 2 * kTzSlabK * N * 16);
-  if (max_slab > f->stage) return false;  // the largest slab must fit one stage
-  f->smem = (size_t)f->r0 + f->w_bytes + (size_t)kStages * f->stage + extra;
+  for (f->stages = kStages; f->stages >= 2; --f->stages) {
+    f->stage = (uint32_t)((kTcSmemLimit - extra - f->r0 - f->w_bytes) / f->stages) & ~1023u;
+    if (max_slab <= f->stage) break;  // the largest slab must fit one stage
+  }
+  if (f->stages < 2) return false;
+  f->smem = (size_t)f->r0 + f->w_bytes + (size_t)f->stages * f->stage + extra;
   return true;
 }
 
@@ -637,6 +651,7 @@ cudaError_t launch_tz_fused(const TzLaunch& L, const TzFused& F, cudaStream_t st
   if (!tc::encode_bf16_map(&wm, F.w, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
   TzArgs a = base_args(L, F.x, Sh::QT);
   a.stage_bytes = stage;
+  a.n_stages = fl.stages;
   a.r0_bytes = r0;
   a.w_bytes = w_bytes;
   a.out = static_cast<__nv_bfloat16*>(F.out);
@@ -679,6 +694,7 @@ bool fused_tz_supported(int K, int C_in, int C_out, int G) {
   FusedLayout f;
   if (K == 3) return fused_layout<3, 1>(C_out / G, &f);
   if (K == 5) return fused_layout<5, 1>(C_out / G, &f);
+  if (K == 9) return fused_layout<9, 2>(C_out / G, &f);
   return false;
 }
 
@@ -687,6 +703,7 @@ cudaError_t launch_fused_tz(const TzLaunch& L, const TzFused& F, cudaStream_t st
   switch (L.K) {
     case 3: return launch_tz_fused<3, 1>(L, F, st);
     case 5: return launch_tz_fused<5, 1>(L, F, st);
+    case 9: return launch_tz_fused<9, 2>(L, F, st);
     default: return cudaErrorInvalidValue;
   }
 }

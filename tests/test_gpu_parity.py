@@ -43,6 +43,8 @@ EDGE = {
     # cutoff of two grid spacings, as on the 721x1440 layer: the packed tensor-core kernels take
     # most rows (the polar rows stay per pair); 70 channels leave a partial second channel tile
     "packed_k3": Workload("packed_k3", 1, 70, 64, 1, 65, 128, 65, 128, (3, 1), 2 * math.pi / 64, "bf16"),
+    # fused tensor-core forward with K = 9: one-half tiles of 64 outputs (ragged last tile)
+    "tz_fused_k9": Workload("tz_fused_k9", 1, 128, 96, 2, 21, 160, 21, 160, (3, 4), 0.5, "bf16"),
 }
 
 
@@ -245,7 +247,7 @@ def test_adjoint_tensor_core_matches_gather(name, monkeypatch):
     check(host(dx_tc), host(dx_g), 8e-3, "dx (tensor cores vs gather)")
 
 
-@pytest.mark.parametrize("name", ["tz_fused_k3", "tz_fused_k5", "weather"])
+@pytest.mark.parametrize("name", ["tz_fused_k3", "tz_fused_k5", "tz_fused_k9", "weather", "grouped"])
 def test_fused_tensor_core_matches_unfused(name):
     """The fused forward (Toeplitz contraction and channel mix on tensor cores, y tile on chip)
     against the unfused path, which rounds the same y to bf16 before the same mix."""
