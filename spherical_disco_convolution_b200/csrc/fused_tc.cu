@@ -163,31 +163,14 @@ size_t fused_tc_smem(const FusedTcArgs& f, int K) {
   return n + (size_t)f.w_chunks * Og * 128 + 64 + 1024;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
 template <int K, int S>
 cudaError_t launch_t(const FusedTcArgs& f, const void* w, cudaStream_t st) {
-  static EncodeTiledFn enc = nullptr;
-  if (!enc) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return cudaErrorNotSupported;
-    enc = reinterpret_cast<EncodeTiledFn>(p);
-  }
   const int Og = f.C_out / f.G, R = (f.C_in / f.G) * K;
   CUtensorMap mw;
   const cuuint64_t dims[2] = {(cuuint64_t)R, (cuuint64_t)f.C_out};
   const cuuint64_t strides[1] = {(cuuint64_t)R * 2};
   const cuuint32_t box[2] = {64, (cuuint32_t)Og};
-  const cuuint32_t es[2] = {1, 1};
-  if (enc(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), dims, strides, box, es,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+  if (!tc::encode_bf16_map(&mw, w, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
   auto kern = fused_tc_kernel<K, S>;
   const size_t smem = fused_tc_smem(f, K);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -264,31 +264,10 @@ __global__ void __launch_bounds__(256) bias_partial_kernel(const __nv_bfloat16* 
 
 // ------------------------------------------------------------------- host
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
 // bf16 tensor map with 128-byte swizzle; dims innermost first, strides in bytes for dims 1..
 bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
               const cuuint32_t* box) {
-  EncodeTiledFn f = encode_fn();
-  if (!f) return false;
-  cuuint32_t es[3] = {1, 1, 1};
-  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, es,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return tc::encode_bf16_map(m, base, rank, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 size_t mix_smem(int BN, int S) { return 1024 + S * (2 * kHalfTile + (size_t)BN * 128) + (2 * S + 2) * 8; }
@@ -304,7 +283,7 @@ int mix_bn(int Mg) {
 }  // namespace
 
 bool mix_tc_supported(int Mg, int Rg, int N) {
-  return encode_fn() != nullptr && Mg % 16 == 0 && Rg % 8 == 0 && N % 8 == 0 && (mix_bn(Mg) % 16 == 0);
+  return tc::encode_tiled_fn() != nullptr && Mg % 16 == 0 && Rg % 8 == 0 && N % 8 == 0 && (mix_bn(Mg) % 16 == 0);
 }
 
 cudaError_t launch_mix_tc(const MixArgs& a, cudaStream_t st) {
@@ -329,7 +308,7 @@ cudaError_t launch_mix_tc(const MixArgs& a, cudaStream_t st) {
 }
 
 bool dw_tc_supported(int Og, int Rg, int N) {
-  return encode_fn() != nullptr && Og % 16 == 0 && Og <= 256 && N % 8 == 0 && Rg >= 1;
+  return tc::encode_tiled_fn() != nullptr && Og % 16 == 0 && Og <= 256 && N % 8 == 0 && Rg >= 1;
 }
 
 cudaError_t launch_dw_tc(const DwArgs& a, cudaStream_t st) {
