@@ -18,17 +18,19 @@
 //     buffer); the hi and lo parts of Psi either sit side by side in N (N = 16K, summed in the
 //     epilogue) or are two MMAs into the same columns (N = 8K rounded up to 16, K > 8).
 //
-// Persistent CTAs, 6 warps.  Warp 0 (all lanes) fills a ring of stages, each holding as many
-// (source row, window slab) pairs of one tile as fit: the x windows by 16-byte cp.async copies
-// (lanes cover 4 octets x 8 channels, so global reads are 64-byte runs and shared writes
-// 128-byte rows), each Psi slab by one bulk copy, and a table of slab offsets for the MMA
-// issuer.  Each lane's copies arrive on the stage's barrier by themselves when they land
-// (cp.async.mbarrier.arrive.noinc), so the producer never waits for its own copies; the MMA
-// issuer orders them before its tensor-core reads with a generic-to-async proxy fence after the
-// barrier wait.  Warp 1 lane 0 issues the MMAs;
-// warps 2..5 read the accumulator of the previous tile back (each warp its TMEM lane quadrant)
-// into a [64 channels][K][16T] bf16 tile in shared memory that one TMA store writes to y.  Every wait is bounded (tc_common.cuh): on expiry the kernel records the timeout
-// and stops.
+// Persistent CTAs, 10 warps.  Four producer warps (0, 7, 8, 9) fill a ring of stages, each
+// holding as many (source row, window slab) pairs of one tile as fit: the x windows by 16-byte
+// cp.async copies (lanes cover 4 octets x 8 channels, so global reads are 64-byte runs and
+// shared writes 128-byte rows; each warp copies 2 of the 8 channel groups, since one warp alone
+// cannot issue copies fast enough), each Psi slab by one bulk copy, and a table of slab offsets
+// for the MMA issuers.  Each lane's copies arrive on the stage's barrier by themselves when they
+// land (cp.async.mbarrier.arrive.noinc), so no producer waits for its own copies; the MMA
+// issuers order them before their tensor-core reads with a generic-to-async proxy fence after
+// the barrier wait.  Lane 0 of warps 1 and 6 issues the MMAs (even and odd groups of 16
+// outputs); warps 2..5 read the accumulator of the previous tile back (each warp its TMEM lane
+// quadrant) into a [64 channels][K][16T] bf16 tile in shared memory that one TMA store writes
+// to y.  Every wait is bounded (tc_common.cuh): on expiry the kernel records the timeout and
+// stops.
 //
 // Fused forward (FUSED): a tile is 128 outputs of one output row for the 64 input channels of
 // one (batch, group), contracted as two halves of 64 outputs.  The epilogue warps round each
@@ -50,7 +52,8 @@ namespace {
 
 constexpr int kCT = 64;                       // channels per tile
 constexpr uint32_t kOctBytes = kCT * 16;      // one staged octet: 64 channels x 8 bf16
-constexpr int kThreads = 224;  // producer, MMA issuer, four epilogue warps, second MMA issuer
+constexpr int kProducers = 4;  // copy warps: 0 and 7..6+kProducers-1
+constexpr int kThreads = 32 * (6 + kProducers);  // producer, MMA issuer, four epilogue warps, MMA issuer, producers
 constexpr uint32_t kTmemCols = 512;
 constexpr int kStages = 4;                    // most stages (barriers are laid out for this many)
 constexpr int kMaxSlabs = 24;                 // slab table entries per stage
@@ -144,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tc_kernel(const __grid_c
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      tc::mbar_init(&full[s], 33);  // 32 producer lanes' copy completions + the closing arrival
+      tc::mbar_init(&full[s], 32 * kProducers + 1);  // every producer lane's copy completions + the closing arrival
       tc::mbar_init(&empty[s], 2);  // both MMA issuers commit
     }
     for (int b = 0; b < 2; ++b) {
@@ -166,8 +169,13 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tc_kernel(const __grid_c
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ---------------------------------------------------------------- producer warp
+  if (warp == 0 || warp >= 7) {
+    // ---------------------------------------------------------------- producer warps
+    // kProducers warps run the same stage packing (so they agree on every stage and offset)
+    // and each copies its share of the 8 channel groups; the first also writes the stage
+    // tables, issues the bulk copies and closes the stages.
+    constexpr int CG = 8 / kProducers;
+    const int pw = warp == 0 ? 0 : warp - 6;
     const size_t chan = (size_t)a.n_lat_in * a.n_lon;
     const int csub = lane >> 2, osub = lane & 3;  // channel within 8, octet within 4
     uint32_t n = 0;                               // stages opened so far
@@ -189,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tc_kernel(const __grid_c
     };
     // closes stage n: every lane's copies arrive on its barrier when they have landed
     auto close = [&](int flags) {
-      if (lane == 0) {
+      if (lane == 0 && pw == 0) {
         meta[st * kMetaWords] = cnt | flags;
         tc::mbar_arrive(&full[st]);
       }
@@ -241,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tc_kernel(const __grid_c
             if (!(ok = open())) break;
           }
           uint8_t* base = sS + (size_t)st * a.stage_bytes;
-          if (lane == 0) {
+          if (lane == 0 && pw == 0) {
             meta[st * kMetaWords + 1 + 2 * cnt] = nk | (int)(used >> 4) << 8;
             meta[st * kMetaWords + 2 + 2 * cnt] = (int)((used + xbytes) >> 4);
             if (nk) {
@@ -260,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tc_kernel(const __grid_c
               const __nv_bfloat16* src = xrow + oo * 8;
               uint8_t* d = dst + o * kOctBytes;
 #pragma unroll
-              for (int cg = 0; cg < 8; ++cg) {
+              for (int cg = pw * CG; cg < pw * CG + CG; ++cg) {
                 const bool v = (cmask >> cg) & 1u;
                 tc::cp_async16(d + cg * 128, v ? src + (size_t)cg * 8 * chan : a.x, v ? 16u : 0u);
               }
