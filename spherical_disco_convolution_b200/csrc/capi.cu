@@ -82,7 +82,6 @@ void free_plan(DevPlan* d) {
 constexpr int kChannelsPerCta = 16;
 constexpr int kPackStrip = 32;  // output rows per strip of a packed plan
 constexpr int kPackKs = 4;      // widest window (K-steps of 16 longitudes) a packed entry takes
-constexpr int kPackPairs = 24;  // slabs per output row from which the adjoint is packed
 constexpr int kStageFloats = 12288;          // 48 KB of staging for the unfused gathers
 constexpr size_t kSmemLimit = 227 * 1024;    // dynamic shared memory per CTA on sm_100
 constexpr size_t kFusedTileBytes = 160 * 1024;
@@ -538,21 +537,18 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
       e = upload_tz(h->tz, &h->dtz);
       if (e == cudaSuccess) e = upload_tz(h->tza, &h->dtza);
       h->tz_ok = e == cudaSuccess;
-      // Packed forms.  Measured on one B200, packing pays where an output row reaches many
-      // source rows (the K = 9 adjoint: about 63 (k, j) rows per output row); with fewer (the
-      // K = 3 layers: 5 forward, 15 adjoint) the per-pair kernels are faster, because staging,
-      // not the MMA count, bounds both.  So by default the adjoint is packed from kPackPairs
-      // slabs per output row on, the forward never; DISCO_PACKED=1 packs wherever a packed plan
-      // exists, DISCO_PACKED=0 never.
+      // Packed forms (one staged source row feeds up to 16 output rows).  Measured on one
+      // B200 with four producer warps, the per-pair kernels are faster on every layer tried,
+      // the K = 9 adjoint included (about 63 (k, j) rows per output row), because staging,
+      // not the MMA count, bounds both.  So the packed kernels run only when DISCO_PACKED=1.
       const char* pk = std::getenv("DISCO_PACKED");
-      const bool force = pk && pk[0] == '1', never = pk && pk[0] == '0';
+      const bool force = pk && pk[0] == '1';
       int T, NR;
       if (e == cudaSuccess && force && disco::packed_shape(g.K, false, &T, &NR)) {
         h->pf = disco::make_packed_plan(g, h->entries, false, T, NR, kPackStrip, kPackKs);
         if (!h->pf.strips.empty()) e = upload_pk(h->pf, h->tz, &h->dpf);
       }
-      const bool dense_adj = h->tza.slabs.size() >= (size_t)kPackPairs * g.nlat_in;
-      if (e == cudaSuccess && !never && (force || dense_adj) && disco::packed_shape(1, true, &T, &NR)) {
+      if (e == cudaSuccess && force && disco::packed_shape(1, true, &T, &NR)) {
         h->pa = disco::make_packed_plan(g, h->entries, true, T, NR, kPackStrip, kPackKs);
         if (!h->pa.strips.empty()) e = upload_pk(h->pa, h->tza, &h->dpa);
       }

@@ -9,8 +9,9 @@
 // accumulates in one of NR tensor-memory slots (slot = strip-relative row mod NR, T groups of
 // 16 outputs apart by NR*Nr columns) from its first source row to its last.
 //
-// Roles as in contract_tc.cu (6 warps, persistent CTAs): warp 0 stages entries (x window by
-// cp.async with copy-completion arrivals, the packed block by one bulk copy); warp 1 lane 0
+// Roles as in contract_tc.cu (persistent CTAs): warps 0 and 6.. stage entries (the x window by
+// cp.async with copy-completion arrivals, each warp a share of the channels; the packed block
+// by one bulk copy from warp 0); warp 1 lane 0
 // waits until a slot's previous row is drained before the first contribution of a new row,
 // issues the MMAs (split in two where the slot range wraps) and commits a "row complete"
 // barrier per finished row; warps 2..5 drain finished rows (TMEM -> bf16 -> shared tile -> TMA
@@ -30,7 +31,8 @@ namespace {
 
 constexpr int kCT = 64;
 constexpr uint32_t kOctBytes = kCT * 16;
-constexpr int kThreads = 192;
+constexpr int kProducers = 4;  // copy warps: 0 and 6..4+kProducers
+constexpr int kThreads = 32 * (5 + kProducers);  // producers, MMA issuer, four epilogue warps
 constexpr uint32_t kTmemCols = 512;
 constexpr int kStages = 4;
 constexpr int kMaxEnt = 24;
@@ -88,7 +90,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tcp_kernel(const __grid_
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      tc::mbar_init(&full[s], 33);
+      tc::mbar_init(&full[s], 32 * kProducers + 1);
       tc::mbar_init(&empty[s], 1);
     }
     for (int s = 0; s < NR; ++s) {
@@ -105,7 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tcp_kernel(const __grid_
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  if (warp >= 2) {  // every slot starts at zero
+  if (warp >= 2 && warp <= 5) {  // every slot starts at zero
     const uint32_t lb = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     for (uint32_t c = 0; c < kTmemCols; c += 16) tc::tmem_st16_zero(lb + c);
     tc::tmem_wait_st();
@@ -114,8 +116,12 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tcp_kernel(const __grid_
   __syncthreads();
   tc::fence_after_sync();
 
-  if (warp == 0) {
-    // ---------------------------------------------------------------- producer warp
+  if (warp == 0 || warp >= 6) {
+    // ---------------------------------------------------------------- producer warps
+    // kProducers warps run the same stage packing and each copies its share of the 8 channel
+    // groups; the first also writes the stage tables, issues the bulk copies and closes stages.
+    constexpr int CG = 8 / kProducers;
+    const int pw = warp == 0 ? 0 : warp - 5;
     const size_t chan = (size_t)a.n_src_rows * a.n_lon;
     const int csub = lane >> 2, osub = lane & 3;
     uint32_t n = 0;
@@ -135,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tcp_kernel(const __grid_
       return true;
     };
     auto close = [&](int flags) {
-      if (lane == 0) {
+      if (lane == 0 && pw == 0) {
         meta[st * kMetaWords] = cnt | flags;
         tc::mbar_arrive(&full[st]);
       }
@@ -171,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tcp_kernel(const __grid_
           if (!(ok = open())) break;
         }
         uint8_t* base = sS + (size_t)st * a.stage_bytes;
-        if (lane == 0) {
+        if (lane == 0 && pw == 0) {
           int* m = meta + st * kMetaWords + 1 + kEntWords * cnt;
           m[0] = w2;
           m[1] = newm;
@@ -191,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tcp_kernel(const __grid_
           const __nv_bfloat16* src = xrow + oo * 8;
           uint8_t* d = dst + o * kOctBytes;
 #pragma unroll
-          for (int cg = 0; cg < 8; ++cg) {
+          for (int cg = pw * CG; cg < pw * CG + CG; ++cg) {
             const bool v = (cmask >> cg) & 1u;
             tc::cp_async16(d + cg * 128, v ? src + (size_t)cg * 8 * chan : a.x, v ? 16u : 0u);
           }
@@ -280,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tcp_kernel(const __grid_
         }
       }
     }
-  } else {
+  } else if (warp <= 5) {
     // ---------------------------------------------------------------- epilogue warps
     const int quad = warp & 3;
     const int m = quad * 32 + lane;
