@@ -65,7 +65,22 @@ typedef enum {
 
 typedef enum { DISCO_F32 = 0, DISCO_BF16 = 1 } disco_dtype;
 
-enum { DISCO_GRID_EQUIANGULAR = 0 };           /* theta_i = pi*i/(nlat-1), poles included */
+/* Latitude grids (grid_in / grid_out).  The DISCO constructor takes grid_in / grid_out (page
+ * "torch_harmonics.DiscreteContinuousConvS2", signature; default "equiangular"); the four
+ * names are listed with the same parameters on the page of the module
+ * "torch_harmonics.distributed.distributed_spectral_convolution" (class docstring,
+ * Parameters).  Neither page defines them; they are read as the textbook rules on
+ * t = cos(theta).  Nodes run north to south and the quadrature weights sum to 2 (times
+ * 2*pi/nlon_in per point). */
+enum {
+  DISCO_GRID_EQUIANGULAR = 0,             /* theta_i = pi*i/(nlat-1), poles included;
+                                             Clenshaw-Curtis weights */
+  DISCO_GRID_LEGENDRE_GAUSS = 1,          /* the nlat Gauss-Legendre nodes and weights; no poles */
+  DISCO_GRID_LOBATTO = 2,                 /* the nlat Gauss-Lobatto-Legendre nodes (poles
+                                             included) and weights; nlat >= 2 */
+  DISCO_GRID_EQUIANGULAR_TRAPEZOIDAL = 3  /* equiangular nodes, trapezoidal weights in t:
+                                             w_i = (t_{i-1} - t_{i+1}) / 2, ends one-sided */
+};
 enum { DISCO_BASIS_PIECEWISE_LINEAR = 0 };
 enum { DISCO_NORM_NODAL = 0 };                 /* every (k, j) row of Psi sums to one */
 
@@ -89,7 +104,7 @@ enum {
  * no default cutoff, so theta_cutoff is required. */
 typedef struct {
   int nlat_in, nlon_in, nlat_out, nlon_out;
-  int grid_in, grid_out;      /* DISCO_GRID_EQUIANGULAR only */
+  int grid_in, grid_out;      /* DISCO_GRID_* (any of the four) */
   int kernel_shape[2];        /* {n_r, n_alpha} */
   int basis_type;             /* DISCO_BASIS_PIECEWISE_LINEAR only */
   int basis_norm_mode;        /* DISCO_NORM_NODAL only */

@@ -44,6 +44,8 @@ class _Spec(ctypes.Structure):
         ("nlat_out", ctypes.c_int), ("nlon_out", ctypes.c_int),
         ("n_r", ctypes.c_int), ("n_alpha", ctypes.c_int),
         ("theta_cutoff", ctypes.c_double),
+        ("th_in", ctypes.POINTER(ctypes.c_double)), ("w_in", ctypes.POINTER(ctypes.c_double)),
+        ("th_out", ctypes.POINTER(ctypes.c_double)),
     ]
 
 
@@ -93,9 +95,70 @@ def _f64(a):
     return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
 
 
+GRIDS = ("equiangular", "legendre-gauss", "lobatto", "equiangular-trapezoidal")
+_GRID_CACHE: dict = {}
+
+
+def latitude_grid(name: str, nlat: int):
+    """(theta, w): colatitudes north to south and quadrature weights on t = cos(theta), summing to 2.
+
+    The DISCO constructor takes grid_in / grid_out (page "torch_harmonics.DiscreteContinuousConvS2",
+    signature); the four names are listed on the page of the module
+    "torch_harmonics.distributed.distributed_spectral_convolution" (class docstring, Parameters).
+    Neither page defines them, so each is read as the textbook rule of that name:
+      - equiangular: theta_i = pi*i/(nlat-1), poles included, Clenshaw-Curtis weights;
+      - legendre-gauss: Gauss-Legendre nodes, here by Golub-Welsch (the eigenvalues of the
+        Jacobi matrix of the Legendre recurrence), weights 2 / ((1 - t^2) P_n'(t)^2);
+      - lobatto: Gauss-Lobatto-Legendre: t = +-1 and the n-2 roots of P'_{n-1}, which are the
+        Gauss nodes of the weight 1 - t^2 (Golub-Welsch on its recurrence), weights
+        2 / (m (m+1) P_m(t)^2) with m = n-1;
+      - equiangular-trapezoidal: equiangular nodes, the trapezoidal rule in t (the integral of
+        the piecewise-linear interpolant in t).
+    """
+    key = (name, nlat)
+    if key in _GRID_CACHE:
+        return _GRID_CACHE[key]
+    n = nlat
+    if n < 2:
+        raise ValueError("a latitude grid needs nlat >= 2")
+    if name in ("equiangular", "equiangular-trapezoidal"):
+        theta = np.pi * np.arange(n) / (n - 1)
+        if name == "equiangular":
+            w = cc_weights(n)
+        else:
+            t = np.cos(theta)
+            w = np.empty(n)
+            for i in range(n):
+                w[i] = 0.5 * (t[max(i - 1, 0)] - t[min(i + 1, n - 1)])
+    elif name == "legendre-gauss":
+        k = np.arange(1, n, dtype=np.float64)
+        off = k / np.sqrt(4.0 * k * k - 1.0)
+        t = np.sort(np.linalg.eigvalsh(np.diag(off, 1) + np.diag(off, -1)))[::-1]
+        dP = np.polynomial.legendre.legval(t, np.polynomial.legendre.legder(np.eye(n + 1)[n]))
+        w = 2.0 / ((1.0 - t * t) * dP ** 2)
+        theta = np.arccos(np.clip(t, -1.0, 1.0))
+    elif name == "lobatto":
+        m = n - 1
+        if n > 2:
+            k = np.arange(1, n - 2, dtype=np.float64)
+            off = np.sqrt(k * (k + 2.0) / ((2.0 * k + 1.0) * (2.0 * k + 3.0)))
+            inner = np.linalg.eigvalsh(np.diag(off, 1) + np.diag(off, -1)) if n > 3 else np.zeros(1)
+        else:
+            inner = np.zeros(0)
+        t = np.concatenate([[1.0], np.sort(inner)[::-1], [-1.0]])
+        Pm = np.polynomial.legendre.legval(t, np.eye(m + 1)[m])
+        w = 2.0 / (m * (m + 1.0) * Pm ** 2)
+        theta = np.arccos(np.clip(t, -1.0, 1.0))
+    else:
+        raise ValueError(f"unknown grid {name!r}; one of {GRIDS}")
+    out = (np.ascontiguousarray(theta, dtype=np.float64), np.ascontiguousarray(w, dtype=np.float64))
+    _GRID_CACHE[key] = out
+    return out
+
+
 @dataclass(frozen=True)
 class Spec:
-    """Layer geometry: in/out grid shapes, kernel_shape (n_r, n_alpha), theta_cutoff."""
+    """Layer geometry: in/out grid shapes, kernel_shape (n_r, n_alpha), theta_cutoff, latitude grids."""
 
     nlat_in: int
     nlon_in: int
@@ -104,6 +167,8 @@ class Spec:
     n_r: int
     n_alpha: int
     theta_cutoff: float
+    grid_in: str = "equiangular"
+    grid_out: str = "equiangular"
 
     @property
     def K(self) -> int:
@@ -114,8 +179,15 @@ class Spec:
         return self.nlon_in // self.nlon_out
 
     def _c(self):
+        # non-equiangular grids pass their arrays (kept alive by the grid cache)
+        th_in = w_in = th_out = None
+        if self.grid_in != "equiangular":
+            th_in, w_in = latitude_grid(self.grid_in, self.nlat_in)
+        if self.grid_out != "equiangular":
+            th_out = latitude_grid(self.grid_out, self.nlat_out)[0]
         return ctypes.byref(_Spec(self.nlat_in, self.nlon_in, self.nlat_out, self.nlon_out,
-                                  self.n_r, self.n_alpha, float(self.theta_cutoff)))
+                                  self.n_r, self.n_alpha, float(self.theta_cutoff),
+                                  _d(th_in), _d(w_in), _d(th_out)))
 
 
 class OracleError(RuntimeError):

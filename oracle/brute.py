@@ -11,7 +11,8 @@ only if the p-shift reduction, the longitude index map, the bearing
 convention and the normalisation are all right.
 
 Readings (the same as the oracle's, taken from the pages' silence): grids
-with poles, Clenshaw-Curtis weights, bearing east of local north, radial and
+with poles and Clenshaw-Curtis weights by default (the other latitude grids
+take the oracle's nodes and weights), bearing east of local north, radial and
 azimuthal hats, inclusive cutoff with tie threshold 1e-10, nodal rows that
 sum to one.  The Clenshaw-Curtis weights here come from a linear solve of the
 exactness conditions on polynomials of degree <= n, not from the closed form.
@@ -36,6 +37,15 @@ def cc_weights_vandermonde(nlat: int) -> np.ndarray:
     even = m % 2 == 0
     rhs[even] = 2.0 / (1.0 - m[even].astype(np.float64) ** 2)
     return np.linalg.solve(V, rhs)
+
+
+def _grid(name: str, nlat: int):
+    """Nodes and weights of the non-equiangular grids: the oracle's (pinned on their own by the
+    tests against closed forms and numpy's Gauss-Legendre rule); this module re-checks what is
+    built from them."""
+    from . import latitude_grid
+
+    return latitude_grid(name, nlat)
 
 
 def _unit(theta, lam):
@@ -76,17 +86,25 @@ def basis_values(r, alpha, n_r: int, n_alpha: int, theta_c: float) -> np.ndarray
 def psi_point(spec, j: int, q: int) -> np.ndarray:
     """Normalised basis x quadrature at every input point for output point (j, q):
     array (K, nlat_in, nlon_in) indexed by ABSOLUTE input longitude."""
-    th_o = np.pi * j / (spec.nlat_out - 1)
+    grid_in = getattr(spec, "grid_in", "equiangular")
+    grid_out = getattr(spec, "grid_out", "equiangular")
+    if grid_out == "equiangular":
+        th_o = np.pi * j / (spec.nlat_out - 1)
+    else:
+        th_o = _grid(grid_out, spec.nlat_out)[0][j]
     la_o = 2 * np.pi * q / spec.nlon_out
-    th = np.pi * np.arange(spec.nlat_in) / (spec.nlat_in - 1)
+    if grid_in == "equiangular":
+        th = np.pi * np.arange(spec.nlat_in) / (spec.nlat_in - 1)
+        qw = cc_weights_vandermonde(spec.nlat_in)
+    else:
+        th, qw = _grid(grid_in, spec.nlat_in)
     la = 2 * np.pi * np.arange(spec.nlon_in) / spec.nlon_in
     P = _unit(th[:, None], la[None, :]) @ _to_pole(th_o, la_o).T
     r = np.arctan2(np.hypot(P[..., 0], P[..., 1]), P[..., 2])
     # rotated frame: local north of the output point lies along -x, east along +y
     alpha = np.arctan2(P[..., 1], -P[..., 0])
     phi = basis_values(r, alpha, spec.n_r, spec.n_alpha, spec.theta_cutoff)
-    qw = cc_weights_vandermonde(spec.nlat_in) * 2 * np.pi / spec.nlon_in
-    phi = phi * qw[None, :, None]
+    phi = phi * (qw * 2 * np.pi / spec.nlon_in)[None, :, None]
     s = phi.sum(axis=(1, 2), keepdims=True)
     assert np.all(s > 0)
     return phi / s

@@ -15,9 +15,12 @@
 // longitude (p-shift symmetry).  The pages leave the basis formulas, the
 // quadrature rule, the rotation convention, the normalisation and the
 // backward formulas open; the readings taken here are:
-//   * grids: theta_i = pi*i/(nlat-1) (poles included), lambda_p = 2*pi*p/nlon;
-//   * quadrature: Clenshaw-Curtis weights in cos(theta) (Waldvogel's closed
-//     form), point weight w_i * 2*pi/nlon_in (total 4*pi);
+//   * grids: lambda_p = 2*pi*p/nlon; by default theta_i = pi*i/(nlat-1)
+//     (poles included) with Clenshaw-Curtis weights in cos(theta) (Waldvogel's
+//     closed form); the other latitude grids the constructor names
+//     (grid_in / grid_out) arrive as colatitude and weight arrays computed
+//     by the Python side of the oracle; point weight w_i * 2*pi/nlon_in
+//     (total 4*pi);
 //   * distance r and bearing alpha (east of local north) of an input point
 //     seen from the output point: haversine for r, atan2 for alpha;
 //   * basis "piecewise linear": radial hats at r_k = k*theta_c/(n_r-1); the
@@ -61,6 +64,9 @@ const double kGapHi = 1e-9;      // around a threshold
 struct Spec {
   int nlat_in, nlon_in, nlat_out, nlon_out, n_r, n_alpha;
   double theta_cutoff;
+  const double* th_in;   // input colatitudes, or NULL for the equiangular grid
+  const double* w_in;    // their quadrature weights on cos(theta) (with th_in)
+  const double* th_out;  // output colatitudes, or NULL for the equiangular grid
 };
 
 struct Entry {
@@ -135,13 +141,17 @@ int validate(const Spec& s) {
 // Returns 0, or -1 for a value inside a gap band, -2 for a row of zero mass.
 int dense_row(const Spec& s, int j, double* psi) {
   const int K = num_basis(s);
-  const double th_out = kPi * j / (s.nlat_out - 1);
+  const double th_out = s.th_out ? s.th_out[j] : kPi * j / (s.nlat_out - 1);
   std::vector<double> w(s.nlat_in);
-  cc_weights(s.nlat_in, w.data());
+  if (s.th_in) {
+    for (int i = 0; i < s.nlat_in; ++i) w[i] = s.w_in[i];
+  } else {
+    cc_weights(s.nlat_in, w.data());
+  }
   const double tc = s.theta_cutoff;
   int status = 0;
   for (int i = 0; i < s.nlat_in; ++i) {
-    const double th_in = kPi * i / (s.nlat_in - 1);
+    const double th_in = s.th_in ? s.th_in[i] : kPi * i / (s.nlat_in - 1);
     const double qw = w[i] * 2.0 * kPi / s.nlon_in;
     for (int p = 0; p < s.nlon_in; ++p) {
       double r, alpha;
@@ -173,10 +183,14 @@ extern "C" {
 struct orc_spec {
   int nlat_in, nlon_in, nlat_out, nlon_out, n_r, n_alpha;
   double theta_cutoff;
+  const double* th_in;
+  const double* w_in;
+  const double* th_out;
 };
 
 static Spec to_spec(const orc_spec* o) {
-  return Spec{o->nlat_in, o->nlon_in, o->nlat_out, o->nlon_out, o->n_r, o->n_alpha, o->theta_cutoff};
+  return Spec{o->nlat_in, o->nlon_in, o->nlat_out, o->nlon_out, o->n_r, o->n_alpha, o->theta_cutoff,
+              o->th_in, o->w_in, o->th_out};
 }
 
 int orc_num_basis(const orc_spec* o) { return num_basis(to_spec(o)); }
@@ -222,6 +236,7 @@ void* orc_psi_build(const orc_spec* o, int* status) {
   if (bad) { *status = bad; return nullptr; }
   Psi* h = new Psi;
   h->s = s;
+  h->s.th_in = h->s.w_in = h->s.th_out = nullptr;  // the caller's arrays are not kept
   h->K = K;
   h->row.assign((size_t)s.nlat_out * K + 1, 0);
   for (int j = 0; j < s.nlat_out; ++j)

@@ -5,7 +5,7 @@ of the convolution runs in libdisco's CUDA kernels (there is no CPU path).
 The layer mirrors the constructor of the page
 "torch_harmonics.DiscreteContinuousConvS2": in/out channels and shapes,
 kernel_shape, basis_type='piecewise linear', basis_norm_mode='nodal',
-groups, equiangular grids, bias, theta_cutoff and `fused`.  With
+groups, grid_in / grid_out, bias, theta_cutoff and `fused`.  With
 fused=False the K-expanded intermediate is saved for backward; with
 fused=True only x is saved and the intermediate is recomputed in backward
 (K times less activation memory, one extra contraction).
@@ -46,7 +46,7 @@ class Psi:
     """Precomputed sparse convolution tensor of one layer geometry, on one device."""
 
     def __init__(self, nlat_in: int, nlon_in: int, nlat_out: int, nlon_out: int, kernel_shape, theta_cutoff: float,
-                 device=None):
+                 device=None, grid_in: str = "equiangular", grid_out: str = "equiangular"):
         dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.device = dev
         self.index = dev.index if dev.index is not None else torch.cuda.current_device()
@@ -54,7 +54,11 @@ class Psi:
         self.out_shape = (nlat_out, nlon_out)
         self.kernel_shape = kernel_shape
         self.theta_cutoff = float(theta_cutoff)
-        self.spec = D.make_spec(nlat_in, nlon_in, nlat_out, nlon_out, kernel_shape, theta_cutoff)
+        if grid_in not in D.GRID_CODES or grid_out not in D.GRID_CODES:
+            raise ValueError(f"grids are one of {sorted(D.GRID_CODES)}")
+        self.grid_in, self.grid_out = grid_in, grid_out
+        self.spec = D.make_spec(nlat_in, nlon_in, nlat_out, nlon_out, kernel_shape, theta_cutoff,
+                                D.GRID_CODES[grid_in], D.GRID_CODES[grid_out])
         with torch.cuda.device(self.index):
             self.handle = D.disco_psi_build(self.spec, self.index)
         self.K, self.nnz = D.disco_psi_info(self.handle)
@@ -169,7 +173,8 @@ class _DiscoFusedFn(torch.autograd.Function):
 
 
 class DiscreteContinuousConvS2(torch.nn.Module):
-    """DISCO convolution on the 2-sphere (equiangular grids, piecewise-linear basis, nodal norm)."""
+    """DISCO convolution on the 2-sphere (piecewise-linear basis, nodal norm; grid_in / grid_out one of
+    "equiangular", "legendre-gauss", "lobatto", "equiangular-trapezoidal")."""
 
     def __init__(self, in_channels, out_channels, in_shape, out_shape, kernel_shape, basis_type="piecewise linear",
                  basis_norm_mode="nodal", groups=1, grid_in="equiangular", grid_out="equiangular", bias=True,
@@ -177,8 +182,6 @@ class DiscreteContinuousConvS2(torch.nn.Module):
         super().__init__()
         if basis_type != "piecewise linear" or basis_norm_mode != "nodal":
             raise NotImplementedError("only basis_type='piecewise linear' with basis_norm_mode='nodal'")
-        if grid_in != "equiangular" or grid_out != "equiangular":
-            raise NotImplementedError("only equiangular grids")
         if theta_cutoff is None:
             raise ValueError("theta_cutoff is required (no default is defined for it)")
         if not optimized_kernel:
@@ -186,7 +189,8 @@ class DiscreteContinuousConvS2(torch.nn.Module):
         if in_channels % groups or out_channels % groups:
             raise ValueError("groups must divide in_channels and out_channels")
         self.groups, self.fused = groups, fused
-        self.psi = Psi(in_shape[0], in_shape[1], out_shape[0], out_shape[1], kernel_shape, theta_cutoff, device)
+        self.psi = Psi(in_shape[0], in_shape[1], out_shape[0], out_shape[1], kernel_shape, theta_cutoff, device,
+                       grid_in, grid_out)
         K = self.psi.K
         scale = 1.0 / math.sqrt((in_channels // groups) * K)
         self.weight = torch.nn.Parameter(

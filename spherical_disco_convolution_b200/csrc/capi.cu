@@ -464,8 +464,9 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
   if (!out) return fail(DISCO_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   if (!spec) return fail(DISCO_ERR_INVALID_ARG, "spec is NULL");
-  if (spec->grid_in != DISCO_GRID_EQUIANGULAR || spec->grid_out != DISCO_GRID_EQUIANGULAR)
-    return fail(DISCO_ERR_UNSUPPORTED, "only equiangular grids are supported");
+  if (spec->grid_in < DISCO_GRID_EQUIANGULAR || spec->grid_in > DISCO_GRID_EQUIANGULAR_TRAPEZOIDAL ||
+      spec->grid_out < DISCO_GRID_EQUIANGULAR || spec->grid_out > DISCO_GRID_EQUIANGULAR_TRAPEZOIDAL)
+    return fail(DISCO_ERR_UNSUPPORTED, "unknown latitude grid");
   if (spec->basis_type != DISCO_BASIS_PIECEWISE_LINEAR)
     return fail(DISCO_ERR_UNSUPPORTED, "only the piecewise-linear basis is supported");
   if (spec->basis_norm_mode != DISCO_NORM_NODAL)
@@ -487,6 +488,8 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
   g.theta_cutoff = spec->theta_cutoff;
   g.K = g.n_alpha == 1 ? g.n_r : 1 + (g.n_r - 1) * g.n_alpha;
   g.stride = g.nlon_in / g.nlon_out;
+  g.grid_in = spec->grid_in;
+  g.grid_out = spec->grid_out;
   if (g.K > disco::kMaxK) return fail(DISCO_ERR_UNSUPPORTED, "more basis functions than the kernels support");
   if (g.stride > disco::kMaxStride) return fail(DISCO_ERR_UNSUPPORTED, "nlon_in / nlon_out above 4");
   disco_psi* h = new (std::nothrow) disco_psi;

@@ -5,9 +5,15 @@
 // the north pole, times quadrature weights; one row per output latitude j
 // (p-shift symmetry).  The page leaves the formulas open; this builder takes
 // these readings:
-//   * equiangular grids with poles: theta_i = pi*i/(nlat-1), lambda_p = 2*pi*p/nlon;
-//   * Clenshaw-Curtis quadrature in cos(theta), computed from the Chebyshev
-//     coefficients of the interpolant; point weight w_i * 2*pi / nlon_in;
+//   * longitudes lambda_p = 2*pi*p/nlon; latitude grids (the grid_in / grid_out choices
+//     "equiangular", "legendre-gauss", "lobatto", "equiangular-trapezoidal", which the page
+//     names but does not define) read as the textbook rules on t = cos(theta):
+//       - equiangular: theta_i = pi*i/(nlat-1), poles included, Clenshaw-Curtis weights
+//         computed from the Chebyshev coefficients of the interpolant;
+//       - legendre-gauss: the nlat Gauss-Legendre nodes and weights (no poles);
+//       - lobatto: the nlat Gauss-Lobatto-Legendre nodes (poles included) and weights;
+//       - equiangular-trapezoidal: equiangular nodes, trapezoidal weights in t;
+//     nodes run north to south; point weight w_i * 2*pi / nlon_in;
 //   * the input point is rotated with R_y(-theta'_j) (output point (theta'_j, 0)
 //     to the pole); distance r = atan2(|(x', y')|, z'), bearing east of local
 //     north alpha = atan2(y', -x');
@@ -57,6 +63,89 @@ std::vector<double> clenshaw_curtis(int nlat) {
   return w;
 }
 
+// Legendre polynomial P_n(t) and its derivative, by the three-term recurrence.
+void legendre(int n, double t, double* pn, double* dpn) {
+  double p0 = 1.0, p1 = t;
+  if (n == 0) {
+    *pn = 1.0;
+    *dpn = 0.0;
+    return;
+  }
+  for (int m = 2; m <= n; ++m) {
+    const double p2 = ((2.0 * m - 1.0) * t * p1 - (m - 1.0) * p0) / m;
+    p0 = p1;
+    p1 = p2;
+  }
+  *pn = p1;
+  // (1 - t^2) P_n' = n (P_{n-1} - t P_n); never evaluated at t = +-1 here
+  *dpn = n * (p0 - t * p1) / (1.0 - t * t);
+}
+
+}  // namespace
+
+bool latitude_grid(int grid, int nlat, std::vector<double>& theta, std::vector<double>& weight) {
+  if (nlat < 2) return false;
+  theta.assign(nlat, 0.0);
+  weight.assign(nlat, 0.0);
+  switch (grid) {
+    case 0:  // equiangular, Clenshaw-Curtis
+    case 3: {  // equiangular, trapezoidal in t
+      for (int i = 0; i < nlat; ++i) theta[i] = kPiD * i / (nlat - 1);
+      if (grid == 0) {
+        weight = clenshaw_curtis(nlat);
+      } else {
+        for (int i = 0; i < nlat; ++i) {
+          const double lo = std::cos(theta[std::max(i - 1, 0)]), hi = std::cos(theta[std::min(i + 1, nlat - 1)]);
+          weight[i] = 0.5 * (lo - hi);
+        }
+      }
+      return true;
+    }
+    case 1: {  // Gauss-Legendre: roots of P_n, Newton from cos(pi (i + 3/4) / (n + 1/2))
+      const int n = nlat;
+      for (int i = 0; i < n; ++i) {
+        double t = std::cos(kPiD * (i + 0.75) / (n + 0.5)), pn = 0.0, dpn = 1.0;
+        for (int it = 0; it < 100; ++it) {
+          legendre(n, t, &pn, &dpn);
+          const double dt = pn / dpn;
+          t -= dt;
+          if (std::fabs(dt) < 1e-16) break;
+        }
+        legendre(n, t, &pn, &dpn);
+        theta[i] = std::acos(t);
+        weight[i] = 2.0 / ((1.0 - t * t) * dpn * dpn);
+      }
+      return true;
+    }
+    case 2: {  // Gauss-Lobatto-Legendre: +-1 and the roots of P'_{n-1}
+      const int m = nlat - 1;
+      const double end = 2.0 / (m * (m + 1.0));
+      theta[0] = 0.0;
+      theta[m] = kPiD;
+      weight[0] = weight[m] = end;
+      for (int i = 1; i < m; ++i) {
+        // Newton on P'_m, with P''_m from Legendre's equation, starting at the Chebyshev-Lobatto point
+        double t = std::cos(kPiD * i / m), pm = 0.0, dpm = 1.0;
+        for (int it = 0; it < 100; ++it) {
+          legendre(m, t, &pm, &dpm);
+          const double d2 = (2.0 * t * dpm - m * (m + 1.0) * pm) / (1.0 - t * t);
+          const double dt = dpm / d2;
+          t -= dt;
+          if (std::fabs(dt) < 1e-16) break;
+        }
+        legendre(m, t, &pm, &dpm);
+        theta[i] = std::acos(t);
+        weight[i] = end / (pm * pm);
+      }
+      return true;
+    }
+    default:
+      return false;
+  }
+}
+
+namespace {
+
 inline double radial_hat(double r, int kr, double width) {
   return std::max(0.0, 1.0 - std::fabs(r - kr * width) / width);
 }
@@ -104,7 +193,11 @@ void circular_interval(const std::vector<int>& ps, int n, int* start, int* span)
 int build_psi_entries(const Geometry& g, std::vector<PsiEntry>& out, std::string& msg) {
   const int K = g.K;
   const double tc = g.theta_cutoff;
-  const std::vector<double> qw = clenshaw_curtis(g.nlat_in);
+  std::vector<double> th_in, qw, th_out, unused;
+  if (!latitude_grid(g.grid_in, g.nlat_in, th_in, qw) || !latitude_grid(g.grid_out, g.nlat_out, th_out, unused)) {
+    msg = "unknown latitude grid";
+    return 2;
+  }
   std::vector<double> cl(g.nlon_in), sl(g.nlon_in);
   for (int p = 0; p < g.nlon_in; ++p) {
     cl[p] = std::cos(2.0 * kPiD * p / g.nlon_in);
@@ -114,12 +207,12 @@ int build_psi_entries(const Geometry& g, std::vector<PsiEntry>& out, std::string
   std::vector<int> bad(g.nlat_out, 0);
 #pragma omp parallel for schedule(dynamic)
   for (int j = 0; j < g.nlat_out; ++j) {
-    const double tho = kPiD * j / (g.nlat_out - 1);
+    const double tho = th_out[j];
     const double ct = std::cos(tho), st = std::sin(tho);
     std::vector<double> phi(K);
     std::vector<PsiEntry>& row = rows[j];
     for (int i = 0; i < g.nlat_in; ++i) {
-      const double thi = kPiD * i / (g.nlat_in - 1);
+      const double thi = th_in[i];
       if (std::fabs(thi - tho) > tc + 1e-9) continue;
       const double si = std::sin(thi), ci = std::cos(thi);
       const double wq = qw[i] * 2.0 * kPiD / g.nlon_in;

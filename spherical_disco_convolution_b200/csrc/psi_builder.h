@@ -15,7 +15,14 @@ struct Geometry {
   double theta_cutoff;
   int K;        // number of basis functions
   int stride;   // nlon_in / nlon_out
+  int grid_in = 0, grid_out = 0;  // latitude grids (DISCO_GRID_* codes)
 };
+
+// Colatitudes theta[0..nlat) (north to south) of a latitude grid, and its quadrature weights
+// on t = cos(theta) (they sum to 2).  grid: 0 equiangular (Clenshaw-Curtis), 1 Legendre-Gauss,
+// 2 Lobatto (Gauss-Lobatto-Legendre), 3 equiangular with trapezoidal weights.  Returns false
+// for an unknown grid or too few points.
+bool latitude_grid(int grid, int nlat, std::vector<double>& theta, std::vector<double>& weight);
 
 struct PsiEntry {
   int k, j, i, p;   // basis, output row, input row, longitude offset in [0, nlon_in)

@@ -32,6 +32,11 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "ALLO
 DISCO_F32 = 0
 DISCO_BF16 = 1
 DISCO_GRID_EQUIANGULAR = 0
+DISCO_GRID_LEGENDRE_GAUSS = 1
+DISCO_GRID_LOBATTO = 2
+DISCO_GRID_EQUIANGULAR_TRAPEZOIDAL = 3
+GRID_CODES = {"equiangular": DISCO_GRID_EQUIANGULAR, "legendre-gauss": DISCO_GRID_LEGENDRE_GAUSS,
+              "lobatto": DISCO_GRID_LOBATTO, "equiangular-trapezoidal": DISCO_GRID_EQUIANGULAR_TRAPEZOIDAL}
 DISCO_BASIS_PIECEWISE_LINEAR = 0
 DISCO_NORM_NODAL = 0
 

@@ -304,3 +304,38 @@ def test_packed_kernel_matches_per_pair(name, monkeypatch):
     check(host(dx_p), host(dx_pp), 8e-3, "dx packed vs per pair")
     y_ref = oracle_psi(name).contract(inp["x"] if sel is None else inp["x"][:, sel])
     check(host(y_p), y_ref, 4e-3, "y packed vs oracle")
+
+
+# Layers on the other latitude grids of the constructor's grid_in / grid_out: only Psi changes, so
+# the same kernels must reproduce the oracle.  One bf16 layer on the tensor-core paths (64
+# channels, TMA-aligned rows), one fp32 stride-2 layer on the gather paths.
+GRID_EDGE = {
+    "gauss_to_lobatto_bf16": (Workload("gauss_to_lobatto_bf16", 2, 64, 64, 1, 33, 64, 33, 64, (3, 1), 0.3, "bf16"),
+                              "legendre-gauss", "lobatto"),
+    "trap_to_gauss_f32": (Workload("trap_to_gauss_f32", 2, 6, 9, 3, 19, 24, 10, 12, (3, 4), 0.7, "f32"),
+                          "equiangular-trapezoidal", "legendre-gauss"),
+}
+
+
+@pytest.mark.parametrize("name", list(GRID_EDGE))
+def test_other_grids_match_oracle(name):
+    wl, gi, go = GRID_EDGE[name]
+    inp = make_inputs(wl, 0)
+    P = oracle.Psi(oracle.Spec(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape[0],
+                               wl.kernel_shape[1], wl.theta_cutoff, gi, go))
+    psi = conv.Psi(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape, wl.theta_cutoff, "cuda:0",
+                   grid_in=gi, grid_out=go)
+    x, w, b, dout = (dev(inp[k], wl) for k in ("x", "w", "bias", "dout"))
+    out, y = conv.disco_forward(psi, x, w, b, wl.groups)
+    out_f, _ = conv.disco_forward(psi, x, w, b, wl.groups, fused=True)
+    dx = conv.disco_backward_input(psi, dout, w, wl.C_in, wl.groups)
+    dw, db = conv.disco_backward_weight(psi, dout, x=x, groups=wl.groups)
+    torch.cuda.synchronize()
+    out_ref = P.forward(inp["x"], inp["w"], inp["bias"], groups=wl.groups)
+    check(host(out), out_ref, tol(wl), "out")
+    check(host(y), P.contract(inp["x"]), tol(wl), "y")
+    check(host(out_f), out_ref, tol(wl), "fused out")
+    check(host(dx), P.backward_input(inp["dout"], inp["w"], wl.C_in, groups=wl.groups), tol(wl), "dx")
+    dw_ref, db_ref = P.backward_weight(inp["dout"], inp["x"], groups=wl.groups)
+    check(host(dw), dw_ref, tol(wl), "dw")
+    check(host(db), db_ref, tol(wl), "dbias")

@@ -50,6 +50,78 @@ def test_psi_export_matches_oracle(name):
     np.testing.assert_allclose(v, vo, rtol=1e-12, atol=1e-11 * np.abs(vo).max())
 
 
+GRID_LAYERS = [
+    # (nlat_in, nlon_in, nlat_out, nlon_out, kernel_shape, theta_cutoff, grid_in, grid_out)
+    (24, 48, 24, 48, (3, 1), 2 * math.pi / 24, "legendre-gauss", "legendre-gauss"),
+    (25, 48, 13, 24, (3, 4), 2 * math.pi / 20, "lobatto", "equiangular-trapezoidal"),
+    (21, 40, 17, 40, (4, 1), 3 * math.pi / 32, "equiangular-trapezoidal", "legendre-gauss"),
+    (33, 64, 33, 64, (3, 1), 2 * math.pi / 32, "legendre-gauss", "lobatto"),
+]
+
+
+@pytest.mark.parametrize("layer", GRID_LAYERS, ids=lambda l: f"{l[6]}->{l[7]}")
+def test_psi_export_matches_oracle_on_other_grids(layer):
+    """The library's latitude grids (Newton on the Legendre recurrence) give the oracle's Psi
+    (Golub-Welsch nodes): the same pattern bit for bit, the values to rounding."""
+    nli, nlo_i, nlo, nlo_o, ks, tc, gi, go = layer
+    s = D.make_spec(nli, nlo_i, nlo, nlo_o, ks, tc, D.GRID_CODES[gi], D.GRID_CODES[go])
+    o = oracle.Spec(nli, nlo_i, nlo, nlo_o, ks[0], ks[1], tc, gi, go)
+    h = D.disco_psi_build(s, -1)
+    try:
+        k, j, i, p, v = D.disco_psi_export(h)
+    finally:
+        D.disco_psi_destroy(h)
+    ko, jo, io, po, vo = oracle.Psi(o).entries()
+    assert np.array_equal(k, ko) and np.array_equal(j, jo) and np.array_equal(i, io) and np.array_equal(p, po)
+    np.testing.assert_allclose(v, vo, rtol=1e-11, atol=1e-11 * np.abs(vo).max())
+
+
+@pytest.mark.parametrize("grid", ["legendre-gauss", "lobatto", "equiangular-trapezoidal"])
+def test_full_size_grid_rows_match_oracle(grid):
+    """721 x 1440 latitude grids (the weather layer's size, where a node solve that loses digits
+    or lands on the wrong root would show): sampled Psi rows, poles and equator included,
+    against the oracle's dense rows."""
+    wl = WORKLOADS["weather"]
+    s = D.make_spec(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape, wl.theta_cutoff,
+                    D.GRID_CODES[grid], D.GRID_CODES[grid])
+    o = oracle.Spec(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape[0], wl.kernel_shape[1],
+                    wl.theta_cutoff, grid, grid)
+    h = D.disco_psi_build(s, -1)
+    try:
+        k, j, i, p, v = D.disco_psi_export(h)
+    finally:
+        D.disco_psi_destroy(h)
+    for jj in (0, 1, 180, wl.nlat_out // 2, wl.nlat_out - 2, wl.nlat_out - 1):
+        dense = oracle.psi_dense_row(o, jj)
+        sel = j == jj
+        got = np.zeros_like(dense)
+        got[k[sel], i[sel], p[sel]] = v[sel]
+        assert np.array_equal(got != 0, dense != 0), (grid, jj)
+        np.testing.assert_allclose(got, dense, rtol=0, atol=1e-9 * np.abs(dense).max())
+
+
+def test_grids_change_psi_and_unknown_grids_are_rejected():
+    base = D.make_spec(24, 48, 24, 48, (3, 1), 2 * math.pi / 24)
+    h = D.disco_psi_build(base, -1)
+    try:
+        v0 = D.disco_psi_export(h)[4]
+    finally:
+        D.disco_psi_destroy(h)
+    gauss = D.make_spec(24, 48, 24, 48, (3, 1), 2 * math.pi / 24, D.DISCO_GRID_LEGENDRE_GAUSS,
+                        D.DISCO_GRID_LEGENDRE_GAUSS)
+    h = D.disco_psi_build(gauss, -1)
+    try:
+        v1 = D.disco_psi_export(h)[4]
+    finally:
+        D.disco_psi_destroy(h)
+    assert v0.shape != v1.shape or not np.allclose(v0, v1)
+    for gi, go in ((4, 0), (0, 4), (-1, 0)):
+        bad = D.make_spec(24, 48, 24, 48, (3, 1), 2 * math.pi / 24, gi, go)
+        with pytest.raises(D.DiscoError) as e:
+            D.disco_psi_build(bad, -1)
+        assert e.value.status == D.DISCO_ERR_UNSUPPORTED
+
+
 def _bc(x):
     return x.reshape((-1,) + x.shape[2:])
 
@@ -117,7 +189,7 @@ def test_status_codes():
     assert not h.value
     bad = D.make_spec(17, 32, 17, 24, 3, 0.3)
     assert lib.disco_psi_build(ctypes.byref(bad), -1, ctypes.byref(h)) == D.DISCO_ERR_UNSUPPORTED
-    bad = D.make_spec(17, 32, 17, 32, 3, 0.3, grid_in=1)
+    bad = D.make_spec(17, 32, 17, 32, 3, 0.3, grid_in=4)  # no such grid
     assert lib.disco_psi_build(ctypes.byref(bad), -1, ctypes.byref(h)) == D.DISCO_ERR_UNSUPPORTED
     bad = D.make_spec(1, 32, 17, 32, 3, 0.3)
     assert lib.disco_psi_build(ctypes.byref(bad), -1, ctypes.byref(h)) == D.DISCO_ERR_INVALID_ARG

@@ -30,6 +30,10 @@ TINY = spec_of(WORKLOADS["tiny"])
 ANISO = oracle.Spec(9, 16, 9, 16, 3, 4, 3 * math.pi / 16)
 DOWN = oracle.Spec(9, 16, 5, 8, 3, 4, 3 * math.pi / 16)
 DOWN_ISO = oracle.Spec(13, 24, 7, 12, 3, 1, 2 * math.pi / 12)
+# the other latitude grids of the constructor's grid_in / grid_out
+GAUSS = oracle.Spec(10, 16, 8, 16, 3, 1, 3 * math.pi / 16, "legendre-gauss", "legendre-gauss")
+LOBATTO_DOWN = oracle.Spec(11, 24, 6, 12, 3, 4, 2 * math.pi / 10, "lobatto", "equiangular-trapezoidal")
+TRAP_GAUSS = oracle.Spec(9, 16, 7, 8, 3, 1, 3 * math.pi / 16, "equiangular-trapezoidal", "legendre-gauss")
 
 
 # ---------------------------------------------------------------- quadrature
@@ -59,6 +63,90 @@ def test_cc_weights_integrate_polynomials_exactly(nlat):
 @pytest.mark.parametrize("nlat", [5, 9, 17, 33, 721])
 def test_cc_weights_match_linear_solve(nlat):
     np.testing.assert_allclose(oracle.cc_weights(nlat), brute.cc_weights_vandermonde(nlat), atol=1e-14)
+
+
+def _monomial_integral(m: int) -> float:
+    return 2.0 / (m + 1) if m % 2 == 0 else 0.0
+
+
+@pytest.mark.parametrize("nlat", [2, 3, 7, 16, 91, 361, 721])
+def test_legendre_gauss_grid_matches_numpy(nlat):
+    """Golub-Welsch nodes and their weights against numpy's Gauss-Legendre rule (a library
+    routine), ordered north to south."""
+    theta, w = oracle.latitude_grid("legendre-gauss", nlat)
+    t_np, w_np = np.polynomial.legendre.leggauss(nlat)
+    order = np.argsort(-t_np)
+    np.testing.assert_allclose(np.cos(theta), t_np[order], rtol=0, atol=1e-13)
+    # numpy's own weights drift from the exact ones by up to ~3e-9 relative at 721 points (measured
+    # against a Newton solve in 80-bit precision; this grid is closer), hence the tolerance
+    np.testing.assert_allclose(w, w_np[order], rtol=1e-8, atol=0)
+
+
+def test_lobatto_grid_closed_forms():
+    """Gauss-Lobatto-Legendre rules with 3, 4 and 5 points, from their textbook closed forms."""
+    cases = {
+        3: ([1.0, 0.0, -1.0], [1 / 3, 4 / 3, 1 / 3]),
+        4: ([1.0, 1 / math.sqrt(5), -1 / math.sqrt(5), -1.0], [1 / 6, 5 / 6, 5 / 6, 1 / 6]),
+        5: ([1.0, math.sqrt(3 / 7), 0.0, -math.sqrt(3 / 7), -1.0], [1 / 10, 49 / 90, 32 / 45, 49 / 90, 1 / 10]),
+    }
+    for n, (t, w) in cases.items():
+        theta, wq = oracle.latitude_grid("lobatto", n)
+        np.testing.assert_allclose(np.cos(theta), t, rtol=0, atol=1e-15)
+        np.testing.assert_allclose(wq, w, rtol=0, atol=1e-15)
+
+
+def test_trapezoidal_grid_closed_forms():
+    """Equiangular nodes with trapezoidal weights in cos(theta): 3 and 4 points by hand."""
+    theta, w = oracle.latitude_grid("equiangular-trapezoidal", 3)
+    np.testing.assert_allclose(theta, [0.0, math.pi / 2, math.pi], atol=0)
+    np.testing.assert_allclose(w, [0.5, 1.0, 0.5], atol=1e-16)
+    theta, w = oracle.latitude_grid("equiangular-trapezoidal", 4)
+    np.testing.assert_allclose(w, [0.25, 0.75, 0.75, 0.25], atol=1e-15)
+
+
+# degree up to which each rule integrates polynomials in t exactly
+_EXACT = {"equiangular": lambda n: n - 1, "legendre-gauss": lambda n: 2 * n - 1,
+          "lobatto": lambda n: 2 * n - 3, "equiangular-trapezoidal": lambda n: 1}
+
+
+@pytest.mark.parametrize("grid", oracle.GRIDS)
+@pytest.mark.parametrize("nlat", [2, 3, 6, 17, 64])
+def test_latitude_grids_are_quadrature_rules(grid, nlat):
+    """Every grid: colatitudes rise from north to south inside [0, pi], mirror-symmetric about the
+    equator, positive weights summing to 2, exact on the polynomials its rule is exact for, and
+    (a degree beyond that) not exact, so the exactness check has teeth."""
+    theta, w = oracle.latitude_grid(grid, nlat)
+    assert theta.shape == w.shape == (nlat,)
+    assert np.all(np.diff(theta) > 0) and theta[0] >= 0 and theta[-1] <= math.pi
+    np.testing.assert_allclose(theta + theta[::-1], math.pi, atol=1e-13)
+    np.testing.assert_allclose(w, w[::-1], rtol=1e-12, atol=0)
+    assert np.all(w > 0)
+    t = np.cos(theta)
+    deg = min(_EXACT[grid](nlat), 40)
+    for m in range(deg + 1):
+        assert abs(np.dot(w, t ** m) - _monomial_integral(m)) < 1e-12, (grid, nlat, m)
+    if _EXACT[grid](nlat) < 40:
+        m = _EXACT[grid](nlat) + 1
+        m += m % 2  # odd monomials vanish by symmetry for every rule
+        assert abs(np.dot(w, t ** m) - _monomial_integral(m)) > 1e-11, (grid, nlat, m)
+
+
+def test_trapezoidal_grid_converges_at_second_order():
+    errs = []
+    for n in (33, 65, 129):
+        theta, w = oracle.latitude_grid("equiangular-trapezoidal", n)
+        errs.append(abs(np.dot(w, np.exp(np.cos(theta))) - (math.e - 1 / math.e)))
+    assert 3.5 < errs[0] / errs[1] < 4.5 and 3.5 < errs[1] / errs[2] < 4.5
+
+
+def test_equiangular_grid_is_the_default():
+    theta, w = oracle.latitude_grid("equiangular", 9)
+    np.testing.assert_array_equal(w, oracle.cc_weights(9))
+    np.testing.assert_allclose(theta, np.pi * np.arange(9) / 8, atol=0)
+    a = oracle.Psi(oracle.Spec(9, 16, 9, 16, 3, 1, 3 * math.pi / 16)).entries()
+    b = oracle.Psi(oracle.Spec(9, 16, 9, 16, 3, 1, 3 * math.pi / 16, "equiangular", "equiangular")).entries()
+    for u, v in zip(a, b):
+        np.testing.assert_array_equal(u, v)
 
 
 # ------------------------------------------------------------------ geometry
@@ -115,7 +203,8 @@ def test_basis_partition_of_unity():
 
 # ----------------------------------------------------------------------- Psi
 
-@pytest.mark.parametrize("spec", [TINY, ANISO, DOWN, DOWN_ISO], ids=["tiny", "aniso", "down", "down_iso"])
+@pytest.mark.parametrize("spec", [TINY, ANISO, DOWN, DOWN_ISO, GAUSS, LOBATTO_DOWN],
+                         ids=["tiny", "aniso", "down", "down_iso", "gauss", "lobatto_down"])
 def test_psi_rows_sum_to_one_and_sparse_matches_dense(spec):
     P = oracle.Psi(spec)
     k, j, i, p, v = P.entries()
@@ -131,7 +220,8 @@ def test_psi_rows_sum_to_one_and_sparse_matches_dense(spec):
         assert np.array_equal(rebuilt, dense)
 
 
-@pytest.mark.parametrize("spec", [TINY, ANISO, DOWN, DOWN_ISO], ids=["tiny", "aniso", "down", "down_iso"])
+@pytest.mark.parametrize("spec", [TINY, ANISO, DOWN, DOWN_ISO, GAUSS, LOBATTO_DOWN, TRAP_GAUSS],
+                         ids=["tiny", "aniso", "down", "down_iso", "gauss", "lobatto_down", "trap_gauss"])
 def test_forward_matches_brute_force_without_p_shift(spec):
     rng = np.random.default_rng(0)
     G, C_in, C_out = 2, 4, 6
