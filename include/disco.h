@@ -121,6 +121,23 @@ typedef struct disco_psi disco_psi;
  * disco_psi_destroy.  On failure *out is NULL. */
 disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** out);
 
+/* Psi of one polar band: the output latitudes j_begin <= j < j_end of the layer spec describes,
+ * as a layer of its own.  This is the per-rank layer of the "halo-exchange" polar mode on the page
+ * "torch_harmonics.distributed.DistributedDiscreteContinuousConvS2" (parameter polar_mode): a
+ * rank computes the output latitudes it owns outright from the input rows they reach.
+ *   j_begin, j_end : output latitude range, 0 <= j_begin < j_end <= spec->nlat_out.
+ *   i_begin, i_end : (out, host) the input rows [i_begin, i_end) the band's Psi reaches.
+ * The handle is a layer with nlat_out = j_end - j_begin and nlat_in = i_end - i_begin (the same
+ * longitudes, K and grids): every compute call takes x restricted to input rows
+ * [i_begin, i_end) and gives out rows [j_begin, j_end); disco_bwd_input gives the band's
+ * contribution to dx on rows [i_begin, i_end), to be summed with the other bands' contributions
+ * over shared rows; disco_bwd_weight gives the band's part of dw / dbias, to be summed over
+ * bands.  Its rows are exactly the full Psi's rows j_begin..j_end-1, re-indexed.  Errors as
+ * disco_psi_build, and INVALID_ARG for an empty or out-of-range row range or NULL i_begin /
+ * i_end.  The caller owns the handle (disco_psi_destroy). */
+disco_status disco_psi_build_band(const disco_spec_t* spec, int j_begin, int j_end, int device, disco_psi** out,
+                                  int* i_begin, int* i_end);
+
 /* Frees host and device memory of a Psi (synchronises the device first).  NULL is a no-op. */
 disco_status disco_psi_destroy(disco_psi* psi);
 

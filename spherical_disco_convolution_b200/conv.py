@@ -46,12 +46,16 @@ class Psi:
     """Precomputed sparse convolution tensor of one layer geometry, on one device."""
 
     def __init__(self, nlat_in: int, nlon_in: int, nlat_out: int, nlon_out: int, kernel_shape, theta_cutoff: float,
-                 device=None, grid_in: str = "equiangular", grid_out: str = "equiangular"):
+                 device=None, grid_in: str = "equiangular", grid_out: str = "equiangular", rows=None):
+        """rows=(j_begin, j_end) builds the Psi of those output latitudes only (a polar band): the
+        handle then takes x on input rows self.in_rows = (i_begin, i_end) and gives out rows
+        j_begin..j_end-1."""
         dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.device = dev
         self.index = dev.index if dev.index is not None else torch.cuda.current_device()
         self.in_shape = (nlat_in, nlon_in)
         self.out_shape = (nlat_out, nlon_out)
+        self.in_rows = (0, nlat_in)
         self.kernel_shape = kernel_shape
         self.theta_cutoff = float(theta_cutoff)
         if grid_in not in D.GRID_CODES or grid_out not in D.GRID_CODES:
@@ -60,7 +64,13 @@ class Psi:
         self.spec = D.make_spec(nlat_in, nlon_in, nlat_out, nlon_out, kernel_shape, theta_cutoff,
                                 D.GRID_CODES[grid_in], D.GRID_CODES[grid_out])
         with torch.cuda.device(self.index):
-            self.handle = D.disco_psi_build(self.spec, self.index)
+            if rows is None:
+                self.handle = D.disco_psi_build(self.spec, self.index)
+            else:
+                self.handle, ib, ie = D.disco_psi_build_band(self.spec, rows[0], rows[1], self.index)
+                self.in_rows = (ib, ie)
+                self.in_shape = (ie - ib, nlon_in)
+                self.out_shape = (rows[1] - rows[0], nlon_out)
         self.K, self.nnz = D.disco_psi_info(self.handle)
 
     def __del__(self):

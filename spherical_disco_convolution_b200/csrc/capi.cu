@@ -460,7 +460,13 @@ disco_status disco_sync_status(void* stream) {
   return DISCO_OK;
 }
 
-disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** out) {
+namespace {
+
+// Psi of the output rows [j_begin, j_end) (j_end < 0: all rows).  A band (not all rows) is
+// re-indexed to a layer of its own: output rows j - j_begin, input rows i - i_begin over the
+// input rows [i_begin, i_end) that its entries reach.
+disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, int device, disco_psi** out,
+                            int* i_begin, int* i_end) {
   if (!out) return fail(DISCO_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   if (!spec) return fail(DISCO_ERR_INVALID_ARG, "spec is NULL");
@@ -494,13 +500,31 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
   if (g.stride > disco::kMaxStride) return fail(DISCO_ERR_UNSUPPORTED, "nlon_in / nlon_out above 4");
   disco_psi* h = new (std::nothrow) disco_psi;
   if (!h) return fail(DISCO_ERR_ALLOC, "host allocation failed");
-  h->g = g;
   std::string msg;
-  const int st = disco::build_psi_entries(g, h->entries, msg);
+  const int st = disco::build_psi_entries(g, h->entries, msg, j_begin, j_end);
   if (st) {
     delete h;
     return fail(static_cast<disco_status>(st), msg);
   }
+  if (j_end < 0) j_end = g.nlat_out;
+  int ib = 0, ie = g.nlat_in;
+  if (j_begin != 0 || j_end != g.nlat_out) {
+    ib = g.nlat_in;
+    ie = 0;
+    for (const disco::PsiEntry& en : h->entries) {
+      ib = std::min(ib, en.i);
+      ie = std::max(ie, en.i + 1);
+    }
+    for (disco::PsiEntry& en : h->entries) {
+      en.j -= j_begin;
+      en.i -= ib;
+    }
+    g.nlat_out = j_end - j_begin;
+    g.nlat_in = ie - ib;
+  }
+  if (i_begin) *i_begin = ib;
+  if (i_end) *i_end = ie;
+  h->g = g;
   h->fwd = disco::make_forward_plan(g, h->entries);
   h->adj = disco::make_adjoint_plan(g, h->entries);
   h->fwdb = disco::make_band_plan(g.nlat_out, h->fwd, 4, 24);
@@ -575,6 +599,21 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
   }
   *out = h;
   return DISCO_OK;
+}
+
+}  // namespace
+
+disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** out) {
+  return psi_build_rows(spec, 0, -1, device, out, nullptr, nullptr);
+}
+
+disco_status disco_psi_build_band(const disco_spec_t* spec, int j_begin, int j_end, int device, disco_psi** out,
+                                  int* i_begin, int* i_end) {
+  if (!spec) return fail(DISCO_ERR_INVALID_ARG, "spec is NULL");
+  if (!i_begin || !i_end) return fail(DISCO_ERR_INVALID_ARG, "i_begin / i_end is NULL");
+  if (j_begin < 0 || j_end <= j_begin || j_end > spec->nlat_out)
+    return fail(DISCO_ERR_INVALID_ARG, "need 0 <= j_begin < j_end <= nlat_out");
+  return psi_build_rows(spec, j_begin, j_end, device, out, i_begin, i_end);
 }
 
 disco_status disco_psi_destroy(disco_psi* psi) {

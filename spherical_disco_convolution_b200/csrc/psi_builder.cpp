@@ -190,7 +190,13 @@ void circular_interval(const std::vector<int>& ps, int n, int* start, int* span)
 
 }  // namespace
 
-int build_psi_entries(const Geometry& g, std::vector<PsiEntry>& out, std::string& msg) {
+int build_psi_entries(const Geometry& g, std::vector<PsiEntry>& out, std::string& msg, int j_begin, int j_end) {
+  if (j_end < 0) j_end = g.nlat_out;
+  if (j_begin < 0 || j_begin >= j_end || j_end > g.nlat_out) {
+    msg = "output row range out of bounds";
+    return 1;
+  }
+  const int n_rows = j_end - j_begin;
   const int K = g.K;
   const double tc = g.theta_cutoff;
   std::vector<double> th_in, qw, th_out, unused;
@@ -203,14 +209,15 @@ int build_psi_entries(const Geometry& g, std::vector<PsiEntry>& out, std::string
     cl[p] = std::cos(2.0 * kPiD * p / g.nlon_in);
     sl[p] = std::sin(2.0 * kPiD * p / g.nlon_in);
   }
-  std::vector<std::vector<PsiEntry>> rows(g.nlat_out);
-  std::vector<int> bad(g.nlat_out, 0);
+  std::vector<std::vector<PsiEntry>> rows(n_rows);
+  std::vector<int> bad(n_rows, 0);
 #pragma omp parallel for schedule(dynamic)
-  for (int j = 0; j < g.nlat_out; ++j) {
+  for (int jr = 0; jr < n_rows; ++jr) {
+    const int j = j_begin + jr;
     const double tho = th_out[j];
     const double ct = std::cos(tho), st = std::sin(tho);
     std::vector<double> phi(K);
-    std::vector<PsiEntry>& row = rows[j];
+    std::vector<PsiEntry>& row = rows[jr];
     for (int i = 0; i < g.nlat_in; ++i) {
       const double thi = th_in[i];
       if (std::fabs(thi - tho) > tc + 1e-9) continue;
@@ -222,11 +229,11 @@ int build_psi_entries(const Geometry& g, std::vector<PsiEntry>& out, std::string
         const double yr = vy;
         const double zr = vx * st + vz * ct;
         const double r = std::atan2(std::hypot(xr, yr), zr);
-        if (r - tc >= kBandLo && r - tc <= kBandHi) bad[j] = 1;
+        if (r - tc >= kBandLo && r - tc <= kBandHi) bad[jr] = 1;
         if (r > tc + kTie) continue;
         basis_all(g, r, std::atan2(yr, -xr), phi.data());
         for (int k = 0; k < K; ++k) {
-          if (phi[k] >= kBandLo && phi[k] <= kBandHi) bad[j] = 1;
+          if (phi[k] >= kBandLo && phi[k] <= kBandHi) bad[jr] = 1;
           if (phi[k] > kTie) row.push_back(PsiEntry{k, j, i, p, phi[k] * wq});
         }
       }
@@ -234,7 +241,7 @@ int build_psi_entries(const Geometry& g, std::vector<PsiEntry>& out, std::string
     std::vector<double> mass(K, 0.0);
     for (const PsiEntry& e : row) mass[e.k] += e.v;
     for (int k = 0; k < K; ++k)
-      if (!(mass[k] > 0.0)) bad[j] = bad[j] ? bad[j] : 2;
+      if (!(mass[k] > 0.0)) bad[jr] = bad[jr] ? bad[jr] : 2;
     for (PsiEntry& e : row) e.v /= mass[e.k];
     std::sort(row.begin(), row.end(), [](const PsiEntry& a, const PsiEntry& b) {
       if (a.k != b.k) return a.k < b.k;
@@ -242,13 +249,14 @@ int build_psi_entries(const Geometry& g, std::vector<PsiEntry>& out, std::string
       return a.p < b.p;
     });
   }
-  for (int j = 0; j < g.nlat_out; ++j) {
-    if (bad[j] == 1) {
+  for (int jr = 0; jr < n_rows; ++jr) {
+    const int j = j_begin + jr;
+    if (bad[jr] == 1) {
       msg = "Psi row " + std::to_string(j) +
             ": a distance or basis value lies within [1e-11, 1e-9] of a threshold (tie too close to call)";
       return 6;
     }
-    if (bad[j] == 2) {
+    if (bad[jr] == 2) {
       msg = "Psi row " + std::to_string(j) + ": a basis function has no support on the input grid";
       return 6;
     }

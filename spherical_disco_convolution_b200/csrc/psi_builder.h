@@ -29,8 +29,10 @@ struct PsiEntry {
   double v;
 };
 
-// Status codes mirror disco_status (0 ok, 1 invalid, 2 unsupported, 6 geometry).
-int build_psi_entries(const Geometry& g, std::vector<PsiEntry>& out, std::string& msg);
+// Status codes mirror disco_status (0 ok, 1 invalid, 2 unsupported, 6 geometry).  Builds the
+// rows j in [j_begin, j_end) (j_end < 0: to the last row); entries keep their global indices.
+int build_psi_entries(const Geometry& g, std::vector<PsiEntry>& out, std::string& msg, int j_begin = 0,
+                      int j_end = -1);
 
 struct GatherPlan {
   std::vector<RowPlan> rows;   // ordered heaviest first

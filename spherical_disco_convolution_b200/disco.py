@@ -89,6 +89,7 @@ def _load():
     DP = ctypes.POINTER(ctypes.c_double)
     sig = {
         "disco_psi_build": [ctypes.POINTER(disco_spec_t), I, ctypes.POINTER(P)],
+        "disco_psi_build_band": [ctypes.POINTER(disco_spec_t), I, I, I, ctypes.POINTER(P), IP, IP],
         "disco_psi_destroy": [P],
         "disco_psi_info": [P, IP, ctypes.POINTER(LL)],
         "disco_psi_export": [P, IP, IP, IP, IP, DP],
@@ -156,6 +157,15 @@ def disco_psi_build(spec: disco_spec_t, device: int) -> ctypes.c_void_p:
     h = ctypes.c_void_p()
     _check(_lib.disco_psi_build(ctypes.byref(spec), device, ctypes.byref(h)))
     return h
+
+
+def disco_psi_build_band(spec: disco_spec_t, j_begin: int, j_end: int, device: int):
+    """(handle, i_begin, i_end): Psi of output rows [j_begin, j_end) over input rows [i_begin, i_end)."""
+    h = ctypes.c_void_p()
+    ib, ie = ctypes.c_int(), ctypes.c_int()
+    _check(_lib.disco_psi_build_band(ctypes.byref(spec), j_begin, j_end, device, ctypes.byref(h), ctypes.byref(ib),
+                                     ctypes.byref(ie)))
+    return h, ib.value, ie.value
 
 
 def disco_psi_destroy(psi) -> None:

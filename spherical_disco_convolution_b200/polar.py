@@ -1,0 +1,190 @@
+"""Polar-band distribution of the DISCO layer: the "halo-exchange" polar mode.
+
+Follows the polar_mode parameter on the page
+"torch_harmonics.distributed.DistributedDiscreteContinuousConvS2": the data is split over
+ranks in the polar (latitude) direction; a rank computes the output latitudes it owns outright,
+borrowing the input rows those latitudes reach from its neighbours, so the K-expanded
+intermediate shrinks with the number of ranks; a filter that reaches past the neighbouring
+rank's rows is refused at construction.  Readings where the page is silent:
+
+  * the latitudes are split into contiguous bands as evenly as possible, the first
+    (n mod P) bands one row longer (input and output grids each split this way);
+  * the backward pass is the adjoint of the forward one: each rank's input gradient on the
+    borrowed rows is sent back to the rows' owners and summed there; dw and dbias are
+    summed over ranks (all-reduce).
+
+Every rank runs the same collective steps in the same order.  torch.distributed carries the
+halo rows (NCCL over NVLink on GPUs, gloo on CPU); the contraction runs in libdisco's kernels
+on each rank's band (disco_psi_build_band).
+"""
+
+from __future__ import annotations
+
+import math
+
+import torch
+import torch.distributed as dist
+
+from . import conv
+from . import disco as D
+
+
+def split_rows(n: int, parts: int):
+    """[(begin, end)] of `parts` contiguous bands covering range(n), sizes differing by at most one."""
+    if parts < 1 or n < parts:
+        raise ValueError(f"cannot split {n} rows over {parts} ranks")
+    q, r = divmod(n, parts)
+    out, b = [], 0
+    for p in range(parts):
+        e = b + q + (1 if p < r else 0)
+        out.append((b, e))
+        b = e
+    return out
+
+
+class PolarBands:
+    """Which rows each rank owns and borrows, for one layer geometry and `world` ranks.
+
+    out_rows[r], in_rows[r]: the output / input latitudes rank r owns.  reach[r]: the input rows
+    [i_begin, i_end) its output rows reach (from the band's Psi).  recv[r]: (src, lo, hi) input
+    row ranges rank r borrows from rank src; send[r]: (dst, lo, hi) ranges it lends to dst.
+    """
+
+    def __init__(self, nlat_in, nlon_in, nlat_out, nlon_out, kernel_shape, theta_cutoff, world: int,
+                 grid_in: str = "equiangular", grid_out: str = "equiangular"):
+        self.world = world
+        self.spec = D.make_spec(nlat_in, nlon_in, nlat_out, nlon_out, kernel_shape, theta_cutoff,
+                                D.GRID_CODES[grid_in], D.GRID_CODES[grid_out])
+        self.geometry = (nlat_in, nlon_in, nlat_out, nlon_out, kernel_shape, theta_cutoff, grid_in, grid_out)
+        self.out_rows = split_rows(nlat_out, world)
+        self.in_rows = split_rows(nlat_in, world)
+        self.reach = []
+        for jb, je in self.out_rows:
+            h, ib, ie = D.disco_psi_build_band(self.spec, jb, je, -1)  # host-only: geometry only
+            D.disco_psi_destroy(h)
+            self.reach.append((ib, ie))
+        self.recv = [[] for _ in range(world)]
+        self.send = [[] for _ in range(world)]
+        for r, (ib, ie) in enumerate(self.reach):
+            lo_ok = self.in_rows[max(r - 1, 0)][0]
+            hi_ok = self.in_rows[min(r + 1, world - 1)][1]
+            if ib < lo_ok or ie > hi_ok:
+                raise ValueError(
+                    f"rank {r}'s output latitudes {self.out_rows[r]} reach input rows [{ib}, {ie}), beyond its "
+                    f"neighbours' rows [{lo_ok}, {hi_ok}): the filter is too wide for {world} polar ranks")
+            for s, (ob, oe) in enumerate(self.in_rows):
+                lo, hi = max(ib, ob), min(ie, oe)
+                if s != r and lo < hi:
+                    self.recv[r].append((s, lo, hi))
+                    self.send[s].append((r, lo, hi))
+
+
+def _exchange(ops):
+    if ops:
+        for req in dist.batch_isend_irecv(ops):
+            req.wait()
+
+
+def halo_gather(bands: PolarBands, rank: int, x_own: torch.Tensor) -> torch.Tensor:
+    """x on the rows rank `rank` reaches, [..., i_end - i_begin, nlon], from x on its own rows."""
+    ob, oe = bands.in_rows[rank]
+    ib, ie = bands.reach[rank]
+    if x_own.shape[-2] != oe - ob:
+        raise ValueError(f"rank {rank} holds input rows [{ob}, {oe}); got {x_own.shape[-2]} rows")
+    x_band = x_own.new_empty(x_own.shape[:-2] + (ie - ib, x_own.shape[-1]))
+    lo, hi = max(ib, ob), min(ie, oe)
+    if lo < hi:
+        x_band[..., lo - ib:hi - ib, :] = x_own[..., lo - ob:hi - ob, :]
+    ops, keep = [], []
+    for dst, lo, hi in bands.send[rank]:
+        buf = x_own[..., lo - ob:hi - ob, :].contiguous()
+        keep.append(buf)
+        ops.append(dist.P2POp(dist.isend, buf, dst))
+    recvs = []
+    for src, lo, hi in bands.recv[rank]:
+        buf = x_own.new_empty(x_own.shape[:-2] + (hi - lo, x_own.shape[-1]))
+        recvs.append((buf, lo))
+        ops.append(dist.P2POp(dist.irecv, buf, src))
+    _exchange(ops)
+    for buf, lo in recvs:
+        x_band[..., lo - ib:lo - ib + buf.shape[-2], :] = buf
+    return x_band
+
+
+def halo_reduce(bands: PolarBands, rank: int, g_band: torch.Tensor) -> torch.Tensor:
+    """The adjoint of halo_gather: a gradient on the reached rows, summed onto each row's owner."""
+    ob, oe = bands.in_rows[rank]
+    ib, ie = bands.reach[rank]
+    g_own = g_band.new_zeros(g_band.shape[:-2] + (oe - ob, g_band.shape[-1]))
+    lo, hi = max(ib, ob), min(ie, oe)
+    if lo < hi:
+        g_own[..., lo - ob:hi - ob, :] += g_band[..., lo - ib:hi - ib, :]
+    ops, keep, recvs = [], [], []
+    for src, lo, hi in bands.recv[rank]:  # rows borrowed from src go back to src
+        buf = g_band[..., lo - ib:hi - ib, :].contiguous()
+        keep.append(buf)
+        ops.append(dist.P2POp(dist.isend, buf, src))
+    for dst, lo, hi in bands.send[rank]:  # rows lent to dst come back from dst
+        buf = g_band.new_empty(g_band.shape[:-2] + (hi - lo, g_band.shape[-1]))
+        recvs.append((buf, lo))
+        ops.append(dist.P2POp(dist.irecv, buf, dst))
+    _exchange(ops)
+    for buf, lo in recvs:
+        g_own[..., lo - ob:lo - ob + buf.shape[-2], :] += buf
+    return g_own
+
+
+class _PolarFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x_own, w, bias, layer):
+        x_band = halo_gather(layer.bands, layer.rank, x_own)
+        out, y = conv.disco_forward(layer.psi, x_band, w, bias, layer.groups)
+        ctx.layer = layer
+        ctx.has_bias = bias is not None
+        ctx.save_for_backward(y, w)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        y, w = ctx.saved_tensors
+        layer = ctx.layer
+        dout = dout.contiguous()
+        dx_band = conv.disco_backward_input(layer.psi, dout, w, y.shape[1], layer.groups)
+        dx = halo_reduce(layer.bands, layer.rank, dx_band)
+        dw, db = conv.disco_backward_weight(layer.psi, dout, y=y, groups=layer.groups, need_bias=ctx.has_bias)
+        dist.all_reduce(dw)
+        if db is not None:
+            dist.all_reduce(db)
+        return dx, dw, db, None
+
+
+class PolarDiscoConvS2(torch.nn.Module):
+    """DISCO convolution with its latitudes split over the ranks of the default process group.
+
+    Each rank passes x on its own input latitudes (bands.in_rows[rank]) and gets out on its own
+    output latitudes (bands.out_rows[rank]).  Weights and bias are replicated (same seed on every
+    rank, or a broadcast, is the caller's business); their gradients are summed over ranks.
+    """
+
+    def __init__(self, in_channels, out_channels, in_shape, out_shape, kernel_shape, theta_cutoff, groups=1,
+                 grid_in="equiangular", grid_out="equiangular", bias=True, device=None, dtype=torch.float32):
+        super().__init__()
+        if in_channels % groups or out_channels % groups:
+            raise ValueError("groups must divide in_channels and out_channels")
+        self.rank, world = dist.get_rank(), dist.get_world_size()
+        self.groups = groups
+        self.bands = PolarBands(in_shape[0], in_shape[1], out_shape[0], out_shape[1], kernel_shape, theta_cutoff,
+                                world, grid_in, grid_out)
+        jb, je = self.bands.out_rows[self.rank]
+        self.psi = conv.Psi(in_shape[0], in_shape[1], out_shape[0], out_shape[1], kernel_shape, theta_cutoff, device,
+                            grid_in, grid_out, rows=(jb, je))
+        assert self.psi.in_rows == self.bands.reach[self.rank]
+        K = self.psi.K
+        scale = 1.0 / math.sqrt((in_channels // groups) * K)
+        self.weight = torch.nn.Parameter(
+            torch.randn(out_channels, in_channels // groups, K, device=self.psi.device, dtype=dtype) * scale)
+        self.bias = torch.nn.Parameter(torch.zeros(out_channels, device=self.psi.device, dtype=dtype)) if bias \
+            else None
+
+    def forward(self, x_own):
+        return _PolarFn.apply(x_own.contiguous(), self.weight, self.bias, self)

@@ -339,3 +339,39 @@ def test_other_grids_match_oracle(name):
     dw_ref, db_ref = P.backward_weight(inp["dout"], inp["x"], groups=wl.groups)
     check(host(dw), dw_ref, tol(wl), "dw")
     check(host(db), db_ref, tol(wl), "dbias")
+
+
+@pytest.mark.parametrize("name", ["tz_fused_k3", "ragged_down_bf16", "aniso_k9_f32"])
+def test_polar_bands_reassemble_the_full_layer(name):
+    """Three polar bands (disco_psi_build_band), each through the kernels on its own rows, stitched
+    together: out and y by row, dx summed over the rows the bands share, dw and dbias summed,
+    against the oracle's full layer.  This is the per-rank computation of the halo-exchange mode
+    without the transfers."""
+    from spherical_disco_convolution_b200 import polar
+
+    wl, inp = workload(name), inputs(name)
+    w, b = dev(inp["w"], wl), dev(inp["bias"], wl)
+    out = np.zeros(oracle_out(name).shape)
+    out_f = np.zeros_like(out)
+    dx = np.zeros(inp["x"].shape)
+    dw, db = 0.0, 0.0
+    for jb, je in polar.split_rows(wl.nlat_out, 3):
+        psi = conv.Psi(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape, wl.theta_cutoff, "cuda:0",
+                       rows=(jb, je))
+        ib, ie = psi.in_rows
+        xb = dev(inp["x"][:, :, ib:ie], wl)
+        db_ = dev(inp["dout"][:, :, jb:je], wl)
+        o, y = conv.disco_forward(psi, xb, w, b, wl.groups)
+        of, _ = conv.disco_forward(psi, xb, w, b, wl.groups, fused=True)
+        dxb = conv.disco_backward_input(psi, db_, w, wl.C_in, wl.groups)
+        dwb, dbb = conv.disco_backward_weight(psi, db_, y=y, groups=wl.groups)
+        torch.cuda.synchronize()
+        out[:, :, jb:je], out_f[:, :, jb:je] = host(o), host(of)
+        dx[:, :, ib:ie] += host(dxb)
+        dw, db = dw + host(dwb), db + host(dbb)
+    check(out, oracle_out(name), tol(wl), "out from bands")
+    check(out_f, oracle_out(name), tol(wl), "fused out from bands")
+    check(dx, oracle_dx(name), tol(wl), "dx from bands")
+    dw_ref, db_ref = oracle_dw(name)
+    check(dw, dw_ref, tol(wl), "dw from bands")
+    check(db, db_ref, tol(wl), "dbias from bands")
