@@ -135,23 +135,32 @@ def halo_reduce(bands: PolarBands, rank: int, g_band: torch.Tensor) -> torch.Ten
 
 
 class _PolarFn(torch.autograd.Function):
+    """fused=False saves the band's K-expanded y; fused=True saves the halo-extended x and
+    recomputes y in backward (the page's fused flag, orthogonal to the polar mode)."""
+
     @staticmethod
     def forward(ctx, x_own, w, bias, layer):
         x_band = halo_gather(layer.bands, layer.rank, x_own)
-        out, y = conv.disco_forward(layer.psi, x_band, w, bias, layer.groups)
+        out, y = conv.disco_forward(layer.psi, x_band, w, bias, layer.groups, fused=layer.fused)
         ctx.layer = layer
         ctx.has_bias = bias is not None
-        ctx.save_for_backward(y, w)
+        ctx.C_in = x_own.shape[1]
+        ctx.save_for_backward(x_band if layer.fused else y, w)
         return out
 
     @staticmethod
     def backward(ctx, dout):
-        y, w = ctx.saved_tensors
+        saved, w = ctx.saved_tensors
         layer = ctx.layer
         dout = dout.contiguous()
-        dx_band = conv.disco_backward_input(layer.psi, dout, w, y.shape[1], layer.groups)
+        dx_band = conv.disco_backward_input(layer.psi, dout, w, ctx.C_in, layer.groups)
         dx = halo_reduce(layer.bands, layer.rank, dx_band)
-        dw, db = conv.disco_backward_weight(layer.psi, dout, y=y, groups=layer.groups, need_bias=ctx.has_bias)
+        if layer.fused:
+            dw, db = conv.disco_backward_weight(layer.psi, dout, x=saved, groups=layer.groups,
+                                                need_bias=ctx.has_bias)
+        else:
+            dw, db = conv.disco_backward_weight(layer.psi, dout, y=saved, groups=layer.groups,
+                                                need_bias=ctx.has_bias)
         dist.all_reduce(dw)
         if db is not None:
             dist.all_reduce(db)
@@ -167,12 +176,13 @@ class PolarDiscoConvS2(torch.nn.Module):
     """
 
     def __init__(self, in_channels, out_channels, in_shape, out_shape, kernel_shape, theta_cutoff, groups=1,
-                 grid_in="equiangular", grid_out="equiangular", bias=True, device=None, dtype=torch.float32):
+                 grid_in="equiangular", grid_out="equiangular", bias=True, fused=False, device=None,
+                 dtype=torch.float32):
         super().__init__()
         if in_channels % groups or out_channels % groups:
             raise ValueError("groups must divide in_channels and out_channels")
         self.rank, world = dist.get_rank(), dist.get_world_size()
-        self.groups = groups
+        self.groups, self.fused = groups, fused
         self.bands = PolarBands(in_shape[0], in_shape[1], out_shape[0], out_shape[1], kernel_shape, theta_cutoff,
                                 world, grid_in, grid_out)
         jb, je = self.bands.out_rows[self.rank]

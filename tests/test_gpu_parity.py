@@ -375,3 +375,39 @@ def test_polar_bands_reassemble_the_full_layer(name):
     dw_ref, db_ref = oracle_dw(name)
     check(dw, dw_ref, tol(wl), "dw from bands")
     check(db, db_ref, tol(wl), "dbias from bands")
+
+
+def test_polar_layer_on_one_rank_matches_oracle():
+    """PolarDiscoConvS2 through autograd on a one-rank NCCL group (the whole layer is one band;
+    no transfers), unfused and fused, against the oracle."""
+    import datetime
+    import socket
+
+    import torch.distributed as dist
+
+    from spherical_disco_convolution_b200 import polar
+
+    name = "ragged_down_bf16"
+    wl, inp = workload(name), inputs(name)
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60), device_id=torch.device("cuda:0"))
+    try:
+        for fused in (False, True):
+            layer = polar.PolarDiscoConvS2(wl.C_in, wl.C_out, (wl.nlat_in, wl.nlon_in), (wl.nlat_out, wl.nlon_out),
+                                           wl.kernel_shape, wl.theta_cutoff, groups=wl.groups, bias=False,
+                                           fused=fused, device="cuda:0", dtype=torch.bfloat16)
+            with torch.no_grad():
+                layer.weight.copy_(dev(inp["w"], wl))
+            x = dev(inp["x"], wl).requires_grad_(True)
+            out = layer(x)
+            out.backward(dev(inp["dout"], wl))
+            torch.cuda.synchronize()
+            check(host(out), oracle_out(name), tol(wl), "polar layer out")
+            check(host(x.grad), oracle_dx(name), tol(wl), "polar layer dx")
+            check(host(layer.weight.grad), oracle_dw(name)[0], tol(wl), "polar layer dw")
+    finally:
+        dist.destroy_process_group()
