@@ -9,12 +9,12 @@
 // accumulates in one of NR tensor-memory slots (slot = strip-relative row mod NR, T groups of
 // 16 outputs apart by NR*Nr columns) from its first source row to its last.
 //
-// Roles as in contract_tc.cu (persistent CTAs): warps 0 and 6.. stage entries (the x window by
+// Roles as in contract_tc.cu (persistent CTAs): warps 0 and 6..8 stage entries (the x window by
 // cp.async with copy-completion arrivals, each warp a share of the channels; the packed block
-// by one bulk copy from warp 0); warp 1 lane 0
-// waits until a slot's previous row is drained before the first contribution of a new row,
-// issues the MMAs (split in two where the slot range wraps) and commits a "row complete"
-// barrier per finished row; warps 2..5 drain finished rows (TMEM -> bf16 -> shared tile -> TMA
+// by one bulk copy from warp 0); lane 0 of warps 1 and 9 (the even and the odd groups of 16
+// outputs) each wait until a slot's previous row is drained before the first contribution of
+// a new row, issue their MMAs (split in two where the slot range wraps) and commit a "row
+// complete" barrier per finished row; warps 2..5 drain finished rows (TMEM -> bf16 -> shared tile -> TMA
 // store), write zeros back into the slot and release it.  Every MMA accumulates: slots start at
 // zero and are zeroed on release.  Every wait is bounded (tc_common.cuh).
 #include <cuda.h>
@@ -32,7 +32,8 @@ namespace {
 constexpr int kCT = 64;
 constexpr uint32_t kOctBytes = kCT * 16;
 constexpr int kProducers = 4;  // copy warps: 0 and 6..4+kProducers
-constexpr int kThreads = 32 * (5 + kProducers);  // producers, MMA issuer, four epilogue warps
+constexpr int kIssuer2 = 5 + kProducers;  // warp of the second MMA issuer
+constexpr int kThreads = 32 * (6 + kProducers);  // producers, two MMA issuers, four epilogue warps
 constexpr uint32_t kTmemCols = 512;
 constexpr int kStages = 4;
 constexpr int kMaxEnt = 24;
@@ -91,10 +92,10 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tcp_kernel(const __grid_
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(&full[s], 32 * kProducers + 1);
-      tc::mbar_init(&empty[s], 1);
+      tc::mbar_init(&empty[s], 2);  // both MMA issuers commit
     }
     for (int s = 0; s < NR; ++s) {
-      tc::mbar_init(&tfull[s], 1);
+      tc::mbar_init(&tfull[s], 2);  // both MMA issuers commit
       tc::mbar_init(&tempty[s], 4);
     }
     tc::fence_barrier_init();
@@ -116,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tcp_kernel(const __grid_
   __syncthreads();
   tc::fence_after_sync();
 
-  if (warp == 0 || warp >= 6) {
+  if (warp == 0 || (warp >= 6 && warp < kIssuer2)) {
     // ---------------------------------------------------------------- producer warps
     // kProducers warps run the same stage packing and each copies its share of the 8 channel
     // groups; the first also writes the stage tables, issues the bulk copies and closes stages.
@@ -209,9 +210,12 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tcp_kernel(const __grid_
       close(kLast);
     }
     tc::cp_async_wait_all();
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == kIssuer2) {
     if (lane == 0) {
-      // ---------------------------------------------------------------- MMA issuer
+      // ---------------------------------------------------------------- MMA issuers
+      // two threads issue the MMAs of the even and the odd groups of 16 outputs (disjoint
+      // accumulator columns); each waits for the slots it writes and commits its own MMAs
+      const int gsel = warp == 1 ? 0 : 1;
       const uint64_t a_fix = tc::desc_noswz(0, kOctBytes, 128);
       const uint32_t a_step = (2 * kOctBytes) >> 4;
       uint32_t n = 0;
@@ -258,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_tcp_kernel(const __grid_
             const uint32_t b_step = (2 * NC * 16) >> 4;
             const uint32_t b2off = ((uint32_t)(n1 * Nr) * 16) >> 4;  // second column group
 #pragma unroll 1
-            for (int g = 0; g < T; ++g) {
+            for (int g = gsel; g < T; g += 2) {
               uint64_t ad = a_fix | (uint64_t)(sbase4 + xo + (uint32_t)g * a_step);
               uint64_t bd = b_fix | (uint64_t)(sbase4 + bo);
               const uint32_t d1 = tmem + (uint32_t)g * GS + (uint32_t)(sl0 * Nr);
