@@ -4,7 +4,7 @@ The band handles are host-only (no GPU), so the per-rank contraction here is the
 Psi applied in NumPy; what is checked is everything around it: that a band's Psi is exactly the
 full Psi's rows, that its plans still reproduce the oracle, and that the halo gather, the
 reverse halo sum and the weight-gradient all-reduce reassemble the global oracle's out, dx and
-dw on 2 and 3 ranks.
+dw on 2, 3 and 4 ranks.
 """
 
 import math
@@ -198,7 +198,7 @@ def _worker(rank, world, port, name, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,name", [(2, "iso"), (3, "aniso_down"), (3, "gauss")])
+@pytest.mark.parametrize("world,name", [(2, "iso"), (3, "aniso_down"), (3, "gauss"), (4, "iso")])
 def test_halo_exchange_reassembles_the_oracle(world, name):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
