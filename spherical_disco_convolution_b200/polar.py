@@ -188,7 +188,11 @@ class PolarDiscoConvS2(torch.nn.Module):
         jb, je = self.bands.out_rows[self.rank]
         self.psi = conv.Psi(in_shape[0], in_shape[1], out_shape[0], out_shape[1], kernel_shape, theta_cutoff, device,
                             grid_in, grid_out, rows=(jb, je))
-        assert self.psi.in_rows == self.bands.reach[self.rank]
+        if self.psi.in_rows != self.bands.reach[self.rank]:
+            raise RuntimeError("band Psi and band geometry disagree on the rows reached")
+        # every rank joins one collective before the first point-to-point exchange (a rank
+        # whose band borrows nothing issues no send or receive of its own)
+        dist.barrier()
         K = self.psi.K
         scale = 1.0 / math.sqrt((in_channels // groups) * K)
         self.weight = torch.nn.Parameter(
