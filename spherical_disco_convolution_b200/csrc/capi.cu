@@ -564,10 +564,10 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
       e = upload_tz(h->tz, &h->dtz);
       if (e == cudaSuccess) e = upload_tz(h->tza, &h->dtza);
       h->tz_ok = e == cudaSuccess;
-      // Packed forms (one staged source row feeds up to 16 output rows).  Measured on one
-      // B200 with four producer warps, the per-pair kernels are faster on every layer tried,
-      // the K = 9 adjoint included (about 63 (k, j) rows per output row), because staging,
-      // not the MMA count, bounds both.  So the packed kernels run only when DISCO_PACKED=1.
+      // Packed forms (one staged source row feeds up to 16 output rows, so 2.7-2.9 times fewer
+      // bytes are staged).  Measured on one B200, the per-pair kernels are still faster on
+      // every layer tried (the K = 9 adjoint within 1%, the 721x1440 contraction by 1.9x), so
+      // the packed kernels run only when DISCO_PACKED=1.
       const char* pk = std::getenv("DISCO_PACKED");
       const bool force = pk && pk[0] == '1';
       int T, NR;
