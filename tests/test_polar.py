@@ -101,6 +101,32 @@ def test_band_toeplitz_plan_reproduces_the_oracle_rows():
         np.testing.assert_allclose(y, want, rtol=0, atol=2e-5 * np.abs(y_ref).max())
 
 
+def test_band_adjoint_toeplitz_plan_reproduces_the_oracle():
+    """A band's adjoint plan (source rows (k, j) of the band's dy, output rows the reached input
+    rows) gives the oracle's dx for a dout that is zero outside the band."""
+    layer = LAYERS["iso"]
+    s = _spec(layer)
+    nli, nloi, nlo, nloo = layer[:4]
+    P = oracle.Psi(_ospec(layer))
+    K = P.K
+    rng = np.random.default_rng(4)
+    w = rng.standard_normal((3, 2, K))
+    for jb, je in polar.split_rows(nlo, 4):
+        dout = np.zeros((1, 3, nlo, nloo))
+        dout[:, :, jb:je] = rng.standard_normal((1, 3, je - jb, nloo))
+        dx_ref = P.backward_input(dout, w, 2)
+        h, ib, ie = D.disco_psi_build_band(s, jb, je, -1)
+        try:
+            plan = D.disco_toeplitz_export(h, 1)
+        finally:
+            D.disco_psi_destroy(h)
+        dy = np.einsum("ock,bojq->bckjq", w, dout[:, :, jb:je]).reshape(2, K * (je - jb), nloo)
+        dx = plan_emulator.toeplitz(plan, dy, ie - ib)[:, 0]
+        # nothing outside the reached rows, and the reached rows match
+        assert np.abs(dx_ref[0, :, :ib]).max(initial=0) == 0 and np.abs(dx_ref[0, :, ie:]).max(initial=0) == 0
+        np.testing.assert_allclose(dx, dx_ref[0, :, ib:ie], rtol=0, atol=2e-5 * np.abs(dx_ref).max())
+
+
 def test_too_wide_filter_is_refused():
     """A cutoff that reaches past the neighbouring rank's latitudes raises at construction."""
     nli, nloi, nlo, nloo, ks, _, gi, go = LAYERS["iso"]
