@@ -192,7 +192,8 @@ class PolarDiscoConvS2(torch.nn.Module):
             raise RuntimeError("band Psi and band geometry disagree on the rows reached")
         # every rank joins one collective before the first point-to-point exchange (a rank
         # whose band borrows nothing issues no send or receive of its own)
-        dist.barrier()
+        if world > 1:
+            dist.barrier()
         K = self.psi.K
         scale = 1.0 / math.sqrt((in_channels // groups) * K)
         self.weight = torch.nn.Parameter(
