@@ -316,3 +316,13 @@ def test_packed_plan_reproduces_oracle(name, which):
     assert len(rows) > len(plan["rest"])  # most rows are packed
     np.testing.assert_allclose(got[:, :, rows], ref[:, :, rows], rtol=0, atol=2e-5 * np.abs(ref).max())
     assert np.all(got[:, :, sorted(plan["rest"].tolist())] == 0)
+
+
+def test_layer_rejects_unknown_grid_names_before_building():
+    from spherical_disco_convolution_b200 import conv
+
+    with pytest.raises(ValueError, match="grids are one of"):
+        conv.Psi(17, 32, 17, 32, (3, 1), 0.3, "cuda:0", grid_in="gaussian")
+    with pytest.raises(ValueError, match="grids are one of"):
+        conv.Psi(17, 32, 17, 32, (3, 1), 0.3, "cuda:0", grid_out="healpix")
+    assert sorted(D.GRID_CODES) == sorted(oracle.GRIDS)
