@@ -326,3 +326,28 @@ def test_layer_rejects_unknown_grid_names_before_building():
     with pytest.raises(ValueError, match="grids are one of"):
         conv.Psi(17, 32, 17, 32, (3, 1), 0.3, "cuda:0", grid_out="healpix")
     assert sorted(D.GRID_CODES) == sorted(oracle.GRIDS)
+
+
+@pytest.mark.parametrize("grids", [("legendre-gauss", "legendre-gauss"), ("lobatto", "equiangular-trapezoidal")])
+def test_tensor_core_plans_on_other_grids_reproduce_oracle(grids):
+    """The Toeplitz and packed plans depend on Psi only; on the other latitude grids they still
+    reproduce the oracle (re-enacted on CPU)."""
+    gi, go = grids
+    nli, nlo, nlon, tc = 40, 40, 64, 2 * math.pi / 36
+    s = D.make_spec(nli, nlon, nlo, nlon, (3, 1), tc, D.GRID_CODES[gi], D.GRID_CODES[go])
+    o = oracle.Spec(nli, nlon, nlo, nlon, 3, 1, tc, gi, go)
+    h = D.disco_psi_build(s, -1)
+    try:
+        tz = D.disco_toeplitz_export(h, 0)
+        pk = D.disco_packed_export(h, 0)
+    finally:
+        D.disco_psi_destroy(h)
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((1, 2, nli, nlon))
+    ref = _bc(oracle.Psi(o).contract(x))
+    got = plan_emulator.toeplitz(tz, _bc(x), nlo)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=2e-5 * np.abs(ref).max())
+    got = plan_emulator.packed(pk, _bc(x), nlo)
+    rows = [r for r in range(nlo) if r not in set(pk["rest"].tolist())]
+    assert len(rows) > len(pk["rest"])  # most rows are packed
+    np.testing.assert_allclose(got[:, :, rows], ref[:, :, rows], rtol=0, atol=2e-5 * np.abs(ref).max())
