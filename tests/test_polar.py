@@ -127,6 +127,34 @@ def test_band_adjoint_toeplitz_plan_reproduces_the_oracle():
         np.testing.assert_allclose(dx, dx_ref[0, :, ib:ie], rtol=0, atol=2e-5 * np.abs(dx_ref).max())
 
 
+@pytest.mark.parametrize("world", [2, 3, 5, 8])
+@pytest.mark.parametrize("cut", [1, 2, 3])
+def test_exchange_plan_covers_each_reach_exactly(world, cut):
+    """For every rank: its own rows plus what it borrows tile its reach with no overlap; every
+    borrowed range is a neighbour's own rows; sends mirror receives."""
+    nlat = 65
+    try:
+        bands = polar.PolarBands(nlat, 64, nlat, 64, (3, 1), cut * math.pi / (nlat - 1) + 1e-3, world)
+    except ValueError:
+        assert world * (cut + 1) > nlat  # refused only when bands are thinner than the reach
+        return
+    for r in range(world):
+        ib, ie = bands.reach[r]
+        ob, oe = bands.in_rows[r]
+        covered = np.zeros(ie - ib, dtype=int)
+        lo, hi = max(ib, ob), min(ie, oe)
+        if lo < hi:
+            covered[lo - ib:hi - ib] += 1
+        for src, lo, hi in bands.recv[r]:
+            assert abs(src - r) == 1
+            sb, se = bands.in_rows[src]
+            assert sb <= lo < hi <= se
+            covered[lo - ib:hi - ib] += 1
+            assert (r, lo, hi) in bands.send[src]
+        assert np.all(covered == 1)
+    assert sum(len(x) for x in bands.send) == sum(len(x) for x in bands.recv)
+
+
 def test_too_wide_filter_is_refused():
     """A cutoff that reaches past the neighbouring rank's latitudes raises at construction."""
     nli, nloi, nlo, nloo, ks, _, gi, go = LAYERS["iso"]
