@@ -232,6 +232,9 @@ def test_forward_matches_brute_force_without_p_shift(spec):
     out_b, y_b = brute.forward(spec, x, w, b, groups=G)
     np.testing.assert_allclose(y, y_b, rtol=0, atol=1e-12)
     np.testing.assert_allclose(out, out_b, rtol=0, atol=1e-12)
+    # the oracle's weight einsum on its own, from the brute force's y: the group index, the
+    # (c, k) pairing and the bias are fixed by the brute force's independent einsum
+    np.testing.assert_allclose(oracle.Psi(spec).mix(y_b, w, b, groups=G), out_b, rtol=0, atol=1e-12)
 
 
 def test_constant_field_and_impulse_response():
@@ -349,6 +352,25 @@ def test_dense_samples_match_sparse_contraction():
                         rng.integers(0, spec.nlat_out, 50), rng.integers(0, spec.nlon_out, 50)], axis=1)
         got = oracle.contract_dense_samples(spec, x, smp)
         np.testing.assert_allclose(got, y[tuple(smp.T)], atol=1e-13)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["downsample", "weather", "grouped"])
+def test_dense_samples_match_sparse_contraction_at_full_size(name):
+    # the sparse Psi of a full-size layer against the dense quadrature sum over every input point,
+    # on 16 output rows: both poles, the two rows next to each pole, the equator and random rows
+    spec = spec_of(WORKLOADS[name])
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((1, 2, spec.nlat_in, spec.nlon_in))
+    y = oracle.Psi(spec).contract(x)
+    n = spec.nlat_out
+    rows = [0, 1, 2, n - 3, n - 2, n - 1, n // 2]
+    rows += [int(r) for r in rng.choice(np.setdiff1d(np.arange(n), rows), 16 - len(rows), replace=False)]
+    m = len(rows) * 3
+    smp = np.stack([np.zeros(m, int), rng.integers(0, 2, m), rng.integers(0, spec.K, m),
+                    np.repeat(rows, 3), rng.integers(0, spec.nlon_out, m)], axis=1)
+    got = oracle.contract_dense_samples(spec, x, smp)
+    np.testing.assert_allclose(got, y[tuple(smp.T)], rtol=0, atol=1e-12)
 
 
 def test_near_tie_cutoff_is_rejected():
