@@ -233,7 +233,10 @@ disco_status disco_bwd_weight(const disco_psi* psi, int B, int C_in, int C_out, 
  *     identical bits.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call before any
- *     stream capture.
+ *     stream capture.  The address is kept together with the device's current context and
+ *     looked up again when that context changes (after cudaDeviceReset, for example), so
+ *     the first call after such a change also belongs before any capture.
+ *   - DISCO_ERR_CUDA when cudaGetDevice or the address lookup fails.
  *   - All calls share the one array and each call overwrites every entry it later reads,
  *     so nothing from an earlier call leaks into a result.  Calls that can overlap on the
  *     GPU (on different streams, or from threads that do not order their streams) race on
@@ -277,6 +280,37 @@ disco_status disco_plan_export(const disco_psi* psi, int which, int* rows, int* 
  * without a Toeplitz plan.  Host-only handles (device < 0) build the plans too. */
 disco_status disco_toeplitz_info(const disco_psi* psi, int which, int* dims);
 disco_status disco_toeplitz_export(const disco_psi* psi, int which, int* slabs, int* slots, unsigned short* b);
+
+/* Ring plans of the strip-staged tensor-core kernel (bf16 layers with nlon_in == nlon_out, a
+ * multiple of 8): which = 0 the forward plan with mirror rows, 1 the forward plan with plane
+ * pairs, 2 and 3 the same for the adjoint (output rows i of dx, source rows k*nlat_out + j of
+ * dy, one basis function).  For an output row r and a source row s, the forward equation on the
+ * page "torch_harmonics.DiscreteContinuousConvS2" (class description) is a correlation along
+ * the longitude ring with the same coefficients for every output longitude; for 16 outputs
+ * q0 + u and 16*ks source longitudes starting at q0 + 8*lo (lo = floor(pmin / 8)) it is the
+ * banded block B[p', (k, u)] = bf16(Psi_k(8*lo + p' - u)).  A plan is a script replayed for
+ * every tile (a strip of output rows, nb*16 output longitudes, 64 or 128 planes): loads put
+ * windows of source octets (8 longitudes) into ring slots, items apply a range of one block's
+ * K-steps to one load for every block of 16 outputs of the tile.  With mirror rows, M rows
+ * 64..127 of each MMA hold the north-south mirror of the output row and of each source row
+ * (built only when every mirror row's entries equal the row's own, mirrored, to 1e-12).
+ * disco_ring_info fills dims[16] = {K, N = 16K, mirror, nb, wmax (octets per slot), ring slots,
+ * row buffers, K-steps per B slot, B slots, grouped by source (0/1), strips, loads, items,
+ * rows, bf16 values, MMAs of one tile column}.  disco_ring_export copies into caller-owned
+ * HOST arrays: strips (x8: first item, end item, first load, end load, first row, end row,
+ * cost, 0; heaviest first), loads (x2: source row | mirror source row << 16, first octet
+ * relative to q0/8 (signed 16 bits) | octets << 16 | ring slot << 24), items (x4: load |
+ * row << 16 (strip-relative); a_off (signed 16 bits) | ks << 16 | flags << 24 (1 last use of
+ * the load, 2 last item of the row, 4 first item of the row); kb0 | nkb << 8 | octets of the
+ * load << 16 | row buffer << 24 | ring slot << 28; B offset of K-step kb0 in 16-byte units),
+ * rows (x2: r | mirror row
+ * << 16 (0xFFFF none); flags (1 no entries) | row buffer << 8) and the blocks ([ks][2][N][8]
+ * bf16 bits per (row, source) pair, column k*16 + u).  Block b, K-step k of an item reads
+ * octets a_off + 2b + 2k and the next of its load when both lie inside it.  Both return
+ * DISCO_ERR_UNSUPPORTED when that plan was not built.  Host-only handles build them too. */
+disco_status disco_ring_info(const disco_psi* psi, int which, int* dims);
+disco_status disco_ring_export(const disco_psi* psi, int which, int* strips, int* loads, int* items, int* rows,
+                               unsigned short* b);
 
 /* Packed Toeplitz plans (which = 0 forward, 1 adjoint): a source row's blocks for every output
  * row of a strip that it reaches, side by side, so that one staged window and one MMA serve

@@ -150,6 +150,38 @@ void free_pk(DevPk* d) {
   *d = DevPk{};
 }
 
+// Device copy of a ring plan (strip-staged tensor-core contraction).
+struct DevRing {
+  int* strips = nullptr;
+  int* loads = nullptr;
+  int* items = nullptr;
+  int* rows = nullptr;
+  uint16_t* b = nullptr;
+  int n_strips = 0;
+  bool ok = false;
+};
+
+cudaError_t upload_ring(const disco::RingPlan& P, DevRing* d) {
+  cudaError_t e;
+  if ((e = upload(P.strips, &d->strips)) != cudaSuccess) return e;
+  if ((e = upload(P.loads, &d->loads)) != cudaSuccess) return e;
+  if ((e = upload(P.items, &d->items)) != cudaSuccess) return e;
+  if ((e = upload(P.rows, &d->rows)) != cudaSuccess) return e;
+  if ((e = upload(P.b, &d->b)) != cudaSuccess) return e;
+  d->n_strips = (int)(P.strips.size() / 8);
+  d->ok = true;
+  return cudaSuccess;
+}
+
+void free_ring(DevRing* d) {
+  cudaFree(d->strips);
+  cudaFree(d->loads);
+  cudaFree(d->items);
+  cudaFree(d->rows);
+  cudaFree(d->b);
+  *d = DevRing{};
+}
+
 struct disco_psi {
   disco::Geometry g;
   int device = -1;
@@ -163,6 +195,12 @@ struct disco_psi {
   DevTz dtz, dtza;
   disco::PackedPlan pf, pa;           // packed forms of the same (rows they serve)
   DevPk dpf, dpa;
+  // ring plans of the strip-staged kernel: [0] forward with mirror rows, [1] forward with plane
+  // pairs, [2] adjoint with mirror rows, [3] adjoint with plane pairs (empty when not built)
+  disco::RingPlan ring[4];
+  bool ring_built[4] = {false, false, false, false};
+  std::string ring_msg[4];            // why a ring plan was not built
+  DevRing dring[4];
 };
 
 namespace {
@@ -294,6 +332,94 @@ WsLayout layout(const disco_psi* psi, int op, int B, int C_in, int C_out, int gr
 
 namespace {
 
+// Shape of the ring plan for a layer: blocks per tile, ring slots and their size, accumulator
+// row buffers and B slots, chosen so that shared memory (x ring + B slots + two y staging
+// blocks) and tensor memory (row buffers x blocks x 16K columns) fit.  K is the number of basis
+// functions per term (1 for the adjoint).  False when the kernel has no such shape.
+bool ring_params(int K, bool adjoint, disco::RingParams* p) {
+  p->src_order = adjoint ? 1 : 0;
+  p->target_strips = 24;
+  p->max_rows = 64;
+  // {nb, wmax, ns, nrb, bk, nbs, src_order, target strips, most rows per strip}
+  if (adjoint && K == 1) {
+    *p = disco::RingParams{4, 12, 8, 6, 4, 8, 1, 24, 64, {}};
+    return true;
+  }
+  if (!adjoint && K == 3) {
+    *p = disco::RingParams{4, 12, 6, 2, 4, 4, 0, 24, 64, {}};
+    return true;
+  }
+  if (!adjoint && K == 5) {
+    *p = disco::RingParams{4, 8, 5, 1, 4, 4, 0, 24, 64, {}};
+    return true;
+  }
+  return false;
+}
+
+// Ring plans of the strip-staged kernel for a bf16 stride-1 layer: forward and adjoint, each
+// with mirror rows (north-south mirror pairs share their Toeplitz blocks: mirror-symmetric
+// latitude grids and an isotropic basis; checked entry by entry) and with plane pairs.  A plan
+// that cannot be built is left out; the per-pair kernel serves that case.
+void build_ring_plans(disco_psi* h) {
+  const disco::Geometry& g = h->g;
+  const int J = g.nlat_out, I = g.nlat_in, K = g.K;
+  std::vector<disco::RingTerm> fwd, adj;
+  fwd.reserve(h->entries.size());
+  adj.reserve(h->entries.size());
+  for (const disco::PsiEntry& e : h->entries) {
+    fwd.push_back(disco::RingTerm{e.j, e.i, e.k, e.p, e.v});
+    adj.push_back(disco::RingTerm{e.i, e.k * J + e.j, 0, -e.p, e.v});
+  }
+  std::vector<int> mo_f(J), ms_f(I), mo_a(I), ms_a((size_t)K * J), key_a((size_t)K * J);
+  for (int j = 0; j < J; ++j) mo_f[j] = J - 1 - j;
+  for (int i = 0; i < I; ++i) ms_f[i] = mo_a[i] = I - 1 - i;
+  for (int k = 0; k < K; ++k)
+    for (int j = 0; j < J; ++j) {
+      ms_a[(size_t)k * J + j] = k * J + (J - 1 - j);
+      key_a[(size_t)k * J + j] = j * K + k;  // sources of one output row j adjacent, basis function inside
+    }
+  const std::vector<int> none;
+  for (int which = 0; which < 4; ++which) {
+    const bool adjoint = which >= 2, mirror = (which & 1) == 0;
+    disco::RingParams prm;
+    if (!ring_params(adjoint ? 1 : K, adjoint, &prm)) {
+      h->ring_msg[which] = "the strip-staged kernel has no shape for this number of basis functions";
+      continue;
+    }
+    if (adjoint) prm.src_key = key_a;
+    std::string msg;
+    h->ring_built[which] =
+        adjoint ? disco::make_ring_plan(I, K * J, g.nlon_in, 1, adj, mirror ? mo_a : none, mirror ? ms_a : none, prm,
+                                        h->ring[which], msg)
+                : disco::make_ring_plan(J, I, g.nlon_in, K, fwd, mirror ? mo_f : none, mirror ? ms_f : none, prm,
+                                        h->ring[which], msg);
+    if (!h->ring_built[which]) {
+      h->ring[which] = disco::RingPlan{};
+      h->ring_msg[which] = msg;
+    }
+  }
+}
+
+// Ring plan for a call with BC planes: mirror rows for at most 64 planes, plane pairs above 64;
+// -1 when the layer has none (the per-pair kernel runs).  The adjoint plans are built for
+// inspection only: on one B200 the strip-staged adjoint measured slower than the per-pair one
+// (721x1440: 0.85 against 0.72 ms; 361x720 with 512 planes: 4.92 against 4.68 ms), so the
+// device copies are not made and the adjoint keeps the per-pair kernel.
+int ring_choice(const disco_psi* psi, int BC, bool adjoint) {
+  if (adjoint) return -1;
+  const int base = 0;
+  if (BC <= 64) return psi->dring[base].ok ? base : -1;
+  return psi->dring[base + 1].ok ? base + 1 : -1;
+}
+
+disco::RingLaunch ring_launch(const disco_psi* psi, int which, int BC, int n_src_rows, int n_out_rows) {
+  const disco::RingPlan& P = psi->ring[which];
+  const DevRing& d = psi->dring[which];
+  disco::RingLaunch L{d.strips, d.loads, d.items, d.rows, d.b, d.n_strips, P.K, P.nb, P.wmax, P.ns, P.nrb,
+                      P.bk, P.nbs, P.mirror, BC, n_src_rows, n_out_rows, psi->g.nlon_in};
+  return L;
+}
+
 // Runs a banded gather as two launches so that the few bands with long staged rows do not set
 // the shared-memory size (and so the occupancy) of all the others: heavy bands run on the
 // plan's side stream, forked from and joined back to the caller's stream; light bands run on
@@ -338,6 +464,13 @@ disco_status launch_contract(const disco_psi* psi, int BC, disco_dtype dtype, co
   const disco::Geometry& g = psi->g;
   if (dtype == DISCO_BF16 && psi->tz_ok && !(reinterpret_cast<uintptr_t>(x) & 15) &&
       !(reinterpret_cast<uintptr_t>(y) & 15)) {
+    const int which = ring_choice(psi, BC, false);
+    if (which >= 0) {
+      // strip-staged kernel: each source row loaded once per tile for all the rows it reaches
+      cudaError_t e = disco::launch_contract_ring(ring_launch(psi, which, BC, g.nlat_in, g.nlat_out), x, y, st);
+      if (e != cudaSuccess) return cuda_fail(e, what);
+      return DISCO_OK;
+    }
     // Toeplitz blocks of Psi on tensor cores: the packed kernel for the rows its plan serves,
     // the per-pair kernel for the others (all rows without a packed plan)
     disco::TzLaunch L{psi->dtz.slabs, psi->dtz.row_begin, psi->dtz.slots, psi->dtz.b, psi->tz.K, psi->tz.parts,
@@ -400,6 +533,13 @@ disco_status launch_adjoint(const disco_psi* psi, int BC, disco_dtype dtype, con
   const disco::Geometry& g = psi->g;
   const bool bf16 = dtype == DISCO_BF16;
   if (bf16 && psi->tz_ok && !(reinterpret_cast<uintptr_t>(dx) & 15) && !(reinterpret_cast<uintptr_t>(dy) & 15)) {
+    const int which = ring_choice(psi, BC, true);
+    if (which >= 0) {
+      cudaError_t e =
+          disco::launch_contract_ring(ring_launch(psi, which, BC, g.K * g.nlat_out, g.nlat_in), dy, dx, st);
+      if (e != cudaSuccess) return cuda_fail(e, "adjoint contraction launch");
+      return DISCO_OK;
+    }
     // Toeplitz blocks of the reversed Psi on tensor cores: dy rows (k, j) are the source rows
     const disco::ToeplitzPlan& P = psi->tza;
     disco::TzLaunch T{psi->dtza.slabs, psi->dtza.row_begin, psi->dtza.slots, psi->dtza.b, P.K, P.parts, P.N,
@@ -455,7 +595,7 @@ disco_status disco_sync_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronisation");
   if (disco::take_mix_tc_status() | disco::take_fused_tc_status() | disco::take_contract_tc_status() |
-      disco::take_contract_tcp_status())
+      disco::take_contract_tcp_status() | disco::take_contract_ring_status())
     return fail(DISCO_ERR_TIMEOUT, "a bounded device-side wait expired");
   return DISCO_OK;
 }
@@ -546,6 +686,7 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
       h->pf = disco::make_packed_plan(g, h->entries, false, T, NR, kPackStrip, kPackKs);
     if (disco::packed_shape(1, true, &T, &NR))
       h->pa = disco::make_packed_plan(g, h->entries, true, T, NR, kPackStrip, kPackKs);
+    build_ring_plans(h);
   }
   if (device >= 0) {
     int prev = -1;
@@ -564,6 +705,13 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
       e = upload_tz(h->tz, &h->dtz);
       if (e == cudaSuccess) e = upload_tz(h->tza, &h->dtza);
       h->tz_ok = e == cudaSuccess;
+      // strip-staged kernel (DISCO_RING=0 keeps the per-pair kernels)
+      const char* rg = std::getenv("DISCO_RING");
+      if (e == cudaSuccess && !(rg && rg[0] == '0')) {
+        build_ring_plans(h);
+        for (int w = 0; w < 2 && e == cudaSuccess; ++w)
+          if (h->ring_built[w] && disco::ring_kernel_k(h->ring[w].K)) e = upload_ring(h->ring[w], &h->dring[w]);
+      }
       // Packed forms (one staged source row feeds up to 16 output rows, so 2.7-2.9 times fewer
       // bytes are staged).  Measured on one B200, the per-pair kernels are still faster on
       // every layer tried (the K = 9 adjoint within 1%, the 721x1440 contraction by 1.9x), so
@@ -593,6 +741,7 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
       free_tz(&h->dtza);
       free_pk(&h->dpf);
       free_pk(&h->dpa);
+      for (int w = 0; w < 4; ++w) free_ring(&h->dring[w]);
       delete h;
       return fail(DISCO_ERR_ALLOC, std::string("Psi upload failed: ") + cudaGetErrorString(e));
     }
@@ -631,6 +780,7 @@ disco_status disco_psi_destroy(disco_psi* psi) {
     free_tz(&psi->dtza);
     free_pk(&psi->dpf);
     free_pk(&psi->dpa);
+    for (int w = 0; w < 4; ++w) free_ring(&psi->dring[w]);
     if (psi->side) cudaStreamDestroy(psi->side);
     if (psi->fork) cudaEventDestroy(psi->fork);
     if (psi->join) cudaEventDestroy(psi->join);
@@ -710,6 +860,32 @@ disco_status disco_toeplitz_export(const disco_psi* psi, int which, int* slabs, 
   if (P.slots.empty()) return fail(DISCO_ERR_UNSUPPORTED, "no Toeplitz plan for this layer");
   std::memcpy(slabs, P.slabs.data(), P.slabs.size() * sizeof(disco::TzSlab));
   std::memcpy(slots, P.slots.data(), P.slots.size() * sizeof(int));
+  std::memcpy(b, P.b.data(), P.b.size() * sizeof(uint16_t));
+  return DISCO_OK;
+}
+
+disco_status disco_ring_info(const disco_psi* psi, int which, int* dims) {
+  if (!psi || !dims || which < 0 || which > 3) return fail(DISCO_ERR_INVALID_ARG, "bad ring plan query");
+  if (!psi->ring_built[which])
+    return fail(DISCO_ERR_UNSUPPORTED, "no ring plan of this kind for this layer: " + psi->ring_msg[which]);
+  const disco::RingPlan& P = psi->ring[which];
+  const int v[16] = {P.K, P.N, P.mirror, P.nb, P.wmax, P.ns, P.nrb, P.bk, P.nbs, P.src_order,
+                     (int)(P.strips.size() / 8), (int)(P.loads.size() / 2), (int)(P.items.size() / 4),
+                     (int)(P.rows.size() / 2), (int)P.b.size(), (int)std::min<long long>(P.mmas, INT32_MAX)};
+  std::memcpy(dims, v, sizeof(v));
+  return DISCO_OK;
+}
+
+disco_status disco_ring_export(const disco_psi* psi, int which, int* strips, int* loads, int* items, int* rows,
+                               unsigned short* b) {
+  if (!psi || !strips || !loads || !items || !rows || !b || which < 0 || which > 3)
+    return fail(DISCO_ERR_INVALID_ARG, "bad ring plan export");
+  if (!psi->ring_built[which]) return fail(DISCO_ERR_UNSUPPORTED, "no ring plan of this kind for this layer");
+  const disco::RingPlan& P = psi->ring[which];
+  std::memcpy(strips, P.strips.data(), P.strips.size() * sizeof(int));
+  std::memcpy(loads, P.loads.data(), P.loads.size() * sizeof(int));
+  std::memcpy(items, P.items.data(), P.items.size() * sizeof(int));
+  std::memcpy(rows, P.rows.data(), P.rows.size() * sizeof(int));
   std::memcpy(b, P.b.data(), P.b.size() * sizeof(uint16_t));
   return DISCO_OK;
 }
@@ -946,19 +1122,45 @@ namespace {
 
 std::mutex g_noalloc_mu;
 constexpr int kNoAllocMaxDevices = 64;
-float* g_noalloc_addr[kNoAllocMaxDevices] = {};
+// Per device: the context the address was looked up in, and the address.  A device reset (or any
+// other change of the current context on that device) reloads the library's module, so the
+// address is looked up again whenever the current context differs from the recorded one.
+struct NoAllocEntry {
+  void* ctx;
+  float* addr;
+};
+NoAllocEntry g_noalloc[kNoAllocMaxDevices] = {};
 
-// Device address of the scratch array on the current device `dev` (looked up once per device).
+typedef int (*CtxGetCurrentFn)(void**);
+
+// cuCtxGetCurrent through the runtime's driver entry point (no link against libcuda); NULL when
+// the driver does not provide it, in which case the address is looked up on every call.
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrentFn>(p);
+    return static_cast<CtxGetCurrentFn>(nullptr);
+  }();
+  return fn;
+}
+
+// Device address of the scratch array on the current device `dev`.
 disco_status noalloc_scratch(int dev, float** out) {
   if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(DISCO_ERR_UNSUPPORTED, "device ordinal above 63");
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
+  void* ctx = nullptr;
+  const CtxGetCurrentFn get = ctx_get_current_fn();
+  const bool known = get && get(&ctx) == 0 && ctx != nullptr;
+  if (!known || !g_noalloc[dev].addr || g_noalloc[dev].ctx != ctx) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static scratch");
-    g_noalloc_addr[dev] = static_cast<float*>(p);
+    g_noalloc[dev] = NoAllocEntry{known ? ctx : nullptr, static_cast<float*>(p)};
   }
-  *out = g_noalloc_addr[dev];
+  *out = g_noalloc[dev].addr;
   return DISCO_OK;
 }
 
@@ -984,7 +1186,8 @@ extern "C" disco_status disco_bwd_weight_noalloc(const disco_psi* psi, int B, in
   const int nc = (N + nchunk - 1) / nchunk;
   nchunk = (N + nc - 1) / nc;
   int dev = -1;
-  cudaGetDevice(&dev);
+  const cudaError_t de = cudaGetDevice(&dev);
+  if (de != cudaSuccess) return cuda_fail(de, "cudaGetDevice");
   float* scratch = nullptr;
   s = noalloc_scratch(dev, &scratch);
   if (s) return s;

@@ -72,6 +72,22 @@ bool packed_shape(int K, bool adjoint, int* T, int* NR);
 cudaError_t launch_contract_tcp(const TpLaunch& L, const void* x, void* y, cudaStream_t st, int grid_cap);
 int take_contract_tcp_status();
 
+// Strip-staged tensor-core contraction over a ring plan (contract_ring.cu, RingPlan in
+// psi_builder.h); src is [BC][n_src_rows][nlon], dst [BC][K][n_out_rows][nlon], bf16.
+struct RingLaunch {
+  const int* strips;   // device arrays of the ring plan
+  const int* loads;
+  const int* items;
+  const int* rows;
+  const void* b;
+  int n_strips;
+  int K, nb, wmax, ns, nrb, bk, nbs, mirror;
+  int BC, n_src_rows, n_out_rows, nlon;
+};
+bool ring_kernel_k(int K);
+cudaError_t launch_contract_ring(const RingLaunch& L, const void* src, void* dst, cudaStream_t st);
+int take_contract_ring_status();
+
 // Fused forward on the same plan: out = bias + mix(w, contraction(x)) with the y tile kept in
 // shared memory; for K = 3 or 5 and 64 input channels per group (bf16, stride 1).
 struct TzFused {

@@ -92,6 +92,12 @@ struct TzSlab {
 };
 constexpr int kTzSlabK = 4;  // most 16-longitude K-steps in one slab
 
+// Flags of the ring plan records (RingPlan in psi_builder.h, contract_ring.cu).
+constexpr int kRowEmpty = 1;      // row flag: no entries, the epilogue writes zeros
+constexpr int kItemLast = 1;      // item flag: last use of its load (the slot may be refilled)
+constexpr int kItemRowEnd = 2;    // item flag: last item of its row (the accumulator is complete)
+constexpr int kItemRowStart = 4;  // item flag: first item of its row
+
 // Staged elements of one source row for a block of qb outputs (a multiple of kAlign).  A task's
 // window starts at t0 + m0*step (t0 <= span - 1, m0 <= qb - kTaskR) and holds
 // (kTaskR - 1)*step + kChunkW elements, so the last element read is span + (qb - 1)*step + 6.

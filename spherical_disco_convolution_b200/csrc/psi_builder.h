@@ -123,6 +123,69 @@ struct PackedPlan {
 PackedPlan make_packed_plan(const Geometry& g, const std::vector<PsiEntry>& e, bool adjoint, int T, int NR,
                             int strip_rows, int ksmax);
 
+// Ring plan of the strip-staged tensor-core contraction (contract_ring.cu).
+//
+// The correlation of an output row r with a source row s (p-shift symmetry, page
+// "torch_harmonics.DiscreteContinuousConvS2", class description) is, for 16 consecutive
+// outputs, a product with a banded Toeplitz block: B[p', (k, u)] = Psi_k(8*lo + p' - u) for a
+// window of 16*ks source longitudes starting 8*lo after the first output (lo = floor(pmin/8)).
+// A tile covers nb such blocks of 16 outputs of a strip of consecutive output rows.  The plan is
+// a script replayed for every tile: `loads` put source-row windows (octets of 8 longitudes)
+// into a ring of shared-memory slots, `items` apply one Toeplitz block (a range of its K-steps)
+// to one loaded window for every block of the tile.  A source whose windows for all the rows of
+// a strip fit one slot is loaded once and shared by every row that reaches it; a longer window
+// is loaded in chunks, each used by one row.  M rows 0..63 of an MMA are 64 planes of the row,
+// rows 64..127 either the mirror row (mirror = 1: the north-south mirror of the output row and
+// of each source row, whose Psi blocks are the same) or the next 64 planes (mirror = 0).
+struct RingPlan {
+  int K = 0, N = 0;       // basis functions per term, MMA columns (16 outputs per function)
+  int mirror = 0;
+  int nb = 0;             // blocks of 16 outputs per tile
+  int wmax = 0;           // octets per ring slot
+  int ns = 0;             // ring slots
+  int nrb = 0;            // accumulator row buffers (tensor memory)
+  int bk = 0;             // Toeplitz K-steps per B slot
+  int nbs = 0;            // B slots
+  int src_order = 0;      // 0: items grouped by output row; 1: grouped by source
+  std::vector<int> strips;  // 8 ints per strip, heaviest first: item0, item1, load0, load1, row0, row1, cost, 0
+  std::vector<int> loads;   // 2 ints per load (see below)
+  std::vector<int> items;   // 4 ints per item (see ring_item_*)
+  std::vector<int> rows;    // 2 ints per row, in accumulator order: r | rbar << 16, flags (kRowEmpty)
+  std::vector<uint16_t> b;  // Toeplitz blocks (bf16 bits), per (row, source) pair ks K-steps of [2][N][8]
+  long long mmas = 0;       // MMAs of one tile column (all strips, one q-tile, one plane tile)
+  long long load_octets = 0;  // octets loaded per tile column
+};
+// (flags kRowEmpty, kItemLast, kItemRowEnd, kItemRowStart: plan.h)
+// load ints:  [0] source row | mirror source row << 16 (0xFFFF: none); [1] first octet (signed
+//             16 bits, relative to q0/8) | octets << 16 | ring slot << 24
+// item ints:  [0] load (strip-relative) | row (strip-relative) << 16; [1] a_off (signed 16 bits:
+//             octet of the pair's window start relative to the load's first octet) | ks << 16 |
+//             flags << 24; [2] kb0 | nkb << 8 | octets of the load << 16 | row buffer << 24 |
+//             ring slot << 28; [3] B
+//             offset of K-step kb0 in 16-byte units.  Block b, K-step k (kb0 <= k < kb0 + nkb,
+//             k < ks) reads octets a_off + 2b + 2k and the next one of the load, when both lie
+//             inside it; every (block, K-step) of a pair is covered by exactly one item.
+// row ints:   [0] r | rbar << 16 (rbar = r: self-mirror row, 0xFFFF: no mirror row);
+//             [1] flags | row buffer << 8
+
+struct RingTerm {
+  int out_row, src_row, k, off;
+  double v;
+};
+struct RingParams {
+  int nb, wmax, ns, nrb, bk, nbs;
+  int src_order;
+  int target_strips, max_rows;
+  std::vector<int> src_key;  // order of sources when items are grouped by source (empty: row index)
+};
+// Builds the ring plan from terms out[.., k, out_row, q] += v * src[.., src_row, q + off].
+// mirror_out / mirror_src: the mirror row of each output / source row (empty: no mirror mode).
+// Returns false (msg set) when the terms are not mirror-symmetric in mirror mode or when an
+// invariant of the ring protocol cannot be met.
+bool make_ring_plan(int n_out_rows, int n_src_rows, int nlon, int K, std::vector<RingTerm> terms,
+                    const std::vector<int>& mirror_out, const std::vector<int>& mirror_src, const RingParams& prm,
+                    RingPlan& P, std::string& msg);
+
 // Adjoint gather plan: output rows i of dx, sources rows (k, j) of dy, one accumulator,
 // output longitude l = stride*m + rho.
 GatherPlan make_adjoint_plan(const Geometry& g, const std::vector<PsiEntry>& e);

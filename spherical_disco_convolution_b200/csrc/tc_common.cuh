@@ -81,6 +81,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// mbar_wait for roles that may wait long (producers waiting for free slots, epilogue warps
+// waiting for rows, a second role on the same barrier): between polls the thread sleeps, up to
+// max_sleep_ns, so that spinning warps do not flood the shared-memory instruction queue that the
+// copying and MMA-issuing warps need.  Same bound and status as mbar_wait.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t max_sleep_ns = 256) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  uint32_t ns = 32;
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    __nanosleep(ns);
+    if (ns < max_sleep_ns) ns <<= 1;
+    if (globaltimer() - t0 > kWaitNs) {
+      atomicExch(&g_device_status, 5);
+      return false;
+    }
+  }
+}
+
 // 2D / 3D tiled TMA loads into shared memory, completion counted on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
   asm volatile(
@@ -141,6 +160,11 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void*
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until the committed bulk stores have finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Waits until at most N of the committed bulk stores are still reading shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read_le() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
 // Waits until the committed bulk stores are complete.
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // Named barrier over `count` threads (whole warps).

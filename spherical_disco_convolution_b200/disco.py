@@ -110,6 +110,8 @@ def _load():
         "disco_toeplitz_export": [P, I, IP, IP, ctypes.POINTER(ctypes.c_ushort)],
         "disco_packed_info": [P, I, IP],
         "disco_packed_export": [P, I, IP, IP, ctypes.POINTER(ctypes.c_ushort), IP],
+        "disco_ring_info": [P, I, IP],
+        "disco_ring_export": [P, I, IP, IP, IP, IP, ctypes.POINTER(ctypes.c_ushort)],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -234,6 +236,32 @@ def disco_packed_export(psi, which: int):
     _check(_lib.disco_packed_export(psi, which, ip(strips), ip(ent), b.ctypes.data_as(ctypes.POINTER(ctypes.c_ushort)),
                                     ip(rest)))
     return dict(K=K, Nr=Nr, NR=NR, T=T, strips=strips, entries=ent, b=b, rest=rest[:n_rest])
+
+
+RING_DIMS = ("K", "N", "mirror", "nb", "wmax", "ns", "nrb", "bk", "nbs", "src_order", "n_strips", "n_loads",
+             "n_items", "n_rows", "n_b", "mmas")
+
+
+def disco_ring_info(psi, which: int) -> dict:
+    """Shape of a ring plan: which = 0/1 forward (mirror rows / plane pairs), 2/3 adjoint."""
+    dims = np.zeros(16, dtype=np.int32)
+    _check(_lib.disco_ring_info(psi, which, dims.ctypes.data_as(ctypes.POINTER(ctypes.c_int))))
+    return dict(zip(RING_DIMS, (int(v) for v in dims)))
+
+
+def disco_ring_export(psi, which: int) -> dict:
+    """Ring plan records (see include/disco.h) as NumPy arrays."""
+    d = disco_ring_info(psi, which)
+    strips = np.zeros((d["n_strips"], 8), dtype=np.int32)
+    loads = np.zeros((d["n_loads"], 2), dtype=np.int32)
+    items = np.zeros((d["n_items"], 4), dtype=np.int32)
+    rows = np.zeros((d["n_rows"], 2), dtype=np.int32)
+    b = np.zeros(max(d["n_b"], 1), dtype=np.uint16)
+    ip = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))  # noqa: E731
+    _check(_lib.disco_ring_export(psi, which, ip(strips), ip(loads), ip(items), ip(rows),
+                                  b.ctypes.data_as(ctypes.POINTER(ctypes.c_ushort))))
+    d.update(strips=strips, loads=loads, items=items, rows=rows, b=b[:d["n_b"]])
+    return d
 
 
 def disco_workspace_size(psi, op, B, C_in, C_out, groups, dtype) -> int:

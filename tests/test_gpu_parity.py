@@ -226,9 +226,19 @@ def test_contract_tensor_core_matches_gather(name, monkeypatch):
                         "cuda:0")
     y_g = conv.disco_contract(psi_simt, x)
     torch.cuda.synchronize()
-    y_ref = oracle_psi(name).contract(inp["x"] if sel is None else inp["x"][:, sel])
-    check(host(y_tc), y_ref, 4e-3, "y (tensor cores)")
-    check(host(y_tc), host(y_g), 8e-3, "y (tensor cores vs gather)")
+    x_ref = inp["x"] if sel is None else inp["x"][:, sel]
+    y_ref = oracle_psi(name).contract(x_ref)
+    # The tensor-core blocks hold each Psi value rounded once to bf16 and y is rounded once to
+    # bf16 (8 significant bits: relative error <= u = 2^-8 each): with Psi >= 0 and every (k, j)
+    # row summing to one, the error is at most u (max|x| + max|y|), plus the same y rounding on the
+    # gather side.
+    u = 2.0 ** -8
+    bound = u * (np.abs(x_ref).max() + np.abs(y_ref).max())
+    err = np.abs(host(y_tc) - y_ref).max()
+    assert err <= 1.05 * bound, f"y (tensor cores): max err {err:.3e} > bound {bound:.3e}"
+    err_g = np.abs(host(y_tc) - host(y_g)).max()
+    assert err_g <= 1.05 * (bound + u * np.abs(y_ref).max()), f"y (tensor cores vs gather): {err_g:.3e}"
+    check(host(y_tc), y_ref, tol(wl), "y (tensor cores, bf16 tolerance)")
 
 
 @pytest.mark.parametrize("name", ["tc_small_bf16", "packed_k3", "weather", "grouped"])
@@ -291,6 +301,7 @@ def test_packed_kernel_matches_per_pair(name, monkeypatch):
     if sel is not None:
         x = x[:, sel].contiguous()
     dout, w = dev(inp["dout"], wl), dev(inp["w"], wl)
+    monkeypatch.setenv("DISCO_RING", "0")
     monkeypatch.setenv("DISCO_PACKED", "1")
     psi_p = conv.Psi(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape, wl.theta_cutoff, "cuda:0")
     y_p = conv.disco_contract(psi_p, x)
