@@ -54,6 +54,7 @@ def parse():
     ap.add_argument("--workload", default="weather")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the activation-memory and other-workload records")
     return ap.parse_args()
 
 
@@ -190,9 +191,10 @@ def cpu_sample_workload(wl):
     return wl.scaled(B=1, C_in=c, C_out=c, groups=g)
 
 
-def oracle_steps(wl, steps, warmup: int, min_seconds: float = 0.0):
+def oracle_steps(wl, steps, warmup: int, min_seconds: float = 0.0, threads: int = 0):
     """Times the CPU oracle on the channel sample: per step forward, forward again (the fused mode
-    computes the same out), dx, dw.  With min_seconds, repeats steps until that much time has passed.
+    computes the same out), dx, dw.  With min_seconds, repeats steps until that much time has passed;
+    threads > 0 sets the oracle's OpenMP thread count first.
     Returns (units per second, cores, sample description, seconds, steps)."""
     import oracle
     from spherical_disco_convolution_b200.workloads import make_inputs
@@ -201,6 +203,8 @@ def oracle_steps(wl, steps, warmup: int, min_seconds: float = 0.0):
     inp = make_inputs(sw, 0)
     P = oracle.Psi(oracle.Spec(sw.nlat_in, sw.nlon_in, sw.nlat_out, sw.nlon_out, sw.kernel_shape[0],
                                sw.kernel_shape[1], sw.theta_cutoff))
+    if threads > 0:
+        oracle.set_num_threads(threads)
 
     def step():
         P.forward(inp["x"], inp["w"], inp["bias"], groups=sw.groups)
@@ -220,6 +224,27 @@ def oracle_steps(wl, steps, warmup: int, min_seconds: float = 0.0):
     desc = (f"oracle fp64 on B={sw.B}, C {sw.C_in}->{sw.C_out} of the {sw.nlat_in}x{sw.nlon_in} grid "
             f"(Psi build untimed), {done} step(s) of fwd+fwd+dx+dw in {dt:.1f} s")
     return u / dt, oracle.num_threads(), desc, dt, done
+
+
+def cpu_baseline(wl) -> dict:
+    """The oracle timed on all host cores and on one thread, median of three runs each, on a
+    channel sample of the workload (about 20-40 s of CPU work in all)."""
+    import oracle
+
+    cores = os.cpu_count() or 1
+    runs_all = [oracle_steps(wl, 1, 1 if i == 0 else 0, min_seconds=2.0, threads=cores) for i in range(3)]
+    runs_one = [oracle_steps(wl, 1, 0, threads=1) for _ in range(3)]
+    oracle.set_num_threads(cores)
+    v_all = statistics.median(r[0] for r in runs_all)
+    v_one = statistics.median(r[0] for r in runs_one)
+    sw = cpu_sample_workload(wl)
+    note = (f"{runs_all[0][2]}; median of 3 runs on {cores} threads, and of 3 one-step runs on 1 thread "
+            f"({v_one:.4g} {UNIT}).  The sample has {sw.C_in} of {wl.C_in} channels: the oracle's weight "
+            f"einsum costs C_in/G*K = {sw.C_in // sw.groups * sw.K} multiply-adds per output point here "
+            f"against {wl.C_in // wl.groups * wl.K} on the full layer, so the sample overstates its "
+            f"throughput there")
+    return {"value": v_all, "unit": UNIT, "cores": runs_all[0][1], "kind": "oracle", "sample": note,
+            "one_thread": {"value": v_one, "unit": UNIT, "cores": 1}}
 
 
 def run_reference(args):
@@ -253,6 +278,107 @@ def workload_config(wl) -> dict:
             "l2": "inputs larger than L2 (x and y exceed 126 MB); no flush"}
 
 
+# ------------------------------------------------------ extra GPU records
+
+def activation_memory(wl, dev, dt, x) -> dict:
+    """What the autograd layer keeps for backward after one forward, unfused (y) and fused (x, which
+    the caller holds anyway): torch allocator bytes after the forward minus before it, less out."""
+    import torch
+
+    from spherical_disco_convolution_b200 import conv
+
+    res = {}
+    for fused in (False, True):
+        layer = conv.DiscreteContinuousConvS2(wl.C_in, wl.C_out, (wl.nlat_in, wl.nlon_in), (wl.nlat_out, wl.nlon_out),
+                                              wl.kernel_shape, groups=wl.groups, theta_cutoff=wl.theta_cutoff,
+                                              fused=fused, device=dev, dtype=dt)
+        torch.cuda.synchronize(dev)
+        base = torch.cuda.memory_allocated(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        out = layer(x)
+        torch.cuda.synchronize(dev)
+        kept = torch.cuda.memory_allocated(dev) - base - out.numel() * out.element_size()
+        peak = torch.cuda.max_memory_allocated(dev) - base
+        res["fused" if fused else "unfused"] = (kept / 1e6, peak / 1e6)
+        del out, layer
+        torch.cuda.synchronize(dev)
+    es = 2 if wl.dtype == "bf16" else 4
+    y_mb = wl.B * wl.C_in * wl.K * wl.nlat_out * wl.nlon_out * es / 1e6
+    return {"unfused_mb": res["unfused"][0], "fused_mb": res["fused"][0],
+            "saving_mb": res["unfused"][0] - res["fused"][0], "y_mb": y_mb,
+            "forward_peak_mb": {"unfused": res["unfused"][1], "fused": res["fused"][1]},
+            "how": "torch.cuda.memory_allocated after minus before one autograd forward, less out"}
+
+
+def workload_record(name: str, dev, steps: int = 5, warmup: int = 3) -> dict:
+    """Per-op times of another workload (same ops as the headline step, CUDA events on the
+    launching stream, median over the timed steps) with GB/s and the HBM roofline fraction."""
+    import numpy as np
+    import torch
+
+    from spherical_disco_convolution_b200 import conv
+    from spherical_disco_convolution_b200 import disco as D
+    from spherical_disco_convolution_b200.workloads import WORKLOADS, make_inputs
+
+    wl = WORKLOADS[name]
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    dcode = D.DISCO_BF16 if wl.dtype == "bf16" else D.DISCO_F32
+    psi = conv.Psi(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape, wl.theta_cutoff, dev)
+    inp = make_inputs(wl, 0)
+    t = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dt).to(dev) for k, v in inp.items() if v is not None}
+    sh = wl.shapes()
+    y, dy = (torch.empty(sh["y"], dtype=dt, device=dev) for _ in range(2))
+    out, out_f = (torch.empty(sh["out"], dtype=dt, device=dev) for _ in range(2))
+    dx = torch.empty(sh["x"], dtype=dt, device=dev)
+    dw = torch.empty(sh["w"], dtype=dt, device=dev)
+    db = torch.empty(sh["bias"], dtype=dt, device=dev) if "bias" in t else None
+    ws_dy, n_dy = psi.workspace(D.DISCO_OP_EINSUM_ADJOINT, wl.B, wl.C_in, wl.C_out, wl.groups, dcode)
+    ws_dw, n_dw = psi.workspace(D.DISCO_OP_BWD_WEIGHT, wl.B, wl.C_in, wl.C_out, wl.groups, dcode)
+    stream = torch.cuda.current_stream(dev)
+    st = stream.cuda_stream
+    p = lambda v: None if v is None else v.data_ptr()  # noqa: E731
+    h, B, Ci, Co, G = psi.handle, wl.B, wl.C_in, wl.C_out, wl.groups
+    calls = [
+        ("contract", lambda: D.disco_contract(h, B, Ci, dcode, p(t["x"]), p(y), st)),
+        ("einsum", lambda: D.disco_einsum(h, B, Ci, Co, G, dcode, p(y), p(t["w"]), p(t.get("bias")), p(out), st)),
+        ("fused", lambda: D.disco_fwd_fused(h, B, Ci, Co, G, dcode, p(t["x"]), p(t["w"]), p(t.get("bias")),
+                                            p(out_f), None, 0, st)),
+        ("dx", lambda: (D.disco_einsum_adjoint(h, B, Ci, Co, G, dcode, p(t["dout"]), p(t["w"]), p(dy), p(ws_dy),
+                                               n_dy, st),
+                        D.disco_contract_adjoint(h, B, Ci, dcode, p(dy), p(dx), st))),
+        ("dw", lambda: D.disco_bwd_weight(h, B, Ci, Co, G, dcode, p(t["dout"]), p(y), None, p(dw), p(db), p(ws_dw),
+                                          n_dw, st)),
+    ]
+    for _ in range(warmup):
+        for _, c in calls:
+            c()
+    torch.cuda.synchronize(dev)
+    ms = {k: [] for k, _ in calls}
+    for _ in range(steps):
+        for k, c in calls:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            c()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ms[k].append(e0.elapsed_time(e1))
+    peak, _ = measured_peaks()
+    alg = algorithmic_bytes(wl, psi.nnz)
+    ups = units_per_step(wl)
+    ops = {}
+    for k, _ in calls:
+        m = statistics.median(ms[k])
+        ops[k] = {"ms": m, "GBps": alg[k] / (m * 1e-3) / 1e9, "frac_hbm": alg[k] / (m * 1e-3) / 1e9 / peak,
+                  "alg_bytes": alg[k]}
+        if ups[k]:
+            ops[k]["units_per_s"] = ups[k] / (m * 1e-3)
+    train = ops["contract"]["ms"] + ops["einsum"]["ms"] + ops["dx"]["ms"] + ops["dw"]["ms"]
+    return {"config": workload_config(wl), "ops": ops, "training_step_ms": train,
+            "training_step": "contract + einsum + dx + dw (the unfused forward and the backward)",
+            "l2": "no flush: the step's tensors exceed 126 MB" if wl.name == "grouped" else
+                  "no flush between ops; inputs of this layer fit L2, so these times can include L2 hits"}
+
+
 # ------------------------------------------------------------------ GPU arm
 
 def run_gpu(args):
@@ -272,7 +398,7 @@ def run_gpu(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_steps(wl, 1, 0, min_seconds=10.0)  # before any GPU work starts
+        cpu = cpu_baseline(wl)  # before any GPU work starts
 
     psi = conv.Psi(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape, wl.theta_cutoff, dev)
     inp = make_inputs(wl, seed=rank)
@@ -395,6 +521,12 @@ def run_gpu(args):
 
     if rank != 0:
         return 0
+    extra = {}
+    if world == 1 and not args.no_extra:
+        extra["activation_memory"] = activation_memory(wl, dev, dt, x)
+        for name in ("grouped", "downsample"):
+            if name != wl.name:
+                extra[name] = workload_record(name, dev)
     peak, peak_kind = measured_peaks()
     alg = algorithmic_bytes(wl, psi.nnz)
     ops = {op: {"ms": op_ms[op], "GBps": alg[op] / (op_ms[op] * 1e-3) / 1e9,
@@ -414,9 +546,11 @@ def run_gpu(args):
         "gpu_launches": launches,
         "e2e": e2e,
     }
+    if extra:
+        line["activation_memory"] = extra.pop("activation_memory")
+        line["workloads"] = extra
     if cpu is not None:
-        line["cpu_baseline"] = {"value": cpu[0], "unit": UNIT, "cores": cpu[1], "kind": "oracle",
-                                "sample": cpu[2]}
+        line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
     return 0
 

@@ -79,6 +79,8 @@ def _L():
         lib.orc_backward_weight.argtypes = [P] + [ctypes.c_int] * 4 + [D, D, D, D]
         lib.orc_contract_dense_samples.argtypes = [S, ctypes.c_int, ctypes.c_int, D, ctypes.c_int] + [I] * 5 + [D]
         lib.orc_num_threads.restype = ctypes.c_int
+        lib.orc_set_num_threads.argtypes = [ctypes.c_int]
+        lib.orc_set_num_threads.restype = None
         _lib = lib
     return _lib
 
@@ -196,6 +198,11 @@ class OracleError(RuntimeError):
 
 def num_threads() -> int:
     return _L().orc_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's OpenMP loops from now on (for timing it on one core or on all)."""
+    _L().orc_set_num_threads(int(n))
 
 
 def cc_weights(nlat: int) -> np.ndarray:

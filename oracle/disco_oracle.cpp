@@ -466,6 +466,15 @@ int orc_contract_dense_samples(const orc_spec* o, int B, int C, const double* x,
   return status;
 }
 
+// Thread count of the OpenMP loops (n >= 1); used to time the oracle on one core and on all.
+void orc_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();
