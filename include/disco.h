@@ -312,20 +312,15 @@ disco_status disco_ring_info(const disco_psi* psi, int which, int* dims);
 disco_status disco_ring_export(const disco_psi* psi, int which, int* strips, int* loads, int* items, int* rows,
                                unsigned short* b);
 
-/* Packed Toeplitz plans (which = 0 forward, 1 adjoint): a source row's blocks for every output
- * row of a strip that it reaches, side by side, so that one staged window and one MMA serve
- * them all.  disco_packed_info fills dims[8] = {K, columns per output row Nr = 16K, slots NR,
- * groups of 16 outputs per tile T, strips, entries, bf16 values, rows left to the per-pair
- * plan}.  disco_packed_export copies into caller-owned HOST arrays: strips (x4: first entry,
- * end entry, first output row, rows), entries (x8: source row, window start lon_start,
- * ks | n_rows << 8 | first row o_a << 16 (strip-relative), block offset in 16-byte units,
- * mask of rows starting here, first completed row | mask of completed rows << 16, 0, 0),
- * blocks ([2*ks octets][n_rows*Nr][8] bf16 bits, column r*Nr + (h*K + k)*8 + u holding part h
- * of Psi_k for output row o_a + r at offset lon_start + p' - u) and the rows left to the
- * per-pair plan.  DISCO_ERR_UNSUPPORTED for layers without a packed plan. */
-disco_status disco_packed_info(const disco_psi* psi, int which, int* dims);
-disco_status disco_packed_export(const disco_psi* psi, int which, int* strips, int* entries, unsigned short* b,
-                                 int* rest);
+/* Self test of the failure path of the bounded device-side waits (the pages have no
+ * counterpart; it exercises the timeout status that every compute call can report).  Launches
+ * on `stream` a one-thread kernel that waits on an mbarrier nothing ever arrives on, gives up
+ * after limit_us microseconds (1 to 1000000) and records DISCO_ERR_TIMEOUT the way an expired
+ * wait inside a compute kernel does; the kernel then exits, so nothing is left waiting and the
+ * context stays usable.  A following disco_sync_status on the stream reports
+ * DISCO_ERR_TIMEOUT and clears the status.  INVALID_ARG for a limit out of range, CUDA for a
+ * launch error.  Asynchronous; allocates nothing. */
+disco_status disco_wait_selftest(unsigned int limit_us, void* stream);
 
 /* Synchronises `stream` and reports device-side failures of the calls queued on it
  * before: DISCO_ERR_CUDA for an asynchronous CUDA error, DISCO_ERR_TIMEOUT when a

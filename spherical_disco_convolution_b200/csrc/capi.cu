@@ -80,8 +80,6 @@ void free_plan(DevPlan* d) {
 }
 
 constexpr int kChannelsPerCta = 16;
-constexpr int kPackStrip = 32;  // output rows per strip of a packed plan
-constexpr int kPackKs = 4;      // widest window (K-steps of 16 longitudes) a packed entry takes
 constexpr int kStageFloats = 12288;          // 48 KB of staging for the unfused gathers
 constexpr size_t kSmemLimit = 227 * 1024;    // dynamic shared memory per CTA on sm_100
 constexpr size_t kFusedTileBytes = 160 * 1024;
@@ -112,42 +110,6 @@ void free_tz(DevTz* d) {
   cudaFree(d->slots);
   cudaFree(d->b);
   *d = DevTz{};
-}
-
-// Device copy of a packed Toeplitz plan and the row records of the rows it leaves to the
-// per-pair kernel.
-struct DevPk {
-  int* ent = nullptr;
-  int* strips = nullptr;
-  uint16_t* b = nullptr;
-  int* rest = nullptr;
-  int n_strips = 0, n_rest = 0;
-  bool ok = false;
-};
-
-cudaError_t upload_pk(const disco::PackedPlan& P, const disco::ToeplitzPlan& per_pair, DevPk* d) {
-  std::vector<char> is_rest(per_pair.row_begin.size(), 0);
-  for (int r : P.rest) is_rest[r] = 1;
-  std::vector<int> rest;  // the per-pair plan's row records of the rest rows, same order
-  for (size_t q = 0; q + 3 < per_pair.slots.size(); q += 4)
-    if (is_rest[per_pair.slots[q]]) rest.insert(rest.end(), per_pair.slots.begin() + q, per_pair.slots.begin() + q + 4);
-  d->n_strips = (int)(P.strips.size() / 4);
-  d->n_rest = (int)(rest.size() / 4);
-  cudaError_t e;
-  if ((e = upload(P.dev, &d->ent)) != cudaSuccess) return e;
-  if ((e = upload(P.strips, &d->strips)) != cudaSuccess) return e;
-  if ((e = upload(P.b, &d->b)) != cudaSuccess) return e;
-  if ((e = upload(rest, &d->rest)) != cudaSuccess) return e;
-  d->ok = true;
-  return cudaSuccess;
-}
-
-void free_pk(DevPk* d) {
-  cudaFree(d->ent);
-  cudaFree(d->strips);
-  cudaFree(d->b);
-  cudaFree(d->rest);
-  *d = DevPk{};
 }
 
 // Device copy of a ring plan (strip-staged tensor-core contraction).
@@ -193,8 +155,6 @@ struct disco_psi {
   bool tz_ok = false;                 // tensor-core contraction available (bf16 signals)
   disco::ToeplitzPlan tz, tza;        // forward (x -> y) and adjoint (dy -> dx) Toeplitz plans
   DevTz dtz, dtza;
-  disco::PackedPlan pf, pa;           // packed forms of the same (rows they serve)
-  DevPk dpf, dpa;
   // ring plans of the strip-staged kernel: [0] forward with mirror rows, [1] forward with plane
   // pairs, [2] adjoint with mirror rows, [3] adjoint with plane pairs (empty when not built)
   disco::RingPlan ring[4];
@@ -471,20 +431,9 @@ disco_status launch_contract(const disco_psi* psi, int BC, disco_dtype dtype, co
       if (e != cudaSuccess) return cuda_fail(e, what);
       return DISCO_OK;
     }
-    // Toeplitz blocks of Psi on tensor cores: the packed kernel for the rows its plan serves,
-    // the per-pair kernel for the others (all rows without a packed plan)
+    // Toeplitz blocks of Psi on tensor cores, one (output row, source row) pair at a time
     disco::TzLaunch L{psi->dtz.slabs, psi->dtz.row_begin, psi->dtz.slots, psi->dtz.b, psi->tz.K, psi->tz.parts,
                       psi->tz.N, BC, g.nlat_in, g.nlat_out, g.nlon_in};
-    if (psi->dpf.ok) {
-      const disco::PackedPlan& P = psi->pf;
-      disco::TpLaunch T{psi->dpf.ent, psi->dpf.strips, psi->dpf.b, P.K, P.T, P.NR, kPackKs,
-                        BC, g.nlat_in, g.nlat_out, g.nlon_in, psi->dpf.n_strips};
-      cudaError_t e = disco::launch_contract_tcp(T, x, y, st, 1 << 30);
-      if (e != cudaSuccess) return cuda_fail(e, what);
-      L.slots = psi->dpf.rest;
-      L.n_slots = psi->dpf.n_rest;
-      if (L.n_slots == 0) return DISCO_OK;
-    }
     cudaError_t e = disco::launch_contract_tc(L, x, y, st);
     if (e != cudaSuccess) return cuda_fail(e, what);
     return DISCO_OK;
@@ -544,16 +493,6 @@ disco_status launch_adjoint(const disco_psi* psi, int BC, disco_dtype dtype, con
     const disco::ToeplitzPlan& P = psi->tza;
     disco::TzLaunch T{psi->dtza.slabs, psi->dtza.row_begin, psi->dtza.slots, psi->dtza.b, P.K, P.parts, P.N,
                       BC, g.K * g.nlat_out, g.nlat_in, g.nlon_in};
-    if (psi->dpa.ok) {
-      const disco::PackedPlan& Q = psi->pa;
-      disco::TpLaunch L{psi->dpa.ent, psi->dpa.strips, psi->dpa.b, Q.K, Q.T, Q.NR, kPackKs,
-                        BC, g.K * g.nlat_out, g.nlat_in, g.nlon_in, psi->dpa.n_strips};
-      cudaError_t e = disco::launch_contract_tcp(L, dy, dx, st, 1 << 30);
-      if (e != cudaSuccess) return cuda_fail(e, "adjoint contraction launch");
-      T.slots = psi->dpa.rest;
-      T.n_slots = psi->dpa.n_rest;
-      if (T.n_slots == 0) return DISCO_OK;
-    }
     cudaError_t e = disco::launch_contract_tc(T, dy, dx, st);
     if (e != cudaSuccess) return cuda_fail(e, "adjoint contraction launch");
     return DISCO_OK;
@@ -591,11 +530,18 @@ const char* disco_last_error(void) { return g_last_error.c_str(); }
 
 unsigned long long disco_launch_count(void) { return disco::g_launches.load(); }
 
+disco_status disco_wait_selftest(unsigned int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return fail(DISCO_ERR_INVALID_ARG, "limit_us must be in [1, 1000000]");
+  const cudaError_t e = disco::launch_wait_selftest(limit_us, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "wait self-test launch");
+  return DISCO_OK;
+}
+
 disco_status disco_sync_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronisation");
   if (disco::take_mix_tc_status() | disco::take_fused_tc_status() | disco::take_contract_tc_status() |
-      disco::take_contract_tcp_status() | disco::take_contract_ring_status())
+      disco::take_contract_ring_status())
     return fail(DISCO_ERR_TIMEOUT, "a bounded device-side wait expired");
   return DISCO_OK;
 }
@@ -681,11 +627,6 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
     // host-only handle: the Toeplitz plans are built for inspection (disco_toeplitz_export)
     h->tz = disco::make_toeplitz_plan(g, h->entries);
     h->tza = disco::make_adjoint_toeplitz_plan(g, h->entries);
-    int T, NR;
-    if (disco::packed_shape(g.K, false, &T, &NR))
-      h->pf = disco::make_packed_plan(g, h->entries, false, T, NR, kPackStrip, kPackKs);
-    if (disco::packed_shape(1, true, &T, &NR))
-      h->pa = disco::make_packed_plan(g, h->entries, true, T, NR, kPackStrip, kPackKs);
     build_ring_plans(h);
   }
   if (device >= 0) {
@@ -712,21 +653,6 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
         for (int w = 0; w < 2 && e == cudaSuccess; ++w)
           if (h->ring_built[w] && disco::ring_kernel_k(h->ring[w].K)) e = upload_ring(h->ring[w], &h->dring[w]);
       }
-      // Packed forms (one staged source row feeds up to 16 output rows, so 2.7-2.9 times fewer
-      // bytes are staged).  Measured on one B200, the per-pair kernels are still faster on
-      // every layer tried (the K = 9 adjoint within 1%, the 721x1440 contraction by 1.9x), so
-      // the packed kernels run only when DISCO_PACKED=1.
-      const char* pk = std::getenv("DISCO_PACKED");
-      const bool force = pk && pk[0] == '1';
-      int T, NR;
-      if (e == cudaSuccess && force && disco::packed_shape(g.K, false, &T, &NR)) {
-        h->pf = disco::make_packed_plan(g, h->entries, false, T, NR, kPackStrip, kPackKs);
-        if (!h->pf.strips.empty()) e = upload_pk(h->pf, h->tz, &h->dpf);
-      }
-      if (e == cudaSuccess && force && disco::packed_shape(1, true, &T, &NR)) {
-        h->pa = disco::make_packed_plan(g, h->entries, true, T, NR, kPackStrip, kPackKs);
-        if (!h->pa.strips.empty()) e = upload_pk(h->pa, h->tza, &h->dpa);
-      }
     }
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->fork, cudaEventDisableTiming);
@@ -739,8 +665,6 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
       free_plan(&h->dadjb);
       free_tz(&h->dtz);
       free_tz(&h->dtza);
-      free_pk(&h->dpf);
-      free_pk(&h->dpa);
       for (int w = 0; w < 4; ++w) free_ring(&h->dring[w]);
       delete h;
       return fail(DISCO_ERR_ALLOC, std::string("Psi upload failed: ") + cudaGetErrorString(e));
@@ -778,8 +702,6 @@ disco_status disco_psi_destroy(disco_psi* psi) {
     free_plan(&psi->dadjb);
     free_tz(&psi->dtz);
     free_tz(&psi->dtza);
-    free_pk(&psi->dpf);
-    free_pk(&psi->dpa);
     for (int w = 0; w < 4; ++w) free_ring(&psi->dring[w]);
     if (psi->side) cudaStreamDestroy(psi->side);
     if (psi->fork) cudaEventDestroy(psi->fork);
@@ -887,34 +809,6 @@ disco_status disco_ring_export(const disco_psi* psi, int which, int* strips, int
   std::memcpy(items, P.items.data(), P.items.size() * sizeof(int));
   std::memcpy(rows, P.rows.data(), P.rows.size() * sizeof(int));
   std::memcpy(b, P.b.data(), P.b.size() * sizeof(uint16_t));
-  return DISCO_OK;
-}
-
-disco_status disco_packed_info(const disco_psi* psi, int which, int* dims) {
-  if (!psi || !dims || which < 0 || which > 1) return fail(DISCO_ERR_INVALID_ARG, "bad packed plan query");
-  const disco::PackedPlan& P = which == 0 ? psi->pf : psi->pa;
-  if (P.Nr == 0) return fail(DISCO_ERR_UNSUPPORTED, "no packed plan for this layer");
-  dims[0] = P.K;
-  dims[1] = P.Nr;
-  dims[2] = P.NR;
-  dims[3] = P.T;
-  dims[4] = (int)(P.strips.size() / 4);
-  dims[5] = (int)P.entries.size();
-  dims[6] = (int)P.b.size();
-  dims[7] = (int)P.rest.size();
-  return DISCO_OK;
-}
-
-disco_status disco_packed_export(const disco_psi* psi, int which, int* strips, int* entries, unsigned short* b,
-                                 int* rest) {
-  if (!psi || !strips || !entries || !b || !rest || which < 0 || which > 1)
-    return fail(DISCO_ERR_INVALID_ARG, "bad packed plan export");
-  const disco::PackedPlan& P = which == 0 ? psi->pf : psi->pa;
-  if (P.Nr == 0) return fail(DISCO_ERR_UNSUPPORTED, "no packed plan for this layer");
-  std::memcpy(strips, P.strips.data(), P.strips.size() * sizeof(int));
-  std::memcpy(entries, P.dev.data(), P.dev.size() * sizeof(int));
-  std::memcpy(b, P.b.data(), P.b.size() * sizeof(uint16_t));
-  std::memcpy(rest, P.rest.data(), P.rest.size() * sizeof(int));
   return DISCO_OK;
 }
 

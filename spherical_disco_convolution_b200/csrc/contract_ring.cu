@@ -501,7 +501,23 @@ cudaError_t launch_ring(const RingLaunch& L, const void* src, void* dst, cudaStr
   return e;
 }
 
+// Self test of the bounded waits: one thread waits on an mbarrier that nothing arrives on, for at
+// most limit_ns, and records the timeout in this file's status word like every expired wait.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  tc::mbar_init(&bar, 1);
+  tc::fence_barrier_init();
+  tc::mbar_wait_for(&bar, 0, limit_ns);
+}
+
 }  // namespace
+
+cudaError_t launch_wait_selftest(unsigned int limit_us, cudaStream_t st) {
+  wait_selftest_kernel<<<1, 32, 0, st>>>(1000ull * limit_us);
+  count_launch();
+  return cudaGetLastError();
+}
 
 bool ring_kernel_k(int K) { return K == 1 || K == 3 || K == 5 || K == 9; }
 

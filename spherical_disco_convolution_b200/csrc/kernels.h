@@ -59,19 +59,6 @@ struct TzLaunch {
 bool toeplitz_geometry(int K, int stride, int nlon_in, int nlon_out);
 bool contract_tc_supported(int K, int stride, int nlon_in, int nlon_out);
 cudaError_t launch_contract_tc(const TzLaunch& L, const void* x, void* y, cudaStream_t st);
-// Packed form (contract_tcp.cu): a source row staged once per tile and applied to all the
-// output rows it reaches in one MMA; the rows of a packed plan only (make_packed_plan).
-struct TpLaunch {
-  const int* ent;      // 8 ints per entry (PackedPlan::dev)
-  const int* strips;   // 4 ints per strip
-  const void* b;       // packed blocks (bf16)
-  int K, T, NR, ksmax;
-  int BC, n_src_rows, n_out_rows, nlon, n_strips;
-};
-bool packed_shape(int K, bool adjoint, int* T, int* NR);
-cudaError_t launch_contract_tcp(const TpLaunch& L, const void* x, void* y, cudaStream_t st, int grid_cap);
-int take_contract_tcp_status();
-
 // Strip-staged tensor-core contraction over a ring plan (contract_ring.cu, RingPlan in
 // psi_builder.h); src is [BC][n_src_rows][nlon], dst [BC][K][n_out_rows][nlon], bf16.
 struct RingLaunch {
@@ -85,6 +72,9 @@ struct RingLaunch {
   int BC, n_src_rows, n_out_rows, nlon;
 };
 bool ring_kernel_k(int K);
+// One-thread kernel whose wait on an mbarrier nothing arrives on expires after limit_us; the
+// expiry is reported by take_contract_ring_status like any bounded wait of the ring kernel.
+cudaError_t launch_wait_selftest(unsigned int limit_us, cudaStream_t st);
 cudaError_t launch_contract_ring(const RingLaunch& L, const void* src, void* dst, cudaStream_t st);
 int take_contract_ring_status();
 

@@ -90,39 +90,6 @@ ToeplitzPlan make_toeplitz_plan(const Geometry& g, const std::vector<PsiEntry>& 
 // (one basis function), offsets -p:  dx[c, i, l] = sum_{k,j} sum_p Psi_k(j, i, p) dy[c, k, j, l - p].
 ToeplitzPlan make_adjoint_toeplitz_plan(const Geometry& g, const std::vector<PsiEntry>& e);
 
-// Packed Toeplitz plan: a source row's blocks for all the output rows it reaches, side by side
-// in the MMA's N dimension, so one staged window and one MMA serve several output rows.
-// Consecutive output rows form strips; within a strip the source rows come in the order in
-// which their output rows advance, and each output row accumulates in one of NR tensor-memory
-// slots (slot = (row - strip start) mod NR) from its first source row to its last.  Rows that
-// the packing cannot serve (a window wider than ksmax K-steps, too many rows per source row,
-// more than NR rows live at once) are left to the per-pair plan (`rest`).
-struct PackedEntry {
-  int s;          // source row
-  int lon_start;  // window start relative to the first output of a group (multiple of 8)
-  int ks;         // K-steps of 16 longitudes
-  int boff;       // block offset in 16-byte units: [2*ks octets][n_rows*Nr][8] bf16
-  int o_a, n_rows;  // output rows o_a .. o_a + n_rows - 1 (strip-relative)
-  int new_mask;   // bit r: output row o_a + r gets its first contribution here
-  int done_begin, done_end;  // output rows completed after this entry: done[done_begin..done_end)
-  int done_base, done_mask;  // the same rows as done_base + bit index (increasing)
-};
-struct PackedPlan {
-  int K = 0, Nr = 0, NR = 0, T = 0;  // Nr = 16K columns per output row (hi and lo parts)
-  std::vector<int> strips;           // per strip: {entry_begin, entry_end, first row, rows}
-  std::vector<PackedEntry> entries;
-  std::vector<int> done;             // strip-relative output rows, in completion order
-  std::vector<uint16_t> b;
-  std::vector<int> rest;             // output rows left to the per-pair plan
-  std::vector<int> dev;              // per entry 8 ints for the device: {s, lon_start,
-                                     // ks | n_rows << 8 | o_a << 16, boff, new_mask,
-                                     // done_base | done_mask << 16, 0, 0}
-  long long mmas_per_group = 0;      // sum over entries of ks (one group of 16 outputs)
-};
-
-PackedPlan make_packed_plan(const Geometry& g, const std::vector<PsiEntry>& e, bool adjoint, int T, int NR,
-                            int strip_rows, int ksmax);
-
 // Ring plan of the strip-staged tensor-core contraction (contract_ring.cu).
 //
 // The correlation of an output row r with a source row s (p-shift symmetry, page

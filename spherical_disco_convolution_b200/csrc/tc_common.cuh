@@ -81,6 +81,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Waits for the phase with the given parity for at most limit_ns of wall time; false (and the
+// status word set to the timeout code) when the limit passes first.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    __nanosleep(256);
+    if (globaltimer() - t0 > limit_ns) {
+      atomicExch(&g_device_status, 5);
+      return false;
+    }
+  }
+}
+
 // mbar_wait for roles that may wait long (producers waiting for free slots, epilogue warps
 // waiting for rows, a second role on the same barrier): between polls the thread sleeps, up to
 // max_sleep_ns, so that spinning warps do not flood the shared-memory instruction queue that the

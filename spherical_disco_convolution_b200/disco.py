@@ -105,11 +105,10 @@ def _load():
         "disco_bwd_weight_noalloc": [P, I, I, I, I, I, P, P, P, P, P],
         "disco_plan_info": [P, I, IP],
         "disco_sync_status": [P],
+        "disco_wait_selftest": [ctypes.c_uint, P],
         "disco_plan_export": [P, I, IP, IP, IP, ctypes.POINTER(ctypes.c_float), IP],
         "disco_toeplitz_info": [P, I, IP],
         "disco_toeplitz_export": [P, I, IP, IP, ctypes.POINTER(ctypes.c_ushort)],
-        "disco_packed_info": [P, I, IP],
-        "disco_packed_export": [P, I, IP, IP, ctypes.POINTER(ctypes.c_ushort), IP],
         "disco_ring_info": [P, I, IP],
         "disco_ring_export": [P, I, IP, IP, IP, IP, ctypes.POINTER(ctypes.c_ushort)],
     }
@@ -145,6 +144,10 @@ def _check(status: int):
 
 def disco_sync_status(stream) -> None:
     _check(_lib.disco_sync_status(stream))
+
+
+def disco_wait_selftest(limit_us: int, stream) -> None:
+    _check(_lib.disco_wait_selftest(limit_us, stream))
 
 
 def disco_launch_count() -> int:
@@ -221,21 +224,6 @@ def disco_toeplitz_export(psi, which: int):
     _check(_lib.disco_toeplitz_export(psi, which, ip(slabs), ip(slots),
                                       b.ctypes.data_as(ctypes.POINTER(ctypes.c_ushort))))
     return dict(K=K, parts=parts, N=N, slabs=slabs, slots=slots, b=b, kslab=kslab, ksteps=ksteps)
-
-
-def disco_packed_export(psi, which: int):
-    """Packed Toeplitz plan: which=0 forward, which=1 adjoint."""
-    dims = np.zeros(8, dtype=np.int32)
-    _check(_lib.disco_packed_info(psi, which, dims.ctypes.data_as(ctypes.POINTER(ctypes.c_int))))
-    K, Nr, NR, T, n_strips, n_ent, n_b, n_rest = (int(v) for v in dims)
-    strips = np.zeros((n_strips, 4), dtype=np.int32)
-    ent = np.zeros((n_ent, 8), dtype=np.int32)
-    b = np.zeros(n_b, dtype=np.uint16)
-    rest = np.zeros(max(n_rest, 1), dtype=np.int32)
-    ip = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))  # noqa: E731
-    _check(_lib.disco_packed_export(psi, which, ip(strips), ip(ent), b.ctypes.data_as(ctypes.POINTER(ctypes.c_ushort)),
-                                    ip(rest)))
-    return dict(K=K, Nr=Nr, NR=NR, T=T, strips=strips, entries=ent, b=b, rest=rest[:n_rest])
 
 
 RING_DIMS = ("K", "N", "mirror", "nb", "wmax", "ns", "nrb", "bk", "nbs", "src_order", "n_strips", "n_loads",

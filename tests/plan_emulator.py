@@ -87,51 +87,6 @@ def toeplitz(plan, src, n_out_rows):
     return out
 
 
-def packed(plan, src, n_out_rows):
-    """Re-enacts the packed tensor-core kernel on a packed plan, in fp64, and checks its slot
-    protocol: every strip row starts once and completes once, after its last entry, and the
-    rows live at any entry sit in distinct slots (row mod NR).
-
-    src (B*C, source rows, nlon) -> out (B*C, K, n_out_rows, nlon), zero on the rows the plan
-    leaves to the per-pair kernel."""
-    K, Nr, NR = plan["K"], plan["Nr"], plan["NR"]
-    BC, _, nlon = src.shape
-    out = np.zeros((BC, K, n_out_rows, nlon))
-    vals = _bf16_values(plan["b"])
-    q = np.arange(nlon)
-    u = q % 8
-    q8 = q - u
-    for e0, e1, o0, nrows in plan["strips"]:
-        started, finished = set(), set()
-        for s_row, lon_start, w2, boff, new_mask, done, _, _ in plan["entries"][e0:e1]:
-            ks, n_rows, o_a = w2 & 0xFF, (w2 >> 8) & 0xFF, w2 >> 16
-            for r in range(n_rows):
-                o = o_a + r
-                if (new_mask >> r) & 1:
-                    assert o not in started
-                    started.add(o)
-                assert o in started and o not in finished, "contribution outside the row's life"
-            live = started - finished
-            assert len({o % NR for o in live}) == len(live), "two live rows share a slot"
-            n = 16 * ks
-            NC = n_rows * Nr
-            blk = vals[8 * boff: 8 * boff + 2 * ks * NC * 8].reshape(2 * ks, NC, 8)
-            bm = blk.transpose(0, 2, 1).reshape(n, n_rows, Nr)  # [p'][row][column]
-            idx = (q8[:, None] + lon_start + np.arange(n)[None, :]) % nlon
-            xs = src[:, s_row, :][:, idx]  # [c, q, p']
-            for r in range(n_rows):
-                wsum = (bm[:, r, : 8 * K] + bm[:, r, 8 * K: 16 * K]).reshape(n, K, 8)
-                coef = wsum[np.arange(n)[None, :], :, u[:, None]]  # [q, p', k]
-                out[:, :, o0 + o_a + r, :] += np.einsum("cqp,qpk->ckq", xs, coef)
-            base, mask = done & 0xFFFF, (done >> 16) & 0xFFFF
-            for bit in range(16):
-                if (mask >> bit) & 1:
-                    assert base + bit in started and base + bit not in finished
-                    finished.add(base + bit)
-        assert started == finished == set(range(nrows)), "a strip row never starts or never completes"
-    return out
-
-
 def _s16(v):
     v = int(v) & 0xFFFF
     return v - 0x10000 if v & 0x8000 else v

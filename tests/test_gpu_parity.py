@@ -40,9 +40,9 @@ EDGE = {
     # ragged last 128-output block, and K = 5 with one contraction accumulator buffer
     "tz_fused_k3": Workload("tz_fused_k3", 2, 128, 64, 2, 33, 192, 33, 192, (3, 1), 0.3, "bf16"),
     "tz_fused_k5": Workload("tz_fused_k5", 1, 64, 48, 1, 25, 64, 25, 64, (5, 1), 0.45, "bf16", bias=False),
-    # cutoff of two grid spacings, as on the 721x1440 layer: the packed tensor-core kernels take
-    # most rows (the polar rows stay per pair); 70 channels leave a partial second channel tile
-    "packed_k3": Workload("packed_k3", 1, 70, 64, 1, 65, 128, 65, 128, (3, 1), 2 * math.pi / 64, "bf16"),
+    # cutoff of two grid spacings, as on the 721x1440 layer: full-ring polar windows; 70 channels
+    # take the plane-pair form of the strip-staged contraction with a partial second group of 64
+    "ring_k3": Workload("ring_k3", 1, 70, 64, 1, 65, 128, 65, 128, (3, 1), 2 * math.pi / 64, "bf16"),
     # fused tensor-core forward with K = 9: one-half tiles of 64 outputs (ragged last tile)
     "tz_fused_k9": Workload("tz_fused_k9", 1, 128, 96, 2, 21, 160, 21, 160, (3, 4), 0.5, "bf16"),
 }
@@ -211,7 +211,7 @@ def test_invalid_calls_raise():
     assert e.value.status == D.DISCO_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("name", ["tc_small_bf16", "packed_k3", "weather", "grouped"])
+@pytest.mark.parametrize("name", ["tc_small_bf16", "ring_k3", "weather", "grouped"])
 def test_contract_tensor_core_matches_gather(name, monkeypatch):
     """The Toeplitz tensor-core contraction (bf16, stride 1) against the gather kernels and the
     oracle: both paths round y to bf16 once, so they agree to a few bf16 units."""
@@ -241,7 +241,7 @@ def test_contract_tensor_core_matches_gather(name, monkeypatch):
     check(host(y_tc), y_ref, tol(wl), "y (tensor cores, bf16 tolerance)")
 
 
-@pytest.mark.parametrize("name", ["tc_small_bf16", "packed_k3", "weather", "grouped"])
+@pytest.mark.parametrize("name", ["tc_small_bf16", "ring_k3", "weather", "grouped"])
 def test_adjoint_tensor_core_matches_gather(name, monkeypatch):
     """dx through the reversed-Psi Toeplitz blocks on tensor cores against the gather kernels and
     the oracle (bf16, stride 1)."""
@@ -289,32 +289,6 @@ def test_input_gradient_halves_compose(name):
     torch.cuda.synchronize()
     assert torch.equal(dx, dx_ref)
     check(host(dx), oracle_dx(name), tol(wl), "dx from the two halves")
-
-
-@pytest.mark.parametrize("name", ["packed_k3", "weather", "grouped"])
-def test_packed_kernel_matches_per_pair(name, monkeypatch):
-    """The packed Toeplitz kernels (a staged source row applied to all its output rows in one
-    MMA) against the per-pair kernels, for the contraction and the adjoint."""
-    wl, inp = workload(name), inputs(name)
-    sel = y_channels(wl)
-    x = dev(inp["x"], wl)
-    if sel is not None:
-        x = x[:, sel].contiguous()
-    dout, w = dev(inp["dout"], wl), dev(inp["w"], wl)
-    monkeypatch.setenv("DISCO_RING", "0")
-    monkeypatch.setenv("DISCO_PACKED", "1")
-    psi_p = conv.Psi(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape, wl.theta_cutoff, "cuda:0")
-    y_p = conv.disco_contract(psi_p, x)
-    dx_p = conv.disco_backward_input(psi_p, dout, w, wl.C_in, wl.groups)
-    monkeypatch.setenv("DISCO_PACKED", "0")
-    psi_pp = conv.Psi(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape, wl.theta_cutoff, "cuda:0")
-    y_pp = conv.disco_contract(psi_pp, x)
-    dx_pp = conv.disco_backward_input(psi_pp, dout, w, wl.C_in, wl.groups)
-    torch.cuda.synchronize()
-    check(host(y_p), host(y_pp), 8e-3, "y packed vs per pair")
-    check(host(dx_p), host(dx_pp), 8e-3, "dx packed vs per pair")
-    y_ref = oracle_psi(name).contract(inp["x"] if sel is None else inp["x"][:, sel])
-    check(host(y_p), y_ref, 4e-3, "y packed vs oracle")
 
 
 # Layers on the other latitude grids of the constructor's grid_in / grid_out: only Psi changes, so

@@ -57,6 +57,9 @@ LAYERS = [
     ("gauss", (24, 48, 24, (3,), 2 * math.pi / 24, 1, 1)),
     ("aniso", (17, 32, 17, (3, 4), 3 * math.pi / 16, 0, 0)),
     ("k5", (33, 64, 33, (5,), 4 * math.pi / 32, 0, 0)),
+    # cutoff of two grid spacings as on the 721x1440 layer: full-ring windows near the poles,
+    # loaded in chunks, and wrapping around the ring
+    ("two_spacings", (65, 128, 65, (3,), 2 * math.pi / 64, 0, 0)),
 ]
 
 
