@@ -308,6 +308,38 @@ disco_status disco_toeplitz_export(const disco_psi* psi, int which, int* slabs, 
  * bf16 bits per (row, source) pair, column k*16 + u).  Block b, K-step k of an item reads
  * octets a_off + 2b + 2k and the next of its load when both lie inside it.  Both return
  * DISCO_ERR_UNSUPPORTED when that plan was not built.  Host-only handles build them too. */
+/* Tile-script plans of the TMA-staged strip kernel (bf16 layers with nlon_in == nlon_out, a
+ * multiple of 8 and at least 64; K in {1, 3, 5}), same four kinds as the ring plans.  They
+ * hold the same products as the ring plans (Toeplitz blocks of Psi on 16 outputs, strips of
+ * output rows, 64 output longitudes per tile), with one script per (strip, longitude tile)
+ * (scripts strip-major, tile-minor):
+ *   tiles (x16: first load, end load, first copy, end copy, first row, end row, start of the
+ *     command stream of issuers 0..3 and its end, B batches, cost, 0, 0, 0);
+ *   loads (x4: source row | mirror source row << 16; ring slot | chunk mask << 8; first
+ *     longitude of chunk 0 (may be negative or past nlon: the staged box reads zeros there);
+ *     the script's batch that holds the load's last use).  Chunk c (bit c of the mask) stages the 64 longitudes from x0 + 56c of the row (M
+ *     rows 0..63) and of the mirror row or the next 64 planes (M rows 64..127), as 64 x 128-byte
+ *     rows in the 128-byte swizzle, at byte 32768*slot + 16384*c (+8192 for rows 64..127);
+ *   copies (x4: B offset in 16-byte units; bytes; byte offset in the B slot; flags (1 first of
+ *     a batch, 2 last of a batch) | bytes of the batch << 8);
+ *   cmds (issuer words: bit 31 clear: an MMA, A at 16*(bits 0-13) in the ring, B at
+ *     16*(bits 14-23) in the current B slot, row buffer bits 24-26, accumulate bit 27; bit 31
+ *     set: the commit of the current batch (8), then waits for the next batch (1), for the load
+ *     of slot bits 8-11 (2), for row buffer bits 12-14 to be free (4)).  The completion of a
+ *     batch releases its B slot and every ring slot and finished row whose last use it holds;
+ *   rows (x2: r | mirror row << 16; flags (1 no entries) | row buffer << 8 | the script's
+ *     batch that holds the row's last MMA << 12);
+ *   cta_tiles (n_ctas + 1 offsets, then the scripts of each CTA);
+ *   b (the Toeplitz blocks, [ks][2][N][8] bf16 bits per (row, source) pair).
+ * disco_tile_info fills dims[20] = {K, N, mirror, nb, ring slots, row buffers, B slots, bytes
+ * per B slot, grouped by source, strips, longitude tiles, CTAs, loads, copies, command words,
+ * rows, bf16 values, MMAs, TMA boxes, cta_tiles ints}; disco_tile_export copies every array
+ * into caller-owned HOST arrays of those sizes (tiles: 12 x strips x tiles).  Both return
+ * DISCO_ERR_UNSUPPORTED when that plan was not built.  Host-only handles build them too. */
+disco_status disco_tile_info(const disco_psi* psi, int which, int* dims);
+disco_status disco_tile_export(const disco_psi* psi, int which, int* tiles, int* loads, int* copies, unsigned int* cmds,
+                               int* rows, int* cta_tiles, unsigned short* b);
+
 disco_status disco_ring_info(const disco_psi* psi, int which, int* dims);
 disco_status disco_ring_export(const disco_psi* psi, int which, int* strips, int* loads, int* items, int* rows,
                                unsigned short* b);

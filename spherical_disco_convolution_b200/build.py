@@ -38,11 +38,18 @@ def build(force: bool = False, verbose: bool = False) -> str:
     build_dir = os.path.join(HERE, "_build")
     os.makedirs(build_dir, exist_ok=True)
     procs = []
+    headers = glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
+        glob.glob(os.path.join(INCLUDE, "*.h"))
+    t_hdr = max((os.path.getmtime(h) for h in headers), default=0.0)
     for src in sources():
         obj = os.path.join(build_dir, os.path.basename(src) + ".o")
+        objs.append(obj)
+        # an object newer than its source, every header and this script is reused
+        if not force and os.path.exists(obj) and \
+                os.path.getmtime(obj) > max(os.path.getmtime(src), t_hdr, os.path.getmtime(__file__)):
+            continue
         cmd = [nvcc, *ARCH, *FLAGS, "-I", INCLUDE, "-c", src, "-o", obj]
         procs.append((cmd, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)))
-        objs.append(obj)
     failed = False
     for cmd, p in procs:
         out, _ = p.communicate()

@@ -144,6 +144,47 @@ void free_ring(DevRing* d) {
   *d = DevRing{};
 }
 
+// Device copy of a tile-script plan (TMA-staged strip contraction).
+struct DevTile {
+  int* tiles = nullptr;
+  int* loads = nullptr;
+  int* copies = nullptr;
+  uint32_t* cmds = nullptr;
+  int* rows = nullptr;
+  int* cta_tiles = nullptr;
+  uint16_t* b = nullptr;
+  bool ok = false;
+};
+
+cudaError_t upload_tile(const disco::TilePlan& P, DevTile* d) {
+  cudaError_t e;
+  if ((e = upload(P.tiles, &d->tiles)) != cudaSuccess) return e;
+  if ((e = upload(P.loads, &d->loads)) != cudaSuccess) return e;
+  if ((e = upload(P.copies, &d->copies)) != cudaSuccess) return e;
+  {
+    // the issuers read their streams four words at a time with three groups ahead
+    std::vector<uint32_t> padded(P.cmds);
+    padded.resize(P.cmds.size() + 64, 0u);
+    if ((e = upload(padded, &d->cmds)) != cudaSuccess) return e;
+  }
+  if ((e = upload(P.rows, &d->rows)) != cudaSuccess) return e;
+  if ((e = upload(P.cta_tiles, &d->cta_tiles)) != cudaSuccess) return e;
+  if ((e = upload(P.b, &d->b)) != cudaSuccess) return e;
+  d->ok = true;
+  return cudaSuccess;
+}
+
+void free_tile(DevTile* d) {
+  cudaFree(d->tiles);
+  cudaFree(d->loads);
+  cudaFree(d->copies);
+  cudaFree(d->cmds);
+  cudaFree(d->rows);
+  cudaFree(d->cta_tiles);
+  cudaFree(d->b);
+  *d = DevTile{};
+}
+
 struct disco_psi {
   disco::Geometry g;
   int device = -1;
@@ -161,6 +202,11 @@ struct disco_psi {
   bool ring_built[4] = {false, false, false, false};
   std::string ring_msg[4];            // why a ring plan was not built
   DevRing dring[4];
+  // tile-script plans of the TMA-staged strip kernel, same four kinds as the ring plans
+  disco::TilePlan tile[4];
+  bool tile_built[4] = {false, false, false, false};
+  std::string tile_msg[4];
+  DevTile dtile[4];
 };
 
 namespace {
@@ -360,6 +406,88 @@ void build_ring_plans(disco_psi* h) {
   }
 }
 
+// Shape of the tile-script plan: five ring slots of two chunks (160 KB), three B slots (1 KB of
+// batch record and about 9 KB of Toeplitz K-steps each), the row
+// buffers that tensor memory holds (512 columns / (4 blocks x 16K)), and the y staging of the
+// epilogue (32 KB) within 227 KB of shared memory.
+bool tile_params(int K, bool adjoint, int n_ctas, disco::TileParams* p) {
+  if (!(K == 1 || K == 3 || K == 5)) return false;
+  p->nb = 4;
+  p->ns = 5;
+  p->nrb = std::min(8, 512 / (4 * 16 * K));
+  p->nbs = 3;
+  const int kstep = 2 * 16 * K * 16;
+  p->bslot_bytes = disco::kMetaBytes + (9216 / kstep) * kstep;  // the batch record, then the K-steps
+  p->src_order = adjoint ? 1 : 0;
+  p->target_strips = 24;
+  p->max_rows = 64;
+  p->n_ctas = n_ctas;
+  return true;
+}
+
+void build_tile_plans(disco_psi* h, int n_ctas) {
+  const disco::Geometry& g = h->g;
+  const int J = g.nlat_out, I = g.nlat_in, K = g.K;
+  std::vector<disco::RingTerm> fwd, adj;
+  fwd.reserve(h->entries.size());
+  adj.reserve(h->entries.size());
+  for (const disco::PsiEntry& e : h->entries) {
+    fwd.push_back(disco::RingTerm{e.j, e.i, e.k, e.p, e.v});
+    adj.push_back(disco::RingTerm{e.i, e.k * J + e.j, 0, -e.p, e.v});
+  }
+  std::vector<int> mo_f(J), ms_f(I), mo_a(I), ms_a((size_t)K * J), key_a((size_t)K * J);
+  for (int j = 0; j < J; ++j) mo_f[j] = J - 1 - j;
+  for (int i = 0; i < I; ++i) ms_f[i] = mo_a[i] = I - 1 - i;
+  for (int k = 0; k < K; ++k)
+    for (int j = 0; j < J; ++j) {
+      ms_a[(size_t)k * J + j] = k * J + (J - 1 - j);
+      key_a[(size_t)k * J + j] = j * K + k;
+    }
+  const std::vector<int> none;
+  for (int which = 0; which < 4; ++which) {
+    const bool adjoint = which >= 2, mirror = (which & 1) == 0;
+    disco::TileParams prm;
+    if (!tile_params(adjoint ? 1 : K, adjoint, n_ctas, &prm) || g.nlon_in < 64) {
+      h->tile_msg[which] = "the TMA-staged strip kernel has no shape for this layer";
+      continue;
+    }
+    if (adjoint) prm.src_key = key_a;
+    std::string msg;
+    h->tile_built[which] =
+        adjoint ? disco::make_tile_plan(I, K * J, g.nlon_in, 1, adj, mirror ? mo_a : none, mirror ? ms_a : none, prm,
+                                        h->tile[which], msg)
+                : disco::make_tile_plan(J, I, g.nlon_in, K, fwd, mirror ? mo_f : none, mirror ? ms_f : none, prm,
+                                        h->tile[which], msg);
+    if (!h->tile_built[which]) {
+      h->tile[which] = disco::TilePlan{};
+      h->tile_msg[which] = msg;
+    }
+  }
+}
+
+// Tile-script plan for a call with BC planes (mirror rows up to 64 planes, plane pairs above);
+// -1 when the layer has none.  DISCO_RING2=0 turns the kernel off, DISCO_RING2_ADJ=0 keeps the
+// adjoint on the other kernels.
+int tile_choice(const disco_psi* psi, int BC, bool adjoint) {
+  const char* off = std::getenv("DISCO_RING2");
+  if (off && off[0] == '0') return -1;
+  if (adjoint) {
+    const char* a = std::getenv("DISCO_RING2_ADJ");
+    if (a && a[0] == '0') return -1;
+  }
+  const int base = adjoint ? 2 : 0;
+  if (BC <= 64) return psi->dtile[base].ok ? base : -1;
+  return psi->dtile[base + 1].ok ? base + 1 : -1;
+}
+
+disco::Ring2Launch tile_launch(const disco_psi* psi, int which, int BC, int n_src_rows, int n_out_rows) {
+  const disco::TilePlan& P = psi->tile[which];
+  const DevTile& d = psi->dtile[which];
+  disco::Ring2Launch L{d.tiles, d.loads, d.copies, d.cmds, d.rows, d.cta_tiles, d.b, P.n_ctas, P.n_qt, P.K, P.nb,
+                       P.ns, P.nrb, P.nbs, P.bslot_bytes, P.mirror, BC, n_src_rows, n_out_rows, psi->g.nlon_in};
+  return L;
+}
+
 // Ring plan for a call with BC planes: mirror rows for at most 64 planes, plane pairs above 64;
 // -1 when the layer has none (the per-pair kernel runs).  The adjoint plans are built for
 // inspection only: on one B200 the strip-staged adjoint measured slower than the per-pair one
@@ -424,6 +552,13 @@ disco_status launch_contract(const disco_psi* psi, int BC, disco_dtype dtype, co
   const disco::Geometry& g = psi->g;
   if (dtype == DISCO_BF16 && psi->tz_ok && !(reinterpret_cast<uintptr_t>(x) & 15) &&
       !(reinterpret_cast<uintptr_t>(y) & 15)) {
+    const int wt = tile_choice(psi, BC, false);
+    if (wt >= 0) {
+      // TMA-staged strip kernel over the tile scripts
+      cudaError_t e = disco::launch_contract_ring2(tile_launch(psi, wt, BC, g.nlat_in, g.nlat_out), x, y, st);
+      if (e != cudaSuccess) return cuda_fail(e, what);
+      return DISCO_OK;
+    }
     const int which = ring_choice(psi, BC, false);
     if (which >= 0) {
       // strip-staged kernel: each source row loaded once per tile for all the rows it reaches
@@ -482,6 +617,13 @@ disco_status launch_adjoint(const disco_psi* psi, int BC, disco_dtype dtype, con
   const disco::Geometry& g = psi->g;
   const bool bf16 = dtype == DISCO_BF16;
   if (bf16 && psi->tz_ok && !(reinterpret_cast<uintptr_t>(dx) & 15) && !(reinterpret_cast<uintptr_t>(dy) & 15)) {
+    const int wt = tile_choice(psi, BC, true);
+    if (wt >= 0) {
+      cudaError_t e =
+          disco::launch_contract_ring2(tile_launch(psi, wt, BC, g.K * g.nlat_out, g.nlat_in), dy, dx, st);
+      if (e != cudaSuccess) return cuda_fail(e, "adjoint contraction launch");
+      return DISCO_OK;
+    }
     const int which = ring_choice(psi, BC, true);
     if (which >= 0) {
       cudaError_t e =
@@ -541,7 +683,7 @@ disco_status disco_sync_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronisation");
   if (disco::take_mix_tc_status() | disco::take_fused_tc_status() | disco::take_contract_tc_status() |
-      disco::take_contract_ring_status())
+      disco::take_contract_ring_status() | disco::take_contract_ring2_status())
     return fail(DISCO_ERR_TIMEOUT, "a bounded device-side wait expired");
   return DISCO_OK;
 }
@@ -628,6 +770,7 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
     h->tz = disco::make_toeplitz_plan(g, h->entries);
     h->tza = disco::make_adjoint_toeplitz_plan(g, h->entries);
     build_ring_plans(h);
+    build_tile_plans(h, 148);
   }
   if (device >= 0) {
     int prev = -1;
@@ -652,6 +795,11 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
         build_ring_plans(h);
         for (int w = 0; w < 2 && e == cudaSuccess; ++w)
           if (h->ring_built[w] && disco::ring_kernel_k(h->ring[w].K)) e = upload_ring(h->ring[w], &h->dring[w]);
+        int sms = 148;
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+        if (e == cudaSuccess) build_tile_plans(h, sms);
+        for (int w = 0; w < 4 && e == cudaSuccess; ++w)
+          if (h->tile_built[w] && disco::ring2_kernel_k(h->tile[w].K)) e = upload_tile(h->tile[w], &h->dtile[w]);
       }
     }
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
@@ -666,6 +814,7 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
       free_tz(&h->dtz);
       free_tz(&h->dtza);
       for (int w = 0; w < 4; ++w) free_ring(&h->dring[w]);
+      for (int w = 0; w < 4; ++w) free_tile(&h->dtile[w]);
       delete h;
       return fail(DISCO_ERR_ALLOC, std::string("Psi upload failed: ") + cudaGetErrorString(e));
     }
@@ -703,6 +852,7 @@ disco_status disco_psi_destroy(disco_psi* psi) {
     free_tz(&psi->dtz);
     free_tz(&psi->dtza);
     for (int w = 0; w < 4; ++w) free_ring(&psi->dring[w]);
+    for (int w = 0; w < 4; ++w) free_tile(&psi->dtile[w]);
     if (psi->side) cudaStreamDestroy(psi->side);
     if (psi->fork) cudaEventDestroy(psi->fork);
     if (psi->join) cudaEventDestroy(psi->join);
@@ -798,6 +948,34 @@ disco_status disco_ring_info(const disco_psi* psi, int which, int* dims) {
   return DISCO_OK;
 }
 
+disco_status disco_tile_info(const disco_psi* psi, int which, int* dims) {
+  if (!psi || !dims || which < 0 || which > 3) return fail(DISCO_ERR_INVALID_ARG, "bad tile plan query");
+  if (!psi->tile_built[which])
+    return fail(DISCO_ERR_UNSUPPORTED, "no tile plan of this kind for this layer: " + psi->tile_msg[which]);
+  const disco::TilePlan& P = psi->tile[which];
+  auto c = [](long long v) { return (int)std::min<long long>(v, INT32_MAX); };
+  const int v[20] = {P.K, P.N, P.mirror, P.nb, P.ns, P.nrb, P.nbs, P.bslot_bytes, P.src_order, P.n_strips, P.n_qt,
+                     P.n_ctas, c((long long)P.loads.size() / 4), c((long long)P.copies.size() / 4), c((long long)P.cmds.size()),
+                     c((long long)P.rows.size() / 2), c((long long)P.b.size()), c(P.mmas), c(P.boxes),
+                     c((long long)P.cta_tiles.size())};
+  std::memcpy(dims, v, sizeof(v));
+  return DISCO_OK;
+}
+disco_status disco_tile_export(const disco_psi* psi, int which, int* tiles, int* loads, int* copies, unsigned int* cmds,
+                               int* rows, int* cta_tiles, unsigned short* b) {
+  if (!psi || !tiles || !loads || !copies || !cmds || !rows || !cta_tiles || !b || which < 0 || which > 3)
+    return fail(DISCO_ERR_INVALID_ARG, "bad tile plan export");
+  if (!psi->tile_built[which]) return fail(DISCO_ERR_UNSUPPORTED, "no tile plan of this kind for this layer");
+  const disco::TilePlan& P = psi->tile[which];
+  std::memcpy(tiles, P.tiles.data(), P.tiles.size() * sizeof(int));
+  std::memcpy(loads, P.loads.data(), P.loads.size() * sizeof(int));
+  std::memcpy(copies, P.copies.data(), P.copies.size() * sizeof(int));
+  std::memcpy(cmds, P.cmds.data(), P.cmds.size() * sizeof(uint32_t));
+  std::memcpy(rows, P.rows.data(), P.rows.size() * sizeof(int));
+  std::memcpy(cta_tiles, P.cta_tiles.data(), P.cta_tiles.size() * sizeof(int));
+  std::memcpy(b, P.b.data(), P.b.size() * sizeof(uint16_t));
+  return DISCO_OK;
+}
 disco_status disco_ring_export(const disco_psi* psi, int which, int* strips, int* loads, int* items, int* rows,
                                unsigned short* b) {
   if (!psi || !strips || !loads || !items || !rows || !b || which < 0 || which > 3)

@@ -71,6 +71,23 @@ struct RingLaunch {
   int K, nb, wmax, ns, nrb, bk, nbs, mirror;
   int BC, n_src_rows, n_out_rows, nlon;
 };
+// TMA-staged strip contraction over a tile-script plan (contract_ring2.cu, TilePlan in
+// psi_builder.h); src is [BC][n_src_rows][nlon], dst [BC][K][n_out_rows][nlon], bf16.
+struct Ring2Launch {
+  const int* tiles;  // device arrays of the tile-script plan
+  const int* loads;
+  const int* copies;
+  const uint32_t* cmds;
+  const int* rows;
+  const int* cta_tiles;
+  const void* b;
+  int n_ctas, n_qt;
+  int K, nb, ns, nrb, nbs, bslot_bytes, mirror;
+  int BC, n_src_rows, n_out_rows, nlon;
+};
+bool ring2_kernel_k(int K);
+cudaError_t launch_contract_ring2(const Ring2Launch& L, const void* src, void* dst, cudaStream_t st);
+int take_contract_ring2_status();
 bool ring_kernel_k(int K);
 // One-thread kernel whose wait on an mbarrier nothing arrives on expires after limit_us; the
 // expiry is reported by take_contract_ring_status like any bounded wait of the ring kernel.

@@ -98,6 +98,22 @@ constexpr int kItemLast = 1;      // item flag: last use of its load (the slot m
 constexpr int kItemRowEnd = 2;    // item flag: last item of its row (the accumulator is complete)
 constexpr int kItemRowStart = 4;  // item flag: first item of its row
 
+// Tile-script plan (TilePlan in psi_builder.h, contract_ring2.cu).
+constexpr int kTileInts = 16;  // per script: load0, load1, copy0, copy1, row0, row1, record0, record1, 0, 0, 0,
+                               // batches, cost, 0, 0, 0
+// Copy flags: first / last copy of a batch, the copy of the batch record (source: the records).
+constexpr int kCopyBatchStart = 1, kCopyBatchEnd = 2, kCopyMeta = 4;
+// A batch's B slot holds its record in the first kMetaBytes: a header of four words (MMA counts
+// of issuers 0..3 in bytes 0..3; word offsets of the lists of issuers 1..3 in 10-bit fields;
+// load starts: count | ring slots << 3 + 4i; row starts: count | row buffers << 3 + 3i) and
+// each issuer's MMA words.  MMA word: A address >> 4 relative to the x ring (bits 0-13), B
+// offset >> 4 in the B slot (bits 14-23), row buffer (bits 24-26), accumulate (bit 27).
+constexpr int kMetaBytes = 1024;
+constexpr int kMaxMetaWords = kMetaBytes / 4;
+constexpr int kMaxLoadStarts = 6, kMaxRowStarts = 4;
+constexpr int kChunkBytes = 16384;  // one staged chunk: 2 groups x 64 planes x 128 bytes
+constexpr int kSlotBytes = 2 * kChunkBytes;
+
 // Staged elements of one source row for a block of qb outputs (a multiple of kAlign).  A task's
 // window starts at t0 + m0*step (t0 <= span - 1, m0 <= qb - kTaskR) and holds
 // (kTaskR - 1)*step + kChunkW elements, so the last element read is span + (qb - 1)*step + 6.

@@ -153,6 +153,43 @@ bool make_ring_plan(int n_out_rows, int n_src_rows, int nlon, int K, std::vector
                     const std::vector<int>& mirror_out, const std::vector<int>& mirror_src, const RingParams& prm,
                     RingPlan& P, std::string& msg);
 
+// Tile-script plan of the TMA-staged strip contraction (contract_ring2.cu).  Same products as
+// RingPlan (Toeplitz blocks of the p-shift symmetry, strips of output rows, nb blocks of 16
+// outputs per tile), with one script per (strip, longitude tile) so that every index, shared-
+// memory address and seam crossing is fixed on the host:
+//   * a load is a source-row window staged by TMA as up to two chunks of 8 octets (64 longitudes,
+//     128-byte swizzled rows of 64 planes, 16 KB with both M groups); chunk c starts 7c octets
+//     after the window, so every K-step (two octets) lies inside one chunk.  A window that
+//     crosses the longitude seam is split into pieces, each staged at its own shift with zeros
+//     outside [0, nlon) (the TMA fill), and a K-step that straddles the seam is applied to both;
+//   * B copies move each batch's record and its items' Toeplitz K-steps into a B slot (one
+//     barrier each); the record lists, for each of the four MMA issuers (issuer b owns block b),
+//     its MMAs with absolute operand addresses, and the loads and rows that start in the batch;
+//   * the completion of a batch (one commit per issuer) releases its B slot and every ring slot
+//     and finished row whose last use it holds.
+struct TileParams {
+  int nb = 4, ns = 5, nrb = 2, nbs = 3, bslot_bytes = 12288;
+  int src_order = 0;
+  int target_strips = 24, max_rows = 64;
+  int n_ctas = 148;
+  std::vector<int> src_key;
+};
+struct TilePlan {
+  int K = 0, N = 0, mirror = 0, nb = 0, ns = 0, nrb = 0, nbs = 0, bslot_bytes = 0, src_order = 0;
+  int n_strips = 0, n_qt = 0, n_ctas = 0;
+  std::vector<int> tiles;     // kTileInts per script (strip-major, then longitude tile)
+  std::vector<int> loads;     // 4 ints: s | sbar << 16; slot | chunk mask << 8; x0 (longitude of chunk 0); 0
+  std::vector<int> copies;    // 4 ints: B offset (16-byte units); bytes; offset in the B slot; flags | batch bytes << 8
+  std::vector<uint32_t> cmds; // batch records (header and the issuers' MMA words, kMetaBytes in plan.h)
+  std::vector<int> rows;      // 2 ints: r | rbar << 16; flags | row buffer << 8 (start order, empty rows last)
+  std::vector<int> cta_tiles; // n_ctas + 1 offsets, then the scripts of each CTA
+  std::vector<uint16_t> b;    // Toeplitz blocks, per (row, source) pair ks K-steps of [2][N][8]
+  long long mmas = 0, boxes = 0, copies_bytes = 0, items = 0;  // totals over all scripts
+};
+bool make_tile_plan(int n_out_rows, int n_src_rows, int nlon, int K, std::vector<RingTerm> terms,
+                    const std::vector<int>& mirror_out, const std::vector<int>& mirror_src, const TileParams& prm,
+                    TilePlan& P, std::string& msg);
+
 // Adjoint gather plan: output rows i of dx, sources rows (k, j) of dy, one accumulator,
 // output longitude l = stride*m + rho.
 GatherPlan make_adjoint_plan(const Geometry& g, const std::vector<PsiEntry>& e);

@@ -111,6 +111,8 @@ def _load():
         "disco_toeplitz_export": [P, I, IP, IP, ctypes.POINTER(ctypes.c_ushort)],
         "disco_ring_info": [P, I, IP],
         "disco_ring_export": [P, I, IP, IP, IP, IP, ctypes.POINTER(ctypes.c_ushort)],
+        "disco_tile_info": [P, I, IP],
+        "disco_tile_export": [P, I, IP, IP, IP, ctypes.POINTER(ctypes.c_uint), IP, IP, ctypes.POINTER(ctypes.c_ushort)],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -235,6 +237,36 @@ def disco_ring_info(psi, which: int) -> dict:
     dims = np.zeros(16, dtype=np.int32)
     _check(_lib.disco_ring_info(psi, which, dims.ctypes.data_as(ctypes.POINTER(ctypes.c_int))))
     return dict(zip(RING_DIMS, (int(v) for v in dims)))
+
+
+TILE_DIMS = ("K", "N", "mirror", "nb", "ns", "nrb", "nbs", "bslot_bytes", "src_order", "n_strips", "n_qt",
+             "n_ctas", "n_loads", "n_copies", "n_cmds", "n_rows", "n_b", "mmas", "boxes", "n_cta_ints")
+
+
+def disco_tile_info(psi, which: int) -> dict:
+    """Shape of a tile-script plan: which = 0/1 forward (mirror rows / plane pairs), 2/3 adjoint."""
+    dims = np.zeros(20, dtype=np.int32)
+    _check(_lib.disco_tile_info(psi, which, dims.ctypes.data_as(ctypes.POINTER(ctypes.c_int))))
+    return dict(zip(TILE_DIMS, (int(v) for v in dims)))
+
+
+def disco_tile_export(psi, which: int) -> dict:
+    """Tile-script plan records (see include/disco.h) as NumPy arrays."""
+    d = disco_tile_info(psi, which)
+    tiles = np.zeros((d["n_strips"] * d["n_qt"], 16), dtype=np.int32)
+    loads = np.zeros((d["n_loads"], 4), dtype=np.int32)
+    copies = np.zeros((d["n_copies"], 4), dtype=np.int32)
+    cmds = np.zeros(max(d["n_cmds"], 1), dtype=np.uint32)
+    rows = np.zeros((d["n_rows"], 2), dtype=np.int32)
+    cta = np.zeros(d["n_cta_ints"], dtype=np.int32)
+    b = np.zeros(max(d["n_b"], 1), dtype=np.uint16)
+    ip = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))  # noqa: E731
+    _check(_lib.disco_tile_export(psi, which, ip(tiles), ip(loads), ip(copies),
+                                  cmds.ctypes.data_as(ctypes.POINTER(ctypes.c_uint)), ip(rows), ip(cta),
+                                  b.ctypes.data_as(ctypes.POINTER(ctypes.c_ushort))))
+    d.update(tiles=tiles, loads=loads, copies=copies, cmds=cmds[:d["n_cmds"]], rows=rows, cta_tiles=cta,
+             b=b[:d["n_b"]])
+    return d
 
 
 def disco_ring_export(psi, which: int) -> dict:
