@@ -104,6 +104,45 @@ struct WarpStream {
 };
 
 
+// A window of 32 records of a plan array held by a warp (one per lane) with the next 32 in
+// flight; at(l) (l increasing, warp-uniform) returns record l + lane to each lane (records past
+// the end read as zeros).
+template <typename T>
+struct WarpWindow {
+  const T* p;
+  int end, base;
+  T cur, nxt;
+  __device__ __forceinline__ T fetch(int b) const {
+    const int i = b + (int)(threadIdx.x & 31);
+    T v{};
+    if (i < end) v = p[i];
+    return v;
+  }
+  __device__ __forceinline__ void start(const T* p_, int begin, int end_) {
+    p = p_;
+    end = end_;
+    base = begin;
+    cur = fetch(base);
+    nxt = fetch(base + 32);
+  }
+  __device__ __forceinline__ T at(int l) {
+    while (l >= base + 32) {
+      base += 32;
+      cur = nxt;
+      nxt = fetch(base + 32);
+    }
+    const int i = l - base + (int)(threadIdx.x & 31);  // 0 .. 62
+    const T a = shfl_any(cur, i & 31), b = shfl_any(nxt, i & 31);
+    return i < 32 ? a : b;
+  }
+  __device__ __forceinline__ static T shfl_any(const T& v, int src) {
+    if constexpr (sizeof(T) == 16)
+      return shfl4(v, src);
+    else
+      return shfl2(v, src);
+  }
+};
+
 struct Script {
   int load0, load1, copy0, copy1, row0, row1, nbatch;
 };
@@ -241,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
             }
           }
           ok = __shfl_sync(0xffffffffu, good, 0) != 0;
-          const uint32_t r = gbase + (uint32_t)ld.w + 1;
+          const uint32_t r = gbase + (uint32_t)(ld.w & 0xFFFF) + 1;
 #pragma unroll
           for (int s = 0; s < kMaxSlots; ++s)
             if (s == slot) rel[s] = r;
@@ -251,11 +290,13 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------------ B copies
-    // each batch: wait until its B slot's previous batch has completed, then its items' K-steps
+    // each batch: wait until its B slot's previous batch has completed, arm the slot's barrier
+    // with the batch's bytes, and issue its copies (the record, then the items' K-steps), one
+    // per lane
     int bslot = 0;
     uint32_t nbatch = 0;  // batches started by this CTA
     bool ok = true;
-    WarpStream<int4> cs;
+    WarpWindow<int4> win;
     for (int t = t_begin; t < t_end && ok; ++t) {
       const Script sc = read_script(a, my[t], -1);
       if (lane == 0 && t + 1 < t_end) {
@@ -263,25 +304,26 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
         l2_prefetch(a.copies + nx.copy0, (uint32_t)(nx.copy1 - nx.copy0) * 16u);
       }
       for (int pt = 0; pt < a.n_pt && ok; ++pt) {
-        cs.start(a.copies, sc.copy0, sc.copy1);
-        for (int n = sc.copy0; n < sc.copy1 && ok; ++n) {
-          const int4 cp = cs.get(n);
-          const int flags = cp.w & 0xFF;
+        win.start(a.copies, sc.copy0, sc.copy1);
+        for (int c = sc.copy0; c < sc.copy1 && ok;) {
+          const int4 cp = win.at(c);  // copy c + lane; copy c is the batch record's
+          const int w0 = __shfl_sync(0xffffffffu, cp.w, 0);
+          const int n = (w0 >> 24) & 0xFF;
           int good = 1;
           if (lane == 0) {
-            if ((flags & kCopyBatchStart) && nbatch >= (uint32_t)a.nbs) good = wait_batches(done, nbatch - a.nbs + 1, 256);
-            if (good) {
-              if (flags & kCopyBatchStart) tc::mbar_arrive_expect_tx(&bfull[bslot], (uint32_t)(cp.w >> 8));
-              const uint8_t* src = (flags & kCopyMeta) ? reinterpret_cast<const uint8_t*>(a.cmds) : a.b;
-              tc::bulk_load(sB + (size_t)bslot * a.bslot_bytes + cp.z, src + (size_t)(uint32_t)cp.x * 16,
-                            (uint32_t)cp.y, &bfull[bslot]);
-            }
+            if (nbatch >= (uint32_t)a.nbs) good = wait_batches(done, nbatch - a.nbs + 1, 256);
+            if (good) tc::mbar_arrive_expect_tx(&bfull[bslot], (uint32_t)((w0 >> 8) & 0xFFFF));
           }
           ok = __shfl_sync(0xffffffffu, good, 0) != 0;
-          if (flags & kCopyBatchEnd) {
-            ++nbatch;
-            bslot = (bslot + 1 == a.nbs) ? 0 : bslot + 1;
+          if (!ok) break;
+          if (lane < n) {
+            const uint8_t* src = (cp.w & kCopyMeta) ? reinterpret_cast<const uint8_t*>(a.cmds) : a.b;
+            tc::bulk_load(sB + (size_t)bslot * a.bslot_bytes + cp.z, src + (size_t)(uint32_t)cp.x * 16, (uint32_t)cp.y,
+                          &bfull[bslot]);
           }
+          c += n;
+          ++nbatch;
+          bslot = (bslot + 1 == a.nbs) ? 0 : bslot + 1;
         }
       }
     }
@@ -297,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
         const Script sc = read_script(a, my[t], -1);
         for (int pt = 0; pt < a.n_pt && ok; ++pt)
           for (int b = 0; b < sc.nbatch; ++b) {
-            if (!tc::mbar_wait_sleep(&bempty[bslot], (bpar >> bslot) & 1u, 128)) {
+            if (!tc::mbar_wait_sleep(&bempty[bslot], (bpar >> bslot) & 1u, 32)) {
               ok = false;
               break;
             }
@@ -349,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
             const int nrs = (int)(h.w & 7u);
             for (int j = 0; j < nrs && ok; ++j) {
               const int rb = (int)((h.w >> (3 + 3 * j)) & 7u);
-              if ((rused & (1u << rb)) && !tc::mbar_wait_sleep(&tempty[rb], ((rpar >> rb) & 1u) ^ 1u, 128)) ok = false;
+              if ((rused & (1u << rb)) && !tc::mbar_wait_sleep(&tempty[rb], ((rpar >> rb) & 1u) ^ 1u, 32)) ok = false;
               rpar ^= 1u << rb;
               rused |= 1u << rb;
             }
@@ -406,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
           const int rb = (rec.y >> 8) & 0xF;
           if (!empty) {
             int good = 1;
-            if (lane == 0) good = wait_batches(done, gbase + (uint32_t)(rec.y >> 12) + 1, 256);
+            if (lane == 0) good = wait_batches(done, gbase + (uint32_t)(rec.y >> 12) + 1, 64);
             ok = __shfl_sync(0xffffffffu, good, 0) != 0;
             if (!ok) break;
             tc::fence_after_sync();
@@ -424,55 +466,49 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
             }
           }
           const uint32_t tb = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(rb * kNb * N);
-#pragma unroll 1
-          for (int k = 0; k < K; ++k) {
+          // the row's values as bf16 pairs: pk[k][8b + e] = outputs 16b + 2e, +1 of kernel index k
+          // (for K <= 3 all of them are read before the buffer is released, so the MMA issuers
+          // may start the buffer's next row while they are staged and stored)
+          constexpr int KP = K <= 3 ? K : 1;
+          uint32_t pk[KP][32];
+          auto load_pack = [&](int k, uint32_t (&dst)[32]) {
             uint32_t v[4 * 16];
-            if (!empty) {
 #pragma unroll
-              for (int b = 0; b < kNb; ++b)
-                asm volatile(
-                    "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
-                    "%13, %14, %15}, [%16];"
-                    : "=r"(v[16 * b + 0]), "=r"(v[16 * b + 1]), "=r"(v[16 * b + 2]), "=r"(v[16 * b + 3]),
-                      "=r"(v[16 * b + 4]), "=r"(v[16 * b + 5]), "=r"(v[16 * b + 6]), "=r"(v[16 * b + 7]),
-                      "=r"(v[16 * b + 8]), "=r"(v[16 * b + 9]), "=r"(v[16 * b + 10]), "=r"(v[16 * b + 11]),
-                      "=r"(v[16 * b + 12]), "=r"(v[16 * b + 13]), "=r"(v[16 * b + 14]), "=r"(v[16 * b + 15])
-                    : "r"(tb + (uint32_t)(b * N + 16 * k)));
-              asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            for (int b = 0; b < kNb; ++b)
+              asm volatile(
+                  "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+                  "%13, %14, %15}, [%16];"
+                  : "=r"(v[16 * b + 0]), "=r"(v[16 * b + 1]), "=r"(v[16 * b + 2]), "=r"(v[16 * b + 3]),
+                    "=r"(v[16 * b + 4]), "=r"(v[16 * b + 5]), "=r"(v[16 * b + 6]), "=r"(v[16 * b + 7]),
+                    "=r"(v[16 * b + 8]), "=r"(v[16 * b + 9]), "=r"(v[16 * b + 10]), "=r"(v[16 * b + 11]),
+                    "=r"(v[16 * b + 12]), "=r"(v[16 * b + 13]), "=r"(v[16 * b + 14]), "=r"(v[16 * b + 15])
+                  : "r"(tb + (uint32_t)(b * N + 16 * k)));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-              for (int i = 0; i < 64; ++i) asm volatile("" : "+r"(v[i]));
-              if (k == K - 1) {
-                // accumulator drained: the MMA issuers may start another row in the buffer
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&tempty[rb]);
-              }
-            } else {
+            for (int i = 0; i < 64; ++i) asm volatile("" : "+r"(v[i]));
 #pragma unroll
-              for (int i = 0; i < 64; ++i) v[i] = 0u;
+            for (int i = 0; i < 32; ++i) {
+              const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+              dst[i] = *reinterpret_cast<const uint32_t*>(&h);
             }
+          };
+          auto release = [&]() {
+            // accumulator drained: the MMA issuers may start another row in the buffer
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&tempty[rb]);
+          };
+          auto stage_store = [&](int k, const uint32_t (&src)[32]) {
             // the buffer is free once the store issued two stores ago has read it
             if (lane == 0) tc::bulk_wait_read_le<1>();
             __syncwarp();
             uint8_t* buf = wy + (size_t)(nst & 1) * kYBuf;
             uint8_t* rowp = buf + (size_t)lane * 128;
 #pragma unroll
-            for (int b = 0; b < kNb; ++b) {
-              uint4 w0, w1;
-              uint32_t* p0 = reinterpret_cast<uint32_t*>(&w0);
-              uint32_t* p1 = reinterpret_cast<uint32_t*>(&w1);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(v[16 * b + 2 * e]),
-                                                                __uint_as_float(v[16 * b + 2 * e + 1]));
-                const __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(v[16 * b + 8 + 2 * e]),
-                                                                __uint_as_float(v[16 * b + 8 + 2 * e + 1]));
-                p0[e] = *reinterpret_cast<const uint32_t*>(&h0);
-                p1[e] = *reinterpret_cast<const uint32_t*>(&h1);
-              }
-              // row = plane (lane) of 128 bytes; 16-byte chunk c = 2b (+1) lands at c ^ (lane % 8)
-              *reinterpret_cast<uint4*>(rowp + (((2 * b) ^ (lane & 7)) << 4)) = w0;
-              *reinterpret_cast<uint4*>(rowp + (((2 * b + 1) ^ (lane & 7)) << 4)) = w1;
+            for (int c = 0; c < 8; ++c) {
+              // row = plane (lane) of 128 bytes; 16-byte chunk c lands at c ^ (lane % 8)
+              *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) =
+                  make_uint4(src[4 * c], src[4 * c + 1], src[4 * c + 2], src[4 * c + 3]);
             }
             tc::fence_proxy_async();
             __syncwarp();
@@ -481,6 +517,32 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
               tc::bulk_commit();
             }
             ++nst;
+          };
+          if constexpr (K <= 3) {
+            if (!empty) {
+#pragma unroll
+              for (int k = 0; k < K; ++k) load_pack(k, pk[k]);
+              release();
+            } else {
+#pragma unroll
+              for (int k = 0; k < K; ++k)
+#pragma unroll
+                for (int i = 0; i < 32; ++i) pk[k][i] = 0u;
+            }
+#pragma unroll
+            for (int k = 0; k < K; ++k) stage_store(k, pk[k]);
+          } else {
+#pragma unroll 1
+            for (int k = 0; k < K; ++k) {
+              if (!empty) {
+                load_pack(k, pk[0]);
+                if (k == K - 1) release();
+              } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) pk[0][i] = 0u;
+              }
+              stage_store(k, pk[0]);
+            }
           }
         }
         gbase += (uint32_t)sc.nbatch;

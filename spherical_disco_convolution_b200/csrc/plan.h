@@ -102,6 +102,7 @@ constexpr int kItemRowStart = 4;  // item flag: first item of its row
 constexpr int kTileInts = 16;  // per script: load0, load1, copy0, copy1, row0, row1, record0, record1, 0, 0, 0,
                                // batches, cost, 0, 0, 0
 // Copy flags: first / last copy of a batch, the copy of the batch record (source: the records).
+// The record's copy carries the batch's total bytes << 8 and its number of copies << 24.
 constexpr int kCopyBatchStart = 1, kCopyBatchEnd = 2, kCopyMeta = 4;
 // A batch's B slot holds its record in the first kMetaBytes: a header of four words (MMA counts
 // of issuers 0..3 in bytes 0..3; word offsets of the lists of issuers 1..3 in 10-bit fields;

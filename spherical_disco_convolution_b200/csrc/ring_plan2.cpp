@@ -351,7 +351,7 @@ bool build_tiles(int n_out, int n_src, int n, int K, std::vector<RingTerm> terms
       int nbatch = 0, fill = 0;
       {
         std::vector<char> lin(loads.size(), 0), rin(nrows, 0);
-        int nl = 0, nr = 0, n_new_l = 0, n_new_r = 0, n_words = 0;
+        int nl = 0, nr = 0, n_new_l = 0, n_new_r = 0, n_words = 0, n_items = 0;
         auto open_batch = [&](size_t t0) {
           // windows and rows used before t0 and again at or after it stay live
           std::fill(lin.begin(), lin.end(), 0);
@@ -363,7 +363,7 @@ bool build_tiles(int n_out, int n_src, int n, int K, std::vector<RingTerm> terms
             if (rfirst[rw] >= 0 && rfirst[rw] < (int)t0 && rlast[rw] >= (int)t0) rin[rw] = 1, ++nr;
           ++nbatch;
           fill = 0;
-          n_new_l = n_new_r = n_words = 0;
+          n_new_l = n_new_r = n_words = n_items = 0;
         };
         const int b_cap = prm.bslot_bytes - kMetaBytes;
         for (size_t t = 0; t < items.size(); ++t) {
@@ -373,7 +373,8 @@ bool build_tiles(int n_out, int n_src, int n, int K, std::vector<RingTerm> terms
           const int words = (int)items[t].mmas.size();
           const bool full = fill + bytes > b_cap || nl + (lin[L] ? 0 : 1) > prm.ns ||
                             nr + (rin[rw] ? 0 : 1) > prm.nrb || n_new_l + new_l > kMaxLoadStarts ||
-                            n_new_r + new_r > kMaxRowStarts || 4 + n_words + words > kMaxMetaWords;
+                            n_new_r + new_r > kMaxRowStarts || 4 + n_words + words > kMaxMetaWords ||
+                            n_items + 1 > 31;
           if (t == 0 || full) {
             open_batch(t);
             if (nl + (lin[L] ? 0 : 1) > prm.ns || nr + (rin[rw] ? 0 : 1) > prm.nrb) {
@@ -386,6 +387,7 @@ bool build_tiles(int n_out, int n_src, int n, int K, std::vector<RingTerm> terms
           n_new_l += new_l;
           n_new_r += new_r;
           n_words += words;
+          ++n_items;
           if (4 + n_words > kMaxMetaWords) {
             msg = "tile plan: an item with more MMAs than a batch holds";
             return false;
@@ -486,7 +488,7 @@ bool build_tiles(int n_out, int n_src, int n, int K, std::vector<RingTerm> terms
         P.loads.push_back(l.s | sbar << 16);
         P.loads.push_back(l.slot | l.mask << 8);
         P.loads.push_back(8 * l.origin);
-        P.loads.push_back(bat(l.last));
+        P.loads.push_back(bat(l.last) | bat(l.first) << 16);
         P.boxes += 2 * __builtin_popcount(l.mask);
       }
       rec[1] = (int)(P.loads.size() / 4);
@@ -516,8 +518,8 @@ bool build_tiles(int n_out, int n_src, int n, int K, std::vector<RingTerm> terms
         for (int bt = 0; bt < nbatch; ++bt) {
           const size_t t0 = t;
           while (t < items.size() && items[t].batch == bt) ++t;
-          if (t0 == t) {
-            msg = "tile plan: an empty batch";
+          if (t0 == t || t - t0 > 31 || nbatch > 0xFFFF) {
+            msg = "tile plan: an empty batch, more than 31 items in a batch or too many batches";
             return false;
           }
           std::vector<std::vector<uint32_t>> lists(nb);
@@ -572,7 +574,7 @@ bool build_tiles(int n_out, int n_src, int n, int K, std::vector<RingTerm> terms
           P.copies.push_back((int)(m0 / 4));
           P.copies.push_back(meta_bytes);
           P.copies.push_back(0);
-          P.copies.push_back(kCopyBatchStart | kCopyMeta | total << 8);
+          P.copies.push_back(kCopyBatchStart | kCopyMeta | total << 8 | (int)(1 + t - t0) << 24);
           for (size_t u = t0; u < t; ++u) {
             const Item& it = items[u];
             const Pair& pr = pairs[it.pair];

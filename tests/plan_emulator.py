@@ -251,15 +251,17 @@ def tile(plan, src, n_out_rows):
         batches, cur = [], None
         for c in copies:
             off16, nbytes, dst, fl = (int(v) for v in c)
-            flags, total = fl & 0xFF, fl >> 8
+            flags, total = fl & 0xFF, (fl >> 8) & 0xFFFF
             if flags & 1:
                 assert cur is None and flags & 4, "a batch does not start with its record"
-                cur = {"total": total, "data": bytearray(bslot), "filled": 0, "kend": META}
+                cur = {"total": total, "data": bytearray(bslot), "filled": 0, "kend": META,
+                       "ncopies": (fl >> 24) & 0xFF, "seen": 0}
             assert cur is not None and dst % 16 == 0 and dst + nbytes <= bslot and nbytes % 16 == 0
             srcb = rbytes if flags & 4 else bbytes
             assert 16 * off16 + nbytes <= len(srcb), "copy outside its source array"
             cur["data"][dst: dst + nbytes] = srcb[16 * off16: 16 * off16 + nbytes]
             cur["filled"] += nbytes
+            cur["seen"] += 1
             if flags & 4:
                 assert dst == 0 and nbytes <= META
             else:
@@ -267,6 +269,7 @@ def tile(plan, src, n_out_rows):
                 cur["kend"] = max(cur["kend"], dst + nbytes)
             if flags & 2:
                 assert cur["filled"] == cur["total"] <= bslot, "batch bytes disagree with its copies"
+                assert cur["seen"] == cur["ncopies"] <= 32, "batch copy count disagrees with its copies"
                 batches.append(cur)
                 cur = None
         assert cur is None and len(batches) == nbatch, "batch count disagrees with the script"
@@ -278,7 +281,7 @@ def tile(plan, src, n_out_rows):
         by_slot = {}
         for L, ld in enumerate(loads):
             slot, mask = int(ld[1]) & 0xFF, (int(ld[1]) >> 8) & 0xFF
-            assert slot < ns and 0 < mask < 4 and 0 <= int(ld[3]) < nbatch
+            assert slot < ns and 0 < mask < 4 and 0 <= (int(ld[3]) & 0xFFFF) < nbatch
             by_slot.setdefault(slot, []).append(L)
         # rows by buffer, in start order
         by_buf, start_order = {}, []
@@ -337,7 +340,9 @@ def tile(plan, src, n_out_rows):
                         seq = by_slot.get(slot, [])
                         assert slot_use[slot] < len(seq), "slot started more often than loaded"
                         if slot in slot_load:
-                            assert bcur > int(loads[slot_load[slot]][3]), "slot refilled before its release batch"
+                            assert bcur > (int(loads[slot_load[slot]][3]) & 0xFFFF), \
+                                "slot refilled before its release batch"
+                        assert int(loads[seq[slot_use[slot]]][3]) >> 16 == bcur, "load's first batch field wrong"
                         slot_load[slot] = seq[slot_use[slot]]
                         slot_use[slot] += 1
                     for j in range(int(h[3]) & 7):
@@ -361,7 +366,7 @@ def tile(plan, src, n_out_rows):
                         assert pos <= 6 and slot in slot_load, "A outside a started slot or its chunk"
                         ld = loads[slot_load[slot]]
                         assert (int(ld[1]) >> 8) & (1 << c), "A in a chunk that was not staged"
-                        assert bcur <= int(ld[3]), "A read after its load's release batch"
+                        assert bcur <= (int(ld[3]) & 0xFFFF), "A read after its load's release batch"
                         assert META <= boff and boff + kstep <= bt["kend"], "B outside the slot's K-steps"
                         assert rb in buf_row, "MMA into a row buffer not started"
                         R = buf_row[rb]
