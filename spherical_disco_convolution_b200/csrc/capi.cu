@@ -406,16 +406,16 @@ void build_ring_plans(disco_psi* h) {
   }
 }
 
-// Shape of the tile-script plan: five ring slots of two chunks (160 KB), three B slots (1 KB of
+// Shape of the tile-script plan: five ring slots of two chunks (160 KB), four B slots (1 KB of
 // batch record and about 9 KB of Toeplitz K-steps each), the row
 // buffers that tensor memory holds (512 columns / (4 blocks x 16K)), and the y staging of the
-// epilogue (32 KB) within 227 KB of shared memory.
+// epilogue (16 KB) within 227 KB of shared memory.
 bool tile_params(int K, bool adjoint, int n_ctas, disco::TileParams* p) {
   if (!(K == 1 || K == 3 || K == 5)) return false;
   p->nb = 4;
   p->ns = 5;
   p->nrb = std::min(8, 512 / (4 * 16 * K));
-  p->nbs = 3;
+  p->nbs = 4;
   const int kstep = 2 * 16 * K * 16;
   p->bslot_bytes = disco::kMetaBytes + (9216 / kstep) * kstep;  // the batch record, then the K-steps
   p->src_order = adjoint ? 1 : 0;

@@ -22,8 +22,8 @@
 // Roles: one thread stages the windows with TMA boxes, one thread copies the B batches, four
 // MMA issuers (issuer b: block b) issue the MMA lists of each batch's record, one thread follows the
 // completion of the batches, and four epilogue warps read finished rows from tensor memory,
-// round them to bf16 and store them with TMA, one kernel index at a time through two staging
-// buffers per warp.  The issuers commit once per B batch: the completion of a batch releases its
+// round them to bf16 and store them with TMA, one kernel index at a time through one staging
+// buffer per warp.  The issuers commit once per B batch: the completion of a batch releases its
 // B slot, and also every ring slot and finished row whose last use it holds (the host chose the
 // batches, slots and row buffers so that none is needed before it is released).
 // Every mbarrier wait is bounded (tc_common.cuh): on expiry the kernel records the timeout in the
@@ -203,8 +203,8 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sX = smem;                                          // ns slots of two chunks
   uint8_t* sB = sX + (size_t)a.ns * kSlotBytes;                // nbs B slots
-  uint8_t* sY = sB + (((size_t)a.nbs * a.bslot_bytes + 1023) & ~(size_t)1023);  // 4 warps x 2 buffers
-  uint64_t* xfull = reinterpret_cast<uint64_t*>(sY + 8 * kYBuf);
+  uint8_t* sY = sB + (((size_t)a.nbs * a.bslot_bytes + 1023) & ~(size_t)1023);  // one buffer per epilogue warp
+  uint64_t* xfull = reinterpret_cast<uint64_t*>(sY + 4 * kYBuf);
   uint64_t* bfull = xfull + kMaxSlots;
   uint64_t* bempty = bfull + kMaxBslots;
   uint64_t* tempty = bempty + kMaxBslots;
@@ -423,11 +423,10 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
     // ------------------------------------------------------------------ epilogue warps
     // each warp drains its TMEM lane quadrant (32 planes of group quad / 2) once the batch that
     // holds the row's last MMA has completed, one kernel index at a time, into a [32 planes][64
-    // outputs] bf16 buffer (128-byte rows, 128-byte swizzle) stored with one TMA store; two
-    // buffers per warp alternate
+    // outputs] bf16 buffer (128-byte rows, 128-byte swizzle) stored with one TMA store
     const int quad = warp;
     const int grp = quad >> 1, pl0 = (quad & 1) * 32;
-    uint8_t* wy = sY + (size_t)warp * 2 * kYBuf;
+    uint8_t* wy = sY + (size_t)warp * kYBuf;
     if (lane == 0) tc::prefetch_map(&ymap);
     uint32_t gbase = 0;
     int nst = 0;  // stores issued by this warp
@@ -499,10 +498,10 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
             if (lane == 0) tc::mbar_arrive(&tempty[rb]);
           };
           auto stage_store = [&](int k, const uint32_t (&src)[32]) {
-            // the buffer is free once the store issued two stores ago has read it
-            if (lane == 0) tc::bulk_wait_read_le<1>();
+            // the buffer is free once the previous store has read it
+            if (lane == 0) tc::bulk_wait_read0();
             __syncwarp();
-            uint8_t* buf = wy + (size_t)(nst & 1) * kYBuf;
+            uint8_t* buf = wy;
             uint8_t* rowp = buf + (size_t)lane * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -584,7 +583,7 @@ cudaError_t launch_k(const Ring2Launch& L, const void* src, void* dst, cudaStrea
   a.bslot_bytes = (uint32_t)L.bslot_bytes;
   const size_t bars = 8 * (kMaxSlots + 2 * kMaxBslots + kMaxBufs + 1) + 16;
   const size_t smem = 1024 + (size_t)L.ns * kSlotBytes + (((size_t)L.nbs * L.bslot_bytes + 1023) & ~(size_t)1023) +
-                      8 * kYBuf + bars;
+                      4 * kYBuf + bars;
   if (smem > kTcSmemLimit) return cudaErrorInvalidValue;
   // x as [BC][n_src_rows][nlon]: boxes of 64 longitudes x 1 row x 64 planes, 128-byte swizzle
   CUtensorMap xm, ym;
