@@ -207,6 +207,10 @@ struct disco_psi {
   bool tile_built[4] = {false, false, false, false};
   std::string tile_msg[4];
   DevTile dtile[4];
+  // the forward plan of the fused variant (mirror rows; fewer B slots: the mix weights take room)
+  disco::TilePlan tile_fused;
+  bool tile_fused_built = false;
+  DevTile dtile_fused;
 };
 
 namespace {
@@ -425,6 +429,23 @@ bool tile_params(int K, bool adjoint, int n_ctas, disco::TileParams* p) {
   return true;
 }
 
+// The fused variant keeps the mix weights (K x 8 KB) in shared memory and the mix accumulators
+// (128 columns) in tensor memory: three B slots of 1 KB of record and four K-steps, and the row
+// buffers that the remaining 384 columns hold.
+bool tile_params_fused(int K, int n_ctas, disco::TileParams* p) {
+  if (!(K == 1 || K == 3)) return false;
+  p->nb = 4;
+  p->ns = 5;
+  p->nrb = std::min(8, 384 / (4 * 16 * K));
+  p->nbs = 3;
+  p->bslot_bytes = disco::kMetaBytes + 4 * (2 * 16 * K * 16);
+  p->src_order = 0;
+  p->target_strips = 24;
+  p->max_rows = 64;
+  p->n_ctas = n_ctas;
+  return true;
+}
+
 void build_tile_plans(disco_psi* h, int n_ctas) {
   const disco::Geometry& g = h->g;
   const int J = g.nlat_out, I = g.nlat_in, K = g.K;
@@ -462,6 +483,12 @@ void build_tile_plans(disco_psi* h, int n_ctas) {
       h->tile[which] = disco::TilePlan{};
       h->tile_msg[which] = msg;
     }
+  }
+  disco::TileParams pf;
+  if (tile_params_fused(K, n_ctas, &pf) && g.nlon_in >= 64) {
+    std::string msg;
+    h->tile_fused_built = disco::make_tile_plan(J, I, g.nlon_in, K, fwd, mo_f, ms_f, pf, h->tile_fused, msg);
+    if (!h->tile_fused_built) h->tile_fused = disco::TilePlan{};
   }
 }
 
@@ -800,6 +827,7 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
         if (e == cudaSuccess) build_tile_plans(h, sms);
         for (int w = 0; w < 4 && e == cudaSuccess; ++w)
           if (h->tile_built[w] && disco::ring2_kernel_k(h->tile[w].K)) e = upload_tile(h->tile[w], &h->dtile[w]);
+        if (e == cudaSuccess && h->tile_fused_built) e = upload_tile(h->tile_fused, &h->dtile_fused);
       }
     }
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
@@ -815,6 +843,7 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
       free_tz(&h->dtza);
       for (int w = 0; w < 4; ++w) free_ring(&h->dring[w]);
       for (int w = 0; w < 4; ++w) free_tile(&h->dtile[w]);
+      free_tile(&h->dtile_fused);
       delete h;
       return fail(DISCO_ERR_ALLOC, std::string("Psi upload failed: ") + cudaGetErrorString(e));
     }
@@ -853,6 +882,7 @@ disco_status disco_psi_destroy(disco_psi* psi) {
     free_tz(&psi->dtza);
     for (int w = 0; w < 4; ++w) free_ring(&psi->dring[w]);
     for (int w = 0; w < 4; ++w) free_tile(&psi->dtile[w]);
+    free_tile(&psi->dtile_fused);
     if (psi->side) cudaStreamDestroy(psi->side);
     if (psi->fork) cudaEventDestroy(psi->fork);
     if (psi->join) cudaEventDestroy(psi->join);
@@ -1048,6 +1078,21 @@ disco_status disco_fwd_fused(const disco_psi* psi, int B, int C_in, int C_out, i
   const bool bf16 = dtype == DISCO_BF16;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int Cg = C_in / groups;
+  const char* rf = std::getenv("DISCO_RING2_FUSED");
+  const char* r2 = std::getenv("DISCO_RING2");
+  if (bf16 && psi->dtile_fused.ok && !(rf && rf[0] == '0') && !(r2 && r2[0] == '0') && C_in == 64 && groups == 1 &&
+      C_out <= 64 && !(reinterpret_cast<uintptr_t>(x) & 15) && !(reinterpret_cast<uintptr_t>(out) & 15) &&
+      !(reinterpret_cast<uintptr_t>(w) & 1) && !(reinterpret_cast<uintptr_t>(bias) & 1)) {
+    // TMA-staged strip contraction with the channel mix on tensor cores in its epilogue
+    const disco::TilePlan& P = psi->tile_fused;
+    const DevTile& d = psi->dtile_fused;
+    disco::Ring2Launch L{d.tiles, d.loads, d.copies, d.cmds, d.rows, d.cta_tiles, d.b, P.n_ctas, P.n_qt, P.K, P.nb,
+                         P.ns, P.nrb, P.nbs, P.bslot_bytes, P.mirror, B * C_in, g.nlat_in, g.nlat_out, g.nlon_in};
+    disco::Ring2Fused F{x, w, bias, out, C_in, C_out};
+    cudaError_t e = disco::launch_fused_ring2(L, F, st);
+    if (e != cudaSuccess) return cuda_fail(e, "fused strip-contraction launch");
+    return DISCO_OK;
+  }
   if (bf16 && psi->tz_ok && disco::fused_tz_supported(g.K, C_in, C_out, groups) &&
       !(reinterpret_cast<uintptr_t>(x) & 15) && !(reinterpret_cast<uintptr_t>(w) & 15)) {
     // Toeplitz contraction and channel mix, both on tensor cores, y tile in shared memory

@@ -57,6 +57,10 @@ struct Args {
   int n_ctas, n_qt, n_pt, plane_tile, mirror, BC;
   int ns, nbs, nrb;
   uint32_t bslot_bytes;
+  // fused forward: out = W y + bias instead of y
+  const __nv_bfloat16* w;     // [C_out][64][K]
+  const __nv_bfloat16* bias;  // [C_out] or null
+  int C_out;
 };
 
 __device__ __forceinline__ int4 shfl4(const int4& v, int src) {
@@ -193,23 +197,26 @@ __device__ __forceinline__ bool wait_batches(const uint32_t* done, uint32_t targ
   }
 }
 
-template <int K>
+template <int K, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                       const __grid_constant__ CUtensorMap ymap,
                                                                       Args a) {
   constexpr int N = 16 * K;
+  constexpr uint32_t kWBytes = kFused ? (uint32_t)K * 8192u : 0u;  // W_k tiles [64 o][64 c] of the mix
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sX = smem;                                          // ns slots of two chunks
   uint8_t* sB = sX + (size_t)a.ns * kSlotBytes;                // nbs B slots
-  uint8_t* sY = sB + (((size_t)a.nbs * a.bslot_bytes + 1023) & ~(size_t)1023);  // one buffer per epilogue warp
+  uint8_t* sW = sB + (((size_t)a.nbs * a.bslot_bytes + 1023) & ~(size_t)1023);  // fused: the mix weights
+  uint8_t* sY = sW + kWBytes;  // one buffer per epilogue warp (fused: also the mix's y operand)
   uint64_t* xfull = reinterpret_cast<uint64_t*>(sY + 4 * kYBuf);
   uint64_t* bfull = xfull + kMaxSlots;
   uint64_t* bempty = bfull + kMaxBslots;
   uint64_t* tempty = bempty + kMaxBslots;
   uint64_t* drain = tempty + kMaxBufs;
-  uint32_t* done = reinterpret_cast<uint32_t*>(drain + 1);  // batches completed
+  uint64_t* mixb = drain + 1;  // fused: the mix MMAs of mirror group 0 / 1 completed
+  uint32_t* done = reinterpret_cast<uint32_t*>(mixb + 2);  // batches completed
   uint32_t* tmem_slot = done + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -221,6 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
     }
     for (int s = 0; s < kMaxBufs; ++s) tc::mbar_init(&tempty[s], 4);
     tc::mbar_init(drain, kIssuers);
+    tc::mbar_init(&mixb[0], 1);
+    tc::mbar_init(&mixb[1], 1);
     *done = 0;
     tc::fence_barrier_init();
   }
@@ -419,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
       tc::mbar_wait(drain, 0);
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 4 && !kFused) {
     // ------------------------------------------------------------------ epilogue warps
     // each warp drains its TMEM lane quadrant (32 planes of group quad / 2) once the batch that
     // holds the row's last MMA has completed, one kernel index at a time, into a [32 planes][64
@@ -548,6 +557,172 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
       }
     }
     if (lane == 0) tc::bulk_wait0();
+  } else if (warp < 4) {
+    // ------------------------------------------------------------------ fused epilogue warps
+    // out[b, o, j, q] = bias[o] + sum_{c, k} W[o, c, k] y[b, c, k, j, q] for the 64 channels c
+    // of one batch element (the plane tile).  Per row: each warp drains its TMEM lane quadrant
+    // (32 channels of mirror group quad / 2) and releases the buffer; then, one kernel index k
+    // at a time, the two warps of a group write y_k of their channels into their staging
+    // buffers ([c][64 q], 128-byte swizzle: the MN-major B operand of the mix) and the group's
+    // first warp issues the mix MMAs D_g[o, q] += W_k[o, c] y_k[c, q] (M = 128: rows 64..127
+    // read past W_k and are never used; N = 64; K = the 64 channels in four steps); finally
+    // warps 0 and 1 (TMEM lanes 0..63 = the output channels) read D_0 and D_1, add the bias and
+    // store out for the row and its mirror row.
+    const int quad = warp;
+    const int grp = quad >> 1;
+    uint8_t* wy = sY + (size_t)warp * kYBuf;
+    if (lane == 0) tc::prefetch_map(&ymap);
+    // W_k[o][c] into shared memory, K-major with the 128-byte swizzle; rows o >= C_out are zero
+    for (int i = threadIdx.x; i < K * 64 * 64; i += 128) {
+      const int k = i >> 12, o = (i >> 6) & 63, c = i & 63;
+      const __nv_bfloat16 v = o < a.C_out ? a.w[((size_t)o * 64 + c) * K + k] : __float2bfloat16(0.0f);
+      *reinterpret_cast<__nv_bfloat16*>(sW + (size_t)k * 8192 + o * 128 + ((((c >> 3) ^ (o & 7))) << 4) + (c & 7) * 2) = v;
+    }
+    tc::fence_proxy_async();
+    tc::named_bar_sync(1, 128);
+    constexpr uint32_t midesc = tc::idesc_bf16(128, 64, false, true);
+    const uint32_t dmix = tmem + (uint32_t)(a.nrb * kNb * N);  // D_0 at +0, D_1 at +64 columns
+    const int o_lane = quad * 32 + lane;                        // output channel of this lane (warps 0, 1)
+    const float bv = (quad < 2 && a.bias && o_lane < a.C_out) ? __bfloat162float(a.bias[o_lane]) : 0.0f;
+    uint32_t gbase = 0, mpar = 0;
+    bool ok = true;
+    WarpStream<int2> rs;
+    for (int t = t_begin; t < t_end && ok; ++t) {
+      const int si = my[t];
+      const Script sc = read_script(a, si, -1);
+      const int q0 = (si % a.n_qt) * (16 * kNb);
+      for (int pt = 0; pt < a.n_pt && ok; ++pt) {
+        rs.start(a.rows, sc.row0, sc.row1);
+        for (int rr = sc.row0; rr < sc.row1 && ok; ++rr) {
+          const int2 rec = rs.get(rr);
+          const int r = rec.x & 0xFFFF, rbar = (rec.x >> 16) & 0xFFFF;
+          const bool empty = rec.y & kRowEmpty;
+          const int rb = (rec.y >> 8) & 0xF;
+          if (!empty) {
+            int good = 1;
+            if (lane == 0) good = wait_batches(done, gbase + (uint32_t)(rec.y >> 12) + 1, 64);
+            ok = __shfl_sync(0xffffffffu, good, 0) != 0;
+          }
+          // one decision for the four warps before the named barriers of the row
+          ok = tc::named_bar_and(1, 128, ok);
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint32_t tb = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(rb * kNb * N);
+          uint32_t pk[K][32];
+          if (!empty) {
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+              uint32_t v[4 * 16];
+#pragma unroll
+              for (int b = 0; b < kNb; ++b)
+                asm volatile(
+                    "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+                    "%13, %14, %15}, [%16];"
+                    : "=r"(v[16 * b + 0]), "=r"(v[16 * b + 1]), "=r"(v[16 * b + 2]), "=r"(v[16 * b + 3]),
+                      "=r"(v[16 * b + 4]), "=r"(v[16 * b + 5]), "=r"(v[16 * b + 6]), "=r"(v[16 * b + 7]),
+                      "=r"(v[16 * b + 8]), "=r"(v[16 * b + 9]), "=r"(v[16 * b + 10]), "=r"(v[16 * b + 11]),
+                      "=r"(v[16 * b + 12]), "=r"(v[16 * b + 13]), "=r"(v[16 * b + 14]), "=r"(v[16 * b + 15])
+                    : "r"(tb + (uint32_t)(b * N + 16 * k)));
+              asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+              for (int i = 0; i < 64; ++i) asm volatile("" : "+r"(v[i]));
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const __nv_bfloat162 h =
+                    __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                pk[k][i] = *reinterpret_cast<const uint32_t*>(&h);
+              }
+            }
+            // accumulator drained: the MMA issuers may start another row in the buffer
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&tempty[rb]);
+          } else {
+#pragma unroll
+            for (int k = 0; k < K; ++k)
+#pragma unroll
+              for (int i = 0; i < 32; ++i) pk[k][i] = 0u;
+          }
+          // the mix, one kernel index at a time
+#pragma unroll
+          for (int k = 0; k < K; ++k) {
+            // the staging buffer is free: the previous out store from it has read it (warps 0, 1)
+            // and the previous mix round that read it has completed (waited below)
+            if (lane == 0) tc::bulk_wait_read0();
+            __syncwarp();
+            uint8_t* rowp = wy + (size_t)lane * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) =
+                  make_uint4(pk[k][4 * c], pk[k][4 * c + 1], pk[k][4 * c + 2], pk[k][4 * c + 3]);
+            tc::fence_proxy_async();
+            tc::named_bar_sync(2 + grp, 64);
+            if ((quad & 1) == 0 && lane == 0) {
+              tc::fence_after_sync();
+              const uint32_t wk = tc::smem_u32(sW) + (uint32_t)k * 8192u;
+              const uint32_t yg = tc::smem_u32(sY) + (uint32_t)grp * 8192u;
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                tc::mma_bf16(dmix + (uint32_t)(64 * grp), tc::desc_sw128(wk + 32u * j, 16, 1024),
+                             tc::desc_sw128(yg + 2048u * j, 16, 1024), midesc, (k > 0 || j > 0) ? 1u : 0u);
+              tc::mma_commit(&mixb[grp]);
+            }
+            int good = 1;
+            if (lane == 0) good = tc::mbar_wait_sleep(&mixb[grp], (mpar >> grp) & 1u, 64);
+            ok = __shfl_sync(0xffffffffu, good, 0) != 0 && ok;
+            mpar ^= 1u << grp;
+            tc::fence_after_sync();
+          }
+          // both groups' mixes are complete (one decision for the four warps): warps 0 and 1 read
+          // D_0 and D_1
+          tc::fence_before_sync();
+          ok = tc::named_bar_and(1, 128, ok);
+          if (!ok) break;
+          tc::fence_after_sync();
+          if (quad < 2) {
+            uint32_t d[2][2][32];  // [group][half of the 64 outputs][column]
+#pragma unroll
+            for (int g = 0; g < 2; ++g)
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+                tc::tmem_ld_chunks<2>(dmix + ((uint32_t)(quad * 32) << 16) + (uint32_t)(64 * g + 32 * h), d[g][h]);
+            // D read: the group-1 issuer (warp 2) may start the next row's mix
+            tc::fence_before_sync();
+            tc::named_bar_sync(1, 128);
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+              const int orow = g == 0 ? r : rbar;
+              const bool st = g == 0 || (rbar != r && rbar != 0xFFFF);
+              if (lane == 0) tc::bulk_wait_read0();
+              __syncwarp();
+              uint8_t* rowp = wy + (size_t)lane * 128;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                uint32_t q4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(d[g][c >> 2][8 * (c & 3) + 2 * e]) + bv,
+                                                                 __uint_as_float(d[g][c >> 2][8 * (c & 3) + 2 * e + 1]) + bv);
+                  q4[e] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+                *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) = make_uint4(q4[0], q4[1], q4[2], q4[3]);
+              }
+              tc::fence_proxy_async();
+              __syncwarp();
+              if (lane == 0) {
+                if (st && quad * 32 < a.C_out) tc::tma_store_4d(&ymap, wy, q0, orow, quad * 32, pt);
+                tc::bulk_commit();
+              }
+            }
+          } else {
+            tc::fence_before_sync();
+            tc::named_bar_sync(1, 128);
+          }
+        }
+        gbase += (uint32_t)sc.nbatch;
+      }
+    }
+    if (lane == 0) tc::bulk_wait0();
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -557,8 +732,8 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
   }
 }
 
-template <int K>
-cudaError_t launch_k(const Ring2Launch& L, const void* src, void* dst, cudaStream_t st) {
+template <int K, bool kFused>
+cudaError_t launch_k(const Ring2Launch& L, const void* src, void* dst, const Ring2Fused* F, cudaStream_t st) {
   constexpr int N = 16 * K;
   if (L.K != K || L.nb != kNb || L.ns > kMaxSlots || L.nrb > kMaxBufs || L.nbs > kMaxBslots || L.nrb * kNb * N > 512 ||
       L.n_ctas < 1 || L.nlon < 64 || L.bslot_bytes % 16)
@@ -581,9 +756,19 @@ cudaError_t launch_k(const Ring2Launch& L, const void* src, void* dst, cudaStrea
   a.nbs = L.nbs;
   a.nrb = L.nrb;
   a.bslot_bytes = (uint32_t)L.bslot_bytes;
-  const size_t bars = 8 * (kMaxSlots + 2 * kMaxBslots + kMaxBufs + 1) + 16;
+  if (kFused) {
+    // one batch element of 64 channels per plane tile, mirror rows, the mix in tensor memory
+    // after the row buffers
+    if (!F || !L.mirror || L.BC % 64 || F->C_in != 64 || F->C_out < 1 || F->C_out > 64 ||
+        L.nrb * kNb * N + 128 > 512 || (reinterpret_cast<uintptr_t>(F->w) & 1))
+      return cudaErrorInvalidValue;
+    a.w = static_cast<const __nv_bfloat16*>(F->w);
+    a.bias = static_cast<const __nv_bfloat16*>(F->bias);
+    a.C_out = F->C_out;
+  }
+  const size_t bars = 8 * (kMaxSlots + 2 * kMaxBslots + kMaxBufs + 3) + 16;
   const size_t smem = 1024 + (size_t)L.ns * kSlotBytes + (((size_t)L.nbs * L.bslot_bytes + 1023) & ~(size_t)1023) +
-                      4 * kYBuf + bars;
+                      (kFused ? (size_t)K * 8192 : 0) + 4 * kYBuf + bars;
   if (smem > kTcSmemLimit) return cudaErrorInvalidValue;
   // x as [BC][n_src_rows][nlon]: boxes of 64 longitudes x 1 row x 64 planes, 128-byte swizzle
   CUtensorMap xm, ym;
@@ -593,15 +778,23 @@ cudaError_t launch_k(const Ring2Launch& L, const void* src, void* dst, cudaStrea
     const cuuint32_t box[3] = {64, 1, 64};
     if (!tc::encode_bf16_map(&xm, src, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
   }
-  // y as [BC][K][n_out_rows][nlon]: boxes of 64 longitudes x 1 row x 1 kernel index x 32 planes
-  {
+  if (!kFused) {
+    // y as [BC][K][n_out_rows][nlon]: boxes of 64 longitudes x 1 row x 1 kernel index x 32 planes
     const cuuint64_t dims[4] = {(cuuint64_t)L.nlon, (cuuint64_t)L.n_out_rows, (cuuint64_t)K, (cuuint64_t)L.BC};
     const cuuint64_t strides[3] = {(cuuint64_t)L.nlon * 2, (cuuint64_t)L.n_out_rows * L.nlon * 2,
                                    (cuuint64_t)K * L.n_out_rows * L.nlon * 2};
     const cuuint32_t box[4] = {64, 1, 1, 32};
     if (!tc::encode_bf16_map(&ym, dst, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
+  } else {
+    // out as [B][C_out][n_out_rows][nlon]: boxes of 64 longitudes x 1 row x 32 channels x 1
+    const int Bn = L.BC / 64;
+    const cuuint64_t dims[4] = {(cuuint64_t)L.nlon, (cuuint64_t)L.n_out_rows, (cuuint64_t)F->C_out, (cuuint64_t)Bn};
+    const cuuint64_t strides[3] = {(cuuint64_t)L.nlon * 2, (cuuint64_t)L.n_out_rows * L.nlon * 2,
+                                   (cuuint64_t)F->C_out * L.n_out_rows * L.nlon * 2};
+    const cuuint32_t box[4] = {64, 1, 32, 1};
+    if (!tc::encode_bf16_map(&ym, dst, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
   }
-  const void* kernel = reinterpret_cast<const void*>(&contract_ring2_kernel<K>);
+  const void* kernel = reinterpret_cast<const void*>(&contract_ring2_kernel<K, kFused>);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   void* args[] = {&xm, &ym, &a};
@@ -618,9 +811,19 @@ cudaError_t launch_contract_ring2(const Ring2Launch& L, const void* src, void* d
   if ((reinterpret_cast<uintptr_t>(src) & 15) || (reinterpret_cast<uintptr_t>(dst) & 15) || L.nlon % 8)
     return cudaErrorInvalidValue;
   switch (L.K) {
-    case 1: return launch_k<1>(L, src, dst, st);
-    case 3: return launch_k<3>(L, src, dst, st);
-    case 5: return launch_k<5>(L, src, dst, st);
+    case 1: return launch_k<1, false>(L, src, dst, nullptr, st);
+    case 3: return launch_k<3, false>(L, src, dst, nullptr, st);
+    case 5: return launch_k<5, false>(L, src, dst, nullptr, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_fused_ring2(const Ring2Launch& L, const Ring2Fused& F, cudaStream_t st) {
+  if ((reinterpret_cast<uintptr_t>(F.x) & 15) || (reinterpret_cast<uintptr_t>(F.out) & 15) || L.nlon % 8)
+    return cudaErrorInvalidValue;
+  switch (L.K) {
+    case 1: return launch_k<1, true>(L, F.x, F.out, &F, st);
+    case 3: return launch_k<3, true>(L, F.x, F.out, &F, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -85,6 +85,16 @@ struct Ring2Launch {
   int K, nb, ns, nrb, nbs, bslot_bytes, mirror;
   int BC, n_src_rows, n_out_rows, nlon;
 };
+// Fused forward on the same kernel (mirror rows, C_in = 64 channels per batch element, groups 1,
+// C_out <= 64): out [B][C_out][n_out_rows][nlon] = bias + the channel mix of the contraction.
+struct Ring2Fused {
+  const void* x;
+  const void* w;     // [C_out][64][K] bf16
+  const void* bias;  // [C_out] bf16 or null
+  void* out;
+  int C_in, C_out;
+};
+cudaError_t launch_fused_ring2(const Ring2Launch& L, const Ring2Fused& F, cudaStream_t st);
 bool ring2_kernel_k(int K);
 cudaError_t launch_contract_ring2(const Ring2Launch& L, const void* src, void* dst, cudaStream_t st);
 int take_contract_ring2_status();

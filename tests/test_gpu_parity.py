@@ -45,6 +45,11 @@ EDGE = {
     "ring_k3": Workload("ring_k3", 1, 70, 64, 1, 65, 128, 65, 128, (3, 1), 2 * math.pi / 64, "bf16"),
     # fused tensor-core forward with K = 9: one-half tiles of 64 outputs (ragged last tile)
     "tz_fused_k9": Workload("tz_fused_k9", 1, 128, 96, 2, 21, 160, 21, 160, (3, 4), 0.5, "bf16"),
+    # fused forward on the TMA-staged strip kernel (64 channels per batch element, mirror rows):
+    # two batch elements, 48 output channels, a ragged last longitude tile and full-ring polar
+    # windows; and 64 output channels without bias
+    "ring_fused_k3": Workload("ring_fused_k3", 2, 64, 48, 1, 49, 160, 49, 160, (3, 1), 2 * math.pi / 48, "bf16"),
+    "ring_fused_nb": Workload("ring_fused_nb", 1, 64, 64, 1, 33, 96, 33, 96, (3, 1), 0.3, "bf16", bias=False),
 }
 
 
