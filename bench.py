@@ -41,8 +41,9 @@ UNIT = "grid-points*channels/s"
 PSI_ENTRY_BYTES = 13  # algorithmic Psi bytes per entry: fp32 value + int32 i + int32 p + int8 k
 OPS = ("contract", "einsum", "fused", "dx", "dw")
 # single-launch kernels of the step, timed one by one for the roofline: the contraction, the weight
-# einsum, the fused forward and the adjoint contraction of dx (dx = its dy einsum + this kernel)
-KERNELS = ("contract", "einsum", "fused", "adjoint")
+# einsum, the fused forward and the input gradient (one launch on this layer: the transposed
+# contraction of dout with the mix by W^T in its epilogue)
+KERNELS = ("contract", "einsum", "fused", "dx")
 
 
 def parse():
@@ -76,7 +77,7 @@ def algorithmic_bytes(wl, nnz: int) -> dict:
     b = wl.C_out * es
     psi = nnz * PSI_ENTRY_BYTES
     return {"contract": x + psi + y, "einsum": y + w + b + out, "fused": x + psi + w + b + out,
-            "dx": out + w + psi + x, "dw": out + y + w + b, "adjoint": y + psi + x}
+            "dx": out + w + psi + x, "dw": out + y + w + b}
 
 
 def measured_peaks() -> tuple:
@@ -327,12 +328,12 @@ def workload_record(name: str, dev, steps: int = 5, warmup: int = 3) -> dict:
     inp = make_inputs(wl, 0)
     t = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dt).to(dev) for k, v in inp.items() if v is not None}
     sh = wl.shapes()
-    y, dy = (torch.empty(sh["y"], dtype=dt, device=dev) for _ in range(2))
+    y = torch.empty(sh["y"], dtype=dt, device=dev)
     out, out_f = (torch.empty(sh["out"], dtype=dt, device=dev) for _ in range(2))
     dx = torch.empty(sh["x"], dtype=dt, device=dev)
     dw = torch.empty(sh["w"], dtype=dt, device=dev)
     db = torch.empty(sh["bias"], dtype=dt, device=dev) if "bias" in t else None
-    ws_dy, n_dy = psi.workspace(D.DISCO_OP_EINSUM_ADJOINT, wl.B, wl.C_in, wl.C_out, wl.groups, dcode)
+    ws_dx, n_dx = psi.workspace(D.DISCO_OP_BWD_INPUT, wl.B, wl.C_in, wl.C_out, wl.groups, dcode)
     ws_dw, n_dw = psi.workspace(D.DISCO_OP_BWD_WEIGHT, wl.B, wl.C_in, wl.C_out, wl.groups, dcode)
     stream = torch.cuda.current_stream(dev)
     st = stream.cuda_stream
@@ -343,9 +344,7 @@ def workload_record(name: str, dev, steps: int = 5, warmup: int = 3) -> dict:
         ("einsum", lambda: D.disco_einsum(h, B, Ci, Co, G, dcode, p(y), p(t["w"]), p(t.get("bias")), p(out), st)),
         ("fused", lambda: D.disco_fwd_fused(h, B, Ci, Co, G, dcode, p(t["x"]), p(t["w"]), p(t.get("bias")),
                                             p(out_f), None, 0, st)),
-        ("dx", lambda: (D.disco_einsum_adjoint(h, B, Ci, Co, G, dcode, p(t["dout"]), p(t["w"]), p(dy), p(ws_dy),
-                                               n_dy, st),
-                        D.disco_contract_adjoint(h, B, Ci, dcode, p(dy), p(dx), st))),
+        ("dx", lambda: D.disco_bwd_input(h, B, Ci, Co, G, dcode, p(t["dout"]), p(t["w"]), p(dx), p(ws_dx), n_dx, st)),
         ("dw", lambda: D.disco_bwd_weight(h, B, Ci, Co, G, dcode, p(t["dout"]), p(y), None, p(dw), p(db), p(ws_dw),
                                           n_dw, st)),
     ]
@@ -413,8 +412,7 @@ def run_gpu(args):
     dx = torch.empty(sh["x"], dtype=dt, device=dev)
     dw = torch.empty(sh["w"], dtype=dt, device=dev)
     db = torch.empty(sh["bias"], dtype=dt, device=dev) if bias is not None else None
-    ws_dy, n_dy = psi.workspace(D.DISCO_OP_EINSUM_ADJOINT, wl.B, wl.C_in, wl.C_out, wl.groups, dcode)
-    dy = torch.empty(sh["y"], dtype=dt, device=dev)  # dx = adjoint contraction of dy = w^T dout
+    ws_dx, n_dx = psi.workspace(D.DISCO_OP_BWD_INPUT, wl.B, wl.C_in, wl.C_out, wl.groups, dcode)
     ws_dw, n_dw = psi.workspace(D.DISCO_OP_BWD_WEIGHT, wl.B, wl.C_in, wl.C_out, wl.groups, dcode)
     stream = torch.cuda.current_stream(dev)
     st = stream.cuda_stream
@@ -434,16 +432,12 @@ def run_gpu(args):
         D.disco_fwd_fused(h, B, Ci, Co, G, dcode, p(x), p(w), p(bias), p(out_f), None, 0, st)
         if ev:
             ev[3].record(stream)
-        # dx in its two C-ABI halves (together they are disco_bwd_input), timed apart
-        D.disco_einsum_adjoint(h, B, Ci, Co, G, dcode, p(dout), p(w), p(dy), p(ws_dy), n_dy, st)
+        D.disco_bwd_input(h, B, Ci, Co, G, dcode, p(dout), p(w), p(dx), p(ws_dx), n_dx, st)
         if ev:
             ev[4].record(stream)
-        D.disco_contract_adjoint(h, B, Ci, dcode, p(dy), p(dx), st)
-        if ev:
-            ev[5].record(stream)
         D.disco_bwd_weight(h, B, Ci, Co, G, dcode, p(dout), p(y), None, p(dw), p(db), p(ws_dw), n_dw, st)
         if ev:
-            ev[6].record(stream)
+            ev[5].record(stream)
 
     def barrier():
         if world > 1:
@@ -452,7 +446,7 @@ def run_gpu(args):
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     barrier()
     torch.cuda.synchronize()
@@ -474,9 +468,8 @@ def run_gpu(args):
     units = sum(ups.values()) * args.steps
     el_max, units_all = aggregate(elapsed, units, world, dev)
     span = lambda i, j: statistics.mean(e[i].elapsed_time(e[j]) for e in evs)  # noqa: E731
-    op_ms = {"contract": span(0, 1), "einsum": span(1, 2), "fused": span(2, 3), "dx": span(3, 5), "dw": span(5, 6)}
-    kern_ms = {"contract": op_ms["contract"], "einsum": op_ms["einsum"], "fused": op_ms["fused"],
-               "adjoint": span(4, 5)}
+    op_ms = {"contract": span(0, 1), "einsum": span(1, 2), "fused": span(2, 3), "dx": span(3, 4), "dw": span(4, 5)}
+    kern_ms = {"contract": op_ms["contract"], "einsum": op_ms["einsum"], "fused": op_ms["fused"], "dx": op_ms["dx"]}
 
     # end to end through the C ABI from pinned host buffers: inputs in, results out, every step
     e2e = None

@@ -211,6 +211,12 @@ struct disco_psi {
   disco::TilePlan tile_fused;
   bool tile_fused_built = false;
   DevTile dtile_fused;
+  // the input gradient with dy mixed in: the transposed contraction of dout with the K basis
+  // functions kept (z[o, k, i, q] = sum_{j, p} Psi_k(j, i, p) dout[o, j, q - p]), then
+  // dx[c] = sum_{o, k} W[o, c, k] z[o, k] in the epilogue
+  disco::TilePlan tile_fused_adj;
+  bool tile_fused_adj_built = false;
+  DevTile dtile_fused_adj;
 };
 
 namespace {
@@ -489,6 +495,12 @@ void build_tile_plans(disco_psi* h, int n_ctas) {
     std::string msg;
     h->tile_fused_built = disco::make_tile_plan(J, I, g.nlon_in, K, fwd, mo_f, ms_f, pf, h->tile_fused, msg);
     if (!h->tile_fused_built) h->tile_fused = disco::TilePlan{};
+    std::vector<disco::RingTerm> adjk;
+    adjk.reserve(h->entries.size());
+    for (const disco::PsiEntry& e : h->entries) adjk.push_back(disco::RingTerm{e.i, e.j, e.k, -e.p, e.v});
+    h->tile_fused_adj_built =
+        disco::make_tile_plan(I, J, g.nlon_in, K, std::move(adjk), mo_a, mo_f, pf, h->tile_fused_adj, msg);
+    if (!h->tile_fused_adj_built) h->tile_fused_adj = disco::TilePlan{};
   }
 }
 
@@ -828,6 +840,7 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
         for (int w = 0; w < 4 && e == cudaSuccess; ++w)
           if (h->tile_built[w] && disco::ring2_kernel_k(h->tile[w].K)) e = upload_tile(h->tile[w], &h->dtile[w]);
         if (e == cudaSuccess && h->tile_fused_built) e = upload_tile(h->tile_fused, &h->dtile_fused);
+        if (e == cudaSuccess && h->tile_fused_adj_built) e = upload_tile(h->tile_fused_adj, &h->dtile_fused_adj);
       }
     }
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
@@ -844,6 +857,7 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
       for (int w = 0; w < 4; ++w) free_ring(&h->dring[w]);
       for (int w = 0; w < 4; ++w) free_tile(&h->dtile[w]);
       free_tile(&h->dtile_fused);
+      free_tile(&h->dtile_fused_adj);
       delete h;
       return fail(DISCO_ERR_ALLOC, std::string("Psi upload failed: ") + cudaGetErrorString(e));
     }
@@ -883,6 +897,7 @@ disco_status disco_psi_destroy(disco_psi* psi) {
     for (int w = 0; w < 4; ++w) free_ring(&psi->dring[w]);
     for (int w = 0; w < 4; ++w) free_tile(&psi->dtile[w]);
     free_tile(&psi->dtile_fused);
+    free_tile(&psi->dtile_fused_adj);
     if (psi->side) cudaStreamDestroy(psi->side);
     if (psi->fork) cudaEventDestroy(psi->fork);
     if (psi->join) cudaEventDestroy(psi->join);
@@ -1160,6 +1175,23 @@ disco_status disco_bwd_input(const disco_psi* psi, int B, int C_in, int C_out, i
   const WsLayout L = layout(psi, DISCO_OP_BWD_INPUT, B, C_in, C_out, groups, dtype);
   if (!workspace || ws_bytes < L.total) return fail(DISCO_ERR_INVALID_ARG, "workspace missing or too small");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const char* rf = std::getenv("DISCO_RING2_FUSED");
+  const char* r2 = std::getenv("DISCO_RING2");
+  if (dtype == DISCO_BF16 && psi->dtile_fused_adj.ok && !(rf && rf[0] == '0') && !(r2 && r2[0] == '0') &&
+      C_out == 64 && groups == 1 && C_in <= 64 && !(reinterpret_cast<uintptr_t>(dout) & 15) &&
+      !(reinterpret_cast<uintptr_t>(dx) & 15) && !(reinterpret_cast<uintptr_t>(w) & 1)) {
+    // one launch: the transposed contraction of dout with the K basis functions kept, and the
+    // mix with W^T in the epilogue (no dy in memory)
+    const disco::Geometry& g = psi->g;
+    const disco::TilePlan& P = psi->tile_fused_adj;
+    const DevTile& d = psi->dtile_fused_adj;
+    disco::Ring2Launch R{d.tiles, d.loads, d.copies, d.cmds, d.rows, d.cta_tiles, d.b, P.n_ctas, P.n_qt, P.K, P.nb,
+                         P.ns, P.nrb, P.nbs, P.bslot_bytes, P.mirror, B * C_out, g.nlat_out, g.nlat_in, g.nlon_in};
+    disco::Ring2Fused F{dout, w, nullptr, dx, C_out, C_in, 1};
+    cudaError_t e = disco::launch_fused_ring2(R, F, st);
+    if (e != cudaSuccess) return cuda_fail(e, "fused input-gradient launch");
+    return DISCO_OK;
+  }
   char* ws = static_cast<char*>(workspace);
   void* dy = ws + L.dy;
   s = launch_dy(psi, B, C_in, C_out, groups, dtype, dout, w, ws + L.wt, dy, st);

@@ -58,9 +58,9 @@ struct Args {
   int ns, nbs, nrb;
   uint32_t bslot_bytes;
   // fused forward: out = W y + bias instead of y
-  const __nv_bfloat16* w;     // [C_out][64][K]
+  const __nv_bfloat16* w;     // [C_out][64][K], or [64][C_out][K] with w_t (the adjoint's W^T)
   const __nv_bfloat16* bias;  // [C_out] or null
-  int C_out;
+  int C_out, w_t;
 };
 
 __device__ __forceinline__ int4 shfl4(const int4& v, int src) {
@@ -560,7 +560,8 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
   } else if (warp < 4) {
     // ------------------------------------------------------------------ fused epilogue warps
     // out[b, o, j, q] = bias[o] + sum_{c, k} W[o, c, k] y[b, c, k, j, q] for the 64 channels c
-    // of one batch element (the plane tile).  Per row: each warp drains its TMEM lane quadrant
+    // of one batch element (the plane tile); with w_t the same with W[c, o, k] (the input gradient:
+    // y is then the transposed contraction of dout, and out is dx).  Per row: each warp drains its TMEM lane quadrant
     // (32 channels of mirror group quad / 2) and releases the buffer; then, one kernel index k
     // at a time, the two warps of a group write y_k of their channels into their staging
     // buffers ([c][64 q], 128-byte swizzle: the MN-major B operand of the mix) and the group's
@@ -575,7 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
     // W_k[o][c] into shared memory, K-major with the 128-byte swizzle; rows o >= C_out are zero
     for (int i = threadIdx.x; i < K * 64 * 64; i += 128) {
       const int k = i >> 12, o = (i >> 6) & 63, c = i & 63;
-      const __nv_bfloat16 v = o < a.C_out ? a.w[((size_t)o * 64 + c) * K + k] : __float2bfloat16(0.0f);
+      const size_t wi = a.w_t ? ((size_t)c * a.C_out + o) * K + k : ((size_t)o * 64 + c) * K + k;
+      const __nv_bfloat16 v = o < a.C_out ? a.w[wi] : __float2bfloat16(0.0f);
       *reinterpret_cast<__nv_bfloat16*>(sW + (size_t)k * 8192 + o * 128 + ((((c >> 3) ^ (o & 7))) << 4) + (c & 7) * 2) = v;
     }
     tc::fence_proxy_async();
@@ -765,6 +767,7 @@ cudaError_t launch_k(const Ring2Launch& L, const void* src, void* dst, const Rin
     a.w = static_cast<const __nv_bfloat16*>(F->w);
     a.bias = static_cast<const __nv_bfloat16*>(F->bias);
     a.C_out = F->C_out;
+    a.w_t = F->w_t;
   }
   const size_t bars = 8 * (kMaxSlots + 2 * kMaxBslots + kMaxBufs + 3) + 16;
   const size_t smem = 1024 + (size_t)L.ns * kSlotBytes + (((size_t)L.nbs * L.bslot_bytes + 1023) & ~(size_t)1023) +

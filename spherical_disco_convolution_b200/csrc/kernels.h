@@ -87,12 +87,14 @@ struct Ring2Launch {
 };
 // Fused forward on the same kernel (mirror rows, C_in = 64 channels per batch element, groups 1,
 // C_out <= 64): out [B][C_out][n_out_rows][nlon] = bias + the channel mix of the contraction.
+// With w_t, over the transposed-Psi plan and dout as the source, it is the input gradient dx.
 struct Ring2Fused {
   const void* x;
-  const void* w;     // [C_out][64][K] bf16
+  const void* w;     // [C_out][64][K] bf16, or [64][C_out][K] with w_t
   const void* bias;  // [C_out] bf16 or null
   void* out;
   int C_in, C_out;
+  int w_t = 0;       // 1: mix with the transposed weights (the input gradient)
 };
 cudaError_t launch_fused_ring2(const Ring2Launch& L, const Ring2Fused& F, cudaStream_t st);
 bool ring2_kernel_k(int K);

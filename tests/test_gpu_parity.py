@@ -50,6 +50,8 @@ EDGE = {
     # windows; and 64 output channels without bias
     "ring_fused_k3": Workload("ring_fused_k3", 2, 64, 48, 1, 49, 160, 49, 160, (3, 1), 2 * math.pi / 48, "bf16"),
     "ring_fused_nb": Workload("ring_fused_nb", 1, 64, 64, 1, 33, 96, 33, 96, (3, 1), 0.3, "bf16", bias=False),
+    # input gradient on the same kernel (64 output channels, 32 input channels, two batch elements)
+    "ring_dx_k3": Workload("ring_dx_k3", 2, 32, 64, 1, 49, 160, 49, 160, (3, 1), 2 * math.pi / 48, "bf16"),
 }
 
 
@@ -278,7 +280,8 @@ def test_fused_tensor_core_matches_unfused(name):
 @pytest.mark.parametrize("name", ["ragged_iso_f32", "tc_small_bf16", "ragged_down_bf16", "grouped"])
 def test_input_gradient_halves_compose(name):
     """disco_einsum_adjoint followed by disco_contract_adjoint is disco_bwd_input, bit for bit
-    (the same kernels in the same order)."""
+    (the same kernels in the same order), on layers that the one-launch input gradient (64 output
+    channels, groups 1, mirror rows) does not serve; that one is checked against the oracle."""
     wl, inp = workload(name), inputs(name)
     psi = gpu_psi(name)
     dout, w = dev(inp["dout"], wl), dev(inp["w"], wl)
