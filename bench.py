@@ -530,7 +530,8 @@ def run_gpu(args):
     traffic = recorded_traffic(dom, wl.name)
     roof = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["GBps"], "peak": peak, "unit": "GB/s",
             "frac": kernels[dom]["frac_hbm"], "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
-            "headline_contract": {"achieved": kernels["contract"]["GBps"], "frac": kernels["contract"]["frac_hbm"]}}
+            "headline_contract": {"achieved": kernels["contract"]["GBps"], "frac": kernels["contract"]["frac_hbm"],
+                                  "traffic": recorded_traffic("contract", wl.name)}}
     line = {
         "metric": METRIC, "value": units_all / (el_max / 1000.0), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": el_max / args.steps,
