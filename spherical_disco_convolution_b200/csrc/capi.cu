@@ -327,7 +327,14 @@ WsLayout layout(const disco_psi* psi, int op, int B, int C_in, int C_out, int gr
   } else if (op == DISCO_OP_BWD_WEIGHT || op == DISCO_OP_BWD_WEIGHT_RECOMPUTE) {
     const int N = (int)n_out;
     L.tc = dtype == DISCO_BF16 && disco::dw_tc_supported(C_out / groups, (C_in / groups) * g.K, N);
-    L.nc = L.tc ? 8192 : 4096;
+    if (L.tc) {
+      // one CTA per (split, batch, group), about one per SM of a B200 (148): the splits cover the
+      // positions in multiples of the 64-element stage
+      const int want = std::max(1, (148 + B * groups / 2) / (B * groups));
+      L.nc = (int)((((long)N + want - 1) / want + 63) / 64 * 64);
+    } else {
+      L.nc = 4096;
+    }
     L.nchunk = (N + L.nc - 1) / L.nc;
     const size_t nsplit = (size_t)B * L.nchunk;
     size_t off = 0;

@@ -149,36 +149,41 @@ __global__ void __launch_bounds__(128, 2) mix_tc_kernel(const __grid_constant__ 
 
 struct DwTcArgs {
   float* part;
+  float* bpart;  // written here when ones_row (dbias as the product with a row of ones), else null
   int G, Og, Rg, N, nc, nchunk;
+  int n_tiles, stages, ones_row;  // M tiles of 128 rows (r = (c, k)); the spare row of the last tile, -1 none
 };
 
-__global__ void __launch_bounds__(128, 2) dw_tc_kernel(const __grid_constant__ CUtensorMap map_y,
+// dw partials for one split of the spatial positions: D_t[r][o] = sum_n y[b, g, 128t + r, n] dout[b, g, o, n]
+// for every M tile t of the Rg rows in one CTA, so that each dout tile is read once.  With a
+// spare row in the last tile (Rg % 128 != 0) that row is set to ones after each stage lands,
+// which makes it the split's sum of dout: the dbias partial.
+__global__ void __launch_bounds__(128, 1) dw_tc_kernel(const __grid_constant__ CUtensorMap map_y,
                                                        const __grid_constant__ CUtensorMap map_d, DwTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  const int BN = a.Og;
-  const uint32_t a_bytes = 128 * 128;
+  const int BN = a.Og, T = a.n_tiles, S = a.stages;
+  const uint32_t a_bytes = 128 * 128;            // one M tile: 128 rows x 64 K, 128-byte swizzle
   const uint32_t b_bytes = (uint32_t)BN * 128;
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + kStages * a_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kStages * b_bytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* done = empty + kStages;
+  const uint32_t st_bytes = (uint32_t)T * a_bytes + b_bytes;
+  uint8_t* sS = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sS + (size_t)S * st_bytes);
+  uint64_t* empty = full + S;
+  uint64_t* done = empty + S;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
   const int chunk = blockIdx.x;
-  const int r0 = blockIdx.y * 128;
   const int bg = blockIdx.z;
   const int g = bg % a.G, b = bg / a.G;
   const int nb = chunk * a.nc;
   const int nk = (min(a.N, nb + a.nc) - nb + kBK - 1) / kBK;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t ncols = tmem_cols(BN);
+  const uint32_t ncols = tmem_cols(T * BN);
 
   if (threadIdx.x == 0) {
     tc::prefetch_map(&map_y);
     tc::prefetch_map(&map_d);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       tc::mbar_init(&full[s], 1);
       tc::mbar_init(&empty[s], 1);
     }
@@ -196,24 +201,35 @@ __global__ void __launch_bounds__(128, 2) dw_tc_kernel(const __grid_constant__ C
 
   if (warp == 0 && lane == 0) {
     for (int kc = 0; kc < nk; ++kc) {
-      const int s = kc % kStages;
-      if (kc >= kStages && !tc::mbar_wait(&empty[s], ((kc / kStages) & 1) ^ 1)) break;
-      tc::mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes);
-      tc::tma_load_3d(sA + s * a_bytes, &map_y, &full[s], nb + kc * kBK, r0, bg);
-      tc::tma_load_3d(sB + s * b_bytes, &map_d, &full[s], nb + kc * kBK, 0, bg);
+      const int s = kc % S;
+      if (kc >= S && !tc::mbar_wait(&empty[s], ((kc / S) & 1) ^ 1)) break;
+      tc::mbar_arrive_expect_tx(&full[s], st_bytes);
+      uint8_t* st = sS + (size_t)s * st_bytes;
+      for (int t = 0; t < T; ++t) tc::tma_load_3d(st + t * a_bytes, &map_y, &full[s], nb + kc * kBK, 128 * t, bg);
+      tc::tma_load_3d(st + T * a_bytes, &map_d, &full[s], nb + kc * kBK, 0, bg);
     }
   } else if (warp == 1 && lane == 0) {
     const uint32_t idesc = tc::idesc_bf16(128, BN, false, false);
     for (int kc = 0; kc < nk; ++kc) {
-      const int s = kc % kStages;
-      if (!tc::mbar_wait(&full[s], (kc / kStages) & 1)) break;
+      const int s = kc % S;
+      if (!tc::mbar_wait(&full[s], (kc / S) & 1)) break;
+      uint8_t* st = sS + (size_t)s * st_bytes;
+      if (a.ones_row >= 0) {
+        // the spare row of the last tile: 64 K-elements of 1.0 (the swizzle only permutes them)
+        uint4* row = reinterpret_cast<uint4*>(st + (T - 1) * a_bytes + a.ones_row * 128);
+        const uint4 one = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) row[i] = one;
+        tc::fence_proxy_async();
+      }
       tc::fence_after_sync();
-      const uint32_t a0 = tc::smem_u32(sA + s * a_bytes);
-      const uint32_t b0 = tc::smem_u32(sB + s * b_bytes);
+      const uint32_t a0 = tc::smem_u32(st);
+      const uint32_t b0 = tc::smem_u32(st + T * a_bytes);
 #pragma unroll
       for (int kk = 0; kk < kBK / 16; ++kk)
-        tc::mma_bf16(tmem, tc::desc_sw128(a0 + kk * 32, 16, 1024), tc::desc_sw128(b0 + kk * 32, 16, 1024), idesc,
-                     (kc | kk) != 0);
+        for (int t = 0; t < T; ++t)
+          tc::mma_bf16(tmem + (uint32_t)(t * BN), tc::desc_sw128(a0 + t * a_bytes + kk * 32, 16, 1024),
+                       tc::desc_sw128(b0 + kk * 32, 16, 1024), idesc, (kc | kk) != 0);
       tc::mma_commit(&empty[s]);
     }
     tc::mma_commit(done);
@@ -222,15 +238,21 @@ __global__ void __launch_bounds__(128, 2) dw_tc_kernel(const __grid_constant__ C
   const bool ok = tc::mbar_wait(done, 0);
   tc::fence_after_sync();
   if (ok) {
-    const int r = r0 + warp * 32 + lane;
     const size_t split = (size_t)b * a.nchunk + chunk;
     float* P = a.part + ((split * a.G + g) * a.Og) * (size_t)a.Rg;
-    for (int c = 0; c < BN; c += 16) {
-      float v[16];
-      tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
-      if (r < a.Rg)
+    for (int t = 0; t < T; ++t) {
+      const int rl = warp * 32 + lane, r = 128 * t + rl;
+      for (int c = 0; c < BN; c += 16) {
+        float v[16];
+        tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(t * BN + c), v);
+        if (r < a.Rg) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) P[(size_t)(c + i) * a.Rg + r] = nk > 0 ? v[i] : 0.0f;
+          for (int i = 0; i < 16; ++i) P[(size_t)(c + i) * a.Rg + r] = nk > 0 ? v[i] : 0.0f;
+        } else if (t == T - 1 && rl == a.ones_row && a.bpart) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) a.bpart[split * (a.G * a.Og) + g * a.Og + c + i] = nk > 0 ? v[i] : 0.0f;
+        }
+      }
     }
   }
   tc::fence_before_sync();
@@ -271,7 +293,6 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
 }
 
 size_t mix_smem(int BN, int S) { return 1024 + S * (2 * kHalfTile + (size_t)BN * 128) + (2 * S + 2) * 8; }
-size_t dw_smem(int BN) { return 1024 + kStages * (128 * 128 + (size_t)BN * 128) + (2 * kStages + 2) * 8; }
 
 int mix_bn(int Mg) {
   if (Mg <= 256) return Mg;
@@ -308,7 +329,11 @@ cudaError_t launch_mix_tc(const MixArgs& a, cudaStream_t st) {
 }
 
 bool dw_tc_supported(int Og, int Rg, int N) {
-  return tc::encode_tiled_fn() != nullptr && Og % 16 == 0 && Og <= 256 && N % 8 == 0 && Rg >= 1;
+  // every M tile's accumulator in tensor memory and at least two stages in shared memory
+  const int T = (Rg + 127) / 128;
+  const size_t st_bytes = (size_t)T * 128 * 128 + (size_t)Og * 128;
+  return tc::encode_tiled_fn() != nullptr && Og % 16 == 0 && Og <= 256 && N % 8 == 0 && Rg >= 1 && T * Og <= 512 &&
+         2 * st_bytes + 1280 <= kTcSmemLimit;
 }
 
 cudaError_t launch_dw_tc(const DwArgs& a, cudaStream_t st) {
@@ -320,14 +345,19 @@ cudaError_t launch_dw_tc(const DwArgs& a, cudaStream_t st) {
   const cuuint64_t sd[2] = {(cuuint64_t)a.N * 2, (cuuint64_t)a.Og * a.N * 2};
   const cuuint32_t bd[3] = {64, (cuuint32_t)a.Og, 1};
   if (!make_map(&my, a.yv, 3, dy, sy, by) || !make_map(&md, a.dout, 3, dd, sd, bd)) return cudaErrorInvalidValue;
-  DwTcArgs t{a.part, a.G, a.Og, a.Rg, a.N, a.nc, a.nchunk};
-  const size_t smem = dw_smem(a.Og);
+  const int T = (a.Rg + 127) / 128;
+  const size_t st_bytes = (size_t)T * 128 * 128 + (size_t)a.Og * 128;
+  const int S = (int)std::min<size_t>(kStages, (kTcSmemLimit - 1024 - 256) / st_bytes);
+  if (S < 2 || T * a.Og > 512) return cudaErrorInvalidValue;
+  const int ones = (a.bpart && a.Rg % 128) ? a.Rg % 128 : -1;
+  DwTcArgs t{a.part, ones >= 0 ? a.bpart : nullptr, a.G, a.Og, a.Rg, a.N, a.nc, a.nchunk, T, S, ones};
+  const size_t smem = 1024 + (size_t)S * st_bytes + (2 * S + 2) * 8;
   cudaError_t e = cudaFuncSetAttribute(dw_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.nchunk, (a.Rg + 127) / 128, a.B * a.G);
+  dim3 grid(a.nchunk, 1, a.B * a.G);
   dw_tc_kernel<<<grid, 128, smem, st>>>(my, md, t);
   count_launch();
-  if (a.bpart) {
+  if (a.bpart && ones < 0) {
     dim3 g2(a.nchunk, a.B * a.G);
     bias_partial_kernel<<<g2, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.dout), a.bpart, a.G, a.Og, a.N, a.nc,
                                             a.nchunk);
