@@ -442,13 +442,14 @@ bool tile_params(int K, bool adjoint, int n_ctas, disco::TileParams* p) {
   return true;
 }
 
-// The fused variant keeps the mix weights (K x 8 KB) in shared memory and the mix accumulators
-// (128 columns) in tensor memory: three B slots of 1 KB of record and four K-steps, and the row
-// buffers that the remaining 384 columns hold.
+// The fused variant keeps the mix weights (K x 8 KB) and the y staging of every kernel index
+// (K x 16 KB) in shared memory and the mix accumulators (128 columns) in tensor memory: four ring
+// slots, three B slots of 1 KB of record and four K-steps, and the row buffers that the
+// remaining 384 columns hold.
 bool tile_params_fused(int K, int n_ctas, disco::TileParams* p) {
   if (!(K == 1 || K == 3)) return false;
   p->nb = 4;
-  p->ns = 5;
+  p->ns = 4;  // the y staging of every kernel index (K x 16 KB) takes one slot's room
   p->nrb = std::min(8, 384 / (4 * 16 * K));
   p->nbs = 3;
   p->bslot_bytes = disco::kMetaBytes + 4 * (2 * 16 * K * 16);

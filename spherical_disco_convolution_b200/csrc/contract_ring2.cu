@@ -209,8 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
   uint8_t* sX = smem;                                          // ns slots of two chunks
   uint8_t* sB = sX + (size_t)a.ns * kSlotBytes;                // nbs B slots
   uint8_t* sW = sB + (((size_t)a.nbs * a.bslot_bytes + 1023) & ~(size_t)1023);  // fused: the mix weights
-  uint8_t* sY = sW + kWBytes;  // one buffer per epilogue warp (fused: also the mix's y operand)
-  uint64_t* xfull = reinterpret_cast<uint64_t*>(sY + 4 * kYBuf);
+  // one buffer per epilogue warp; fused: one per warp and kernel index ([k][warp][32 rows][128 B],
+  // the mix's y operand: group g of index k is 64 rows at k * 16 KB + g * 8 KB)
+  uint8_t* sY = sW + kWBytes;
+  uint64_t* xfull = reinterpret_cast<uint64_t*>(sY + (kFused ? K : 1) * 4 * kYBuf);
   uint64_t* bfull = xfull + kMaxSlots;
   uint64_t* bempty = bfull + kMaxBslots;
   uint64_t* tempty = bempty + kMaxBslots;
@@ -571,7 +573,6 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
     // store out for the row and its mirror row.
     const int quad = warp;
     const int grp = quad >> 1;
-    uint8_t* wy = sY + (size_t)warp * kYBuf;
     if (lane == 0) tc::prefetch_map(&ymap);
     // W_k[o][c] into shared memory, K-major with the 128-byte swizzle; rows o >= C_out are zero
     for (int i = threadIdx.x; i < K * 64 * 64; i += 128) {
@@ -645,30 +646,35 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
 #pragma unroll
               for (int i = 0; i < 32; ++i) pk[k][i] = 0u;
           }
-          // the mix, one kernel index at a time
+          // the mix: y of every kernel index into this warp's buffers (free: the previous row's mix
+          // has completed and its out stores from buffers 0 and 1 have read them), then the
+          // group's first warp issues all 4K MMAs into the group's accumulator
+          if (lane == 0) tc::bulk_wait_read0();
+          __syncwarp();
 #pragma unroll
           for (int k = 0; k < K; ++k) {
-            // the staging buffer is free: the previous out store from it has read it (warps 0, 1)
-            // and the previous mix round that read it has completed (waited below)
-            if (lane == 0) tc::bulk_wait_read0();
-            __syncwarp();
-            uint8_t* rowp = wy + (size_t)lane * 128;
+            uint8_t* rowp = sY + (size_t)k * 4 * kYBuf + (size_t)warp * kYBuf + (size_t)lane * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
               *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) =
                   make_uint4(pk[k][4 * c], pk[k][4 * c + 1], pk[k][4 * c + 2], pk[k][4 * c + 3]);
-            tc::fence_proxy_async();
-            tc::named_bar_sync(2 + grp, 64);
-            if ((quad & 1) == 0 && lane == 0) {
-              tc::fence_after_sync();
+          }
+          tc::fence_proxy_async();
+          tc::named_bar_sync(2 + grp, 64);
+          if ((quad & 1) == 0 && lane == 0) {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
               const uint32_t wk = tc::smem_u32(sW) + (uint32_t)k * 8192u;
-              const uint32_t yg = tc::smem_u32(sY) + (uint32_t)grp * 8192u;
+              const uint32_t yg = tc::smem_u32(sY) + (uint32_t)k * 4u * kYBuf + (uint32_t)grp * 8192u;
 #pragma unroll
               for (int j = 0; j < 4; ++j)
                 tc::mma_bf16(dmix + (uint32_t)(64 * grp), tc::desc_sw128(wk + 32u * j, 16, 1024),
                              tc::desc_sw128(yg + 2048u * j, 16, 1024), midesc, (k > 0 || j > 0) ? 1u : 0u);
-              tc::mma_commit(&mixb[grp]);
             }
+            tc::mma_commit(&mixb[grp]);
+          }
+          {
             int good = 1;
             if (lane == 0) good = tc::mbar_wait_sleep(&mixb[grp], (mpar >> grp) & 1u, 64);
             ok = __shfl_sync(0xffffffffu, good, 0) != 0 && ok;
@@ -695,9 +701,10 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
             for (int g = 0; g < 2; ++g) {
               const int orow = g == 0 ? r : rbar;
               const bool st = g == 0 || (rbar != r && rbar != 0xFFFF);
-              if (lane == 0) tc::bulk_wait_read0();
-              __syncwarp();
-              uint8_t* rowp = wy + (size_t)lane * 128;
+              // group g's out tile in this warp's buffer of kernel index g (read by the mix, which
+              // has completed)
+              uint8_t* ob = sY + (size_t)g * 4 * kYBuf + (size_t)warp * kYBuf;
+              uint8_t* rowp = ob + (size_t)lane * 128;
 #pragma unroll
               for (int c = 0; c < 8; ++c) {
                 uint32_t q4[4];
@@ -712,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
               tc::fence_proxy_async();
               __syncwarp();
               if (lane == 0) {
-                if (st && quad * 32 < a.C_out) tc::tma_store_4d(&ymap, wy, q0, orow, quad * 32, pt);
+                if (st && quad * 32 < a.C_out) tc::tma_store_4d(&ymap, ob, q0, orow, quad * 32, pt);
                 tc::bulk_commit();
               }
             }
@@ -771,7 +778,7 @@ cudaError_t launch_k(const Ring2Launch& L, const void* src, void* dst, const Rin
   }
   const size_t bars = 8 * (kMaxSlots + 2 * kMaxBslots + kMaxBufs + 3) + 16;
   const size_t smem = 1024 + (size_t)L.ns * kSlotBytes + (((size_t)L.nbs * L.bslot_bytes + 1023) & ~(size_t)1023) +
-                      (kFused ? (size_t)K * 8192 : 0) + 4 * kYBuf + bars;
+                      (kFused ? (size_t)K * 8192 : 0) + (size_t)(kFused ? K : 1) * 4 * kYBuf + bars;
   if (smem > kTcSmemLimit) return cudaErrorInvalidValue;
   // x as [BC][n_src_rows][nlon]: boxes of 64 longitudes x 1 row x 64 planes, 128-byte swizzle
   CUtensorMap xm, ym;
