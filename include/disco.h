@@ -138,6 +138,21 @@ disco_status disco_psi_build(const disco_spec_t* spec, int device, disco_psi** o
 disco_status disco_psi_build_band(const disco_spec_t* spec, int j_begin, int j_end, int device, disco_psi** out,
                                   int* i_begin, int* i_end);
 
+/* Psi of one band of input latitudes: the entries of the layer spec describes whose input row i
+ * lies in [i_begin, i_end), for every output latitude.  This is the per-rank layer of the
+ * "reduce-scatter" polar mode on the page "torch_harmonics.distributed.
+ * DistributedDiscreteContinuousConvS2" (parameter polar_mode): every rank computes a partial sum
+ * over all output latitudes from the input rows it owns, and a reduce-scatter completes and
+ * splits it.  The handle is a layer with nlat_in = i_end - i_begin (its rows re-indexed from 0)
+ * and the full nlat_out: disco_contract / disco_fwd / disco_einsum give the band's partial y and
+ * out (sum them over bands; add the bias once), disco_bwd_input takes dout on every output row
+ * and gives dx on the band's rows, disco_bwd_weight the band's part of dw (sum over bands).
+ * Output rows that no entry of the band reaches are written as zeros by the contraction (and
+ * input rows no entry reaches by the adjoint).  disco_fwd_fused returns UNSUPPORTED on such a
+ * handle when it has rows without entries.  Errors as disco_psi_build, and INVALID_ARG for an
+ * empty or out-of-range row range.  The caller owns the handle (disco_psi_destroy). */
+disco_status disco_psi_build_inputs(const disco_spec_t* spec, int i_begin, int i_end, int device, disco_psi** out);
+
 /* Frees host and device memory of a Psi (synchronises the device first).  NULL is a no-op. */
 disco_status disco_psi_destroy(disco_psi* psi);
 

@@ -46,10 +46,12 @@ class Psi:
     """Precomputed sparse convolution tensor of one layer geometry, on one device."""
 
     def __init__(self, nlat_in: int, nlon_in: int, nlat_out: int, nlon_out: int, kernel_shape, theta_cutoff: float,
-                 device=None, grid_in: str = "equiangular", grid_out: str = "equiangular", rows=None):
+                 device=None, grid_in: str = "equiangular", grid_out: str = "equiangular", rows=None,
+                 inputs=None):
         """rows=(j_begin, j_end) builds the Psi of those output latitudes only (a polar band): the
         handle then takes x on input rows self.in_rows = (i_begin, i_end) and gives out rows
-        j_begin..j_end-1."""
+        j_begin..j_end-1.  inputs=(i_begin, i_end) builds the Psi of those input latitudes over
+        every output latitude (a band's partial sums, the reduce-scatter polar mode)."""
         dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.device = dev
         self.index = dev.index if dev.index is not None else torch.cuda.current_device()
@@ -64,7 +66,11 @@ class Psi:
         self.spec = D.make_spec(nlat_in, nlon_in, nlat_out, nlon_out, kernel_shape, theta_cutoff,
                                 D.GRID_CODES[grid_in], D.GRID_CODES[grid_out])
         with torch.cuda.device(self.index):
-            if rows is None:
+            if inputs is not None:
+                self.handle = D.disco_psi_build_inputs(self.spec, inputs[0], inputs[1], self.index)
+                self.in_rows = (inputs[0], inputs[1])
+                self.in_shape = (inputs[1] - inputs[0], nlon_in)
+            elif rows is None:
                 self.handle = D.disco_psi_build(self.spec, self.index)
             else:
                 self.handle, ib, ie = D.disco_psi_build_band(self.spec, rows[0], rows[1], self.index)

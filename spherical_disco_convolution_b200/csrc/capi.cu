@@ -217,6 +217,11 @@ struct disco_psi {
   disco::TilePlan tile_fused_adj;
   bool tile_fused_adj_built = false;
   DevTile dtile_fused_adj;
+  // rows without entries (handles of a band of input latitudes): output rows of the forward and
+  // input rows of the adjoint, zeroed after each contraction into them
+  std::vector<int> empty_out, empty_in;
+  int* d_empty_out = nullptr;
+  int* d_empty_in = nullptr;
 };
 
 namespace {
@@ -594,7 +599,7 @@ disco_status run_banded(const disco_psi* psi, const disco::GatherPlan& P, disco:
 }
 
 // Forward contraction x -> y with the best gather form for the layer.
-disco_status launch_contract(const disco_psi* psi, int BC, disco_dtype dtype, const void* x, void* y,
+disco_status launch_contract_core(const disco_psi* psi, int BC, disco_dtype dtype, const void* x, void* y,
                              cudaStream_t st, const char* what) {
   const disco::Geometry& g = psi->g;
   if (dtype == DISCO_BF16 && psi->tz_ok && !(reinterpret_cast<uintptr_t>(x) & 15) &&
@@ -659,7 +664,7 @@ disco_status launch_dy(const disco_psi* psi, int B, int C_in, int C_out, int gro
 }
 
 // dx from dy: the adjoint contraction with the best kernel for the layer.
-disco_status launch_adjoint(const disco_psi* psi, int BC, disco_dtype dtype, const void* dy, void* dx,
+disco_status launch_adjoint_core(const disco_psi* psi, int BC, disco_dtype dtype, const void* dy, void* dx,
                             cudaStream_t st) {
   const disco::Geometry& g = psi->g;
   const bool bf16 = dtype == DISCO_BF16;
@@ -710,6 +715,28 @@ disco_status launch_adjoint(const disco_psi* psi, int BC, disco_dtype dtype, con
   return DISCO_OK;
 }
 
+// The contractions with the rows that have no entries (handles of a band of input latitudes)
+// set to zero afterwards, whatever kernel ran.
+disco_status launch_contract(const disco_psi* psi, int BC, disco_dtype dtype, const void* x, void* y,
+                             cudaStream_t st, const char* what) {
+  disco_status s = launch_contract_core(psi, BC, dtype, x, y, st, what);
+  if (s || psi->empty_out.empty()) return s;
+  const disco::Geometry& g = psi->g;
+  cudaError_t e = disco::launch_zero_rows(y, dtype == DISCO_BF16 ? 2 : 4, psi->d_empty_out, (int)psi->empty_out.size(),
+                                          BC * g.K, g.nlat_out, g.nlon_out, st);
+  return e == cudaSuccess ? DISCO_OK : cuda_fail(e, what);
+}
+
+disco_status launch_adjoint(const disco_psi* psi, int BC, disco_dtype dtype, const void* dy, void* dx,
+                            cudaStream_t st) {
+  disco_status s = launch_adjoint_core(psi, BC, dtype, dy, dx, st);
+  if (s || psi->empty_in.empty()) return s;
+  const disco::Geometry& g = psi->g;
+  cudaError_t e = disco::launch_zero_rows(dx, dtype == DISCO_BF16 ? 2 : 4, psi->d_empty_in, (int)psi->empty_in.size(),
+                                          BC, g.nlat_in, g.nlon_in, st);
+  return e == cudaSuccess ? DISCO_OK : cuda_fail(e, "adjoint contraction");
+}
+
 }  // namespace
 
 extern "C" {
@@ -741,7 +768,7 @@ namespace {
 // re-indexed to a layer of its own: output rows j - j_begin, input rows i - i_begin over the
 // input rows [i_begin, i_end) that its entries reach.
 disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, int device, disco_psi** out,
-                            int* i_begin, int* i_end) {
+                            int* i_begin, int* i_end, int in_begin = -1, int in_end = -1) {
   if (!out) return fail(DISCO_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   if (!spec) return fail(DISCO_ERR_INVALID_ARG, "spec is NULL");
@@ -783,7 +810,30 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
   }
   if (j_end < 0) j_end = g.nlat_out;
   int ib = 0, ie = g.nlat_in;
-  if (j_begin != 0 || j_end != g.nlat_out) {
+  if (in_begin >= 0) {
+    // a band of input latitudes: its entries of every output row, input rows re-indexed
+    std::vector<disco::PsiEntry> keep;
+    keep.reserve(h->entries.size());
+    for (const disco::PsiEntry& en : h->entries)
+      if (en.i >= in_begin && en.i < in_end) {
+        disco::PsiEntry e2 = en;
+        e2.i -= in_begin;
+        keep.push_back(e2);
+      }
+    h->entries.swap(keep);
+    g.nlat_in = in_end - in_begin;
+    ib = in_begin;
+    ie = in_end;
+    std::vector<char> has_out(g.nlat_out, 0), has_in(g.nlat_in, 0);
+    for (const disco::PsiEntry& en : h->entries) {
+      has_out[en.j] = 1;
+      has_in[en.i] = 1;
+    }
+    for (int j = 0; j < g.nlat_out; ++j)
+      if (!has_out[j]) h->empty_out.push_back(j);
+    for (int i = 0; i < g.nlat_in; ++i)
+      if (!has_in[i]) h->empty_in.push_back(i);
+  } else if (j_begin != 0 || j_end != g.nlat_out) {
     ib = g.nlat_in;
     ie = 0;
     for (const disco::PsiEntry& en : h->entries) {
@@ -827,6 +877,8 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
     if (e == cudaSuccess) e = upload_plan(h->adj, &h->dadj);
     if (e == cudaSuccess) e = upload_plan(h->fwdb, &h->dfwdb);
     if (e == cudaSuccess) e = upload_plan(h->adjb, &h->dadjb);
+    if (e == cudaSuccess && !h->empty_out.empty()) e = upload(h->empty_out, &h->d_empty_out);
+    if (e == cudaSuccess && !h->empty_in.empty()) e = upload(h->empty_in, &h->d_empty_in);
     // tensor-core contraction for bf16 signals (DISCO_SIMT_CONTRACT=1 keeps the gather kernels)
     const char* simt = std::getenv("DISCO_SIMT_CONTRACT");
     if (e == cudaSuccess && !(simt && simt[0] == '1') &&
@@ -866,6 +918,8 @@ disco_status psi_build_rows(const disco_spec_t* spec, int j_begin, int j_end, in
       for (int w = 0; w < 4; ++w) free_tile(&h->dtile[w]);
       free_tile(&h->dtile_fused);
       free_tile(&h->dtile_fused_adj);
+      cudaFree(h->d_empty_out);
+      cudaFree(h->d_empty_in);
       delete h;
       return fail(DISCO_ERR_ALLOC, std::string("Psi upload failed: ") + cudaGetErrorString(e));
     }
@@ -889,6 +943,13 @@ disco_status disco_psi_build_band(const disco_spec_t* spec, int j_begin, int j_e
   return psi_build_rows(spec, j_begin, j_end, device, out, i_begin, i_end);
 }
 
+disco_status disco_psi_build_inputs(const disco_spec_t* spec, int i_begin, int i_end, int device, disco_psi** out) {
+  if (!spec) return fail(DISCO_ERR_INVALID_ARG, "spec is NULL");
+  if (i_begin < 0 || i_end <= i_begin || i_end > spec->nlat_in)
+    return fail(DISCO_ERR_INVALID_ARG, "need 0 <= i_begin < i_end <= nlat_in");
+  return psi_build_rows(spec, 0, -1, device, out, nullptr, nullptr, i_begin, i_end);
+}
+
 disco_status disco_psi_destroy(disco_psi* psi) {
   if (!psi) return DISCO_OK;
   if (psi->device >= 0) {
@@ -906,6 +967,8 @@ disco_status disco_psi_destroy(disco_psi* psi) {
     for (int w = 0; w < 4; ++w) free_tile(&psi->dtile[w]);
     free_tile(&psi->dtile_fused);
     free_tile(&psi->dtile_fused_adj);
+    cudaFree(psi->d_empty_out);
+    cudaFree(psi->d_empty_in);
     if (psi->side) cudaStreamDestroy(psi->side);
     if (psi->fork) cudaEventDestroy(psi->fork);
     if (psi->join) cudaEventDestroy(psi->join);
@@ -1098,6 +1161,10 @@ disco_status disco_fwd_fused(const disco_psi* psi, int B, int C_in, int C_out, i
   if (!x || !w || !out) return fail(DISCO_ERR_INVALID_ARG, "x, w and out must be non-NULL");
   const disco::Geometry& g = psi->g;
   if (!disco::gather_supports(g.K, g.stride)) return fail(DISCO_ERR_UNSUPPORTED, "K or stride not compiled");
+  if (!psi->empty_out.empty())
+    return fail(DISCO_ERR_UNSUPPORTED,
+                "the fused forward needs an entry in every output row; this handle (a band of input latitudes) "
+                "has rows without: use disco_fwd or disco_contract + disco_einsum");
   const bool bf16 = dtype == DISCO_BF16;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int Cg = C_in / groups;

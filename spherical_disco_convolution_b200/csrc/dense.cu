@@ -7,6 +7,8 @@
 // with n running over the output grid.  The same kernel serves the transposed
 // einsum of the backward pass (dy = w^T dout).  The weight gradient is the
 // split-K GEMM dw[o, r] = sum_n dout[o, n] * y[r, n] reduced in a fixed order.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -208,6 +210,35 @@ cudaError_t launch_dw_partial_simt(bool bf16, const DwArgs& a, cudaStream_t st) 
     dw_partial_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
   else
     dw_partial_kernel<float><<<grid, 256, 0, st>>>(a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+namespace {
+// t[p][rows[r]][0..n) = 0 for every plane p: one CTA per (row, plane block), 16-byte stores.
+// With vec (base address and row length multiples of 16 bytes) 16-byte stores, else bytes.
+__global__ void zero_rows_kernel(uint8_t* t, const int* __restrict__ rows, int n_rows, int planes, int nrows,
+                                 size_t row_bytes, bool vec) {
+  const int r = rows[blockIdx.x];
+  for (int p = blockIdx.y; p < planes; p += gridDim.y) {
+    uint8_t* base = t + ((size_t)p * nrows + r) * row_bytes;
+    if (vec) {
+      for (size_t o = (size_t)threadIdx.x * 16; o < row_bytes; o += (size_t)blockDim.x * 16)
+        *reinterpret_cast<uint4*>(base + o) = make_uint4(0u, 0u, 0u, 0u);
+    } else {
+      for (size_t o = threadIdx.x; o < row_bytes; o += blockDim.x) base[o] = 0;
+    }
+  }
+}
+}  // namespace
+
+cudaError_t launch_zero_rows(void* t, int elem_bytes, const int* rows, int n_rows, int planes, int nrows, int nlon,
+                             cudaStream_t st) {
+  if (n_rows <= 0 || planes <= 0) return cudaSuccess;
+  const size_t row_bytes = (size_t)nlon * elem_bytes;
+  const bool vec = !(reinterpret_cast<uintptr_t>(t) & 15) && !(row_bytes & 15);
+  dim3 grid(n_rows, std::min(planes, 64));
+  zero_rows_kernel<<<grid, 128, 0, st>>>(static_cast<uint8_t*>(t), rows, n_rows, planes, nrows, row_bytes, vec);
   count_launch();
   return cudaGetLastError();
 }

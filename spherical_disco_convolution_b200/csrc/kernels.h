@@ -156,6 +156,9 @@ cudaError_t launch_dw_partial_simt(bool bf16, const DwArgs& a, cudaStream_t st);
 // Tensor-core form for bf16 (Og % 16 == 0, Og <= 256, N % 8 == 0); nc must be a multiple of 64.
 bool dw_tc_supported(int Og, int Rg, int N);
 cudaError_t launch_dw_tc(const DwArgs& a, cudaStream_t st);
+// t[p][rows[i]][0..nlon) = 0 for p < planes, t being [planes][nrows][nlon] of elem_bytes elements.
+cudaError_t launch_zero_rows(void* t, int elem_bytes, const int* rows, int n_rows, int planes, int nrows, int nlon,
+                             cudaStream_t st);
 // dw[g*Og + o, r] = sum_split part[split, g, o, r]; dbias[o] = sum_split bpart[split, o]; fixed order.
 cudaError_t launch_dw_reduce(bool bf16, const float* part, const float* bpart, void* dw, void* dbias, int nsplit,
                              int G, int Og, int Rg, cudaStream_t st);

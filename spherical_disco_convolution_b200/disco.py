@@ -90,6 +90,7 @@ def _load():
     sig = {
         "disco_psi_build": [ctypes.POINTER(disco_spec_t), I, ctypes.POINTER(P)],
         "disco_psi_build_band": [ctypes.POINTER(disco_spec_t), I, I, I, ctypes.POINTER(P), IP, IP],
+        "disco_psi_build_inputs": [ctypes.POINTER(disco_spec_t), I, I, I, ctypes.POINTER(P)],
         "disco_psi_destroy": [P],
         "disco_psi_info": [P, IP, ctypes.POINTER(LL)],
         "disco_psi_export": [P, IP, IP, IP, IP, DP],
@@ -173,6 +174,13 @@ def disco_psi_build_band(spec: disco_spec_t, j_begin: int, j_end: int, device: i
     _check(_lib.disco_psi_build_band(ctypes.byref(spec), j_begin, j_end, device, ctypes.byref(h), ctypes.byref(ib),
                                      ctypes.byref(ie)))
     return h, ib.value, ie.value
+
+
+def disco_psi_build_inputs(spec: disco_spec_t, i_begin: int, i_end: int, device: int):
+    """Psi of input rows [i_begin, i_end) (re-indexed from 0) over every output row."""
+    h = ctypes.c_void_p()
+    _check(_lib.disco_psi_build_inputs(ctypes.byref(spec), i_begin, i_end, device, ctypes.byref(h)))
+    return h
 
 
 def disco_psi_destroy(psi) -> None:

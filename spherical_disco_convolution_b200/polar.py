@@ -203,3 +203,135 @@ class PolarDiscoConvS2(torch.nn.Module):
 
     def forward(self, x_own):
         return _PolarFn.apply(x_own.contiguous(), self.weight, self.bias, self)
+
+
+# ------------------------------------------------------------------ the "reduce-scatter" polar mode
+#
+# polar_mode="reduce-scatter" on the same page: every rank computes a partial sum over all output
+# latitudes from the input latitudes it owns, and a reduce-scatter completes the sums and splits
+# them by output band.  No bound on the angular reach; the partial sums stay at the full nlat_out.
+# Readings where the page is silent:
+#
+#   * the reduce-scatter runs on out (C_out channels), after each rank's weight einsum of its
+#     partial y, not on the K-expanded y: the einsum is linear, so the sums are the same with K
+#     times less collective volume; the bias is added once, on the owner of each output row;
+#   * backward is the adjoint: dout on the rank's output rows is all-gathered to every output row,
+#     each rank's dx is its input band's adjoint, dw and dbias are summed over ranks.
+
+
+class InputBands:
+    """Input latitudes each rank owns (in_rows[r]) and output latitudes it receives the completed
+    sums of (out_rows[r]), both split as evenly as possible into contiguous bands."""
+
+    def __init__(self, nlat_in, nlon_in, nlat_out, nlon_out, kernel_shape, theta_cutoff, world: int,
+                 grid_in: str = "equiangular", grid_out: str = "equiangular"):
+        self.world = world
+        self.spec = D.make_spec(nlat_in, nlon_in, nlat_out, nlon_out, kernel_shape, theta_cutoff,
+                                D.GRID_CODES[grid_in], D.GRID_CODES[grid_out])
+        self.geometry = (nlat_in, nlon_in, nlat_out, nlon_out, kernel_shape, theta_cutoff, grid_in, grid_out)
+        self.in_rows = split_rows(nlat_in, world)
+        self.out_rows = split_rows(nlat_out, world)
+        self.nlat_out = nlat_out
+
+
+def _padded(bands_rows):
+    return max(e - b for b, e in bands_rows)
+
+
+def reduce_scatter_rows(out_rows, rank: int, t: torch.Tensor) -> torch.Tensor:
+    """t[..., J, L] partial on every row -> the sum over ranks on rank's rows out_rows[rank]."""
+    world = len(out_rows)
+    jb, je = out_rows[rank]
+    if world == 1:
+        return t[..., jb:je, :].contiguous()
+    if dist.get_backend() == "nccl":
+        # equal chunks of the longest band (padded with zeros), one reduce-scatter
+        m = _padded(out_rows)
+        chunks = t.new_zeros((world,) + t.shape[:-2] + (m, t.shape[-1]))
+        for r, (b, e) in enumerate(out_rows):
+            chunks[r, ..., : e - b, :] = t[..., b:e, :]
+        own = t.new_empty(t.shape[:-2] + (m, t.shape[-1]))
+        dist.reduce_scatter_tensor(own, chunks.reshape((world * chunks.shape[1],) + chunks.shape[2:]))
+        return own[..., : je - jb, :].contiguous()
+    # backends without reduce-scatter (gloo): the sum everywhere, then the rank's rows
+    s = t.contiguous().clone()
+    dist.all_reduce(s)
+    return s[..., jb:je, :].contiguous()
+
+
+def all_gather_rows(out_rows, rank: int, t_own: torch.Tensor) -> torch.Tensor:
+    """The adjoint of reduce_scatter_rows: every rank's rows, gathered onto every output row."""
+    world = len(out_rows)
+    if world == 1:
+        return t_own.contiguous()
+    m = _padded(out_rows)
+    jb, je = out_rows[rank]
+    pad = t_own.new_zeros(t_own.shape[:-2] + (m, t_own.shape[-1]))
+    pad[..., : je - jb, :] = t_own
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad.contiguous())
+    return torch.cat([parts[r][..., : e - b, :] for r, (b, e) in enumerate(out_rows)], dim=-2).contiguous()
+
+
+class _ReduceScatterFn(torch.autograd.Function):
+    """fused=False saves the band's partial y; fused=True saves x on the band and recomputes y."""
+
+    @staticmethod
+    def forward(ctx, x_own, w, bias, layer):
+        out_part, y = conv.disco_forward(layer.psi, x_own, w, None, layer.groups)
+        out = reduce_scatter_rows(layer.bands.out_rows, layer.rank, out_part)
+        if bias is not None:
+            out = out + bias.view(1, -1, 1, 1).to(out.dtype)
+        ctx.layer = layer
+        ctx.has_bias = bias is not None
+        ctx.C_in = x_own.shape[1]
+        ctx.save_for_backward(x_own if layer.fused else y, w)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout_own):
+        saved, w = ctx.saved_tensors
+        layer = ctx.layer
+        dout_own = dout_own.contiguous()
+        dout = all_gather_rows(layer.bands.out_rows, layer.rank, dout_own)
+        dx = conv.disco_backward_input(layer.psi, dout, w, ctx.C_in, layer.groups)
+        if layer.fused:
+            dw, _ = conv.disco_backward_weight(layer.psi, dout, x=saved, groups=layer.groups, need_bias=False)
+        else:
+            dw, _ = conv.disco_backward_weight(layer.psi, dout, y=saved, groups=layer.groups, need_bias=False)
+        dist.all_reduce(dw)
+        db = None
+        if ctx.has_bias:
+            db = dout_own.float().sum(dim=(0, 2, 3))
+            dist.all_reduce(db)
+            db = db.to(w.dtype)
+        return dx, dw, db, None
+
+
+class PolarReduceScatterConvS2(torch.nn.Module):
+    """DISCO convolution, latitudes split over the ranks of the default process group in the
+    reduce-scatter polar mode: rank r passes x on its input latitudes (bands.in_rows[r]) and gets
+    out on its output latitudes (bands.out_rows[r]).  Weights and bias are replicated; their
+    gradients are summed over ranks."""
+
+    def __init__(self, in_channels, out_channels, in_shape, out_shape, kernel_shape, theta_cutoff, groups=1,
+                 grid_in="equiangular", grid_out="equiangular", bias=True, fused=False, device=None,
+                 dtype=torch.float32):
+        super().__init__()
+        if in_channels % groups or out_channels % groups:
+            raise ValueError("groups must divide in_channels and out_channels")
+        self.rank, world = dist.get_rank(), dist.get_world_size()
+        self.groups, self.fused = groups, fused
+        self.bands = InputBands(in_shape[0], in_shape[1], out_shape[0], out_shape[1], kernel_shape, theta_cutoff,
+                                world, grid_in, grid_out)
+        self.psi = conv.Psi(in_shape[0], in_shape[1], out_shape[0], out_shape[1], kernel_shape, theta_cutoff, device,
+                            grid_in, grid_out, inputs=self.bands.in_rows[self.rank])
+        K = self.psi.K
+        scale = 1.0 / math.sqrt((in_channels // groups) * K)
+        self.weight = torch.nn.Parameter(
+            torch.randn(out_channels, in_channels // groups, K, device=self.psi.device, dtype=dtype) * scale)
+        self.bias = torch.nn.Parameter(torch.zeros(out_channels, device=self.psi.device, dtype=dtype)) if bias \
+            else None
+
+    def forward(self, x_own):
+        return _ReduceScatterFn.apply(x_own.contiguous(), self.weight, self.bias, self)

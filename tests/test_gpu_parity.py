@@ -370,6 +370,49 @@ def test_polar_bands_reassemble_the_full_layer(name):
     check(db, db_ref, tol(wl), "dbias from bands")
 
 
+@pytest.mark.parametrize("name", ["tz_fused_k3", "ragged_down_bf16", "aniso_k9_f32", "ring_k3", "mid"])
+def test_input_bands_reassemble_the_full_layer(name):
+    """Three bands of input latitudes (disco_psi_build_inputs), each through the kernels: the
+    partial y and out summed over the bands (+ the bias once), dx stitched by row, dw summed,
+    against the oracle's full layer; every output row that a band does not reach comes out
+    exactly zero.  This is the per-rank computation of the reduce-scatter mode without the
+    collectives."""
+    from spherical_disco_convolution_b200 import polar
+
+    wl, inp = workload(name), inputs(name)
+    w, b = dev(inp["w"], wl), dev(inp["bias"], wl)
+    dout = dev(inp["dout"], wl)
+    y_sum = np.zeros((wl.B, wl.C_in, wl.K, wl.nlat_out, wl.nlon_out))
+    out = np.zeros(oracle_out(name).shape)
+    dx = np.zeros(inp["x"].shape)
+    dw = 0.0
+    entries = D.disco_psi_export(gpu_psi(name).handle)
+    for ib, ie in polar.split_rows(wl.nlat_in, 3):
+        psi = conv.Psi(wl.nlat_in, wl.nlon_in, wl.nlat_out, wl.nlon_out, wl.kernel_shape, wl.theta_cutoff, "cuda:0",
+                       inputs=(ib, ie))
+        xb = dev(inp["x"][:, :, ib:ie], wl)
+        o, y = conv.disco_forward(psi, xb, w, None, wl.groups)
+        with pytest.raises(D.DiscoError):
+            conv.disco_forward(psi, xb, w, b, wl.groups, fused=True)
+        dxb = conv.disco_backward_input(psi, dout, w, wl.C_in, wl.groups)
+        dwb, _ = conv.disco_backward_weight(psi, dout, y=y, groups=wl.groups, need_bias=False)
+        torch.cuda.synchronize()
+        yh = host(y)
+        reached = np.zeros(wl.nlat_out, dtype=bool)
+        reached[entries[1][(entries[2] >= ib) & (entries[2] < ie)]] = True
+        assert not np.any(yh[:, :, :, ~reached]), "an output row the band does not reach is not zero"
+        y_sum += yh
+        out += host(o)
+        dx[:, :, ib:ie] = host(dxb)
+        dw = dw + host(dwb)
+    out += inp["bias"][None, :, None, None] if inp["bias"] is not None else 0.0
+    check(out, oracle_out(name), tol(wl), "out from input bands")
+    check(dx, oracle_dx(name), tol(wl), "dx from input bands")
+    check(dw, oracle_dw(name)[0], tol(wl), "dw from input bands")
+    if wl.B * wl.C_in <= 512:
+        check(y_sum, oracle_psi(name).contract(inp["x"]), tol(wl), "y from input bands")
+
+
 def test_polar_layer_on_one_rank_matches_oracle():
     """PolarDiscoConvS2 through autograd on a one-rank NCCL group (the whole layer is one band;
     no transfers), unfused and fused, against the oracle."""
