@@ -147,9 +147,9 @@ disco_status disco_psi_build_band(const disco_spec_t* spec, int j_begin, int j_e
  * and the full nlat_out: disco_contract / disco_fwd / disco_einsum give the band's partial y and
  * out (sum them over bands; add the bias once), disco_bwd_input takes dout on every output row
  * and gives dx on the band's rows, disco_bwd_weight the band's part of dw (sum over bands).
- * Output rows that no entry of the band reaches are written as zeros by the contraction (and
- * input rows no entry reaches by the adjoint).  disco_fwd_fused returns UNSUPPORTED on such a
- * handle when it has rows without entries.  Errors as disco_psi_build, and INVALID_ARG for an
+ * Output rows that no entry of the band reaches are written as zeros by the contraction, as the
+ * bias (zeros without one) by disco_fwd_fused, and input rows no entry reaches as zeros by the
+ * adjoint.  Errors as disco_psi_build, and INVALID_ARG for an
  * empty or out-of-range row range.  The caller owns the handle (disco_psi_destroy). */
 disco_status disco_psi_build_inputs(const disco_spec_t* spec, int i_begin, int i_end, int device, disco_psi** out);
 
@@ -227,6 +227,39 @@ disco_status disco_contract_adjoint(const disco_psi* psi, int B, int C, disco_dt
 disco_status disco_bwd_weight(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
                               const void* dout, const void* y, const void* x, void* dw, void* dbias,
                               void* workspace, size_t ws_bytes, void* stream);
+
+/* The weight einsum, its transpose and the weight gradient on a set of points, without a Psi
+ * handle.  They compute the channel-mixing sums of the forward equation on the page
+ * "torch_harmonics.DiscreteContinuousConvS2", section "Forward", and of its adjoint, at each of
+ * npts points of every (b, channel) plane, the points contiguous in the plane:
+ *
+ *   disco_mix:          out[b,o,n] = bias[o] + sum_{c in group(o), k} w[o,c',k] * y[b,c,k,n]
+ *   disco_mix_adjoint:  dy[b,c,k,n] = sum_{o in group(c)} w[o,c',k] * dout[b,o,n]
+ *   disco_mix_weight:   dw[o,c',k] = sum_{b,n} dout[b,o,n] * y[b,c,k,n],  dbias[o] = sum_{b,n} dout[b,o,n]
+ *
+ * y and dy are (B, C_in, K, npts), out and dout (B, C_out, npts), w and dw (C_out, C_in/groups,
+ * K), bias and dbias (C_out), all caller-owned device memory on the current device, in `dtype`.
+ * bias and dbias may be NULL.  The page's distributed layer needs them on the longitudes that
+ * one azimuth rank owns (page "torch_harmonics.distributed.DistributedDiscreteContinuousConvS2",
+ * class description: the einsum runs after the transpose back to longitude shards), a set of
+ * points no Psi handle describes.
+ *
+ * disco_mix_adjoint and disco_mix_weight take scratch through `workspace`, sized by
+ * disco_mix_workspace_size with op DISCO_OP_EINSUM_ADJOINT or DISCO_OP_BWD_WEIGHT (no other op).
+ * All three are asynchronous on `stream` and allocate nothing.  Errors: DISCO_ERR_INVALID_ARG for
+ * a non-positive size, groups not dividing both channel counts, npts above 2^31 - 1, a NULL
+ * required pointer, an unknown dtype or a missing or short workspace; DISCO_ERR_CUDA for a
+ * failed launch.  The weight gradient's reduction order is fixed (bitwise reproducible). */
+disco_status disco_mix_workspace_size(int op, int B, int C_in, int C_out, int groups, int K, long long npts,
+                                      disco_dtype dtype, size_t* bytes);
+disco_status disco_mix(int B, int C_in, int C_out, int groups, int K, long long npts, disco_dtype dtype,
+                       const void* y, const void* w, const void* bias, void* out, void* stream);
+disco_status disco_mix_adjoint(int B, int C_in, int C_out, int groups, int K, long long npts, disco_dtype dtype,
+                               const void* dout, const void* w, void* dy, void* workspace, size_t ws_bytes,
+                               void* stream);
+disco_status disco_mix_weight(int B, int C_in, int C_out, int groups, int K, long long npts, disco_dtype dtype,
+                              const void* dout, const void* y, void* dw, void* dbias, void* workspace, size_t ws_bytes,
+                              void* stream);
 
 /* Weight gradient that allocates nothing (the pages have no counterpart to this entry point).
  *

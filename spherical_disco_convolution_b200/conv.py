@@ -151,6 +151,60 @@ def disco_backward_weight(psi: Psi, dout: torch.Tensor, y=None, x=None, groups: 
     return dw, db
 
 
+def disco_contract_adjoint(psi: Psi, dy: torch.Tensor) -> torch.Tensor:
+    """dx = the adjoint of the contraction applied to dy (B, C, K, nlat_out, nlon_out)."""
+    _need_cuda(dy)
+    B, C = dy.shape[:2]
+    dx = torch.empty((B, C) + psi.in_shape, dtype=dy.dtype, device=dy.device)
+    D.disco_contract_adjoint(psi.handle, B, C, _dtype_code(dy), _ptr(dy), _ptr(dx), _stream(dy.device))
+    return dx
+
+
+def mix(y: torch.Tensor, w: torch.Tensor, bias=None, groups: int = 1) -> torch.Tensor:
+    """The weight einsum on any set of points: y (B, C_in, K, *pts) -> out (B, C_out, *pts)."""
+    _need_cuda(y, w, bias)
+    y = y.contiguous()
+    B, C_in, K = y.shape[:3]
+    pts = y.shape[3:]
+    C_out = w.shape[0]
+    out = torch.empty((B, C_out) + pts, dtype=y.dtype, device=y.device)
+    D.disco_mix(B, C_in, C_out, groups, K, math.prod(pts), _dtype_code(y), _ptr(y), _ptr(w), _ptr(bias), _ptr(out),
+                _stream(y.device))
+    return out
+
+
+def mix_adjoint(dout: torch.Tensor, w: torch.Tensor, C_in: int, groups: int = 1) -> torch.Tensor:
+    """The transposed weight einsum: dout (B, C_out, *pts) -> dy (B, C_in, K, *pts)."""
+    _need_cuda(dout, w)
+    dout = dout.contiguous()
+    B, C_out = dout.shape[:2]
+    pts = dout.shape[2:]
+    K = w.shape[2]
+    dt, n = _dtype_code(dout), math.prod(pts)
+    dy = torch.empty((B, C_in, K) + pts, dtype=dout.dtype, device=dout.device)
+    nb = D.disco_mix_workspace_size(D.DISCO_OP_EINSUM_ADJOINT, B, C_in, C_out, groups, K, n, dt)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dout.device)
+    D.disco_mix_adjoint(B, C_in, C_out, groups, K, n, dt, _ptr(dout), _ptr(w), _ptr(dy), _ptr(ws), nb,
+                        _stream(dout.device))
+    return dy
+
+
+def mix_weight(dout: torch.Tensor, y: torch.Tensor, groups: int = 1, need_bias: bool = True):
+    """(dw, dbias) of the weight einsum on any set of points: dout (B, C_out, *pts), y (B, C_in, K, *pts)."""
+    _need_cuda(dout, y)
+    dout, y = dout.contiguous(), y.contiguous()
+    B, C_out = dout.shape[:2]
+    C_in, K = y.shape[1:3]
+    dt, n = _dtype_code(dout), math.prod(dout.shape[2:])
+    dw = torch.empty((C_out, C_in // groups, K), dtype=dout.dtype, device=dout.device)
+    db = torch.empty((C_out,), dtype=dout.dtype, device=dout.device) if need_bias else None
+    nb = D.disco_mix_workspace_size(D.DISCO_OP_BWD_WEIGHT, B, C_in, C_out, groups, K, n, dt)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dout.device)
+    D.disco_mix_weight(B, C_in, C_out, groups, K, n, dt, _ptr(dout), _ptr(y), _ptr(dw), _ptr(db), _ptr(ws), nb,
+                       _stream(dout.device))
+    return dw, db
+
+
 class _DiscoFn(torch.autograd.Function):
     @staticmethod
     def forward(ctx, x, w, bias, psi, groups):

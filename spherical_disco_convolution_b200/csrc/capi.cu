@@ -316,22 +316,21 @@ cudaError_t launch_mix(bool bf16, const disco::MixArgs& m, cudaStream_t st) {
   return disco::launch_mix_simt(bf16, m, st);
 }
 
-WsLayout layout(const disco_psi* psi, int op, int B, int C_in, int C_out, int groups, disco_dtype dtype) {
+// Scratch of an operation on K kernel indices and n_out output points per plane.
+WsLayout layout_kn(int K, size_t n_out, int op, int B, int C_in, int C_out, int groups, disco_dtype dtype) {
   WsLayout L;
   const size_t es = dtype == DISCO_BF16 ? 2 : 4;
-  const disco::Geometry& g = psi->g;
-  const size_t n_out = (size_t)g.nlat_out * g.nlon_out;
-  const size_t y_elems = (size_t)B * C_in * g.K * n_out;
+  const size_t y_elems = (size_t)B * C_in * K * n_out;
   if (op == DISCO_OP_EINSUM_ADJOINT) {
     L.wt = 0;
-    L.total = align256((size_t)C_out * (C_in / groups) * g.K * es);
+    L.total = align256((size_t)C_out * (C_in / groups) * K * es);
   } else if (op == DISCO_OP_BWD_INPUT) {
     L.wt = 0;
-    L.dy = align256((size_t)C_out * (C_in / groups) * g.K * es);
+    L.dy = align256((size_t)C_out * (C_in / groups) * K * es);
     L.total = L.dy + align256(y_elems * es);
   } else if (op == DISCO_OP_BWD_WEIGHT || op == DISCO_OP_BWD_WEIGHT_RECOMPUTE) {
     const int N = (int)n_out;
-    L.tc = dtype == DISCO_BF16 && disco::dw_tc_supported(C_out / groups, (C_in / groups) * g.K, N);
+    L.tc = dtype == DISCO_BF16 && disco::dw_tc_supported(C_out / groups, (C_in / groups) * K, N);
     if (L.tc) {
       // one CTA per (split, batch, group), about one per SM of a B200 (148): the splits cover the
       // positions in multiples of the 64-element stage
@@ -348,12 +347,16 @@ WsLayout layout(const disco_psi* psi, int op, int B, int C_in, int C_out, int gr
       off = align256(y_elems * es);
     }
     L.part = off;
-    off += align256(nsplit * (size_t)C_out * (C_in / groups) * g.K * sizeof(float));
+    off += align256(nsplit * (size_t)C_out * (C_in / groups) * K * sizeof(float));
     L.bpart = off;
     off += align256(nsplit * (size_t)C_out * sizeof(float));
     L.total = off;
   }
   return L;
+}
+
+WsLayout layout(const disco_psi* psi, int op, int B, int C_in, int C_out, int groups, disco_dtype dtype) {
+  return layout_kn(psi->g.K, (size_t)psi->g.nlat_out * psi->g.nlon_out, op, B, C_in, C_out, groups, dtype);
 }
 
 }  // namespace
@@ -650,16 +653,39 @@ disco_status launch_contract_core(const disco_psi* psi, int BC, disco_dtype dtyp
 }
 
 // dy = w^T dout (the transposed weight einsum): w transposed into `wt`, then the channel mix.
+// dy = W^T dout on N points per plane (the transposed weight einsum)
+disco_status launch_dy_kn(int K, int N, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                          const void* dout, const void* w, void* wt, void* dy, cudaStream_t st) {
+  const bool bf16 = dtype == DISCO_BF16;
+  const int Cg = C_in / groups, Og = C_out / groups;
+  cudaError_t e = disco::launch_transpose_weight(bf16, w, wt, groups, Og, Cg, K, st);
+  if (e != cudaSuccess) return cuda_fail(e, "weight transpose launch");
+  disco::MixArgs m{dout, wt, nullptr, dy, B, groups, Cg * K, Og, N};
+  e = launch_mix(bf16, m, st);
+  if (e != cudaSuccess) return cuda_fail(e, "transposed einsum launch");
+  return DISCO_OK;
+}
+
 disco_status launch_dy(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
                        const void* dout, const void* w, void* wt, void* dy, cudaStream_t st) {
   const disco::Geometry& g = psi->g;
+  return launch_dy_kn(g.K, g.nlat_out * g.nlon_out, B, C_in, C_out, groups, dtype, dout, w, wt, dy, st);
+}
+
+// dw (and dbias when non-NULL) from dout and y on N points per plane, with the split-K partial
+// sums in the scratch that L describes
+disco_status launch_dw_kn(int K, int N, const WsLayout& L, int B, int C_in, int C_out, int groups,
+                          disco_dtype dtype, const void* dout, const void* y, char* ws, void* dw, void* dbias,
+                          cudaStream_t st) {
   const bool bf16 = dtype == DISCO_BF16;
-  const int Cg = C_in / groups, Og = C_out / groups;
-  cudaError_t e = disco::launch_transpose_weight(bf16, w, wt, groups, Og, Cg, g.K, st);
-  if (e != cudaSuccess) return cuda_fail(e, "weight transpose launch");
-  disco::MixArgs m{dout, wt, nullptr, dy, B, groups, Cg * g.K, Og, g.nlat_out * g.nlon_out};
-  e = launch_mix(bf16, m, st);
-  if (e != cudaSuccess) return cuda_fail(e, "transposed einsum launch");
+  const int Og = C_out / groups, Rg = (C_in / groups) * K;
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  float* bpart = dbias ? reinterpret_cast<float*>(ws + L.bpart) : nullptr;
+  disco::DwArgs d{dout, y, part, bpart, B, groups, Og, Rg, N, L.nc, L.nchunk};
+  cudaError_t e = L.tc ? disco::launch_dw_tc(d, st) : disco::launch_dw_partial_simt(bf16, d, st);
+  if (e != cudaSuccess) return cuda_fail(e, "weight-gradient launch");
+  e = disco::launch_dw_reduce(bf16, part, bpart, dw, dbias, B * L.nchunk, groups, Og, Rg, st);
+  if (e != cudaSuccess) return cuda_fail(e, "weight-gradient reduce launch");
   return DISCO_OK;
 }
 
@@ -1151,6 +1177,9 @@ disco_status disco_fwd(const disco_psi* psi, int B, int C_in, int C_out, int gro
   return disco_einsum(psi, B, C_in, C_out, groups, dtype, y, w, bias, out, stream);
 }
 
+static disco_status fwd_fused_core(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                                   const void* x, const void* w, const void* bias, void* out, cudaStream_t st);
+
 disco_status disco_fwd_fused(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
                              const void* x, const void* w, const void* bias, void* out, void* workspace,
                              size_t ws_bytes, void* stream) {
@@ -1161,12 +1190,20 @@ disco_status disco_fwd_fused(const disco_psi* psi, int B, int C_in, int C_out, i
   if (!x || !w || !out) return fail(DISCO_ERR_INVALID_ARG, "x, w and out must be non-NULL");
   const disco::Geometry& g = psi->g;
   if (!disco::gather_supports(g.K, g.stride)) return fail(DISCO_ERR_UNSUPPORTED, "K or stride not compiled");
-  if (!psi->empty_out.empty())
-    return fail(DISCO_ERR_UNSUPPORTED,
-                "the fused forward needs an entry in every output row; this handle (a band of input latitudes) "
-                "has rows without: use disco_fwd or disco_contract + disco_einsum");
-  const bool bf16 = dtype == DISCO_BF16;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = fwd_fused_core(psi, B, C_in, C_out, groups, dtype, x, w, bias, out, st);
+  if (s || psi->empty_out.empty()) return s;
+  // output rows without entries (a band of input latitudes): out = bias there, whatever the
+  // kernel left in them
+  cudaError_t e = disco::launch_fill_rows(dtype == DISCO_BF16, out, psi->d_empty_out, (int)psi->empty_out.size(),
+                                          B * C_out, g.nlat_out, g.nlon_out, bias, C_out, st);
+  return e == cudaSuccess ? DISCO_OK : cuda_fail(e, "fused forward row fill");
+}
+
+static disco_status fwd_fused_core(const disco_psi* psi, int B, int C_in, int C_out, int groups, disco_dtype dtype,
+                                   const void* x, const void* w, const void* bias, void* out, cudaStream_t st) {
+  const disco::Geometry& g = psi->g;
+  const bool bf16 = dtype == DISCO_BF16;
   const int Cg = C_in / groups;
   const char* rf = std::getenv("DISCO_RING2_FUSED");
   const char* r2 = std::getenv("DISCO_RING2");
@@ -1264,6 +1301,9 @@ disco_status disco_bwd_input(const disco_psi* psi, int B, int C_in, int C_out, i
                          P.ns, P.nrb, P.nbs, P.bslot_bytes, P.mirror, B * C_out, g.nlat_out, g.nlat_in, g.nlon_in};
     disco::Ring2Fused F{dout, w, nullptr, dx, C_out, C_in, 1};
     cudaError_t e = disco::launch_fused_ring2(R, F, st);
+    if (e == cudaSuccess && !psi->empty_in.empty())  // input rows no entry reaches: dx = 0 there
+      e = disco::launch_zero_rows(dx, 2, psi->d_empty_in, (int)psi->empty_in.size(), B * C_in, g.nlat_in, g.nlon_in,
+                                  st);
     if (e != cudaSuccess) return cuda_fail(e, "fused input-gradient launch");
     return DISCO_OK;
   }
@@ -1306,25 +1346,76 @@ disco_status disco_bwd_weight(const disco_psi* psi, int B, int C_in, int C_out, 
   const int op = y ? DISCO_OP_BWD_WEIGHT : DISCO_OP_BWD_WEIGHT_RECOMPUTE;
   const WsLayout L = layout(psi, op, B, C_in, C_out, groups, dtype);
   if (!workspace || ws_bytes < L.total) return fail(DISCO_ERR_INVALID_ARG, "workspace missing or too small");
-  const bool bf16 = dtype == DISCO_BF16;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
-  cudaError_t e;
   const void* yv = y;
   if (!y) {
     s = launch_contract(psi, B * C_in, dtype, x, ws + L.ybuf, st, "recompute contraction launch");
     if (s) return s;
     yv = ws + L.ybuf;
   }
-  const int Og = C_out / groups, Rg = (C_in / groups) * g.K;
-  float* part = reinterpret_cast<float*>(ws + L.part);
-  float* bpart = dbias ? reinterpret_cast<float*>(ws + L.bpart) : nullptr;
-  disco::DwArgs d{dout, yv, part, bpart, B, groups, Og, Rg, g.nlat_out * g.nlon_out, L.nc, L.nchunk};
-  e = L.tc ? disco::launch_dw_tc(d, st) : disco::launch_dw_partial_simt(bf16, d, st);
-  if (e != cudaSuccess) return cuda_fail(e, "weight-gradient launch");
-  e = disco::launch_dw_reduce(bf16, part, bpart, dw, dbias, B * L.nchunk, groups, Og, Rg, st);
-  if (e != cudaSuccess) return cuda_fail(e, "weight-gradient reduce launch");
+  return launch_dw_kn(g.K, g.nlat_out * g.nlon_out, L, B, C_in, C_out, groups, dtype, dout, yv, ws, dw, dbias, st);
+}
+
+// ------------------------------------------------------------------ the weight einsum on a set of points
+// The three channel-mixing steps on K kernel indices and npts points per (b, channel) plane, with
+// no Psi handle: the points may be any slice of the output grid that is contiguous in every
+// plane (the longitudes an azimuth rank owns, after the transpose back).
+
+static disco_status check_mix(int B, int C_in, int C_out, int groups, int K, long long npts, disco_dtype dtype) {
+  if (B <= 0 || C_in <= 0 || C_out <= 0 || groups <= 0 || K <= 0 || npts <= 0)
+    return fail(DISCO_ERR_INVALID_ARG, "B, C_in, C_out, groups, K and npts must be positive");
+  if (C_in % groups || C_out % groups) return fail(DISCO_ERR_INVALID_ARG, "groups must divide both C_in and C_out");
+  if (npts > (long long)INT32_MAX) return fail(DISCO_ERR_INVALID_ARG, "npts exceeds 2^31 - 1");
+  if ((long long)(C_in / groups) * K > (long long)INT32_MAX) return fail(DISCO_ERR_INVALID_ARG, "C_in/groups * K too large");
+  if (dtype != DISCO_F32 && dtype != DISCO_BF16) return fail(DISCO_ERR_INVALID_ARG, "unknown dtype");
   return DISCO_OK;
+}
+
+disco_status disco_mix_workspace_size(int op, int B, int C_in, int C_out, int groups, int K, long long npts,
+                                      disco_dtype dtype, size_t* bytes) {
+  if (!bytes) return fail(DISCO_ERR_INVALID_ARG, "NULL argument");
+  disco_status s = check_mix(B, C_in, C_out, groups, K, npts, dtype);
+  if (s) return s;
+  if (op != DISCO_OP_EINSUM_ADJOINT && op != DISCO_OP_BWD_WEIGHT)
+    return fail(DISCO_ERR_INVALID_ARG, "op is DISCO_OP_EINSUM_ADJOINT or DISCO_OP_BWD_WEIGHT");
+  *bytes = layout_kn(K, (size_t)npts, op, B, C_in, C_out, groups, dtype).total;
+  return DISCO_OK;
+}
+
+disco_status disco_mix(int B, int C_in, int C_out, int groups, int K, long long npts, disco_dtype dtype,
+                       const void* y, const void* w, const void* bias, void* out, void* stream) {
+  disco_status s = check_mix(B, C_in, C_out, groups, K, npts, dtype);
+  if (s) return s;
+  if (!y || !w || !out) return fail(DISCO_ERR_INVALID_ARG, "y, w and out must be non-NULL");
+  disco::MixArgs m{y, w, bias, out, B, groups, C_out / groups, (C_in / groups) * K, (int)npts};
+  cudaError_t e = launch_mix(dtype == DISCO_BF16, m, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "einsum launch");
+  return DISCO_OK;
+}
+
+disco_status disco_mix_adjoint(int B, int C_in, int C_out, int groups, int K, long long npts, disco_dtype dtype,
+                               const void* dout, const void* w, void* dy, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  disco_status s = check_mix(B, C_in, C_out, groups, K, npts, dtype);
+  if (s) return s;
+  if (!dout || !w || !dy) return fail(DISCO_ERR_INVALID_ARG, "dout, w and dy must be non-NULL");
+  const WsLayout L = layout_kn(K, (size_t)npts, DISCO_OP_EINSUM_ADJOINT, B, C_in, C_out, groups, dtype);
+  if (!workspace || ws_bytes < L.total) return fail(DISCO_ERR_INVALID_ARG, "workspace missing or too small");
+  return launch_dy_kn(K, (int)npts, B, C_in, C_out, groups, dtype, dout, w, static_cast<char*>(workspace) + L.wt,
+                      dy, static_cast<cudaStream_t>(stream));
+}
+
+disco_status disco_mix_weight(int B, int C_in, int C_out, int groups, int K, long long npts, disco_dtype dtype,
+                              const void* dout, const void* y, void* dw, void* dbias, void* workspace, size_t ws_bytes,
+                              void* stream) {
+  disco_status s = check_mix(B, C_in, C_out, groups, K, npts, dtype);
+  if (s) return s;
+  if (!dout || !y || !dw) return fail(DISCO_ERR_INVALID_ARG, "dout, y and dw must be non-NULL");
+  const WsLayout L = layout_kn(K, (size_t)npts, DISCO_OP_BWD_WEIGHT, B, C_in, C_out, groups, dtype);
+  if (!workspace || ws_bytes < L.total) return fail(DISCO_ERR_INVALID_ARG, "workspace missing or too small");
+  return launch_dw_kn(K, (int)npts, L, B, C_in, C_out, groups, dtype, dout, y, static_cast<char*>(workspace), dw,
+                      dbias, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -243,6 +243,35 @@ cudaError_t launch_zero_rows(void* t, int elem_bytes, const int* rows, int n_row
   return cudaGetLastError();
 }
 
+namespace {
+// t[p][rows[r]][0..nlon) = bias[p % C] for every plane p (a plane is one (b, output channel))
+template <typename T>
+__global__ void fill_rows_kernel(T* t, const int* __restrict__ rows, int planes, int nrows, int nlon,
+                                 const T* __restrict__ bias, int C) {
+  const int r = rows[blockIdx.x];
+  for (int p = blockIdx.y; p < planes; p += gridDim.y) {
+    const T v = bias[p % C];
+    T* base = t + ((size_t)p * nrows + r) * nlon;
+    for (int q = threadIdx.x; q < nlon; q += blockDim.x) base[q] = v;
+  }
+}
+}  // namespace
+
+cudaError_t launch_fill_rows(bool bf16, void* t, const int* rows, int n_rows, int planes, int nrows, int nlon,
+                             const void* bias, int C, cudaStream_t st) {
+  if (!bias) return launch_zero_rows(t, bf16 ? 2 : 4, rows, n_rows, planes, nrows, nlon, st);
+  if (n_rows <= 0 || planes <= 0) return cudaSuccess;
+  dim3 grid(n_rows, std::min(planes, 64));
+  if (bf16)
+    fill_rows_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<__nv_bfloat16*>(t), rows, planes, nrows, nlon,
+                                                          static_cast<const __nv_bfloat16*>(bias), C);
+  else
+    fill_rows_kernel<float><<<grid, 128, 0, st>>>(static_cast<float*>(t), rows, planes, nrows, nlon,
+                                                  static_cast<const float*>(bias), C);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dw_reduce(bool bf16, const float* part, const float* bpart, void* dw, void* dbias, int nsplit,
                              int G, int Og, int Rg, cudaStream_t st) {
   const int per = G * Og * Rg;

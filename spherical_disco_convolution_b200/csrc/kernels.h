@@ -159,6 +159,9 @@ cudaError_t launch_dw_tc(const DwArgs& a, cudaStream_t st);
 // t[p][rows[i]][0..nlon) = 0 for p < planes, t being [planes][nrows][nlon] of elem_bytes elements.
 cudaError_t launch_zero_rows(void* t, int elem_bytes, const int* rows, int n_rows, int planes, int nrows, int nlon,
                              cudaStream_t st);
+// Rows `rows` of every plane set to bias[plane % C] (zero when bias is NULL).
+cudaError_t launch_fill_rows(bool bf16, void* t, const int* rows, int n_rows, int planes, int nrows, int nlon,
+                             const void* bias, int C, cudaStream_t st);
 // dw[g*Og + o, r] = sum_split part[split, g, o, r]; dbias[o] = sum_split bpart[split, o]; fixed order.
 cudaError_t launch_dw_reduce(bool bf16, const float* part, const float* bpart, void* dw, void* dbias, int nsplit,
                              int G, int Og, int Rg, cudaStream_t st);

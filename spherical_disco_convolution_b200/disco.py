@@ -104,6 +104,10 @@ def _load():
         "disco_contract_adjoint": [P, I, I, I, P, P, P],
         "disco_bwd_weight": [P, I, I, I, I, I, P, P, P, P, P, P, Z, P],
         "disco_bwd_weight_noalloc": [P, I, I, I, I, I, P, P, P, P, P],
+        "disco_mix_workspace_size": [I, I, I, I, I, I, LL, I, ctypes.POINTER(Z)],
+        "disco_mix": [I, I, I, I, I, LL, I, P, P, P, P, P],
+        "disco_mix_adjoint": [I, I, I, I, I, LL, I, P, P, P, P, Z, P],
+        "disco_mix_weight": [I, I, I, I, I, LL, I, P, P, P, P, P, Z, P],
         "disco_plan_info": [P, I, IP],
         "disco_sync_status": [P],
         "disco_wait_selftest": [ctypes.c_uint, P],
@@ -333,3 +337,23 @@ def disco_bwd_weight(psi, B, C_in, C_out, groups, dtype, dout, y, x, dw, dbias, 
 
 def disco_bwd_weight_noalloc(psi, B, C_in, C_out, groups, dtype, dout, y, dw, dbias, stream) -> None:
     _check(_lib.disco_bwd_weight_noalloc(psi, B, C_in, C_out, groups, dtype, dout, y, dw, dbias, stream))
+
+
+def disco_mix_workspace_size(op, B, C_in, C_out, groups, K, npts, dtype) -> int:
+    n = ctypes.c_size_t()
+    _check(_lib.disco_mix_workspace_size(op, B, C_in, C_out, groups, K, npts, dtype, ctypes.byref(n)))
+    return n.value
+
+
+def disco_mix(B, C_in, C_out, groups, K, npts, dtype, y, w, bias, out, stream) -> None:
+    _check(_lib.disco_mix(B, C_in, C_out, groups, K, npts, dtype, y, w, bias, out, stream))
+
+
+def disco_mix_adjoint(B, C_in, C_out, groups, K, npts, dtype, dout, w, dy, workspace, ws_bytes, stream) -> None:
+    _check(_lib.disco_mix_adjoint(B, C_in, C_out, groups, K, npts, dtype, dout, w, dy, workspace, ws_bytes, stream))
+
+
+def disco_mix_weight(B, C_in, C_out, groups, K, npts, dtype, dout, y, dw, dbias, workspace, ws_bytes,
+                     stream) -> None:
+    _check(_lib.disco_mix_weight(B, C_in, C_out, groups, K, npts, dtype, dout, y, dw, dbias, workspace, ws_bytes,
+                                 stream))

@@ -85,8 +85,14 @@ def _exchange(ops):
             req.wait()
 
 
-def halo_gather(bands: PolarBands, rank: int, x_own: torch.Tensor) -> torch.Tensor:
-    """x on the rows rank `rank` reaches, [..., i_end - i_begin, nlon], from x on its own rows."""
+def _peer(group, r: int) -> int:
+    """Global rank of rank r of `group` (None: the default group)."""
+    return r if group is None else dist.get_global_rank(group, r)
+
+
+def halo_gather(bands: PolarBands, rank: int, x_own: torch.Tensor, group=None) -> torch.Tensor:
+    """x on the rows rank `rank` reaches, [..., i_end - i_begin, nlon], from x on its own rows;
+    ranks are those of `group` (None: the default group)."""
     ob, oe = bands.in_rows[rank]
     ib, ie = bands.reach[rank]
     if x_own.shape[-2] != oe - ob:
@@ -99,19 +105,19 @@ def halo_gather(bands: PolarBands, rank: int, x_own: torch.Tensor) -> torch.Tens
     for dst, lo, hi in bands.send[rank]:
         buf = x_own[..., lo - ob:hi - ob, :].contiguous()
         keep.append(buf)
-        ops.append(dist.P2POp(dist.isend, buf, dst))
+        ops.append(dist.P2POp(dist.isend, buf, _peer(group, dst), group))
     recvs = []
     for src, lo, hi in bands.recv[rank]:
         buf = x_own.new_empty(x_own.shape[:-2] + (hi - lo, x_own.shape[-1]))
         recvs.append((buf, lo))
-        ops.append(dist.P2POp(dist.irecv, buf, src))
+        ops.append(dist.P2POp(dist.irecv, buf, _peer(group, src), group))
     _exchange(ops)
     for buf, lo in recvs:
         x_band[..., lo - ib:lo - ib + buf.shape[-2], :] = buf
     return x_band
 
 
-def halo_reduce(bands: PolarBands, rank: int, g_band: torch.Tensor) -> torch.Tensor:
+def halo_reduce(bands: PolarBands, rank: int, g_band: torch.Tensor, group=None) -> torch.Tensor:
     """The adjoint of halo_gather: a gradient on the reached rows, summed onto each row's owner."""
     ob, oe = bands.in_rows[rank]
     ib, ie = bands.reach[rank]
@@ -123,11 +129,11 @@ def halo_reduce(bands: PolarBands, rank: int, g_band: torch.Tensor) -> torch.Ten
     for src, lo, hi in bands.recv[rank]:  # rows borrowed from src go back to src
         buf = g_band[..., lo - ib:hi - ib, :].contiguous()
         keep.append(buf)
-        ops.append(dist.P2POp(dist.isend, buf, src))
+        ops.append(dist.P2POp(dist.isend, buf, _peer(group, src), group))
     for dst, lo, hi in bands.send[rank]:  # rows lent to dst come back from dst
         buf = g_band.new_empty(g_band.shape[:-2] + (hi - lo, g_band.shape[-1]))
         recvs.append((buf, lo))
-        ops.append(dist.P2POp(dist.irecv, buf, dst))
+        ops.append(dist.P2POp(dist.irecv, buf, _peer(group, dst), group))
     _exchange(ops)
     for buf, lo in recvs:
         g_own[..., lo - ob:lo - ob + buf.shape[-2], :] += buf
@@ -214,9 +220,10 @@ class PolarDiscoConvS2(torch.nn.Module):
 #
 #   * the reduce-scatter runs on out (C_out channels), after each rank's weight einsum of its
 #     partial y, not on the K-expanded y: the einsum is linear, so the sums are the same with K
-#     times less collective volume; the bias is added once, on the owner of each output row;
+#     times less collective volume; rank 0's partial sum carries the bias, so it is added once;
 #   * backward is the adjoint: dout on the rank's output rows is all-gathered to every output row,
-#     each rank's dx is its input band's adjoint, dw and dbias are summed over ranks.
+#     each rank's dx is its input band's adjoint, dw is summed over ranks and dbias is the sum of
+#     the gathered dout, the same on every rank.
 
 
 class InputBands:
@@ -238,50 +245,67 @@ def _padded(bands_rows):
     return max(e - b for b, e in bands_rows)
 
 
-def reduce_scatter_rows(out_rows, rank: int, t: torch.Tensor) -> torch.Tensor:
-    """t[..., J, L] partial on every row -> the sum over ranks on rank's rows out_rows[rank]."""
-    world = len(out_rows)
-    jb, je = out_rows[rank]
+def reduce_scatter_dim(spans, rank: int, t: torch.Tensor, dim: int, group=None) -> torch.Tensor:
+    """t partial over the ranks of `group` (None: the default group) -> the sum over them of
+    t's slice spans[rank] = (begin, end) along dimension `dim`."""
+    world = len(spans)
+    dim = dim % t.dim()
+    jb, je = spans[rank]
     if world == 1:
-        return t[..., jb:je, :].contiguous()
-    if dist.get_backend() == "nccl":
-        # equal chunks of the longest band (padded with zeros), one reduce-scatter
-        m = _padded(out_rows)
-        chunks = t.new_zeros((world,) + t.shape[:-2] + (m, t.shape[-1]))
-        for r, (b, e) in enumerate(out_rows):
-            chunks[r, ..., : e - b, :] = t[..., b:e, :]
-        own = t.new_empty(t.shape[:-2] + (m, t.shape[-1]))
-        dist.reduce_scatter_tensor(own, chunks.reshape((world * chunks.shape[1],) + chunks.shape[2:]))
-        return own[..., : je - jb, :].contiguous()
-    # backends without reduce-scatter (gloo): the sum everywhere, then the rank's rows
+        return t.narrow(dim, jb, je - jb).contiguous()
+    if dist.get_backend(group) == "nccl":
+        # equal chunks of the longest span (padded with zeros), one reduce-scatter
+        m = _padded(spans)
+        tm = t.movedim(dim, -1)
+        chunks = t.new_zeros((world,) + tm.shape[:-1] + (m,))
+        for r, (b, e) in enumerate(spans):
+            chunks[r, ..., : e - b] = tm[..., b:e]
+        own = t.new_empty(tm.shape[:-1] + (m,))
+        dist.reduce_scatter_tensor(own, chunks.reshape((world * chunks.shape[1],) + chunks.shape[2:]), group=group)
+        return own[..., : je - jb].movedim(-1, dim).contiguous()
+    # backends without reduce-scatter (gloo): the sum everywhere, then the rank's slice
     s = t.contiguous().clone()
-    dist.all_reduce(s)
-    return s[..., jb:je, :].contiguous()
+    dist.all_reduce(s, group=group)
+    return s.narrow(dim, jb, je - jb).contiguous()
 
 
-def all_gather_rows(out_rows, rank: int, t_own: torch.Tensor) -> torch.Tensor:
-    """The adjoint of reduce_scatter_rows: every rank's rows, gathered onto every output row."""
-    world = len(out_rows)
+def all_gather_dim(spans, rank: int, t_own: torch.Tensor, dim: int, group=None) -> torch.Tensor:
+    """The adjoint of reduce_scatter_dim: every rank's slice, concatenated along `dim`."""
+    world = len(spans)
     if world == 1:
         return t_own.contiguous()
-    m = _padded(out_rows)
-    jb, je = out_rows[rank]
-    pad = t_own.new_zeros(t_own.shape[:-2] + (m, t_own.shape[-1]))
-    pad[..., : je - jb, :] = t_own
+    dim = dim % t_own.dim()
+    m = _padded(spans)
+    jb, je = spans[rank]
+    tm = t_own.movedim(dim, -1)
+    pad = t_own.new_zeros(tm.shape[:-1] + (m,))
+    pad[..., : je - jb] = tm
     parts = [torch.empty_like(pad) for _ in range(world)]
-    dist.all_gather(parts, pad.contiguous())
-    return torch.cat([parts[r][..., : e - b, :] for r, (b, e) in enumerate(out_rows)], dim=-2).contiguous()
+    dist.all_gather(parts, pad.contiguous(), group=group)
+    return torch.cat([parts[r][..., : e - b] for r, (b, e) in enumerate(spans)], dim=-1).movedim(-1, dim).contiguous()
+
+
+def reduce_scatter_rows(out_rows, rank: int, t: torch.Tensor, group=None) -> torch.Tensor:
+    """t[..., J, L] partial on every row -> the sum over the ranks of `group` (None: the default
+    group) on rank's rows out_rows[rank]."""
+    return reduce_scatter_dim(out_rows, rank, t, -2, group)
+
+
+def all_gather_rows(out_rows, rank: int, t_own: torch.Tensor, group=None) -> torch.Tensor:
+    """The adjoint of reduce_scatter_rows: every rank's rows, gathered onto every output row."""
+    return all_gather_dim(out_rows, rank, t_own, -2, group)
 
 
 class _ReduceScatterFn(torch.autograd.Function):
-    """fused=False saves the band's partial y; fused=True saves x on the band and recomputes y."""
+    """fused=False saves the band's partial y; fused=True runs the fused forward, saves x on the band
+    and recomputes y in backward."""
 
     @staticmethod
     def forward(ctx, x_own, w, bias, layer):
-        out_part, y = conv.disco_forward(layer.psi, x_own, w, None, layer.groups)
+        # rank 0's partial sum carries the bias, so the reduce-scatter adds it exactly once
+        out_part, y = conv.disco_forward(layer.psi, x_own, w, bias if layer.rank == 0 else None, layer.groups,
+                                         fused=layer.fused)
         out = reduce_scatter_rows(layer.bands.out_rows, layer.rank, out_part)
-        if bias is not None:
-            out = out + bias.view(1, -1, 1, 1).to(out.dtype)
         ctx.layer = layer
         ctx.has_bias = bias is not None
         ctx.C_in = x_own.shape[1]
@@ -295,16 +319,15 @@ class _ReduceScatterFn(torch.autograd.Function):
         dout_own = dout_own.contiguous()
         dout = all_gather_rows(layer.bands.out_rows, layer.rank, dout_own)
         dx = conv.disco_backward_input(layer.psi, dout, w, ctx.C_in, layer.groups)
+        # dw is the band's part (summed over ranks); dbias comes from dout on every output row,
+        # the same complete sum on every rank
         if layer.fused:
-            dw, _ = conv.disco_backward_weight(layer.psi, dout, x=saved, groups=layer.groups, need_bias=False)
+            dw, db = conv.disco_backward_weight(layer.psi, dout, x=saved, groups=layer.groups,
+                                                need_bias=ctx.has_bias)
         else:
-            dw, _ = conv.disco_backward_weight(layer.psi, dout, y=saved, groups=layer.groups, need_bias=False)
+            dw, db = conv.disco_backward_weight(layer.psi, dout, y=saved, groups=layer.groups,
+                                                need_bias=ctx.has_bias)
         dist.all_reduce(dw)
-        db = None
-        if ctx.has_bias:
-            db = dout_own.float().sum(dim=(0, 2, 3))
-            dist.all_reduce(db)
-            db = db.to(w.dtype)
         return dx, dw, db, None
 
 

@@ -373,9 +373,9 @@ def test_polar_bands_reassemble_the_full_layer(name):
 @pytest.mark.parametrize("name", ["tz_fused_k3", "ragged_down_bf16", "aniso_k9_f32", "ring_k3", "mid"])
 def test_input_bands_reassemble_the_full_layer(name):
     """Three bands of input latitudes (disco_psi_build_inputs), each through the kernels: the
-    partial y and out summed over the bands (+ the bias once), dx stitched by row, dw summed,
-    against the oracle's full layer; every output row that a band does not reach comes out
-    exactly zero.  This is the per-rank computation of the reduce-scatter mode without the
+    partial y and out (unfused and fused) summed over the bands (+ the bias once), dx stitched by
+    row, dw summed, against the oracle's full layer; every output row that a band does not reach
+    comes out exactly zero (exactly the bias from the fused forward given one).  This is the per-rank computation of the reduce-scatter mode without the
     collectives."""
     from spherical_disco_convolution_b200 import polar
 
@@ -384,6 +384,7 @@ def test_input_bands_reassemble_the_full_layer(name):
     dout = dev(inp["dout"], wl)
     y_sum = np.zeros((wl.B, wl.C_in, wl.K, wl.nlat_out, wl.nlon_out))
     out = np.zeros(oracle_out(name).shape)
+    out_f = np.zeros_like(out)
     dx = np.zeros(inp["x"].shape)
     dw = 0.0
     entries = D.disco_psi_export(gpu_psi(name).handle)
@@ -392,8 +393,8 @@ def test_input_bands_reassemble_the_full_layer(name):
                        inputs=(ib, ie))
         xb = dev(inp["x"][:, :, ib:ie], wl)
         o, y = conv.disco_forward(psi, xb, w, None, wl.groups)
-        with pytest.raises(D.DiscoError):
-            conv.disco_forward(psi, xb, w, b, wl.groups, fused=True)
+        of, _ = conv.disco_forward(psi, xb, w, None, wl.groups, fused=True)
+        ofb = conv.disco_forward(psi, xb, w, b, wl.groups, fused=True)[0] if b is not None else None
         dxb = conv.disco_backward_input(psi, dout, w, wl.C_in, wl.groups)
         dwb, _ = conv.disco_backward_weight(psi, dout, y=y, groups=wl.groups, need_bias=False)
         torch.cuda.synchronize()
@@ -401,27 +402,90 @@ def test_input_bands_reassemble_the_full_layer(name):
         reached = np.zeros(wl.nlat_out, dtype=bool)
         reached[entries[1][(entries[2] >= ib) & (entries[2] < ie)]] = True
         assert not np.any(yh[:, :, :, ~reached]), "an output row the band does not reach is not zero"
+        assert not np.any(host(of)[:, :, ~reached]), "fused: an output row the band does not reach is not zero"
+        if ofb is not None:  # the bias exactly, on the rows the band does not reach
+            hb = host(ofb)[:, :, ~reached]
+            assert np.array_equal(hb, np.broadcast_to(host(b)[None, :, None, None], hb.shape)), \
+                "fused: unreached rows are not the bias"
         y_sum += yh
         out += host(o)
+        out_f += host(of)
         dx[:, :, ib:ie] = host(dxb)
         dw = dw + host(dwb)
-    out += inp["bias"][None, :, None, None] if inp["bias"] is not None else 0.0
+    if inp["bias"] is not None:
+        out += host(b)[None, :, None, None]
+        out_f += host(b)[None, :, None, None]
     check(out, oracle_out(name), tol(wl), "out from input bands")
+    check(out_f, oracle_out(name), tol(wl), "fused out from input bands")
     check(dx, oracle_dx(name), tol(wl), "dx from input bands")
     check(dw, oracle_dw(name)[0], tol(wl), "dw from input bands")
     if wl.B * wl.C_in <= 512:
         check(y_sum, oracle_psi(name).contract(inp["x"]), tol(wl), "y from input bands")
 
 
+@pytest.mark.parametrize("name,A", [("tz_fused_k3", 2), ("ragged_down_bf16", 3), ("aniso_k9_f32", 2), ("mid", 3)])
+def test_azimuth_shards_reassemble_the_full_layer(name, A):
+    """The per-rank kernels of the azimuth all-to-all on A emulated ranks, without the transfers.
+    Standard mode: the contraction on each channel shard, y cut into longitude shards, the weight
+    einsum, its transpose and the weight gradient on each shard's points (disco_mix*), the
+    adjoint contraction on each channel shard.  Reordered mode: the fused forward of each channel
+    shard with its dense block weight (partial out over full rows, summed), the one-call input
+    gradient and the recomputing weight gradient per shard.  Against the oracle's full layer."""
+    from spherical_disco_convolution_b200 import distributed
+
+    wl, inp = workload(name), inputs(name)
+    sh = distributed.AzimuthShards(wl.nlon_in, wl.nlon_out, wl.C_in, A)
+    psi = gpu_psi(name)
+    x, w, b, dout = dev(inp["x"], wl), dev(inp["w"], wl), dev(inp["bias"], wl), dev(inp["dout"], wl)
+    has_b, G = b is not None, wl.groups
+    # standard
+    y = torch.cat([conv.disco_contract(psi, x[:, cb:ce].contiguous()) for cb, ce in sh.chans], dim=1)
+    out = np.zeros(oracle_out(name).shape)
+    dy = torch.empty_like(y)
+    dw, db = 0.0, 0.0
+    for qb, qe in sh.lon_out:
+        y_a, d_a = y[..., qb:qe].contiguous(), dout[..., qb:qe].contiguous()
+        out[..., qb:qe] = host(conv.mix(y_a, w, b, G))
+        dy[..., qb:qe] = conv.mix_adjoint(d_a, w, wl.C_in, G)
+        dw_a, db_a = conv.mix_weight(d_a, y_a, G, need_bias=has_b)
+        dw = dw + host(dw_a)
+        db = db + (host(db_a) if has_b else 0.0)
+    dx = torch.cat([conv.disco_contract_adjoint(psi, dy[:, cb:ce].contiguous()) for cb, ce in sh.chans], dim=1)
+    torch.cuda.synchronize()
+    check(out, oracle_out(name), tol(wl), "out from azimuth shards")
+    check(host(dx), oracle_dx(name), tol(wl), "dx from azimuth shards")
+    dw_ref, db_ref = oracle_dw(name)
+    check(dw, dw_ref, tol(wl), "dw from azimuth shards")
+    if has_b:
+        check(db, db_ref, tol(wl), "dbias from azimuth shards")
+    # reordered (fused)
+    out_f = np.zeros_like(out)
+    dx_f = np.zeros(inp["x"].shape)
+    dw_f = 0.0
+    for a, (cb, ce) in enumerate(sh.chans):
+        cols, mask = distributed.channel_shard(wl.C_in, wl.C_out, G, (cb, ce))
+        ws = distributed.shard_weight(w, cols, mask)
+        xc = x[:, cb:ce].contiguous()
+        out_f += host(conv.disco_forward(psi, xc, ws, b if a == 0 else None, 1, fused=True)[0])
+        dx_f[:, cb:ce] = host(conv.disco_backward_input(psi, dout, ws, ce - cb, 1))
+        dws, _ = conv.disco_backward_weight(psi, dout, x=xc, groups=1, need_bias=False)
+        dw_f = dw_f + host(distributed.unshard_weight_grad(dws, cols, mask, wl.C_out, wl.C_in // G))
+    torch.cuda.synchronize()
+    check(out_f, oracle_out(name), tol(wl), "fused out from channel shards")
+    check(dx_f, oracle_dx(name), tol(wl), "fused dx from channel shards")
+    check(dw_f, dw_ref, tol(wl), "fused dw from channel shards")
+
+
 def test_polar_layer_on_one_rank_matches_oracle():
-    """PolarDiscoConvS2 through autograd on a one-rank NCCL group (the whole layer is one band;
-    no transfers), unfused and fused, against the oracle."""
+    """PolarDiscoConvS2, PolarReduceScatterConvS2 and DistributedDiscoConvS2 (both polar modes)
+    through autograd on a one-rank NCCL group (the whole layer is one band and one longitude
+    shard; the collectives move nothing), unfused and fused, against the oracle."""
     import datetime
     import socket
 
     import torch.distributed as dist
 
-    from spherical_disco_convolution_b200 import polar
+    from spherical_disco_convolution_b200 import distributed, polar
 
     name = "ragged_down_bf16"
     wl, inp = workload(name), inputs(name)
@@ -445,5 +509,28 @@ def test_polar_layer_on_one_rank_matches_oracle():
             check(host(out), oracle_out(name), tol(wl), "polar layer out")
             check(host(x.grad), oracle_dx(name), tol(wl), "polar layer dx")
             check(host(layer.weight.grad), oracle_dw(name)[0], tol(wl), "polar layer dw")
+        # the reduce-scatter polar mode and the polar x azimuth layer, each on the 1 x 1 grid
+        layers = [("reduce-scatter", fused, polar.PolarReduceScatterConvS2) for fused in (False, True)]
+        layers += [(mode, fused, distributed.DistributedDiscoConvS2) for mode in distributed.POLAR_MODES
+                   for fused in (False, True)]
+        for mode, fused, cls in layers:
+            kw = dict(polar_mode=mode) if cls is distributed.DistributedDiscoConvS2 else {}
+            layer = cls(wl.C_in, wl.C_out, (wl.nlat_in, wl.nlon_in), (wl.nlat_out, wl.nlon_out), wl.kernel_shape,
+                        wl.theta_cutoff, groups=wl.groups, bias=True, fused=fused, device="cuda:0",
+                        dtype=torch.bfloat16, **kw)
+            bias = np.linspace(-1.0, 1.0, wl.C_out)
+            with torch.no_grad():
+                layer.weight.copy_(dev(inp["w"], wl))
+                layer.bias.copy_(dev(bias, wl))
+            x = dev(inp["x"], wl).requires_grad_(True)
+            out = layer(x)
+            out.backward(dev(inp["dout"], wl))
+            torch.cuda.synchronize()
+            what = f"{cls.__name__} {mode} fused={fused}"
+            ref = oracle_psi(name).forward(inp["x"], inp["w"], host(dev(bias, wl)), groups=wl.groups)
+            check(host(out), ref, tol(wl), what + " out")
+            check(host(x.grad), oracle_dx(name), tol(wl), what + " dx")
+            check(host(layer.weight.grad), oracle_dw(name)[0], tol(wl), what + " dw")
+            check(host(layer.bias.grad), inp["dout"].sum(axis=(0, 2, 3)), tol(wl), what + " dbias")
     finally:
         dist.destroy_process_group()

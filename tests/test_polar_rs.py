@@ -69,7 +69,7 @@ def _worker(rank, world, port, name, padded, q):
         if padded:
             # the one-collective path on equal padded chunks, its reduce-scatter emulated by a sum
             # and the rank's chunk (gloo has no reduce-scatter of its own)
-            def rs(out, inp):
+            def rs(out, inp, group=None):
                 s = inp.clone()
                 dist.all_reduce(s)
                 out.copy_(s.reshape((world, -1) + tuple(out.shape[1:]))[rank].reshape(out.shape))
