@@ -40,6 +40,21 @@ def _need_cuda(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError("libdisco takes contiguous CUDA tensors")
+    dts = {t.dtype for t in ts if t is not None}
+    if len(dts) > 1:
+        raise TypeError(f"libdisco takes tensors of one dtype; got {sorted(map(str, dts))}")
+
+
+def _shape(t, want, what):
+    """The C ABI sees only pointers: every tensor's shape is checked here, before a kernel reads it."""
+    if t is not None and tuple(t.shape) != tuple(want):
+        raise ValueError(f"{what} has shape {tuple(t.shape)}, expected {tuple(want)}")
+
+
+def _weight(w, C_out, C_in, groups, K):
+    if groups <= 0 or C_in % groups or C_out % groups:
+        raise ValueError(f"groups={groups} must divide C_in={C_in} and C_out={C_out}")
+    _shape(w, (C_out, C_in // groups, K), "w")
 
 
 class Psi:
@@ -99,6 +114,7 @@ def disco_contract(psi: Psi, x: torch.Tensor) -> torch.Tensor:
     """y = the K-expanded contraction of x with Psi, shape (B, C, K, nlat_out, nlon_out)."""
     _need_cuda(x)
     B, C = x.shape[:2]
+    _shape(x, (B, C) + psi.in_shape, "x")
     y = torch.empty((B, C, psi.K) + psi.out_shape, dtype=x.dtype, device=x.device)
     D.disco_contract(psi.handle, B, C, _dtype_code(x), _ptr(x), _ptr(y), _stream(x.device))
     return y
@@ -109,6 +125,9 @@ def disco_forward(psi: Psi, x: torch.Tensor, w: torch.Tensor, bias=None, groups:
     _need_cuda(x, w, bias)
     B, C_in = x.shape[:2]
     C_out = w.shape[0]
+    _shape(x, (B, C_in) + psi.in_shape, "x")
+    _weight(w, C_out, C_in, groups, psi.K)
+    _shape(bias, (C_out,), "bias")
     dt = _dtype_code(x)
     out = torch.empty((B, C_out) + psi.out_shape, dtype=x.dtype, device=x.device)
     st = _stream(x.device)
@@ -127,6 +146,8 @@ def disco_forward(psi: Psi, x: torch.Tensor, w: torch.Tensor, bias=None, groups:
 def disco_backward_input(psi: Psi, dout: torch.Tensor, w: torch.Tensor, C_in: int, groups: int = 1):
     _need_cuda(dout, w)
     B, C_out = dout.shape[:2]
+    _shape(dout, (B, C_out) + psi.out_shape, "dout")
+    _weight(w, C_out, C_in, groups, psi.K)
     dt = _dtype_code(dout)
     dx = torch.empty((B, C_in) + psi.in_shape, dtype=dout.dtype, device=dout.device)
     ws, n = psi.workspace(D.DISCO_OP_BWD_INPUT, B, C_in, C_out, groups, dt)
@@ -139,8 +160,14 @@ def disco_backward_weight(psi: Psi, dout: torch.Tensor, y=None, x=None, groups: 
                           need_bias: bool = True):
     """(dw, dbias); y given, or x to recompute y."""
     _need_cuda(dout, y, x)
+    if y is None and x is None:
+        raise ValueError("give y, or x to recompute it")
     B, C_out = dout.shape[:2]
     C_in = y.shape[1] if y is not None else x.shape[1]
+    _shape(dout, (B, C_out) + psi.out_shape, "dout")
+    _shape(y, (B, C_in, psi.K) + psi.out_shape, "y")
+    _shape(x, (B, C_in) + psi.in_shape, "x")
+    _weight(None, C_out, C_in, groups, psi.K)
     dt = _dtype_code(dout)
     dw = torch.empty((C_out, C_in // groups, psi.K), dtype=dout.dtype, device=dout.device)
     db = torch.empty((C_out,), dtype=dout.dtype, device=dout.device) if need_bias else None
@@ -155,6 +182,7 @@ def disco_contract_adjoint(psi: Psi, dy: torch.Tensor) -> torch.Tensor:
     """dx = the adjoint of the contraction applied to dy (B, C, K, nlat_out, nlon_out)."""
     _need_cuda(dy)
     B, C = dy.shape[:2]
+    _shape(dy, (B, C, psi.K) + psi.out_shape, "dy")
     dx = torch.empty((B, C) + psi.in_shape, dtype=dy.dtype, device=dy.device)
     D.disco_contract_adjoint(psi.handle, B, C, _dtype_code(dy), _ptr(dy), _ptr(dx), _stream(dy.device))
     return dx
@@ -164,9 +192,13 @@ def mix(y: torch.Tensor, w: torch.Tensor, bias=None, groups: int = 1) -> torch.T
     """The weight einsum on any set of points: y (B, C_in, K, *pts) -> out (B, C_out, *pts)."""
     _need_cuda(y, w, bias)
     y = y.contiguous()
+    if y.dim() < 4:
+        raise ValueError(f"y has shape {tuple(y.shape)}, expected (B, C_in, K, *points)")
     B, C_in, K = y.shape[:3]
     pts = y.shape[3:]
     C_out = w.shape[0]
+    _weight(w, C_out, C_in, groups, K)
+    _shape(bias, (C_out,), "bias")
     out = torch.empty((B, C_out) + pts, dtype=y.dtype, device=y.device)
     D.disco_mix(B, C_in, C_out, groups, K, math.prod(pts), _dtype_code(y), _ptr(y), _ptr(w), _ptr(bias), _ptr(out),
                 _stream(y.device))
@@ -177,9 +209,12 @@ def mix_adjoint(dout: torch.Tensor, w: torch.Tensor, C_in: int, groups: int = 1)
     """The transposed weight einsum: dout (B, C_out, *pts) -> dy (B, C_in, K, *pts)."""
     _need_cuda(dout, w)
     dout = dout.contiguous()
+    if dout.dim() < 3 or w.dim() != 3:
+        raise ValueError("dout is (B, C_out, *points) and w (C_out, C_in/groups, K)")
     B, C_out = dout.shape[:2]
     pts = dout.shape[2:]
     K = w.shape[2]
+    _weight(w, C_out, C_in, groups, K)
     dt, n = _dtype_code(dout), math.prod(pts)
     dy = torch.empty((B, C_in, K) + pts, dtype=dout.dtype, device=dout.device)
     nb = D.disco_mix_workspace_size(D.DISCO_OP_EINSUM_ADJOINT, B, C_in, C_out, groups, K, n, dt)
@@ -195,6 +230,8 @@ def mix_weight(dout: torch.Tensor, y: torch.Tensor, groups: int = 1, need_bias: 
     dout, y = dout.contiguous(), y.contiguous()
     B, C_out = dout.shape[:2]
     C_in, K = y.shape[1:3]
+    _shape(y, (B, C_in, K) + tuple(dout.shape[2:]), "y")
+    _weight(None, C_out, C_in, groups, K)
     dt, n = _dtype_code(dout), math.prod(dout.shape[2:])
     dw = torch.empty((C_out, C_in // groups, K), dtype=dout.dtype, device=dout.device)
     db = torch.empty((C_out,), dtype=dout.dtype, device=dout.device) if need_bias else None

@@ -97,7 +97,8 @@ bool build_tiles(int n_out, int n_src, int n, int K, std::vector<RingTerm> terms
     return false;
   }
   const int R = n / 8;  // octets around the ring
-  const int bk = prm.bslot_bytes / kstep_bytes;
+  // K-steps of one item: the room a B slot has after its batch record
+  const int bk = (prm.bslot_bytes - kMetaBytes) / kstep_bytes;
   // offsets centred in (-n/2, n/2] so that an arc around offset 0 is one contiguous range
   for (RingTerm& t : terms) {
     t.off = ((t.off % n) + n) % n;
@@ -390,6 +391,10 @@ bool build_tiles(int n_out, int n_src, int n, int K, std::vector<RingTerm> terms
           ++n_items;
           if (4 + n_words > kMaxMetaWords) {
             msg = "tile plan: an item with more MMAs than a batch holds";
+            return false;
+          }
+          if (fill + bytes > b_cap) {
+            msg = "tile plan: an item with more K-steps than a B slot holds";
             return false;
           }
           items[t].batch = nbatch - 1;

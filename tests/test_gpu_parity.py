@@ -213,9 +213,26 @@ def test_invalid_calls_raise():
         conv.disco_forward(psi, x, w, None, wl.groups)
     assert e.value.status == D.DISCO_ERR_INVALID_ARG
     x = torch.zeros((1, wl.C_in, wl.nlat_in, wl.nlon_in), device="cuda:0")
-    with pytest.raises(D.DiscoError) as e:
-        conv.disco_forward(psi, x, w, None, 4)  # 4 divides neither 6 nor 9
+    y = torch.zeros((1, wl.C_in, wl.K, wl.nlat_out, wl.nlon_out), device="cuda:0")
+    out = torch.zeros((1, wl.C_out, wl.nlat_out, wl.nlon_out), device="cuda:0")
+    st = torch.cuda.current_stream().cuda_stream
+    with pytest.raises(D.DiscoError) as e:  # the library's own check, under the Python layer's
+        D.disco_fwd(psi.handle, 1, wl.C_in, wl.C_out, 4, D.DISCO_F32, x.data_ptr(), w.data_ptr(), None, y.data_ptr(),
+                    out.data_ptr(), None, 0, st)  # 4 divides neither 6 nor 9
     assert e.value.status == D.DISCO_ERR_INVALID_ARG
+    # the Python layer checks every shape before a kernel sees a pointer
+    with pytest.raises(ValueError):
+        conv.disco_forward(psi, x, w, None, 4)
+    with pytest.raises(ValueError):  # x of another grid
+        conv.disco_contract(psi, torch.zeros((1, wl.C_in, wl.nlat_in, wl.nlon_in + 1), device="cuda:0"))
+    with pytest.raises(ValueError):  # dy without its K axis
+        conv.disco_contract_adjoint(psi, torch.zeros((1, wl.C_in * wl.K, wl.nlat_out, wl.nlon_out), device="cuda:0"))
+    with pytest.raises(ValueError):  # w of another K
+        conv.mix(y, w[:, :, :1].contiguous(), None, wl.groups)
+    with pytest.raises(ValueError):  # y on other points than dout
+        conv.mix_weight(out, y[..., :-1].contiguous(), wl.groups)
+    with pytest.raises(TypeError):  # mixed dtypes
+        conv.disco_forward(psi, x, w.to(torch.bfloat16), None, wl.groups)
 
 
 @pytest.mark.parametrize("name", ["tc_small_bf16", "ring_k3", "weather", "grouped"])
