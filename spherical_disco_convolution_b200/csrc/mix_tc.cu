@@ -147,6 +147,211 @@ __global__ void __launch_bounds__(128, 2) mix_tc_kernel(const __grid_constant__ 
   if (warp == 2) tc::tmem_dealloc(tmem, ncols);
 }
 
+// ------------------------------------------------------------------ persistent form
+// The same GEMM with one CTA per SM looping over the (batch*group, M-tile of outputs, 128-point)
+// tiles, so that the loads of the next tile overlap the epilogue of the last:
+//   warp 4 (lane 0)  streams the `in` stages through a ring, and the W chunks of an M tile with
+//                    the first stage of a tile whose (group, M tile) differs from the previous
+//                    one (after every MMA that read the old W has completed);
+//   warp 5 (lane 0)  issues the MMAs into one of two accumulators in tensor memory;
+//   warps 0..3       drain an accumulator (TMEM lane = grid point), add the bias, stage the
+//                    bf16 tile [m][n] in shared memory and write it with TMA stores.
+// W stays in shared memory across the tiles of one (group, M tile), instead of being re-read
+// with every tile.  Every wait is bounded.
+
+struct MixPArgs {
+  const void* bias;
+  int G, Mg, Rg, N, BN, S, NT, MT, T;  // NT point tiles, MT output tiles, T tiles in all
+  int NO;                              // out staging buffers (2: a tile's stores overlap the next)
+};
+
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
+               "r"(tc::smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(192, 1) mix_tc_persistent_kernel(const __grid_constant__ CUtensorMap map_in,
+                                                                   const __grid_constant__ CUtensorMap map_w,
+                                                                   const __grid_constant__ CUtensorMap map_out,
+                                                                   MixPArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const int BN = a.BN, S = a.S;
+  const int nk = (a.Rg + kBK - 1) / kBK;
+  const uint32_t a_bytes = 2 * kHalfTile;
+  const uint32_t wc_bytes = (uint32_t)BN * 128;  // one 64-wide K chunk of W
+  uint8_t* sA = smem;                             // S stages of [64 K][128 M], MN-major
+  uint8_t* sW = sA + (size_t)S * a_bytes;         // nk chunks of [BN][64 K], K-major
+  uint8_t* sO = sW + (size_t)nk * wc_bytes;       // NO out tiles, each two halves [BN][64 n]
+  const size_t o_bytes = 2 * (size_t)BN * 128;
+  float* sBias = reinterpret_cast<float*>(sO + (size_t)a.NO * o_bytes);  // BN floats
+  uint64_t* full = reinterpret_cast<uint64_t*>(sBias + 256);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;   // [2]
+  uint64_t* tempty = tfull + 2;  // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ncols = tmem_cols(2 * BN);
+
+  if (threadIdx.x == 0) {
+    tc::prefetch_map(&map_in);
+    tc::prefetch_map(&map_w);
+    tc::prefetch_map(&map_out);
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&tfull[b], 1);
+      tc::mbar_init(&tempty[b], 4);
+    }
+    tc::fence_barrier_init();
+  }
+  if (warp == 5) {
+    tc::tmem_alloc(tmem_slot, ncols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  auto wkey = [&](int t) { return t / a.NT; };  // (batch*group, M tile): W and bias change with it
+  // a contiguous run of tiles per CTA: consecutive tiles read the next points of the same planes
+  const int t_lo = (int)((long)a.T * blockIdx.x / gridDim.x), t_hi = (int)((long)a.T * (blockIdx.x + 1) / gridDim.x);
+
+  if (warp == 4) {
+    if (lane == 0) {
+      uint32_t gs = 0;  // stages loaded so far
+      int prev_key = -1;
+      bool ok = true;
+      for (int t = t_lo; t < t_hi && ok; ++t) {
+        const int nt = t % a.NT, rest = t / a.NT, mt = rest % a.MT, bg = rest / a.MT, g = bg % a.G;
+        const bool wload = wkey(t) != prev_key;
+        prev_key = wkey(t);
+        for (int kc = 0; kc < nk && ok; ++kc, ++gs) {
+          const int s = (int)(gs % (uint32_t)S);
+          if (gs >= (uint32_t)S) ok = tc::mbar_wait_sleep(&empty[s], ((gs / S) - 1) & 1u);
+          if (!ok) break;
+          const bool wl = wload && kc == 0;
+          if (wl && gs > 0) {
+            // every MMA that read the old W has completed: the commit of the last stage loaded
+            const uint32_t gp = gs - 1;
+            ok = tc::mbar_wait_sleep(&empty[gp % S], (gp / S) & 1u);
+            if (!ok) break;
+          }
+          tc::mbar_arrive_expect_tx(&full[s], a_bytes + (wl ? (uint32_t)nk * wc_bytes : 0u));
+          if (wl)
+            for (int c = 0; c < nk; ++c)
+              tc::tma_load_2d(sW + (size_t)c * wc_bytes, &map_w, &full[s], c * kBK, g * a.Mg + mt * BN);
+          tc::tma_load_3d(sA + (size_t)s * a_bytes, &map_in, &full[s], nt * 128, kc * kBK, bg);
+          tc::tma_load_3d(sA + (size_t)s * a_bytes + kHalfTile, &map_in, &full[s], nt * 128 + 64, kc * kBK, bg);
+        }
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16(128, BN, true, false);
+      uint32_t gs = 0, i = 0;
+      bool ok = true;
+      for (int t = t_lo; t < t_hi && ok; ++t, ++i) {
+        const uint32_t acc = i & 1u, use = i >> 1;
+        if (use >= 1) ok = tc::mbar_wait_sleep(&tempty[acc], (use - 1) & 1u);
+        if (!ok) break;
+        tc::fence_after_sync();
+        const uint32_t d = tmem + acc * (uint32_t)BN;
+        for (int kc = 0; kc < nk && ok; ++kc, ++gs) {
+          const int s = (int)(gs % (uint32_t)S);
+          ok = tc::mbar_wait(&full[s], (gs / S) & 1u);
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint32_t a0 = tc::smem_u32(sA + (size_t)s * a_bytes);
+          const uint32_t b0 = tc::smem_u32(sW + (size_t)kc * wc_bytes);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = tc::desc_sw128(a0 + kk * 2048, kHalfTile, 1024);
+            const uint64_t bd = tc::desc_sw128(b0 + kk * 32, 16, 1024);
+            tc::mma_bf16(d, ad, bd, idesc, (kc | kk) != 0);
+          }
+          tc::mma_commit(&empty[s]);
+        }
+        if (ok) tc::mma_commit(&tfull[acc]);
+      }
+    }
+  } else {
+    // epilogue: warps 0..3, TMEM lanes 32*warp.., grid point n = 128*nt + 32*warp + lane
+    const int row = warp * 32 + lane;
+    const int half = row >> 6;
+    const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
+    const size_t orow = (size_t)half * BN * 128 + (size_t)(row & 63) * 2;
+    uint32_t i = 0;
+    int prev_key = -1;
+    bool ok = true;
+    for (int t = t_lo; t < t_hi; ++t, ++i) {
+      const int nt = t % a.NT, rest = t / a.NT, mt = rest % a.MT, bg = rest / a.MT, g = bg % a.G;
+      const uint32_t acc = i & 1u, use = i >> 1;
+      if (wkey(t) != prev_key) {
+        // the bias of this (group, M tile); the previous tile's readers are past the barrier below
+        for (int m = threadIdx.x; m < BN; m += 128) {
+          const int o = mt * BN + m;
+          sBias[m] = (bias && o < a.Mg) ? __bfloat162float(bias[g * a.Mg + o]) : 0.0f;
+        }
+        prev_key = wkey(t);
+      }
+      int good = 1;
+      if (lane == 0) good = tc::mbar_wait_sleep(&tfull[acc], use & 1u);
+      ok = __shfl_sync(0xffffffffu, good, 0) != 0;
+      // this tile's out staging is free once the stores that last read it are done with it (the
+      // previous tile's with one buffer, the one before with two); one decision for the four warps
+      uint8_t* ob = sO + (size_t)(i % (uint32_t)a.NO) * o_bytes;
+      if (threadIdx.x == 0) {
+        if (a.NO == 2)
+          tc::bulk_wait_read_le<1>();
+        else
+          tc::bulk_wait_read0();
+      }
+      ok = tc::named_bar_and(1, 128, ok);
+      if (!ok) break;
+      tc::fence_after_sync();
+      const uint32_t tb = tmem + ((uint32_t)(warp * 32) << 16) + acc * (uint32_t)BN;
+      uint8_t* orow_p = ob + orow;
+      int c = 0;
+      // 64 columns per wait: the loads of a group are in flight together
+      for (; c + 64 <= BN; c += 64) {
+        uint32_t v[64];
+        tc::tmem_ld_chunks<4>(tb + (uint32_t)c, v);
+#pragma unroll
+        for (int e = 0; e < 64; ++e)
+          *reinterpret_cast<__nv_bfloat16*>(orow_p + (size_t)(c + e) * 128) =
+              __float2bfloat16_rn(__uint_as_float(v[e]) + sBias[c + e]);
+      }
+      for (; c < BN; c += 16) {
+        uint32_t v[16];
+        tc::tmem_ld_chunks<1>(tb + (uint32_t)c, v);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          *reinterpret_cast<__nv_bfloat16*>(orow_p + (size_t)(c + e) * 128) =
+              __float2bfloat16_rn(__uint_as_float(v[e]) + sBias[c + e]);
+      }
+      // accumulator drained: the MMA issuer may reuse it
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+      tc::fence_proxy_async();
+      tc::named_bar_sync(1, 128);
+      if (threadIdx.x == 0) {
+        tma_store_3d(&map_out, ob, nt * 128, mt * BN, bg);
+        tma_store_3d(&map_out, ob + (size_t)BN * 128, nt * 128 + 64, mt * BN, bg);
+        tc::bulk_commit();
+      }
+    }
+    if (threadIdx.x == 0) tc::bulk_wait0();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 5) tc::tmem_dealloc(tmem, ncols);
+}
+
 struct DwTcArgs {
   float* part;
   float* bpart;  // written here when ones_row (dbias as the product with a row of ones), else null
@@ -307,9 +512,56 @@ bool mix_tc_supported(int Mg, int Rg, int N) {
   return tc::encode_tiled_fn() != nullptr && Mg % 16 == 0 && Rg % 8 == 0 && N % 8 == 0 && (mix_bn(Mg) % 16 == 0);
 }
 
+// Shared memory of the persistent form with S stages (the 1 KB alignment slack included).
+size_t mixp_smem(int BN, int nk, int S, int NO) {
+  return 1024 + (size_t)S * 2 * kHalfTile + (size_t)nk * BN * 128 + (size_t)NO * 2 * BN * 128 + 256 * 4 +
+         (2 * (size_t)S + 4) * 8 + 16;
+}
+
 cudaError_t launch_mix_tc(const MixArgs& a, cudaStream_t st) {
-  CUtensorMap mi, mw;
+  CUtensorMap mi, mw, mo;
   const int BN = mix_bn(a.Mg);
+  const int nk = (a.Rg + kBK - 1) / kBK;
+  // two out staging buffers when four stages still fit beside them, else one
+  int NO = 2, S = 8;
+  while (S >= 4 && mixp_smem(BN, nk, S, NO) > kTcSmemLimit) --S;
+  if (S < 4) {
+    NO = 1;
+    S = 8;
+    while (S >= 2 && mixp_smem(BN, nk, S, NO) > kTcSmemLimit) --S;
+  }
+  // the persistent form where it measured faster: up to 128 outputs per tile (the weight einsum
+  // of the 721x1440 and 361x720 layers); the transposed einsum's 192-row tiles keep the
+  // one-tile kernel, which ran them faster
+  if (S >= 2 && BN <= 128 && !(reinterpret_cast<uintptr_t>(a.out) & 15)) {
+    const cuuint64_t di[3] = {(cuuint64_t)a.N, (cuuint64_t)a.Rg, (cuuint64_t)a.B * a.G};
+    const cuuint64_t si[2] = {(cuuint64_t)a.N * 2, (cuuint64_t)a.Rg * a.N * 2};
+    const cuuint32_t bi[3] = {64, 64, 1};
+    const cuuint64_t dw[2] = {(cuuint64_t)a.Rg, (cuuint64_t)a.G * a.Mg};
+    const cuuint64_t sw[1] = {(cuuint64_t)a.Rg * 2};
+    const cuuint32_t bw[2] = {64, (cuuint32_t)BN};
+    const cuuint64_t dq[3] = {(cuuint64_t)a.N, (cuuint64_t)a.Mg, (cuuint64_t)a.B * a.G};
+    const cuuint64_t sq[2] = {(cuuint64_t)a.N * 2, (cuuint64_t)a.Mg * a.N * 2};
+    const cuuint32_t bq[3] = {64, (cuuint32_t)BN, 1};
+    if (!make_map(&mi, a.in, 3, di, si, bi) || !make_map(&mw, a.wm, 2, dw, sw, bw) ||
+        !tc::encode_bf16_map(&mo, a.out, 3, dq, sq, bq, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    int dev = 0, n_sm = 148;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int NT = (a.N + 127) / 128, MT = (a.Mg + BN - 1) / BN;
+    const long T = (long)NT * MT * a.B * a.G;
+    if (T > 0x7FFFFFFFL) return cudaErrorInvalidValue;
+    MixPArgs p{a.bias, a.G, a.Mg, a.Rg, a.N, BN, S, NT, MT, (int)T, NO};
+    // at least half the shared memory, so that one CTA (and its tensor memory) holds an SM
+    const size_t smem = std::max(mixp_smem(BN, nk, S, NO), (size_t)kTcSmemLimit / 2 + 1024);
+    e = cudaFuncSetAttribute(mix_tc_persistent_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    mix_tc_persistent_kernel<<<(int)std::min<long>(T, n_sm), 192, smem, st>>>(mi, mw, mo, p);
+    count_launch();
+    return cudaGetLastError();
+  }
   const cuuint64_t di[3] = {(cuuint64_t)a.N, (cuuint64_t)a.Rg, (cuuint64_t)a.B * a.G};
   const cuuint64_t si[2] = {(cuuint64_t)a.N * 2, (cuuint64_t)a.Rg * a.N * 2};
   const cuuint32_t bi[3] = {64, 64, 1};
@@ -317,9 +569,9 @@ cudaError_t launch_mix_tc(const MixArgs& a, cudaStream_t st) {
   const cuuint64_t sw[1] = {(cuuint64_t)a.Rg * 2};
   const cuuint32_t bw[2] = {64, (cuuint32_t)BN};
   if (!make_map(&mi, a.in, 3, di, si, bi) || !make_map(&mw, a.wm, 2, dw, sw, bw)) return cudaErrorInvalidValue;
-  const int S = std::min(kStages, (a.Rg + kBK - 1) / kBK);
-  MixTcArgs t{a.out, a.bias, a.G, a.Mg, a.Rg, a.N, BN, S};
-  const size_t smem = mix_smem(BN, S);
+  const int S1 = std::min(kStages, nk);
+  MixTcArgs t{a.out, a.bias, a.G, a.Mg, a.Rg, a.N, BN, S1};
+  const size_t smem = mix_smem(BN, S1);
   cudaError_t e = cudaFuncSetAttribute(mix_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.N + 127) / 128, (a.Mg + BN - 1) / BN, a.B * a.G);
