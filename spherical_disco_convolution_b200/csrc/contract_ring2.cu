@@ -185,6 +185,17 @@ __device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
 __device__ __forceinline__ bool wait_batches(const uint32_t* done, uint32_t target, uint32_t max_sleep_ns) {
   if (ld_acquire(done) >= target) return true;
   const unsigned long long t0 = tc::globaltimer();
+  if (max_sleep_ns == 0) {
+    // no sleep: the x producer and the B warp, whose wake-up would delay the slots they refill
+    while (true) {
+      for (int i = 0; i < 64; ++i)
+        if (ld_acquire(done) >= target) return true;
+      if (tc::globaltimer() - t0 > tc::kWaitNs) {
+        atomicExch(&g_device_status, 5);
+        return false;
+      }
+    }
+  }
   uint32_t ns = 32;
   while (true) {
     if (ld_acquire(done) >= target) return true;
@@ -201,6 +212,9 @@ template <int K, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                       const __grid_constant__ CUtensorMap ymap,
                                                                       Args a) {
+  // the x producer and the B warp spin on the batch counter in the plain contraction; in the
+  // fused forms, whose epilogue warps share their issue slots, they sleep between polls
+  constexpr uint32_t kProducerSleepNs = kFused ? 256u : 0u;
   constexpr int N = 16 * K;
   constexpr uint32_t kWBytes = kFused ? (uint32_t)K * 8192u : 0u;  // W_k tiles [64 o][64 c] of the mix
   extern __shared__ uint8_t smem_raw[];
@@ -276,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
             if (s == slot) need = rel[s];
           int good = 1;
           if (lane == 0) {
-            if (need) good = wait_batches(done, need, 256);
+            if (need) good = wait_batches(done, need, kProducerSleepNs);
             if (good) {
               const int src = ld.x & 0xFFFF, sbar = (ld.x >> 16) & 0xFFFF;
               tc::mbar_arrive_expect_tx(&xfull[slot], (uint32_t)__popc(mask) * (uint32_t)kChunkBytes);
@@ -322,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1) contract_ring2_kernel(const __gri
           const int n = (w0 >> 24) & 0xFF;
           int good = 1;
           if (lane == 0) {
-            if (nbatch >= (uint32_t)a.nbs) good = wait_batches(done, nbatch - a.nbs + 1, 256);
+            if (nbatch >= (uint32_t)a.nbs) good = wait_batches(done, nbatch - a.nbs + 1, kProducerSleepNs);
             if (good) tc::mbar_arrive_expect_tx(&bfull[bslot], (uint32_t)((w0 >> 8) & 0xFFFF));
           }
           ok = __shfl_sync(0xffffffffu, good, 0) != 0;
