@@ -171,6 +171,7 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
                : "memory");
 }
 
+template <int H>  // 128-point halves per tile: a tile reads 128*H consecutive points of each plane
 __global__ void __launch_bounds__(192, 1) mix_tc_persistent_kernel(const __grid_constant__ CUtensorMap map_in,
                                                                    const __grid_constant__ CUtensorMap map_w,
                                                                    const __grid_constant__ CUtensorMap map_out,
@@ -179,12 +180,12 @@ __global__ void __launch_bounds__(192, 1) mix_tc_persistent_kernel(const __grid_
   uint8_t* smem = align1024(smem_raw);
   const int BN = a.BN, S = a.S;
   const int nk = (a.Rg + kBK - 1) / kBK;
-  const uint32_t a_bytes = 2 * kHalfTile;
+  const uint32_t a_bytes = 2 * H * kHalfTile;
   const uint32_t wc_bytes = (uint32_t)BN * 128;  // one 64-wide K chunk of W
-  uint8_t* sA = smem;                             // S stages of [64 K][128 M], MN-major
+  uint8_t* sA = smem;                             // S stages of H x [64 K][128 M], MN-major
   uint8_t* sW = sA + (size_t)S * a_bytes;         // nk chunks of [BN][64 K], K-major
-  uint8_t* sO = sW + (size_t)nk * wc_bytes;       // NO out tiles, each two halves [BN][64 n]
-  const size_t o_bytes = 2 * (size_t)BN * 128;
+  uint8_t* sO = sW + (size_t)nk * wc_bytes;       // NO out tiles, each 2H quarters [BN][64 n]
+  const size_t o_bytes = 2 * H * (size_t)BN * 128;
   float* sBias = reinterpret_cast<float*>(sO + (size_t)a.NO * o_bytes);  // BN floats
   uint64_t* full = reinterpret_cast<uint64_t*>(sBias + 256);
   uint64_t* empty = full + S;
@@ -192,7 +193,7 @@ __global__ void __launch_bounds__(192, 1) mix_tc_persistent_kernel(const __grid_
   uint64_t* tempty = tfull + 2;  // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t ncols = tmem_cols(2 * BN);
+  const uint32_t ncols = tmem_cols(2 * H * BN);
 
   if (threadIdx.x == 0) {
     tc::prefetch_map(&map_in);
@@ -244,8 +245,9 @@ __global__ void __launch_bounds__(192, 1) mix_tc_persistent_kernel(const __grid_
           if (wl)
             for (int c = 0; c < nk; ++c)
               tc::tma_load_2d(sW + (size_t)c * wc_bytes, &map_w, &full[s], c * kBK, g * a.Mg + mt * BN);
-          tc::tma_load_3d(sA + (size_t)s * a_bytes, &map_in, &full[s], nt * 128, kc * kBK, bg);
-          tc::tma_load_3d(sA + (size_t)s * a_bytes + kHalfTile, &map_in, &full[s], nt * 128 + 64, kc * kBK, bg);
+          for (int q = 0; q < 2 * H; ++q)
+            tc::tma_load_3d(sA + (size_t)s * a_bytes + (size_t)q * kHalfTile, &map_in, &full[s], nt * 128 * H + 64 * q,
+                            kc * kBK, bg);
         }
       }
     }
@@ -259,19 +261,22 @@ __global__ void __launch_bounds__(192, 1) mix_tc_persistent_kernel(const __grid_
         if (use >= 1) ok = tc::mbar_wait_sleep(&tempty[acc], (use - 1) & 1u);
         if (!ok) break;
         tc::fence_after_sync();
-        const uint32_t d = tmem + acc * (uint32_t)BN;
+        const uint32_t d = tmem + acc * (uint32_t)(H * BN);
         for (int kc = 0; kc < nk && ok; ++kc, ++gs) {
           const int s = (int)(gs % (uint32_t)S);
           ok = tc::mbar_wait(&full[s], (gs / S) & 1u);
           if (!ok) break;
           tc::fence_after_sync();
-          const uint32_t a0 = tc::smem_u32(sA + (size_t)s * a_bytes);
           const uint32_t b0 = tc::smem_u32(sW + (size_t)kc * wc_bytes);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = tc::desc_sw128(a0 + kk * 2048, kHalfTile, 1024);
-            const uint64_t bd = tc::desc_sw128(b0 + kk * 32, 16, 1024);
-            tc::mma_bf16(d, ad, bd, idesc, (kc | kk) != 0);
+          for (int hh = 0; hh < H; ++hh) {
+            const uint32_t a0 = tc::smem_u32(sA + (size_t)s * a_bytes + (size_t)hh * 2 * kHalfTile);
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t ad = tc::desc_sw128(a0 + kk * 2048, kHalfTile, 1024);
+              const uint64_t bd = tc::desc_sw128(b0 + kk * 32, 16, 1024);
+              tc::mma_bf16(d + (uint32_t)(hh * BN), ad, bd, idesc, (kc | kk) != 0);
+            }
           }
           tc::mma_commit(&empty[s]);
         }
@@ -281,9 +286,7 @@ __global__ void __launch_bounds__(192, 1) mix_tc_persistent_kernel(const __grid_
   } else {
     // epilogue: warps 0..3, TMEM lanes 32*warp.., grid point n = 128*nt + 32*warp + lane
     const int row = warp * 32 + lane;
-    const int half = row >> 6;
     const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(a.bias);
-    const size_t orow = (size_t)half * BN * 128 + (size_t)(row & 63) * 2;
     uint32_t i = 0;
     int prev_key = -1;
     bool ok = true;
@@ -313,25 +316,29 @@ __global__ void __launch_bounds__(192, 1) mix_tc_persistent_kernel(const __grid_
       ok = tc::named_bar_and(1, 128, ok);
       if (!ok) break;
       tc::fence_after_sync();
-      const uint32_t tb = tmem + ((uint32_t)(warp * 32) << 16) + acc * (uint32_t)BN;
-      uint8_t* orow_p = ob + orow;
-      int c = 0;
-      // 64 columns per wait: the loads of a group are in flight together
-      for (; c + 64 <= BN; c += 64) {
-        uint32_t v[64];
-        tc::tmem_ld_chunks<4>(tb + (uint32_t)c, v);
+      for (int hh = 0; hh < H; ++hh) {
+        // point hh*128 + row of the tile: quarter (hh*128 + row) / 64 of the staging
+        const uint32_t tb = tmem + ((uint32_t)(warp * 32) << 16) + acc * (uint32_t)(H * BN) + (uint32_t)(hh * BN);
+        const int pq = hh * 128 + row;
+        uint8_t* orow_p = ob + (size_t)(pq >> 6) * BN * 128 + (size_t)(pq & 63) * 2;
+        int c = 0;
+        // 64 columns per wait: the loads of a group are in flight together
+        for (; c + 64 <= BN; c += 64) {
+          uint32_t v[64];
+          tc::tmem_ld_chunks<4>(tb + (uint32_t)c, v);
 #pragma unroll
-        for (int e = 0; e < 64; ++e)
-          *reinterpret_cast<__nv_bfloat16*>(orow_p + (size_t)(c + e) * 128) =
-              __float2bfloat16_rn(__uint_as_float(v[e]) + sBias[c + e]);
-      }
-      for (; c < BN; c += 16) {
-        uint32_t v[16];
-        tc::tmem_ld_chunks<1>(tb + (uint32_t)c, v);
+          for (int e = 0; e < 64; ++e)
+            *reinterpret_cast<__nv_bfloat16*>(orow_p + (size_t)(c + e) * 128) =
+                __float2bfloat16_rn(__uint_as_float(v[e]) + sBias[c + e]);
+        }
+        for (; c < BN; c += 16) {
+          uint32_t v[16];
+          tc::tmem_ld_chunks<1>(tb + (uint32_t)c, v);
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          *reinterpret_cast<__nv_bfloat16*>(orow_p + (size_t)(c + e) * 128) =
-              __float2bfloat16_rn(__uint_as_float(v[e]) + sBias[c + e]);
+          for (int e = 0; e < 16; ++e)
+            *reinterpret_cast<__nv_bfloat16*>(orow_p + (size_t)(c + e) * 128) =
+                __float2bfloat16_rn(__uint_as_float(v[e]) + sBias[c + e]);
+        }
       }
       // accumulator drained: the MMA issuer may reuse it
       tc::fence_before_sync();
@@ -340,8 +347,8 @@ __global__ void __launch_bounds__(192, 1) mix_tc_persistent_kernel(const __grid_
       tc::fence_proxy_async();
       tc::named_bar_sync(1, 128);
       if (threadIdx.x == 0) {
-        tma_store_3d(&map_out, ob, nt * 128, mt * BN, bg);
-        tma_store_3d(&map_out, ob + (size_t)BN * 128, nt * 128 + 64, mt * BN, bg);
+        for (int q = 0; q < 2 * H; ++q)
+          tma_store_3d(&map_out, ob + (size_t)q * BN * 128, nt * 128 * H + 64 * q, mt * BN, bg);
         tc::bulk_commit();
       }
     }
@@ -513,8 +520,8 @@ bool mix_tc_supported(int Mg, int Rg, int N) {
 }
 
 // Shared memory of the persistent form with S stages (the 1 KB alignment slack included).
-size_t mixp_smem(int BN, int nk, int S, int NO) {
-  return 1024 + (size_t)S * 2 * kHalfTile + (size_t)nk * BN * 128 + (size_t)NO * 2 * BN * 128 + 256 * 4 +
+size_t mixp_smem(int BN, int nk, int S, int NO, int H) {
+  return 1024 + (size_t)S * 2 * H * kHalfTile + (size_t)nk * BN * 128 + (size_t)NO * 2 * H * BN * 128 + 256 * 4 +
          (2 * (size_t)S + 4) * 8 + 16;
 }
 
@@ -522,13 +529,21 @@ cudaError_t launch_mix_tc(const MixArgs& a, cudaStream_t st) {
   CUtensorMap mi, mw, mo;
   const int BN = mix_bn(a.Mg);
   const int nk = (a.Rg + kBK - 1) / kBK;
-  // two out staging buffers when four stages still fit beside them, else one
-  int NO = 2, S = 8;
-  while (S >= 4 && mixp_smem(BN, nk, S, NO) > kTcSmemLimit) --S;
-  if (S < 4) {
-    NO = 1;
+  // the wider tile (128*H points, H = 2, else 1) when its two accumulators fit tensor memory and
+  // its stages fit shared memory at least twice; two out staging buffers when four stages still
+  // fit beside them, else one.  (256 points: weather einsum 0.145 -> 0.134 ms; 512 points, with
+  // room for two stages only, 0.137 ms.)
+  int H = 2, NO = 2, S = 8;
+  for (;; H >>= 1) {
+    NO = 2;
     S = 8;
-    while (S >= 2 && mixp_smem(BN, nk, S, NO) > kTcSmemLimit) --S;
+    while (S >= 4 && mixp_smem(BN, nk, S, NO, H) > kTcSmemLimit) --S;
+    if (S < 4) {
+      NO = 1;
+      S = 8;
+      while (S >= 2 && mixp_smem(BN, nk, S, NO, H) > kTcSmemLimit) --S;
+    }
+    if (H == 1 || (2 * H * BN <= 512 && S >= 2)) break;
   }
   // the persistent form where it measured faster: up to 128 outputs per tile (the weight einsum
   // of the 721x1440 and 361x720 layers); the transposed einsum's 192-row tiles keep the
@@ -550,15 +565,16 @@ cudaError_t launch_mix_tc(const MixArgs& a, cudaStream_t st) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    const int NT = (a.N + 127) / 128, MT = (a.Mg + BN - 1) / BN;
+    const int NT = (a.N + 128 * H - 1) / (128 * H), MT = (a.Mg + BN - 1) / BN;
     const long T = (long)NT * MT * a.B * a.G;
     if (T > 0x7FFFFFFFL) return cudaErrorInvalidValue;
     MixPArgs p{a.bias, a.G, a.Mg, a.Rg, a.N, BN, S, NT, MT, (int)T, NO};
     // at least half the shared memory, so that one CTA (and its tensor memory) holds an SM
-    const size_t smem = std::max(mixp_smem(BN, nk, S, NO), (size_t)kTcSmemLimit / 2 + 1024);
-    e = cudaFuncSetAttribute(mix_tc_persistent_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = std::max(mixp_smem(BN, nk, S, NO, H), (size_t)kTcSmemLimit / 2 + 1024);
+    auto kern = H == 2 ? mix_tc_persistent_kernel<2> : mix_tc_persistent_kernel<1>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    mix_tc_persistent_kernel<<<(int)std::min<long>(T, n_sm), 192, smem, st>>>(mi, mw, mo, p);
+    kern<<<(int)std::min<long>(T, n_sm), 192, smem, st>>>(mi, mw, mo, p);
     count_launch();
     return cudaGetLastError();
   }
