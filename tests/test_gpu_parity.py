@@ -493,6 +493,43 @@ def test_azimuth_shards_reassemble_the_full_layer(name, A):
     check(dw_f, dw_ref, tol(wl), "fused dw from channel shards")
 
 
+@pytest.mark.parametrize("B,C_in,C_out,G,K,npts,bias", [
+    (1, 64, 128, 1, 3, 4104, True),     # 128 outputs per tile, 256-point tiles (all 512 TMEM columns)
+    (2, 64, 64, 2, 3, 1000, False),     # 32 outputs per group, ragged last tile, no bias
+    (1, 32, 16, 1, 5, 776, True),       # 16 outputs, K = 5 (K-chunks past the rows read as zeros)
+    (1, 64, 256, 1, 3, 2056, True),     # 256 outputs: the one-tile kernel
+    (1, 64, 128, 1, 9, 1032, True),     # 128 outputs, K = 9: the persistent kernel with 128-point tiles
+    (1, 64, 64, 1, 3, 1001, True),      # a point count TMA cannot address: the SIMT kernel
+])
+def test_weight_einsum_on_points_matches_fp64(B, C_in, C_out, G, K, npts, bias):
+    """disco_mix, disco_mix_adjoint and disco_mix_weight on bf16 inputs against the same sums in
+    fp64 on the host (the einsum of the forward equation and its two adjoints), over the tile
+    shapes the launcher picks: every output tile size, both point-tile widths, groups, a ragged
+    last tile and no bias."""
+    rng = np.random.default_rng(B * 1000 + C_out + npts)
+    bf = lambda a: torch.from_numpy(a).to(torch.bfloat16)  # noqa: E731
+    y = bf(rng.standard_normal((B, C_in, K, npts)))
+    w = bf(rng.standard_normal((C_out, C_in // G, K)) / math.sqrt(C_in // G * K))
+    b = bf(rng.standard_normal(C_out)) if bias else None
+    dout = bf(rng.standard_normal((B, C_out, npts)))
+    yh, wh, dh = (t.double().numpy() for t in (y, w, dout))
+    Og, Cg = C_out // G, C_in // G
+    ref = np.einsum("gock,bgckn->bgon", wh.reshape(G, Og, Cg, K), yh.reshape(B, G, Cg, K, npts)).reshape(B, C_out, npts)
+    if bias:
+        ref = ref + b.double().numpy()[None, :, None]
+    dy_ref = np.einsum("gock,bgon->bgckn", wh.reshape(G, Og, Cg, K), dh.reshape(B, G, Og, npts)).reshape(yh.shape)
+    dw_ref = np.einsum("bgon,bgckn->gock", dh.reshape(B, G, Og, npts), yh.reshape(B, G, Cg, K, npts)).reshape(wh.shape)
+    dev0 = "cuda:0"
+    out = conv.mix(y.to(dev0), w.to(dev0), None if b is None else b.to(dev0), G)
+    dy = conv.mix_adjoint(dout.to(dev0), w.to(dev0), C_in, G)
+    dw, db = conv.mix_weight(dout.to(dev0), y.to(dev0), G, need_bias=True)
+    torch.cuda.synchronize()
+    check(host(out), ref, 2e-2, "mix")
+    check(host(dy), dy_ref, 2e-2, "mix_adjoint")
+    check(host(dw), dw_ref, 2e-2, "mix_weight dw")
+    check(host(db), dh.sum(axis=(0, 2)), 2e-2, "mix_weight dbias")
+
+
 def test_polar_layer_on_one_rank_matches_oracle():
     """PolarDiscoConvS2, PolarReduceScatterConvS2 and DistributedDiscoConvS2 (both polar modes)
     through autograd on a one-rank NCCL group (the whole layer is one band and one longitude
